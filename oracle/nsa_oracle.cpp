@@ -1,0 +1,634 @@
+// ORACLE — test infrastructure, not product code.
+//
+// A plain, slow, single-threaded fp64 CPU statement of what the LSRM
+// native-sparse-attention (NSA) layer computes.  Only the tests, the smoke
+// check and the benchmark's CPU-baseline leg may load it; the CUDA path shares
+// no code, header, table or helper with it.
+//
+// Sources (the pages this follows; "LSRM page" = hyper.ai "LSRM" summary,
+// "Speed3R page" = gist.science "Speed3R" technical summary):
+//   compression  k_cmp = AvgPool(ResBlock(k_t)), v_cmp likewise  — LSRM page, 方法,
+//                equations k^cmp / v^cmp.  ResBlock is a trained module and is
+//                taken as the identity, so compression is the block mean.
+//   score routing: NSA selects KV blocks by attention scores against the
+//                compressed keys — LSRM page, 方法, 3D-aware routing paragraph.
+//   geometric routing: nearest volume blocks by 3D Euclidean distance between
+//                block centres — LSRM page, same paragraph.
+//   branches: compressed context + selected blocks (fine detail) — LSRM page,
+//                方法 (after the k^cmp equations); window attention computed
+//                locally inside whole blocks — LSRM page, sequence-parallel
+//                paragraph; Speed3R page, 2.1 (compression / selection branches).
+//   gates: Sigmoid(Linear(x)) gate values weight the branch outputs — LSRM page,
+//                方法, gate equations; Speed3R page, 2.1 gated aggregation.
+//
+// Readings where the pages are silent (each also listed in the design notes):
+//   * softmax scale tau = 1/sqrt(d); query head h uses KV group floor(h / (Hq/Hkv)).
+//   * score routing is per (query block, KV group): Score[a,g,j] is the SUM over
+//     the block's tokens and the group's heads of the compressed-branch softmax
+//     probabilities p_cmp[t,h,j]; top-k by (score desc, j asc).
+//   * geometric routing: centroid c[b] = round-half-up(sum of the block's lattice
+//     coordinates / n_b) per axis, i.e. floor((2S + n) / (2n)); distance
+//     D = sum over axes of (c[a] - c[j])^2 in int64; top-k by (D asc, j asc);
+//     one index list per query block, shared by every KV group.
+//   * window: W(t) = { u in block(t) : r(t) - w/2 <= r(u) <= r(t) + w/2 - 1 },
+//     r = position inside the block; w = 0 switches the branch off.
+//   * the selected key set of (a, g) is the union of the forced blocks and the
+//     routed blocks (as a set).
+//   * Speed3R variant (pooled_q = 1): the compressed branch uses the block-mean
+//     query Qbar[beta(t)] and its output is copied to every token of the block;
+//     routing is top-k by the raw pooled logit tau * Qbar . Kbar over the blocks
+//     that are not forced; there is no window branch.
+//
+// Top-k everywhere: a full std::sort on (key, index).  Softmax: max-subtracted
+// in fp64.  Inputs arrive as bf16 bit patterns and are widened exactly (or, for
+// finite-difference checks, as doubles).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+struct Desc {
+  int64_t n_tokens;
+  int32_t n_blocks;
+  int32_t n_q_heads, n_kv_heads, head_dim;
+  int32_t top_k, window;
+  double scale;      // 0 -> 1/sqrt(d)
+  int32_t pooled_q;  // 0 LSRM, 1 Speed3R
+  int32_t n_gates;   // 3 (cmp, slc, win) or 2 (cmp, slc)
+};
+
+inline double bf(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+inline double bf(double x) { return x; }  // fp64 inputs (finite-difference checks)
+
+inline double tau_of(const Desc& D) { return D.scale > 0 ? D.scale : 1.0 / std::sqrt((double)D.head_dim); }
+
+inline int64_t floor_div(int64_t a, int64_t b) {  // b > 0
+  int64_t q = a / b;
+  if ((a % b != 0) && (a < 0)) --q;
+  return q;
+}
+
+// softmax-weighted sum over a key list: keys/values are row pointers.
+// out[d] = sum_u p_u v_u, p = softmax(tau q.k_u); returns the natural-log LSE.
+double attend(const std::vector<double>& q, const std::vector<const double*>& keys,
+              const std::vector<const double*>& vals, int d, double tau, double* out) {
+  const size_t n = keys.size();
+  for (int c = 0; c < d; ++c) out[c] = 0.0;
+  if (n == 0) return -INFINITY;
+  std::vector<double> s(n);
+  double m = -INFINITY;
+  for (size_t u = 0; u < n; ++u) {
+    double acc = 0.0;
+    for (int c = 0; c < d; ++c) acc += q[c] * keys[u][c];
+    s[u] = tau * acc;
+    m = std::max(m, s[u]);
+  }
+  double l = 0.0;
+  for (size_t u = 0; u < n; ++u) { s[u] = std::exp(s[u] - m); l += s[u]; }
+  for (size_t u = 0; u < n; ++u) {
+    const double p = s[u] / l;
+    for (int c = 0; c < d; ++c) out[c] += p * vals[u][c];
+  }
+  return m + std::log(l);
+}
+
+// widen a [N][H][d] bf16 tensor to double
+template <typename T>
+std::vector<double> widen(const T* x, size_t count) {
+  std::vector<double> r(count);
+  for (size_t i = 0; i < count; ++i) r[i] = bf(x[i]);
+  return r;
+}
+
+template <typename T>
+void mean_pool(const Desc& D, const int32_t* off, const T* x, int32_t H, double* out) {
+  const int d = D.head_dim;
+  for (int32_t b = 0; b < D.n_blocks; ++b) {
+    const int64_t n = (int64_t)off[b + 1] - off[b];
+    for (int32_t h = 0; h < H; ++h)
+      for (int c = 0; c < d; ++c) {
+        double s = 0.0;
+        for (int64_t t = off[b]; t < off[b + 1]; ++t) s += bf(x[(t * H + h) * d + c]);
+        out[((int64_t)b * H + h) * d + c] = n > 0 ? s / (double)n : 0.0;
+      }
+  }
+}
+
+// the key set of the selected branch for (query block a, index row `row`)
+std::vector<int32_t> selected_blocks(const Desc& D, const int32_t* row, int32_t n_forced, const int32_t* forced) {
+  std::vector<int32_t> s(forced, forced + n_forced);
+  for (int i = 0; i < D.top_k; ++i) s.push_back(row[i]);
+  std::sort(s.begin(), s.end());
+  s.erase(std::unique(s.begin(), s.end()), s.end());
+  return s;
+}
+
+// ---- templated statements of each step (T = uint16_t bf16 bits, or double)
+
+// ---- S1: block mean-pool.  out[b][h][c] = (1/n_b) sum_{t in b} x[t][h][c]
+template <typename T>
+int impl_compress(const Desc* D, const int32_t* off, const T* x, int32_t n_heads, double* out) {
+  mean_pool(*D, off, x, n_heads, out);
+  return 0;
+}
+
+// ---- S2b: geometric routing.  idx [B][k]; centroids [B][3] (int64) optional.
+template <typename T>
+int impl_route_geometric(const Desc* D, const int32_t* off, const int32_t* coords, int32_t* idx,
+                           int64_t* centroids) {
+  const int32_t B = D->n_blocks, k = D->top_k;
+  std::vector<int64_t> c((size_t)B * 3);
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t n = (int64_t)off[b + 1] - off[b];
+    for (int a = 0; a < 3; ++a) {
+      int64_t S = 0;
+      for (int64_t t = off[b]; t < off[b + 1]; ++t) S += coords[t * 3 + a];
+      c[(size_t)b * 3 + a] = floor_div(2 * S + n, 2 * n);
+    }
+  }
+  if (centroids) std::memcpy(centroids, c.data(), c.size() * sizeof(int64_t));
+  std::vector<std::pair<int64_t, int32_t>> key((size_t)B);
+  for (int32_t a = 0; a < B; ++a) {
+    for (int32_t j = 0; j < B; ++j) {
+      int64_t dist = 0;
+      for (int ax = 0; ax < 3; ++ax) {
+        const int64_t e = c[(size_t)a * 3 + ax] - c[(size_t)j * 3 + ax];
+        dist += e * e;
+      }
+      key[(size_t)j] = {dist, j};
+    }
+    std::sort(key.begin(), key.end());
+    for (int i = 0; i < k; ++i) idx[(int64_t)a * k + i] = key[(size_t)i].second;
+  }
+  return 0;
+}
+
+// ---- S2a: score routing for the listed query blocks.
+// kc: [B][Hkv][d] compressed keys (double).  idx out [nq][Hkv][k]; score out [nq][Hkv][B] (optional).
+template <typename T>
+int impl_route_score(const Desc* D, const int32_t* off, const T* q, const double* kc,
+                       int32_t n_qb, const int32_t* qblocks, int32_t* idx, double* score) {
+  const int32_t B = D->n_blocks, Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim, k = D->top_k;
+  const int32_t G = Hq / Hkv;
+  const double tau = tau_of(*D);
+  std::vector<double> sc((size_t)Hkv * B), s((size_t)B);
+  std::vector<std::pair<double, int32_t>> key;
+  for (int32_t qi = 0; qi < n_qb; ++qi) {
+    const int32_t a = qblocks[qi];
+    std::fill(sc.begin(), sc.end(), 0.0);
+    for (int64_t t = off[a]; t < off[a + 1]; ++t)
+      for (int32_t h = 0; h < Hq; ++h) {
+        const int32_t g = h / G;
+        double m = -INFINITY;
+        for (int32_t j = 0; j < B; ++j) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += bf(q[(t * Hq + h) * d + c]) * kc[((size_t)j * Hkv + g) * d + c];
+          s[(size_t)j] = tau * acc;
+          m = std::max(m, s[(size_t)j]);
+        }
+        double l = 0.0;
+        for (int32_t j = 0; j < B; ++j) { s[(size_t)j] = std::exp(s[(size_t)j] - m); l += s[(size_t)j]; }
+        for (int32_t j = 0; j < B; ++j) sc[(size_t)g * B + j] += s[(size_t)j] / l;
+      }
+    for (int32_t g = 0; g < Hkv; ++g) {
+      key.resize((size_t)B);
+      for (int32_t j = 0; j < B; ++j) key[(size_t)j] = {-sc[(size_t)g * B + j], j};
+      std::sort(key.begin(), key.end());
+      for (int i = 0; i < k; ++i) idx[((int64_t)qi * Hkv + g) * k + i] = key[(size_t)i].second;
+      if (score) std::memcpy(score + ((int64_t)qi * Hkv + g) * B, sc.data() + (size_t)g * B, sizeof(double) * B);
+    }
+  }
+  return 0;
+}
+
+// ---- Speed3R routing: per (a, h) top-k by tau*Qbar[a,h].Kbar[j,h] over non-forced j.
+// qc [B][H][d], kc [B][H][d]; idx out [nq][H][k]; logits out [nq][H][B] optional.
+template <typename T>
+int impl_route_pooled(const Desc* D, const double* qc, const double* kc, int32_t n_forced,
+                        const int32_t* forced, int32_t n_qb, const int32_t* qblocks, int32_t* idx,
+                        double* logits) {
+  const int32_t B = D->n_blocks, H = D->n_q_heads, d = D->head_dim, k = D->top_k;
+  const double tau = tau_of(*D);
+  std::vector<char> is_forced((size_t)B, 0);
+  for (int32_t i = 0; i < n_forced; ++i) is_forced[(size_t)forced[i]] = 1;
+  std::vector<std::pair<double, int32_t>> key;
+  for (int32_t qi = 0; qi < n_qb; ++qi) {
+    const int32_t a = qblocks[qi];
+    for (int32_t h = 0; h < H; ++h) {
+      key.clear();
+      for (int32_t j = 0; j < B; ++j) {
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += qc[((size_t)a * H + h) * d + c] * kc[((size_t)j * H + h) * d + c];
+        const double lg = tau * acc;
+        if (logits) logits[((int64_t)qi * H + h) * B + j] = lg;
+        if (!is_forced[(size_t)j]) key.push_back({-lg, j});
+      }
+      std::sort(key.begin(), key.end());
+      for (int i = 0; i < k; ++i)
+        idx[((int64_t)qi * H + h) * k + i] = i < (int)key.size() ? key[(size_t)i].second : -1;
+    }
+  }
+  return 0;
+}
+
+// ---- S3: compressed branch for the listed query blocks.  o [tokens of listed blocks][Hq][d]
+// (compacted in list order), lse [..][Hq] (natural log).  kc, vc: [B][Hkv][d];
+// qc: [B][Hq][d] block-mean queries (used when pooled_q = 1).
+template <typename T>
+int impl_cmp_attn(const Desc* D, const int32_t* off, const T* q, const double* kc, const double* vc,
+                    const double* qc, int32_t n_qb, const int32_t* qblocks, double* o, double* lse) {
+  const int32_t B = D->n_blocks, Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim;
+  const int32_t G = Hq / Hkv;
+  const double tau = tau_of(*D);
+  std::vector<const double*> keys((size_t)B), vals((size_t)B);
+  std::vector<double> qv((size_t)d);
+  int64_t row = 0;
+  for (int32_t qi = 0; qi < n_qb; ++qi) {
+    const int32_t a = qblocks[qi];
+    const int64_t row0 = row;
+    for (int64_t t = off[a]; t < off[a + 1]; ++t, ++row)
+      for (int32_t h = 0; h < Hq; ++h) {
+        if (D->pooled_q && t > off[a]) {
+          // pooled query: every token of the block receives the block's output
+          for (int c = 0; c < d; ++c) o[(row * Hq + h) * d + c] = o[(row0 * Hq + h) * d + c];
+          if (lse) lse[row * Hq + h] = lse[row0 * Hq + h];
+          continue;
+        }
+        const int32_t g = h / G;
+        for (int32_t j = 0; j < B; ++j) {
+          keys[(size_t)j] = kc + ((size_t)j * Hkv + g) * d;
+          vals[(size_t)j] = vc + ((size_t)j * Hkv + g) * d;
+        }
+        for (int c = 0; c < d; ++c)
+          qv[(size_t)c] = D->pooled_q ? qc[((size_t)a * Hq + h) * d + c] : bf(q[(t * Hq + h) * d + c]);
+        const double L = attend(qv, keys, vals, d, tau, o + (row * Hq + h) * d);
+        if (lse) lse[row * Hq + h] = L;
+      }
+  }
+  return 0;
+}
+
+// ---- S4: selected branch.  idx rows: [B][idx_heads][k] with idx_heads in {1, Hkv};
+// group g reads row (idx_heads == 1 ? 0 : g).  Forced blocks join every key set.
+template <typename T>
+int impl_select_attn(const Desc* D, const int32_t* off, const T* q, const T* k,
+                       const T* v, const int32_t* idx, int32_t idx_heads, int32_t n_forced,
+                       const int32_t* forced, int32_t n_qb, const int32_t* qblocks, double* o, double* lse) {
+  const int32_t Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim, K = D->top_k;
+  const int32_t G = Hq / Hkv;
+  const double tau = tau_of(*D);
+  std::vector<double> qv((size_t)d);
+  int64_t row = 0;
+  for (int32_t qi = 0; qi < n_qb; ++qi) {
+    const int32_t a = qblocks[qi];
+    // widen the key/value rows of each group's selected set once per query block
+    std::vector<std::vector<double>> kw((size_t)Hkv), vw((size_t)Hkv);
+    for (int32_t g = 0; g < Hkv; ++g) {
+      const int32_t* r = idx + ((int64_t)a * idx_heads + (idx_heads == 1 ? 0 : g)) * K;
+      for (int32_t j : selected_blocks(*D, r, n_forced, forced))
+        for (int64_t u = off[j]; u < off[j + 1]; ++u)
+          for (int c = 0; c < d; ++c) {
+            kw[(size_t)g].push_back(bf(k[(u * Hkv + g) * d + c]));
+            vw[(size_t)g].push_back(bf(v[(u * Hkv + g) * d + c]));
+          }
+    }
+    for (int64_t t = off[a]; t < off[a + 1]; ++t, ++row)
+      for (int32_t h = 0; h < Hq; ++h) {
+        const int32_t g = h / G;
+        const size_t nk = kw[(size_t)g].size() / (size_t)d;
+        std::vector<const double*> keys(nk), vals(nk);
+        for (size_t u = 0; u < nk; ++u) { keys[u] = &kw[(size_t)g][u * d]; vals[u] = &vw[(size_t)g][u * d]; }
+        for (int c = 0; c < d; ++c) qv[(size_t)c] = bf(q[(t * Hq + h) * d + c]);
+        const double L = attend(qv, keys, vals, d, tau, o + (row * Hq + h) * d);
+        if (lse) lse[row * Hq + h] = L;
+      }
+  }
+  return 0;
+}
+
+// ---- S5: window branch, in-block band.
+template <typename T>
+int impl_window_attn(const Desc* D, const int32_t* off, const T* q, const T* k,
+                       const T* v, int32_t n_qb, const int32_t* qblocks, double* o, double* lse) {
+  const int32_t Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim, w = D->window;
+  const int32_t G = Hq / Hkv;
+  const double tau = tau_of(*D);
+  std::vector<double> qv((size_t)d);
+  int64_t row = 0;
+  for (int32_t qi = 0; qi < n_qb; ++qi) {
+    const int32_t a = qblocks[qi];
+    const int64_t n = (int64_t)off[a + 1] - off[a];
+    std::vector<double> kw((size_t)(n * Hkv * d)), vw((size_t)(n * Hkv * d));
+    for (int64_t r = 0; r < n; ++r)
+      for (int32_t g = 0; g < Hkv; ++g)
+        for (int c = 0; c < d; ++c) {
+          kw[(size_t)((r * Hkv + g) * d + c)] = bf(k[((off[a] + r) * Hkv + g) * d + c]);
+          vw[(size_t)((r * Hkv + g) * d + c)] = bf(v[((off[a] + r) * Hkv + g) * d + c]);
+        }
+    for (int64_t r = 0; r < n; ++r, ++row)
+      for (int32_t h = 0; h < Hq; ++h) {
+        const int32_t g = h / G;
+        std::vector<const double*> keys, vals;
+        if (w > 0)
+          for (int64_t u = 0; u < n; ++u)
+            if (u >= r - w / 2 && u <= r + w / 2 - 1) {
+              keys.push_back(&kw[(size_t)((u * Hkv + g) * d)]);
+              vals.push_back(&vw[(size_t)((u * Hkv + g) * d)]);
+            }
+        for (int c = 0; c < d; ++c) qv[(size_t)c] = bf(q[((off[a] + r) * Hq + h) * d + c]);
+        const double L = attend(qv, keys, vals, d, tau, o + (row * Hq + h) * d);
+        if (lse) lse[row * Hq + h] = L;
+      }
+  }
+  return 0;
+}
+
+// ---- S6 + S7: the layer output for the listed query blocks:
+//   O = g_cmp o_cmp + g_slc o_slc (+ g_win o_win).
+// branches (optional): [rows][Hq][n_gates][d]; lse (optional): [rows][Hq][n_gates].
+template <typename T>
+int impl_forward(const Desc* D, const int32_t* off, const T* q, const T* k, const T* v,
+                   const T* gates, const int32_t* idx, int32_t idx_heads, int32_t n_forced,
+                   const int32_t* forced, int32_t n_qb, const int32_t* qblocks, double* out, double* branches,
+                   double* lse) {
+  const int32_t B = D->n_blocks, Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim, NG = D->n_gates;
+  int64_t rows = 0;
+  for (int32_t qi = 0; qi < n_qb; ++qi) rows += (int64_t)off[qblocks[qi] + 1] - off[qblocks[qi]];
+  std::vector<double> kc((size_t)B * Hkv * d), vc((size_t)B * Hkv * d), qc;
+  mean_pool(*D, off, k, Hkv, kc.data());
+  mean_pool(*D, off, v, Hkv, vc.data());
+  if (D->pooled_q) { qc.resize((size_t)B * Hq * d); mean_pool(*D, off, q, Hq, qc.data()); }
+  std::vector<double> oc((size_t)(rows * Hq * d)), os((size_t)(rows * Hq * d)), ow((size_t)(rows * Hq * d), 0.0);
+  std::vector<double> lc((size_t)(rows * Hq)), ls((size_t)(rows * Hq)), lw((size_t)(rows * Hq), -INFINITY);
+  impl_cmp_attn<T>(D, off, q, kc.data(), vc.data(), qc.data(), n_qb, qblocks, oc.data(), lc.data());
+  impl_select_attn<T>(D, off, q, k, v, idx, idx_heads, n_forced, forced, n_qb, qblocks, os.data(), ls.data());
+  if (NG >= 3) impl_window_attn<T>(D, off, q, k, v, n_qb, qblocks, ow.data(), lw.data());
+  int64_t row = 0;
+  for (int32_t qi = 0; qi < n_qb; ++qi) {
+    const int32_t a = qblocks[qi];
+    for (int64_t t = off[a]; t < off[a + 1]; ++t, ++row)
+      for (int32_t h = 0; h < Hq; ++h) {
+        const T* gt = gates + (t * Hq + h) * NG;
+        const double* br[3] = {&oc[(size_t)((row * Hq + h) * d)], &os[(size_t)((row * Hq + h) * d)],
+                               &ow[(size_t)((row * Hq + h) * d)]};
+        const double* lb[3] = {&lc[(size_t)(row * Hq + h)], &ls[(size_t)(row * Hq + h)], &lw[(size_t)(row * Hq + h)]};
+        for (int c = 0; c < d; ++c) {
+          double acc = 0.0;
+          for (int b = 0; b < NG; ++b) acc += bf(gt[b]) * br[b][c];
+          out[(row * Hq + h) * d + c] = acc;
+        }
+        if (branches)
+          for (int b = 0; b < NG; ++b)
+            for (int c = 0; c < d; ++c) branches[((row * Hq + h) * NG + b) * d + c] = br[b][c];
+        if (lse)
+          for (int b = 0; b < NG; ++b) lse[(row * Hq + h) * NG + b] = *lb[b];
+      }
+  }
+  return 0;
+}
+
+// ---- S10: backward of the LSRM layer (pooled_q = 0) with the routing indices fixed.
+// Chain rule through the gated sum, the three softmax attentions and the mean-pool:
+//   dgates[t,h,b] = <dO[t,h], o_b[t,h]>,  dO_b = g_b dO,
+//   per branch: dV_u += sum_t P[t,u] dO_b[t];  dS[t,u] = P[t,u] (dO_b[t].V_u - dO_b[t].o_b[t]);
+//               dQ[t] += tau sum_u dS[t,u] K_u;   dK_u += tau sum_t dS[t,u] Q_t;
+//   compressed keys: dK[u] += dKbar[beta(u)] / n_beta(u) (and V likewise).
+// Outputs cover all tokens: dq [N][Hq][d], dk, dv [N][Hkv][d], dgates [N][Hq][n_gates].
+// nthreads > 1 splits the query blocks across threads; each thread keeps its own
+// key-side accumulators, which are summed in thread order.
+template <typename T>
+int impl_backward(const Desc* D, const int32_t* off, const T* q, const T* k, const T* v,
+                    const T* gates, const int32_t* idx, int32_t idx_heads, const T* dout,
+                    double* dq, double* dk, double* dv, double* dgates, int32_t nthreads) {
+  if (D->pooled_q) return 1;
+  const int32_t B = D->n_blocks, Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim, NG = D->n_gates;
+  const int32_t G = Hq / Hkv, K = D->top_k, w = D->window;
+  const int64_t N = D->n_tokens;
+  const double tau = tau_of(*D);
+  std::vector<double> kc((size_t)B * Hkv * d), vc((size_t)B * Hkv * d);
+  mean_pool(*D, off, k, Hkv, kc.data());
+  mean_pool(*D, off, v, Hkv, vc.data());
+  const std::vector<double> Kw = widen(k, (size_t)(N * Hkv * d)), Vw = widen(v, (size_t)(N * Hkv * d));
+  if (nthreads < 1) nthreads = 1;
+  const size_t kv_sz = (size_t)(N * Hkv * d), kvc_sz = (size_t)B * Hkv * d;
+  std::vector<std::vector<double>> dK(nthreads, std::vector<double>(kv_sz, 0.0)),
+      dV(nthreads, std::vector<double>(kv_sz, 0.0)), dKc(nthreads, std::vector<double>(kvc_sz, 0.0)),
+      dVc(nthreads, std::vector<double>(kvc_sz, 0.0));
+
+  auto work = [&](int tid) {
+    std::vector<double> qv((size_t)d), go((size_t)d), ob((size_t)d), dqv((size_t)d);
+    std::vector<double> s, p;
+    for (int32_t a = tid; a < B; a += nthreads) {
+      // per group: token ids of the selected set
+      std::vector<std::vector<int64_t>> sel((size_t)Hkv);
+      for (int32_t g = 0; g < Hkv; ++g) {
+        const int32_t* r = idx + ((int64_t)a * idx_heads + (idx_heads == 1 ? 0 : g)) * K;
+        for (int32_t j : selected_blocks(*D, r, 0, nullptr))
+          for (int64_t u = off[j]; u < off[j + 1]; ++u) sel[(size_t)g].push_back(u);
+      }
+      const int64_t n_a = (int64_t)off[a + 1] - off[a];
+      for (int64_t t = off[a]; t < off[a + 1]; ++t)
+        for (int32_t h = 0; h < Hq; ++h) {
+          const int32_t g = h / G;
+          for (int c = 0; c < d; ++c) { qv[(size_t)c] = bf(q[(t * Hq + h) * d + c]); dqv[(size_t)c] = 0.0; }
+          const T* gt = gates + (t * Hq + h) * NG;
+          for (int br = 0; br < NG; ++br) {
+            // key list of this branch: pointers into widened K/V (or compressed K/V)
+            std::vector<const double*> kp, vp;
+            std::vector<int64_t> tok;  // token id (or block id for the compressed branch)
+            if (br == 0) {
+              for (int32_t j = 0; j < B; ++j) {
+                kp.push_back(&kc[((size_t)j * Hkv + g) * d]);
+                vp.push_back(&vc[((size_t)j * Hkv + g) * d]);
+                tok.push_back(j);
+              }
+            } else if (br == 1) {
+              for (int64_t u : sel[(size_t)g]) {
+                kp.push_back(&Kw[(size_t)((u * Hkv + g) * d)]);
+                vp.push_back(&Vw[(size_t)((u * Hkv + g) * d)]);
+                tok.push_back(u);
+              }
+            } else if (w > 0) {
+              const int64_t r = t - off[a];
+              for (int64_t ru = 0; ru < n_a; ++ru)
+                if (ru >= r - w / 2 && ru <= r + w / 2 - 1) {
+                  const int64_t u = off[a] + ru;
+                  kp.push_back(&Kw[(size_t)((u * Hkv + g) * d)]);
+                  vp.push_back(&Vw[(size_t)((u * Hkv + g) * d)]);
+                  tok.push_back(u);
+                }
+            }
+            const size_t n = kp.size();
+            if (n == 0) { dgates[(t * Hq + h) * NG + br] = 0.0; continue; }
+            s.assign(n, 0.0);
+            double m = -INFINITY;
+            for (size_t u = 0; u < n; ++u) {
+              double acc = 0.0;
+              for (int c = 0; c < d; ++c) acc += qv[(size_t)c] * kp[u][c];
+              s[u] = tau * acc;
+              m = std::max(m, s[u]);
+            }
+            double l = 0.0;
+            for (size_t u = 0; u < n; ++u) { s[u] = std::exp(s[u] - m); l += s[u]; }
+            p.assign(n, 0.0);
+            for (int c = 0; c < d; ++c) ob[(size_t)c] = 0.0;
+            for (size_t u = 0; u < n; ++u) {
+              p[u] = s[u] / l;
+              for (int c = 0; c < d; ++c) ob[(size_t)c] += p[u] * vp[u][c];
+            }
+            const double gb = bf(gt[br]);
+            double dg = 0.0, Dt = 0.0;
+            for (int c = 0; c < d; ++c) {
+              const double g_out = bf(dout[(t * Hq + h) * d + c]);
+              dg += g_out * ob[(size_t)c];
+              go[(size_t)c] = gb * g_out;
+              Dt += go[(size_t)c] * ob[(size_t)c];
+            }
+            dgates[(t * Hq + h) * NG + br] = dg;
+            for (size_t u = 0; u < n; ++u) {
+              double dp = 0.0;
+              for (int c = 0; c < d; ++c) dp += go[(size_t)c] * vp[u][c];
+              const double ds = p[u] * (dp - Dt);
+              double* dkr;
+              double* dvr;
+              if (br == 0) {
+                dkr = &dKc[tid][((size_t)tok[u] * Hkv + g) * d];
+                dvr = &dVc[tid][((size_t)tok[u] * Hkv + g) * d];
+              } else {
+                dkr = &dK[tid][(size_t)((tok[u] * Hkv + g) * d)];
+                dvr = &dV[tid][(size_t)((tok[u] * Hkv + g) * d)];
+              }
+              for (int c = 0; c < d; ++c) {
+                dqv[(size_t)c] += tau * ds * kp[u][c];
+                dkr[c] += tau * ds * qv[(size_t)c];
+                dvr[c] += p[u] * go[(size_t)c];
+              }
+            }
+          }
+          for (int c = 0; c < d; ++c) dq[(t * Hq + h) * d + c] = dqv[(size_t)c];
+        }
+    }
+  };
+  if (nthreads == 1) work(0);
+  else {
+    std::vector<std::thread> th;
+    for (int i = 0; i < nthreads; ++i) th.emplace_back(work, i);
+    for (auto& x : th) x.join();
+  }
+  for (size_t i = 0; i < kv_sz; ++i) { dk[i] = 0.0; dv[i] = 0.0; }
+  for (int tid = 0; tid < nthreads; ++tid) {
+    for (size_t i = 0; i < kv_sz; ++i) { dk[i] += dK[(size_t)tid][i]; dv[i] += dV[(size_t)tid][i]; }
+  }
+  // mean-pool backward: every token of block b receives dKbar[b] / n_b
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t n = (int64_t)off[b + 1] - off[b];
+    for (int32_t g = 0; g < Hkv; ++g)
+      for (int c = 0; c < d; ++c) {
+        double gk = 0.0, gv = 0.0;
+        for (int tid = 0; tid < nthreads; ++tid) {
+          gk += dKc[(size_t)tid][((size_t)b * Hkv + g) * d + c];
+          gv += dVc[(size_t)tid][((size_t)b * Hkv + g) * d + c];
+        }
+        for (int64_t u = off[b]; u < off[b + 1]; ++u) {
+          dk[(u * Hkv + g) * d + c] += gk / (double)n;
+          dv[(u * Hkv + g) * d + c] += gv / (double)n;
+        }
+      }
+  }
+  return 0;
+}
+
+// ---- a scalar loss L = sum O * dO for the listed blocks (finite-difference checks of the backward)
+template <typename T>
+double impl_loss(const Desc* D, const int32_t* off, const T* q, const T* k, const T* v,
+                   const T* gates, const int32_t* idx, int32_t idx_heads, const T* dout) {
+  const int32_t B = D->n_blocks, Hq = D->n_q_heads, d = D->head_dim;
+  std::vector<int32_t> all((size_t)B);
+  for (int32_t b = 0; b < B; ++b) all[(size_t)b] = b;
+  std::vector<double> out((size_t)(D->n_tokens * Hq * d));
+  impl_forward<T>(D, off, q, k, v, gates, idx, idx_heads, 0, nullptr, B, all.data(), out.data(), nullptr, nullptr);
+  double L = 0.0;
+  for (size_t i = 0; i < out.size(); ++i) L += out[i] * bf(dout[i]);
+  return L;
+}
+
+
+}  // namespace
+
+// ------------------------------------------------------------------------------------------
+// C entry points.  "_bf16" functions take bf16 bit patterns (uint16); "_f64" functions take
+// doubles (used to perturb inputs by tiny steps for finite differences).
+// ------------------------------------------------------------------------------------------
+extern "C" {
+
+int oracle_compress(const Desc* D, const int32_t* off, const uint16_t* x, int32_t n_heads, double* out) {
+  return impl_compress<uint16_t>(D, off, x, n_heads, out);
+}
+int oracle_compress_f64(const Desc* D, const int32_t* off, const double* x, int32_t n_heads, double* out) {
+  return impl_compress<double>(D, off, x, n_heads, out);
+}
+int oracle_route_geometric(const Desc* D, const int32_t* off, const int32_t* coords, int32_t* idx,
+                           int64_t* centroids) {
+  return impl_route_geometric<uint16_t>(D, off, coords, idx, centroids);
+}
+int oracle_route_score(const Desc* D, const int32_t* off, const uint16_t* q, const double* kc, int32_t n_qb,
+                       const int32_t* qblocks, int32_t* idx, double* score) {
+  return impl_route_score<uint16_t>(D, off, q, kc, n_qb, qblocks, idx, score);
+}
+int oracle_route_pooled(const Desc* D, const double* qc, const double* kc, int32_t n_forced, const int32_t* forced,
+                        int32_t n_qb, const int32_t* qblocks, int32_t* idx, double* logits) {
+  return impl_route_pooled<uint16_t>(D, qc, kc, n_forced, forced, n_qb, qblocks, idx, logits);
+}
+int oracle_cmp_attn(const Desc* D, const int32_t* off, const uint16_t* q, const double* kc, const double* vc,
+                    const double* qc, int32_t n_qb, const int32_t* qblocks, double* o, double* lse) {
+  return impl_cmp_attn<uint16_t>(D, off, q, kc, vc, qc, n_qb, qblocks, o, lse);
+}
+int oracle_select_attn(const Desc* D, const int32_t* off, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       const int32_t* idx, int32_t idx_heads, int32_t n_forced, const int32_t* forced, int32_t n_qb,
+                       const int32_t* qblocks, double* o, double* lse) {
+  return impl_select_attn<uint16_t>(D, off, q, k, v, idx, idx_heads, n_forced, forced, n_qb, qblocks, o, lse);
+}
+int oracle_window_attn(const Desc* D, const int32_t* off, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       int32_t n_qb, const int32_t* qblocks, double* o, double* lse) {
+  return impl_window_attn<uint16_t>(D, off, q, k, v, n_qb, qblocks, o, lse);
+}
+int oracle_forward(const Desc* D, const int32_t* off, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const uint16_t* gates, const int32_t* idx, int32_t idx_heads, int32_t n_forced,
+                   const int32_t* forced, int32_t n_qb, const int32_t* qblocks, double* out, double* branches,
+                   double* lse) {
+  return impl_forward<uint16_t>(D, off, q, k, v, gates, idx, idx_heads, n_forced, forced, n_qb, qblocks, out,
+                                branches, lse);
+}
+int oracle_forward_f64(const Desc* D, const int32_t* off, const double* q, const double* k, const double* v,
+                       const double* gates, const int32_t* idx, int32_t idx_heads, int32_t n_forced,
+                       const int32_t* forced, int32_t n_qb, const int32_t* qblocks, double* out, double* branches,
+                       double* lse) {
+  return impl_forward<double>(D, off, q, k, v, gates, idx, idx_heads, n_forced, forced, n_qb, qblocks, out,
+                              branches, lse);
+}
+int oracle_backward(const Desc* D, const int32_t* off, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                    const uint16_t* gates, const int32_t* idx, int32_t idx_heads, const uint16_t* dout, double* dq,
+                    double* dk, double* dv, double* dgates, int32_t nthreads) {
+  return impl_backward<uint16_t>(D, off, q, k, v, gates, idx, idx_heads, dout, dq, dk, dv, dgates, nthreads);
+}
+int oracle_backward_f64(const Desc* D, const int32_t* off, const double* q, const double* k, const double* v,
+                        const double* gates, const int32_t* idx, int32_t idx_heads, const double* dout, double* dq,
+                        double* dk, double* dv, double* dgates, int32_t nthreads) {
+  return impl_backward<double>(D, off, q, k, v, gates, idx, idx_heads, dout, dq, dk, dv, dgates, nthreads);
+}
+double oracle_loss_f64(const Desc* D, const int32_t* off, const double* q, const double* k, const double* v,
+                       const double* gates, const int32_t* idx, int32_t idx_heads, const double* dout) {
+  return impl_loss<double>(D, off, q, k, v, gates, idx, idx_heads, dout);
+}
+
+}  // extern "C"
