@@ -1,0 +1,350 @@
+#!/usr/bin/env python3
+"""Benchmark of the LSRM native-sparse-attention layer forward on B200.
+
+Workload: the LSRM sparse stage with 3D-aware geometric routing — 1384 volume
+bricks on the 0.35-0.45 shell of a 64^3 grid + 16 views of 64x64 image tokens
+with 32 of 64 tiles kept (121344 tokens, 1896 blocks of 64), GQA 32/2, d 32,
+geometric top-16, window 64, seeded synthetic bf16 inputs.
+
+One step = one pass of the whole hot path through the C ABI: block mean-pool
+(lsrm_nsa_compress), geometric routing (lsrm_route_geometric), and the fused
+three-branch attention with the gated combine in its epilogue (lsrm_nsa_attend).
+`value` is tokens/s over all ranks with inputs already in HBM; `e2e` is the same
+metric through lsrm_nsa_forward with pinned host buffers, host<->device copies
+inside the timed region.  `--impl reference` times the fp64 CPU oracle instead
+(a bounded sample of query blocks per step, on the host cores).
+
+Multi-GPU: the layer does not shard on one GPU's worth of work here (one
+instance per GPU), so N ranks run N independent replicas ("scaling": "weak");
+the only collectives are the timing barrier and a max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn fwd tokens/s and effective TFLOP/s vs B200 bf16 tensor peak"
+WORKLOAD = "lsrm_sparse_stage_geometric_top16"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-sample-blocks", type=int, default=24,
+                    help="query blocks of the oracle's bounded CPU sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def algorithmic_flops(w, idx: np.ndarray) -> dict:
+    """4 * d * sum over (token, head) of the keys each branch attends (cmp: B block
+    means; slc: tokens of the routed blocks; win: in-block band)."""
+    off = w.off.astype(np.int64)
+    n = np.diff(off)
+    B, Hq, d = w.n_blocks, w.n_q_heads, w.head_dim
+    N = int(off[-1])
+    cmp = N * Hq * B
+    sel_tokens = n[idx].sum(axis=1) if idx.ndim == 2 else n[idx].sum(axis=-1).mean(axis=1)
+    slc = float((n * sel_tokens).sum()) * Hq
+    win = 0
+    if w.window > 0 and w.n_gates >= 3:
+        for nb in np.unique(n):
+            r = np.arange(nb)
+            lo = np.maximum(0, r - w.window // 2)
+            hi = np.minimum(nb - 1, r + w.window // 2 - 1)
+            win += int((hi - lo + 1).sum()) * int((n == nb).sum())
+        win *= Hq
+    f = 4 * d
+    return {"cmp": f * cmp, "slc": f * slc, "win": f * win, "total": f * (cmp + slc + win)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------------
+# the oracle on the host: cpu_baseline of our arm, and the whole reference arm
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample(w, idx, n_blocks: int, seed: int):
+    """Time the fp64 oracle on a seeded sample of query blocks of the workload (1 thread)."""
+    import oracle as O
+    D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window,
+                   n_gates=w.n_gates)
+    rng = np.random.default_rng(seed)
+    qb = np.sort(rng.choice(w.n_blocks, size=n_blocks, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, qblocks=qb)
+    dt = time.perf_counter() - t0
+    tokens = int((w.off[qb + 1] - w.off[qb]).sum())
+    return tokens, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from workloads import make_workload
+    import oracle as O
+    w = make_workload("sparse", seed=args.seed)
+    D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window)
+    idx, _ = O.route_geometric(D, w.off, w.coords)
+    per_step = 2  # query blocks per step: ~1 s of fp64 work each on one core
+    for s in range(args.warmup):
+        oracle_sample(w, idx, per_step, 1000 + s)
+    tok, tsum = 0, 0.0
+    for s in range(args.steps):
+        t, dt = oracle_sample(w, idx, per_step, s)
+        tok += t
+        tsum += dt
+    value = tok / tsum
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * tsum / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
+                       "heads": "32q/2kv", "head_dim": 32, "top_k": 16, "window": 64,
+                       "sample": f"{per_step} seeded query blocks per step"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{per_step} query blocks ({per_step * 64} tokens) per step, fp64, 1 thread"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+
+    from block_sparse_gqa_nsa_b200 import nsa
+    from block_sparse_gqa_nsa_b200.build import build
+    from workloads import make_workload
+
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    nsa.load_library()
+
+    w = make_workload("sparse", seed=args.seed)
+    N, B, Hq, Hkv, d, k = w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    h_q, h_k, h_v, h_g = bf(w.q), bf(w.k), bf(w.v), bf(w.gates)
+    h_off = torch.from_numpy(w.off.astype(np.int32))
+    h_coords = torch.from_numpy(w.coords.astype(np.int32))
+    q, kk, v, gates = h_q.to(dev), h_k.to(dev), h_v.to(dev), h_g.to(dev)
+    off, coords = h_off.to(dev), h_coords.to(dev)
+    desc = nsa.make_desc(N, B, w.max_block_len, Hq, Hkv, d, k, w.window, 0.0, False, w.n_gates)
+    ws = nsa.workspace(desc, dev)
+    kc = torch.empty(B, Hkv, d, dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+    out = torch.empty(N, Hq, d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        nsa.lsrm_nsa_compress(desc, off, None, kk, v, None, kc, None, vc, None, None, ws)
+        nsa.lsrm_route_geometric(desc, off, coords, idx, ws)
+        if e is not None:
+            e[1].record(stream)
+        nsa.lsrm_nsa_attend(desc, off, q, kk, v, kc, vc, gates, idx, 1, 0, out, None, ws)
+        if e is not None:
+            e[2].record(stream)
+
+    launches_per_step = 4  # compress, centroids, top-k, fused attention
+    for _ in range(max(3, args.warmup)):
+        step()
+    st = nsa.lsrm_nsa_last_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    flops = algorithmic_flops(w, idx.cpu().numpy())
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = t_start.elapsed_time(t_end)
+    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    pre_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * N * args.steps / (total_ms / 1000.0)
+
+    # end to end through lsrm_nsa_forward with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        p_q, p_k, p_v, p_g = h_q.pin_memory(), h_k.pin_memory(), h_v.pin_memory(), h_g.pin_memory()
+        p_off, p_c = h_off.pin_memory(), h_coords.pin_memory()
+        p_out = torch.empty(N, Hq, d, dtype=torch.bfloat16).pin_memory()
+        d_q, d_k, d_v, d_g = torch.empty_like(q), torch.empty_like(kk), torch.empty_like(v), torch.empty_like(gates)
+        d_off, d_c = torch.empty_like(off), torch.empty_like(coords)
+        d_out = torch.empty_like(out)
+        ins = ((d_q, p_q), (d_k, p_k), (d_v, p_v), (d_g, p_g), (d_off, p_off), (d_c, p_c))
+
+        def e2e_step():
+            for dst, src in ins:
+                dst.copy_(src, non_blocking=True)
+            nsa.lsrm_nsa_forward(desc, d_off, d_q, d_k, d_v, d_g, d_c, nsa.ROUTE_GEOMETRIC, d_out, None, None, ws)
+            p_out.copy_(d_out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(src.numel() * src.element_size() for _, src in ins)
+        d2h = p_out.numel() * p_out.element_size()
+        e2e = {"value": world * N * args.steps / (float(te.item()) / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        if not np.array_equal(p_out.view(torch.int16).numpy(), out.view(torch.int16).cpu().numpy()):
+            raise RuntimeError("end-to-end output differs from the device-resident run")
+
+    if rank == 0:
+        peaks, src = measured_peaks()
+        attn_avg = sum(attn_ms) / len(attn_ms)
+        achieved = flops["total"] / (attn_avg / 1000.0) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "n_tokens": N, "n_blocks": B, "heads": f"{Hq}q/{Hkv}kv",
+                           "head_dim": d, "top_k": k, "window": w.window, "route": "geometric",
+                           "parallelism": f"replicas{world}" if world > 1 else "single",
+                           "l2": "inputs larger than L2 (q 249 MB + out 249 MB per step)", "seed": args.seed},
+                "effective_tflops": flops["total"] / (ms_per_step / 1000.0) / 1e12,
+                "flops_per_step": flops,
+                "kernel_ms": {"fused_attention": attn_avg, "compress_and_route": sum(pre_ms) / len(pre_ms)},
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                             "frac": achieved / peak, "traffic": None,
+                             "kernel": "nsa_attn (fused cmp+slc+win attention, gated combine)",
+                             "peak_source": f"{src} bf16_tflops (burst)"},
+                "gpu_launches": launches_per_step * args.steps,
+                "clocks": clocks, "e2e": e2e}
+        if not args.no_cpu_baseline and world == 1:
+            tok, dt = oracle_sample(w, idx.cpu().numpy(), args.cpu_sample_blocks, 7)
+            line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"{args.cpu_sample_blocks} seeded query blocks ({tok} tokens) "
+                                              f"of the same workload, fp64, 1 thread, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,310 @@
+// C entry points of liblsrm_nsa.so: argument validation, workspace carving and
+// kernel launches.  Every pointer is caller-owned device memory; nothing here
+// allocates.  See include/lsrm_nsa.h for the contract of each call.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "lsrm_common.cuh"
+
+namespace lsrm {
+lsrm_status launch_compress(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
+                            float* kc32, void* kc, float* vc32, void* vc, float* qc32, void* qc, cudaStream_t s);
+lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, const int32_t* coords, int32_t* cen,
+                                   int32_t* idx, uint32_t* status, cudaStream_t s);
+lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
+                               int32_t* idx, float* score, uint32_t* status, cudaStream_t s);
+lsrm_status launch_route_pooled(const lsrm_nsa_desc& d, const void* qc, const void* kc, int32_t* idx,
+                                uint32_t* status, cudaStream_t s);
+lsrm_status launch_gate_combine(const lsrm_nsa_desc& d, const float* oc, const float* os, const float* ow,
+                                const void* gates, void* out, cudaStream_t s);
+lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
+                        const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
+                        int route_all, int branches, void* out, float* obranch, float* lse, int lse_stride,
+                        int lse_first, uint32_t* status, cudaStream_t stream);
+lsrm_status launch_pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, const void* vc, float* o_blk,
+                              float* lse_blk, cudaStream_t s);
+lsrm_status launch_pooled_broadcast(const lsrm_nsa_desc& d, const int32_t* off, const float* o_blk,
+                                    const float* lse_blk, float* o_cmp, float* lse, cudaStream_t s);
+lsrm_status launch_attn_pooled_fused(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
+                                     const void* v, const void* gates, const int32_t* idx, const float* o_blk,
+                                     void* out, float* lse, uint32_t* status, cudaStream_t stream);
+lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
+                            const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
+                            unsigned char* ws_bwd, uint32_t* status, cudaStream_t stream);
+}  // namespace lsrm
+
+using namespace lsrm;
+
+namespace {
+
+constexpr int BR_CMP = 1, BR_SLC = 2, BR_WIN = 4;
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// shape checks shared by every call
+lsrm_status check_desc(const lsrm_nsa_desc* d) {
+  if (d == nullptr) return LSRM_ERR_INVALID_ARG;
+  if (d->n_tokens < 1 || d->n_blocks < 1 || d->n_blocks > d->n_tokens) return LSRM_ERR_INVALID_ARG;
+  if (d->n_tokens > (int64_t)INT32_MAX) return LSRM_ERR_UNSUPPORTED;
+  if (d->max_block_len < 1 || d->max_block_len > kMaxBlockLen) return LSRM_ERR_INVALID_ARG;
+  if (d->n_kv_heads < 1 || d->n_q_heads < d->n_kv_heads || d->n_q_heads % d->n_kv_heads) return LSRM_ERR_INVALID_ARG;
+  if (d->head_dim != 32 && d->head_dim != 64) return LSRM_ERR_UNSUPPORTED;
+  if (d->top_k < 1 || d->top_k > d->n_blocks) return LSRM_ERR_INVALID_ARG;
+  if (d->window < 0 || (d->window & 1)) return LSRM_ERR_INVALID_ARG;
+  if (!(d->scale >= 0.0f) || isinf(d->scale)) return LSRM_ERR_INVALID_ARG;
+  if (d->pooled_q != 0 && d->pooled_q != 1) return LSRM_ERR_INVALID_ARG;
+  if (d->n_gates != 2 && d->n_gates != 3) return LSRM_ERR_INVALID_ARG;
+  if (d->n_forced < 0 || (d->n_forced > 0 && d->forced_blocks == nullptr)) return LSRM_ERR_INVALID_ARG;
+  if (d->pooled_q && (d->n_q_heads != d->n_kv_heads || d->n_gates != 2)) return LSRM_ERR_INVALID_ARG;
+  if (d->pooled_q && d->top_k + d->n_forced > d->n_blocks) return LSRM_ERR_INVALID_ARG;
+  return LSRM_OK;
+}
+
+lsrm_status check_ws(const lsrm_nsa_desc* d, void* ws) {
+  if (ws == nullptr || !aligned(ws, 256)) return LSRM_ERR_WORKSPACE;
+  (void)d;
+  return LSRM_OK;
+}
+
+template <typename T>
+T* wsp(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<unsigned char*>(ws) + off);
+}
+
+uint32_t* status_of(void* ws) { return wsp<uint32_t>(ws, 0); }
+
+#define LSRM_TRY(x)                         \
+  do {                                      \
+    lsrm_status _s = (x);                   \
+    if (_s != LSRM_OK) return _s;           \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t lsrm_nsa_workspace_size(const lsrm_nsa_desc* desc) {
+  if (check_desc(desc) != LSRM_OK) return 0;
+  return workspace_layout(*desc).total;
+}
+
+lsrm_status lsrm_nsa_workspace_init(const lsrm_nsa_desc* desc, void* ws, size_t ws_bytes, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (ws_bytes < workspace_layout(*desc).total) return LSRM_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) != cudaSuccess) return LSRM_ERR_CUDA;
+  return LSRM_OK;
+}
+
+lsrm_status lsrm_nsa_compress(const lsrm_nsa_desc* desc, const int32_t* off, const void* q_or_null, const void* k,
+                              const void* v, float* kc32, void* kc, float* vc32, void* vc, float* qc32_or_null,
+                              void* qc_or_null, void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  if (off == nullptr || k == nullptr || v == nullptr) return LSRM_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || (q_or_null && !aligned(q_or_null, 16))) return LSRM_ERR_INVALID_ARG;
+  (void)ws;
+  return launch_compress(*desc, off, q_or_null, k, v, kc32, kc, vc32, vc, qc32_or_null, qc_or_null,
+                         (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_route_score_topk(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const float* kc32,
+                                  int32_t* idx, float* score_or_null, void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (off == nullptr || q == nullptr || kc32 == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
+  return launch_route_score(*desc, off, q, kc32, idx, score_or_null, status_of(ws), (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords, int32_t* idx,
+                                 void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (off == nullptr || coords == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
+  const Workspace w = workspace_layout(*desc);
+  return launch_route_geometric(*desc, off, coords, wsp<int32_t>(ws, w.centroids), idx, status_of(ws),
+                                (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc, int32_t* idx,
+                                   void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (!desc->pooled_q || qc == nullptr || kc == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
+  return launch_route_pooled(*desc, qc, kc, idx, status_of(ws), (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_nsa_cmp_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* kc,
+                              const void* vc, float* o_cmp, float* lse, void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (off == nullptr || q == nullptr || kc == nullptr || vc == nullptr || o_cmp == nullptr)
+    return LSRM_ERR_INVALID_ARG;
+  if (desc->pooled_q) {
+    const Workspace w = workspace_layout(*desc);
+    float* o_blk = wsp<float>(ws, w.obranch);
+    float* l_blk = o_blk + (size_t)desc->n_blocks * desc->n_q_heads * desc->head_dim;
+    LSRM_TRY(launch_pooled_cmp(*desc, q, kc, vc, o_blk, l_blk, (cudaStream_t)stream));
+    return launch_pooled_broadcast(*desc, off, o_blk, l_blk, o_cmp, lse, (cudaStream_t)stream);
+  }
+  return launch_attn(*desc, off, q, nullptr, nullptr, kc, vc, nullptr, nullptr, 1, 0, BR_CMP, nullptr, o_cmp, lse,
+                     1, 0, status_of(ws), (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_nsa_select_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, int32_t idx_heads, float* o_slc, float* lse,
+                                 void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o_slc == nullptr)
+    return LSRM_ERR_INVALID_ARG;
+  if (idx_heads != 1 && idx_heads != desc->n_kv_heads) return LSRM_ERR_INVALID_ARG;
+  return launch_attn(*desc, off, q, k, v, nullptr, nullptr, nullptr, idx, idx_heads, 0, BR_SLC, nullptr, o_slc, lse,
+                     1, 0, status_of(ws), (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_nsa_window_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                                 const void* v, float* o_win, float* lse, void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || o_win == nullptr) return LSRM_ERR_INVALID_ARG;
+  if (desc->window == 0) return LSRM_ERR_INVALID_ARG;
+  return launch_attn(*desc, off, q, k, v, nullptr, nullptr, nullptr, nullptr, 1, 0, BR_WIN, nullptr, o_win, lse, 1,
+                     0, status_of(ws), (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_nsa_gate_combine(const lsrm_nsa_desc* desc, const float* o_cmp, const float* o_slc,
+                                  const float* o_win_or_null, const void* gates, void* out, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  if (o_cmp == nullptr || o_slc == nullptr || gates == nullptr || out == nullptr) return LSRM_ERR_INVALID_ARG;
+  if (desc->n_gates == 3 && o_win_or_null == nullptr) return LSRM_ERR_INVALID_ARG;
+  if (!aligned(o_cmp, 16) || !aligned(o_slc, 16) || !aligned(out, 8) ||
+      (o_win_or_null && !aligned(o_win_or_null, 16)))
+    return LSRM_ERR_INVALID_ARG;
+  return launch_gate_combine(*desc, o_cmp, o_slc, o_win_or_null, gates, out, (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_nsa_attend(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                            const void* v, const void* kc, const void* vc, const void* gates, const int32_t* idx,
+                            int32_t idx_heads, int32_t route_all, void* out, float* lse_or_null, void* ws,
+                            void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (desc->pooled_q) return LSRM_ERR_UNSUPPORTED;
+  if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || kc == nullptr || vc == nullptr ||
+      gates == nullptr || out == nullptr || (!route_all && idx == nullptr))
+    return LSRM_ERR_INVALID_ARG;
+  if (idx_heads != 1 && idx_heads != desc->n_kv_heads) return LSRM_ERR_INVALID_ARG;
+  if (route_all && desc->top_k != desc->n_blocks) return LSRM_ERR_INVALID_ARG;
+  const int branches = BR_CMP | BR_SLC | ((desc->n_gates == 3 && desc->window > 0) ? BR_WIN : 0);
+  return launch_attn(*desc, off, q, k, v, kc, vc, gates, idx, idx_heads, route_all ? 1 : 0, branches, out, nullptr,
+                     lse_or_null, desc->n_gates, 0, status_of(ws), (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                             const void* v, const void* gates, const int32_t* coords_or_null, int32_t route_mode,
+                             void* out, int32_t* idx_inout, float* lse_or_null, void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || gates == nullptr || out == nullptr)
+    return LSRM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return LSRM_ERR_INVALID_ARG;
+  const lsrm_nsa_desc& d = *desc;
+  const Workspace w = workspace_layout(d);
+  cudaStream_t s = (cudaStream_t)stream;
+  float* kc32 = wsp<float>(ws, w.kc32);
+  float* vc32 = wsp<float>(ws, w.vc32);
+  void* kc16 = wsp<void>(ws, w.kc16);
+  void* vc16 = wsp<void>(ws, w.vc16);
+  int32_t* idx = idx_inout != nullptr ? idx_inout : wsp<int32_t>(ws, w.idx);
+
+  if (d.pooled_q) {
+    if (route_mode != LSRM_ROUTE_SCORE && route_mode != LSRM_ROUTE_GIVEN) return LSRM_ERR_INVALID_ARG;
+    if (route_mode == LSRM_ROUTE_GIVEN && idx_inout == nullptr) return LSRM_ERR_INVALID_ARG;
+    float* qc32 = wsp<float>(ws, w.qc32);
+    void* qc16 = wsp<void>(ws, w.qc16);
+    LSRM_TRY(launch_compress(d, off, q, k, v, nullptr, kc16, nullptr, vc16, qc32, qc16, s));
+    if (route_mode == LSRM_ROUTE_SCORE) LSRM_TRY(launch_route_pooled(d, qc16, kc16, idx, status_of(ws), s));
+    float* o_blk = wsp<float>(ws, w.obranch);
+    float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
+    LSRM_TRY(launch_pooled_cmp(d, qc16, kc16, vc16, o_blk, l_blk, s));
+    return launch_attn_pooled_fused(d, off, q, k, v, gates, idx, o_blk, out, lse_or_null, status_of(ws), s);
+  }
+
+  LSRM_TRY(launch_compress(d, off, nullptr, k, v, route_mode == LSRM_ROUTE_SCORE ? kc32 : nullptr, kc16, nullptr,
+                           vc16, nullptr, nullptr, s));
+  int idx_heads = 1, route_all = 0;
+  switch (route_mode) {
+    case LSRM_ROUTE_GIVEN:
+      if (idx_inout == nullptr) return LSRM_ERR_INVALID_ARG;
+      idx_heads = d.n_kv_heads;  // a caller-given index uses the per-group layout
+      break;
+    case LSRM_ROUTE_SCORE:
+      idx_heads = d.n_kv_heads;
+      LSRM_TRY(launch_route_score(d, off, q, kc32, idx, nullptr, status_of(ws), s));
+      break;
+    case LSRM_ROUTE_GEOMETRIC:
+      if (coords_or_null == nullptr) return LSRM_ERR_INVALID_ARG;
+      idx_heads = 1;
+      LSRM_TRY(launch_route_geometric(d, off, coords_or_null, wsp<int32_t>(ws, w.centroids), idx, status_of(ws), s));
+      break;
+    case LSRM_ROUTE_ALL:
+      if (d.top_k != d.n_blocks) return LSRM_ERR_INVALID_ARG;
+      route_all = 1;
+      break;
+    default:
+      return LSRM_ERR_INVALID_ARG;
+  }
+  const int branches = BR_CMP | BR_SLC | ((d.n_gates == 3 && d.window > 0) ? BR_WIN : 0);
+  return launch_attn(d, off, q, k, v, kc16, vc16, gates, idx, idx_heads, route_all, branches, out, nullptr,
+                     lse_or_null, d.n_gates, 0, status_of(ws), s);
+}
+
+lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                              const void* v, const void* gates, const int32_t* idx, int32_t idx_heads,
+                              const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates, void* ws,
+                              void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (desc->pooled_q) return LSRM_ERR_UNSUPPORTED;
+  if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || gates == nullptr || idx == nullptr ||
+      lse == nullptr || dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || dgates == nullptr)
+    return LSRM_ERR_INVALID_ARG;
+  if (idx_heads != 1 && idx_heads != desc->n_kv_heads) return LSRM_ERR_INVALID_ARG;
+  const Workspace w = workspace_layout(*desc);
+  cudaStream_t s = (cudaStream_t)stream;
+  void* kc16 = wsp<void>(ws, w.kc16);
+  void* vc16 = wsp<void>(ws, w.vc16);
+  LSRM_TRY(launch_compress(*desc, off, nullptr, k, v, nullptr, kc16, nullptr, vc16, nullptr, nullptr, s));
+  return launch_backward(*desc, off, q, k, v, kc16, vc16, gates, idx, idx_heads, lse, dout, dq, dk, dv, dgates,
+                         wsp<unsigned char>(ws, w.bwd), status_of(ws), s);
+}
+
+lsrm_status lsrm_nsa_last_device_status(void* ws, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return LSRM_ERR_WORKSPACE;
+  uint32_t word = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return LSRM_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LSRM_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return LSRM_ERR_CUDA;
+  if (word == 0) return LSRM_OK;
+  for (int st = 1; st < 32; ++st)
+    if (word & (1u << (st - 1))) return (lsrm_status)st;
+  return LSRM_ERR_CUDA;
+}
+
+const char* lsrm_status_string(lsrm_status s) {
+  switch (s) {
+    case LSRM_OK: return "ok";
+    case LSRM_ERR_INVALID_ARG: return "invalid argument";
+    case LSRM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LSRM_ERR_CUDA: return "CUDA error";
+    case LSRM_ERR_TIMEOUT: return "device wait timed out";
+    case LSRM_ERR_BOUNDS: return "device bounds check failed";
+    case LSRM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,98 @@
+// Shared device/host helpers of the sm_100a LSRM NSA library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lsrm_nsa.h"
+
+namespace lsrm {
+
+constexpr int kMaxBlockLen = 64;
+
+// ---- device status word (first 4 bytes of the workspace) ---------------------------------------
+// Kernels OR a status bit in; the host reads and clears it.  Bit i set <=> status (i+1) was raised.
+__device__ __forceinline__ void raise_status(uint32_t* status, lsrm_status s) {
+  if (status) atomicOr(status, 1u << ((int)s - 1));
+}
+
+// ---- workspace layout ----------------------------------------------------------------------------
+struct Workspace {
+  size_t status, kc32, vc32, kc16, vc16, qc32, qc16, centroids, idx, obranch, bwd, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
+  Workspace w{};
+  size_t o = 0;
+  const size_t B = (size_t)d.n_blocks, Hkv = (size_t)d.n_kv_heads, Hq = (size_t)d.n_q_heads, D = (size_t)d.head_dim;
+  const size_t N = (size_t)d.n_tokens;
+  w.status = o;    o = align256(o + 16);
+  w.kc32 = o;      o = align256(o + B * Hkv * D * 4);
+  w.vc32 = o;      o = align256(o + B * Hkv * D * 4);
+  w.kc16 = o;      o = align256(o + B * Hkv * D * 2);
+  w.vc16 = o;      o = align256(o + B * Hkv * D * 2);
+  const size_t qcn = d.pooled_q ? B * Hq * D : 0;
+  w.qc32 = o;      o = align256(o + qcn * 4);
+  w.qc16 = o;      o = align256(o + qcn * 2);
+  w.centroids = o; o = align256(o + B * 3 * 4);
+  // routing indices when the caller passes none: [B][max(Hq,Hkv)][k]
+  const size_t ih = d.pooled_q ? Hq : Hkv;
+  w.idx = o;       o = align256(o + B * ih * (size_t)(d.top_k > 0 ? d.top_k : 1) * 4);
+  // pooled compressed-branch output [B][Hq][d] fp32 (Speed3R) + its LSE [B][Hq]
+  w.obranch = o;   o = align256(o + (d.pooled_q ? B * Hq * (D + 1) * 4 : 0));
+  // backward scratch: dKbar/dVbar fp32 [B][Hkv][d] x2, per-row D terms fp32 [N][Hq][3]
+  w.bwd = o;       o = align256(o + (d.pooled_q ? 0 : (2 * B * Hkv * D * 4 + N * Hq * 3 * 4)));
+  w.total = o;
+  return w;
+}
+
+// ---- small PTX wrappers (mma.sync bring-up path) -------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
+  const int n = pred ? 16 : 0;  // src-size 0 zero-fills the destination
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                                  uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + C (fp32)
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+}  // namespace lsrm

@@ -1,0 +1,344 @@
+// S2 routing kernels: geometric (integer centroid distance) and score-based top-k.
+//
+// Geometric routing, LSRM page (hyper.ai "LSRM", 方法, 3D-aware block routing
+// paragraph): every token carries a 3D position; a query block keeps the blocks
+// whose centres are nearest in Euclidean distance.  Centres are integer block
+// means (round half up) and distances exact int64, so the result is bit-exact.
+//
+// Score routing, same paragraph: standard NSA picks the KV blocks with the highest
+// attention scores against the compressed keys.  Here the score of block j for
+// query block a and KV group g is the sum over a's tokens and g's heads of the
+// compressed-branch softmax probability of j.
+//
+// Top-k is done by k rounds of a block-wide arg-min/arg-max (warp shuffles, then
+// shared memory across warps): round r returns the best candidate strictly after
+// the one returned by round r-1 in the total order (key, index), so no per-candidate
+// state is kept and ties always go to the lower block index.
+#include "lsrm_common.cuh"
+
+namespace lsrm {
+
+constexpr int kRouteThreads = 256;
+constexpr int kCoordLimit = 1 << 29;
+
+// ---- centroids -----------------------------------------------------------------------------------
+// One warp per block: c[b][axis] = floor((2 S + n) / (2 n)), S = sum of the block's coordinates.
+__global__ void centroid_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ coords, int32_t B,
+                                int32_t* __restrict__ cen, uint32_t* status) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= B) return;
+  const int t0 = off[warp], t1 = off[warp + 1];
+  long long s[3] = {0, 0, 0};
+  bool bad = false;
+  for (int t = t0 + lane; t < t1; t += 32) {
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      const int c = __ldg(coords + (size_t)t * 3 + a);
+      bad |= (c > kCoordLimit) || (c < -kCoordLimit);
+      s[a] += c;
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s[a] += __shfl_xor_sync(0xffffffffu, s[a], o);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(status, LSRM_ERR_BOUNDS);
+  if (lane < 3) {
+    const long long n = t1 - t0;
+    const long long num = 2 * s[lane] + n, den = 2 * n;
+    long long qv = num / den;
+    if ((num % den != 0) && (num < 0)) --qv;  // floor division
+    cen[(size_t)warp * 3 + lane] = (int32_t)qv;
+  }
+}
+
+struct DistKey {
+  long long d;
+  int j;
+};
+__device__ __forceinline__ bool key_less(const DistKey& a, const DistKey& b) {
+  return a.d < b.d || (a.d == b.d && a.j < b.j);
+}
+
+// One CTA per query block; centroids read from shared memory when they fit.
+template <bool SMEM_CEN>
+__global__ void __launch_bounds__(kRouteThreads)
+geo_topk_kernel(const int32_t* __restrict__ cen, int32_t B, int32_t k, int32_t* __restrict__ idx) {
+  extern __shared__ int32_t s_cen[];
+  __shared__ DistKey s_warp[kRouteThreads / 32];
+  __shared__ DistKey s_last;
+  const int a = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (SMEM_CEN) {
+    for (int i = tid; i < B * 3; i += kRouteThreads) s_cen[i] = cen[i];
+  }
+  const int32_t* C = SMEM_CEN ? s_cen : cen;
+  if (tid == 0) s_last = DistKey{-1, -1};
+  __syncthreads();
+  const long long ax = C[a * 3 + 0], ay = C[a * 3 + 1], az = C[a * 3 + 2];
+  for (int r = 0; r < k; ++r) {
+    const DistKey last = s_last;
+    DistKey best{LLONG_MAX, INT_MAX};
+    for (int j = tid; j < B; j += kRouteThreads) {
+      const long long dx = C[j * 3 + 0] - ax, dy = C[j * 3 + 1] - ay, dz = C[j * 3 + 2] - az;
+      const DistKey cand{dx * dx + dy * dy + dz * dz, j};
+      if (key_less(last, cand) && key_less(cand, best)) best = cand;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      DistKey other{__shfl_xor_sync(0xffffffffu, best.d, o), __shfl_xor_sync(0xffffffffu, best.j, o)};
+      if (key_less(other, best)) best = other;
+    }
+    if (lane == 0) s_warp[warp] = best;
+    __syncthreads();
+    if (tid == 0) {
+      DistKey b = s_warp[0];
+      for (int w = 1; w < kRouteThreads / 32; ++w)
+        if (key_less(s_warp[w], b)) b = s_warp[w];
+      idx[(size_t)a * k + r] = b.j;
+      s_last = b;
+    }
+    __syncthreads();
+  }
+}
+
+lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, const int32_t* coords, int32_t* cen,
+                                   int32_t* idx, uint32_t* status, cudaStream_t stream) {
+  const int B = d.n_blocks;
+  centroid_kernel<<<(B * 32 + 255) / 256, 256, 0, stream>>>(off, coords, B, cen, status);
+  const size_t smem = (size_t)B * 3 * sizeof(int32_t);
+  if (smem <= 48 * 1024) {
+    geo_topk_kernel<true><<<B, kRouteThreads, smem, stream>>>(cen, B, d.top_k, idx);
+  } else {
+    geo_topk_kernel<false><<<B, kRouteThreads, 0, stream>>>(cen, B, d.top_k, idx);
+  }
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
+// ---- score routing -------------------------------------------------------------------------------
+// One CTA per (query block a, KV group g), fp32 throughout.  Pass 1 gets each row's
+// softmax max and normaliser over all B compressed keys; pass 2 accumulates the
+// probabilities per key (per-warp partials summed in a fixed order).  Scores stay in
+// shared memory; then k rounds of arg-max by (score desc, j asc).
+constexpr int kScoreChunk = 128;  // compressed keys staged per step
+constexpr int kMaxScoreRows = 64 * 64;
+
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads)
+score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__ q, const float* __restrict__ kc32,
+                   int32_t B, int32_t Hq, int32_t Hkv, int32_t k, float scale, int32_t* __restrict__ idx,
+                   float* __restrict__ score_out, uint32_t* status) {
+  extern __shared__ float smem[];
+  float* s_k = smem;                                   // [kScoreChunk][D + 1]
+  float* s_part = s_k + kScoreChunk * (D + 1);         // [8 warps][kScoreChunk]
+  float* s_score = s_part + 8 * kScoreChunk;           // [B]
+  float2* s_ml = reinterpret_cast<float2*>(s_score + ((B + 1) & ~1));  // [rows] (max, 1/sum)
+  __shared__ float s_bv[kRouteThreads / 32];
+  __shared__ int s_bj[kRouteThreads / 32];
+  __shared__ float s_lv;
+  __shared__ int s_lj;
+  const int a = blockIdx.x, g = blockIdx.y;
+  const int G = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = off[a];
+  // a block longer than the descriptor allows would overrun the row table: flag it and clip
+  int rows = (off[a + 1] - t0) * G;
+  if (rows > kMaxScoreRows) {
+    if (tid == 0) raise_status(status, LSRM_ERR_BOUNDS);
+    rows = kMaxScoreRows;
+  }
+  const float sl2 = scale * 1.4426950408889634f;  // logits in log2 units
+  const int nchunks = (B + kScoreChunk - 1) / kScoreChunk;
+  constexpr int KPL = kScoreChunk / 32;  // keys per lane per chunk
+
+  auto load_chunk = [&](int c) {
+    __syncthreads();
+    for (int e = tid; e < kScoreChunk * D; e += kRouteThreads) {
+      const int kk = e / D, col = e % D;
+      const int j = c * kScoreChunk + kk;
+      s_k[kk * (D + 1) + col] = j < B ? kc32[((size_t)j * Hkv + g) * D + col] : 0.0f;
+    }
+    __syncthreads();
+  };
+  auto load_q = [&](int r, float* qv) {
+    const int t = t0 + r / G, h = g * G + r % G;
+    const uint16_t* src = q + ((size_t)t * Hq + h) * D;
+#pragma unroll
+    for (int c = 0; c < D; ++c) qv[c] = bf16_to_f32(__ldg(src + c));
+  };
+
+  // pass 1: per-row running max / sum (lane-local over its keys, merged at the end)
+  for (int r0 = 0; r0 < rows; r0 += 8 * 8) {
+    float m[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { m[i] = -INFINITY; l[i] = 0.0f; }
+    for (int c = 0; c < nchunks; ++c) {
+      load_chunk(c);
+#pragma unroll 1
+      for (int i = 0; i < 8; ++i) {
+        const int r = r0 + warp * 8 + i;
+        if (r >= rows) break;
+        float qv[D];
+        load_q(r, qv);
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+          const int kk = lane + 32 * e;
+          const int j = c * kScoreChunk + kk;
+          if (j >= B) continue;
+          float s = 0.0f;
+#pragma unroll
+          for (int cc = 0; cc < D; ++cc) s = fmaf(qv[cc], s_k[kk * (D + 1) + cc], s);
+          s *= sl2;
+          if (s > m[i]) { l[i] = l[i] * exp2f(m[i] - s) + 1.0f; m[i] = s; }
+          else l[i] += exp2f(s - m[i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = r0 + warp * 8 + i;
+      float mi = m[i], li = l[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, mi, o), lo = __shfl_xor_sync(0xffffffffu, li, o);
+        const float mn = fmaxf(mi, mo);
+        li = (mi == -INFINITY ? 0.0f : li * exp2f(mi - mn)) + (mo == -INFINITY ? 0.0f : lo * exp2f(mo - mn));
+        mi = mn;
+      }
+      if (lane == 0 && r < rows) s_ml[r] = make_float2(mi, 1.0f / li);
+    }
+  }
+  __syncthreads();
+  // pass 2: probabilities summed per key, chunk by chunk
+  for (int c = 0; c < nchunks; ++c) {
+    load_chunk(c);
+    float acc[KPL];
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) acc[e] = 0.0f;
+    for (int r = warp; r < rows; r += 8) {
+      float qv[D];
+      load_q(r, qv);
+      const float2 ml = s_ml[r];
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) {
+        const int kk = lane + 32 * e;
+        float s = 0.0f;
+#pragma unroll
+        for (int cc = 0; cc < D; ++cc) s = fmaf(qv[cc], s_k[kk * (D + 1) + cc], s);
+        acc[e] += exp2f(s * sl2 - ml.x) * ml.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) s_part[warp * kScoreChunk + lane + 32 * e] = acc[e];
+    __syncthreads();
+    for (int kk = tid; kk < kScoreChunk; kk += kRouteThreads) {
+      const int j = c * kScoreChunk + kk;
+      if (j < B) {
+        float s = 0.0f;
+        for (int w = 0; w < 8; ++w) s += s_part[w * kScoreChunk + kk];
+        s_score[j] = s;
+        if (score_out) score_out[((size_t)a * Hkv + g) * B + j] = s;
+      }
+    }
+  }
+  // top-k by (score desc, j asc)
+  if (tid == 0) { s_lv = INFINITY; s_lj = -1; }
+  __syncthreads();
+  for (int r = 0; r < k; ++r) {
+    const float lv = s_lv;
+    const int lj = s_lj;
+    float bv = -INFINITY;
+    int bj = INT_MAX;
+    for (int j = tid; j < B; j += kRouteThreads) {
+      const float v = s_score[j];
+      const bool after_last = (v < lv) || (v == lv && j > lj);
+      const bool better = (v > bv) || (v == bv && j < bj);
+      if (after_last && better) { bv = v; bj = j; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
+    }
+    if (lane == 0) { s_bv[warp] = bv; s_bj[warp] = bj; }
+    __syncthreads();
+    if (tid == 0) {
+      float v = s_bv[0];
+      int j = s_bj[0];
+      for (int w = 1; w < kRouteThreads / 32; ++w)
+        if (s_bv[w] > v || (s_bv[w] == v && s_bj[w] < j)) { v = s_bv[w]; j = s_bj[w]; }
+      idx[((size_t)a * Hkv + g) * k + r] = j;
+      s_lv = v;
+      s_lj = j;
+    }
+    __syncthreads();
+  }
+}
+
+size_t score_route_smem(int B, int D) {
+  return (size_t)kScoreChunk * (D + 1) * 4 + 8 * kScoreChunk * 4 + (size_t)((B + 1) & ~1) * 4 +
+         (size_t)kMaxScoreRows * 8;
+}
+
+lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
+                               int32_t* idx, float* score, uint32_t* status, cudaStream_t stream) {
+  const int B = d.n_blocks, D = d.head_dim;
+  if ((size_t)d.max_block_len * (d.n_q_heads / d.n_kv_heads) > (size_t)kMaxScoreRows) return LSRM_ERR_UNSUPPORTED;
+  const size_t smem = score_route_smem(B, D);
+  if (smem > 200 * 1024) return LSRM_ERR_UNSUPPORTED;
+  const float scale = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)D);
+  dim3 grid((unsigned)B, (unsigned)d.n_kv_heads);
+  cudaError_t e;
+  if (D == 32) {
+    e = cudaFuncSetAttribute(score_route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return LSRM_ERR_CUDA;
+    score_route_kernel<32><<<grid, kRouteThreads, smem, stream>>>(off, (const uint16_t*)q, kc32, B, d.n_q_heads,
+                                                                  d.n_kv_heads, d.top_k, scale, idx, score, status);
+  } else {
+    e = cudaFuncSetAttribute(score_route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return LSRM_ERR_CUDA;
+    score_route_kernel<64><<<grid, kRouteThreads, smem, stream>>>(off, (const uint16_t*)q, kc32, B, d.n_q_heads,
+                                                                  d.n_kv_heads, d.top_k, scale, idx, score, status);
+  }
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
+// ---- gated combine ---------------------------------------------------------------------------------
+// out[t,h,:] = sum_b gates[t,h,b] * o_b[t,h,:]  (bf16 out); one thread per 4 output columns.
+__global__ void gate_combine_kernel(const float4* __restrict__ oc, const float4* __restrict__ os,
+                                    const float4* __restrict__ ow, const uint16_t* __restrict__ gates,
+                                    uint2* __restrict__ out, long long n_vec4, int d4, int ng) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_vec4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i / d4;
+    const uint16_t* g = gates + row * ng;
+    const float g0 = bf16_to_f32(g[0]), g1 = bf16_to_f32(g[1]);
+    const float4 a = oc[i], b = os[i];
+    float4 r = make_float4(g0 * a.x + g1 * b.x, g0 * a.y + g1 * b.y, g0 * a.z + g1 * b.z, g0 * a.w + g1 * b.w);
+    if (ow != nullptr && ng >= 3) {
+      const float g2 = bf16_to_f32(g[2]);
+      const float4 c = ow[i];
+      r.x += g2 * c.x; r.y += g2 * c.y; r.z += g2 * c.z; r.w += g2 * c.w;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(r.x, r.y);
+    o.y = pack_bf16x2(r.z, r.w);
+    out[i] = o;
+  }
+}
+
+lsrm_status launch_gate_combine(const lsrm_nsa_desc& d, const float* oc, const float* os, const float* ow,
+                                const void* gates, void* out, cudaStream_t stream) {
+  const long long n_vec4 = d.n_tokens * (long long)d.n_q_heads * d.head_dim / 4;
+  const int threads = 256;
+  const long long blocks = (n_vec4 + threads - 1) / threads;
+  const int grid = (int)(blocks < 148LL * 32 ? blocks : 148LL * 32);
+  gate_combine_kernel<<<grid, threads, 0, stream>>>((const float4*)oc, (const float4*)os, (const float4*)ow,
+                                                    (const uint16_t*)gates, (uint2*)out, n_vec4, d.head_dim / 4,
+                                                    d.n_gates);
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
+}  // namespace lsrm

@@ -1,0 +1,201 @@
+/*
+ * lsrm_nsa.h — C ABI of the B200 (sm_100a) native-sparse-attention layer of the
+ * Large Sparse Reconstruction Model (LSRM), plus its Speed3R pooled-query variant.
+ *
+ * The layer (LSRM page, hyper.ai "LSRM", section 方法):
+ *   - active tokens are grouped into spatial blocks (8x8 image tiles, volume
+ *     bricks; the block grouping paragraph);
+ *   - compression: per-block mean of K and V (equations k^cmp, v^cmp; the
+ *     ResBlock before the pool is a trained module and is not part of this ABI);
+ *   - routing picks top-k KV blocks per query block, from compressed attention
+ *     scores (standard NSA) or from 3D distances between block centres (the
+ *     3D-aware routing paragraph);
+ *   - a compressed branch, a selected-block branch and an in-block window branch
+ *     run softmax attention and a sigmoid-gated sum combines them (gate
+ *     equations w = Sigmoid(Linear(x)); the gate VALUES are inputs here).
+ * Speed3R page (gist.science "Speed3R", section 2.1 Global Sparse Attention):
+ *   Q/K/V are average-pooled per block, the pooled scores pick the top-k blocks,
+ *   the reference frame and camera tokens are always selected (section 2.2), and
+ *   a gate mixes the compressed and selected outputs.
+ *
+ * Notation: N tokens in block-major order; block b owns tokens off[b] .. off[b+1]-1
+ * (n_b = off[b+1] - off[b], 1 <= n_b <= max_block_len <= 64).  Hq query heads,
+ * Hkv KV heads, G = Hq / Hkv, query head h reads KV head h / G.  d = head_dim.
+ * tau = scale (0 means 1/sqrt(d)).
+ *
+ * Layouts (all row-major, contiguous):
+ *   q      bf16 [N][Hq][d]        k, v   bf16 [N][Hkv][d]
+ *   gates  bf16 [N][Hq][n_gates]  order (cmp, slc, win); n_gates = 2 drops win
+ *   off    int32 [B+1]            coords int32 [N][3] lattice coordinates
+ *   out    bf16 [N][Hq][d]
+ *   kc32/vc32 fp32 [B][Hkv][d], kc/vc bf16 [B][Hkv][d] (block means)
+ *   qc32/qc fp32/bf16 [B][Hq][d]  (pooled queries, Speed3R only)
+ *   idx    int32 [B][idx_heads][top_k]; idx_heads = 1 (geometric: one list per
+ *          query block, shared by all KV heads) or Hkv (score routing)
+ *   o_* / lse fp32 [N][Hq][d] / [N][Hq]  (per-branch outputs, natural-log LSE)
+ *
+ * Ownership and errors.  Every array pointer is DEVICE memory owned by the
+ * caller; the library allocates nothing and keeps no global state (all scratch
+ * lives in the caller's workspace, sized by lsrm_nsa_workspace_size and zeroed
+ * once by lsrm_nsa_workspace_init).  The descriptor itself is host memory.
+ * Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ * legacy default stream).  The return value reports argument validation and
+ * launch errors only.  Faults found while running (a routed index outside
+ * [0, B), a coordinate outside [-2^29, 2^29], a bounded wait that gave up) are
+ * written to a status word in the workspace and read back, then cleared, by
+ * lsrm_nsa_last_device_status.  No call traps, asserts or waits without bound.
+ */
+#ifndef LSRM_NSA_H
+#define LSRM_NSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LSRM_API __attribute__((visibility("default")))
+#else
+#define LSRM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LSRM_OK = 0,
+  LSRM_ERR_INVALID_ARG = 1, /* a pointer, size or shape the call cannot accept */
+  LSRM_ERR_UNSUPPORTED = 2, /* valid in principle, not built (e.g. head_dim not 32/64) */
+  LSRM_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  LSRM_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up */
+  LSRM_ERR_BOUNDS = 5,      /* a device-side index/coordinate check failed; access skipped */
+  LSRM_ERR_WORKSPACE = 6    /* workspace missing, misaligned or too small */
+} lsrm_status;
+
+/* route_mode of lsrm_nsa_forward */
+enum { LSRM_ROUTE_GIVEN = 0, LSRM_ROUTE_SCORE = 1, LSRM_ROUTE_GEOMETRIC = 2, LSRM_ROUTE_ALL = 3 };
+
+typedef struct {
+  int64_t n_tokens;       /* N >= 1 */
+  int32_t n_blocks;       /* B >= 1 */
+  int32_t max_block_len;  /* upper bound of every n_b, 1..64 */
+  int32_t n_q_heads;      /* Hq, multiple of n_kv_heads */
+  int32_t n_kv_heads;     /* Hkv >= 1 */
+  int32_t head_dim;       /* d in {32, 64} */
+  int32_t top_k;          /* routed blocks per query block, 1..B */
+  int32_t window;         /* even, 0 switches the window branch off */
+  float scale;            /* softmax scale tau; 0 -> 1/sqrt(d) */
+  int32_t pooled_q;       /* 0 LSRM layer, 1 Speed3R pooled-query variant (MHA, no window) */
+  int32_t n_gates;        /* 3 (cmp, slc, win) or 2 (cmp, slc) */
+  int32_t n_forced;       /* blocks every query selects (Speed3R), 0 for LSRM */
+  const int32_t* forced_blocks; /* device int32 [n_forced], sorted, distinct */
+} lsrm_nsa_desc;
+
+/* Bytes of device workspace the calls below need for this descriptor (a
+ * multiple of 256).  Pass the same workspace to every call of one layer. */
+LSRM_API size_t lsrm_nsa_workspace_size(const lsrm_nsa_desc* desc);
+
+/* Zero the workspace (status word included).  Call once after allocating it. */
+LSRM_API lsrm_status lsrm_nsa_workspace_init(const lsrm_nsa_desc* desc, void* ws, size_t ws_bytes, void* stream);
+
+/* S1 compression (LSRM page, equations k^cmp / v^cmp; Speed3R page 2.1 for the
+ * pooled query): per-block means of K and V (and of Q when q != NULL), written
+ * in fp32 and rounded to bf16.  Any output pointer may be NULL to skip it. */
+LSRM_API lsrm_status lsrm_nsa_compress(const lsrm_nsa_desc* desc, const int32_t* off, const void* q_or_null,
+                              const void* k, const void* v, float* kc32, void* kc, float* vc32, void* vc,
+                              float* qc32_or_null, void* qc_or_null, void* ws, void* stream);
+
+/* S2a score routing (LSRM page, routing paragraph: NSA picks KV blocks by their
+ * attention scores against the compressed keys).  For query block a and KV
+ * group g: Score[a,g,j] = sum over tokens t of a and heads h of g of
+ * softmax_j(tau * q[t,h] . kc32[j,g]); idx[a][g][:] = the top_k j by
+ * (Score desc, j asc).  score_or_null receives fp32 [B][Hkv][B] when given. */
+LSRM_API lsrm_status lsrm_route_score_topk(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const float* kc32,
+                                  int32_t* idx, float* score_or_null, void* ws, void* stream);
+
+/* S2b geometric routing (LSRM page, routing paragraph: nearest blocks by 3D
+ * Euclidean distance between block centres).  Centroid c[b] per axis =
+ * floor((2*S + n_b) / (2*n_b)) with S the sum of the block's coordinates
+ * (round half up); D[a,j] = sum over axes of (c[a]-c[j])^2 in int64;
+ * idx[a][:] = the top_k j by (D asc, j asc).  coords must lie in [-2^29, 2^29]. */
+LSRM_API lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords,
+                                 int32_t* idx, void* ws, void* stream);
+
+/* Speed3R routing (Speed3R page 2.1 selection branch, 2.2 forced frame-0 and
+ * camera blocks): per block a and head h, the top_k blocks j outside the forced
+ * set by (tau * qc[a,h] . kc[j,h] desc, j asc), computed from the bf16 pooled
+ * tensors with fp32 accumulation.  idx is int32 [B][Hq][top_k]. */
+LSRM_API lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc, int32_t* idx,
+                                   void* ws, void* stream);
+
+/* S3 compressed branch (LSRM page, k^cmp/v^cmp give the global coarse context;
+ * Speed3R page 2.1 compression branch).  o_cmp[t,h] = sum_j softmax_j(tau *
+ * q[t,h] . kc[j,g]) vc[j,g] over all B blocks; with pooled_q the query is
+ * qc[beta(t),h] (pass it as q, shape [B][Hq][d]) and the block's output is
+ * written to every token of the block.  kc/vc are bf16 block means. */
+LSRM_API lsrm_status lsrm_nsa_cmp_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* kc,
+                              const void* vc, float* o_cmp, float* lse, void* ws, void* stream);
+
+/* S4 selected branch (LSRM page: selected active blocks give fine detail;
+ * Speed3R page 2.1 selection branch).  Softmax attention of q[t,h] over every
+ * token of the blocks idx[beta(t)][g or 0][0..top_k-1] plus the forced blocks.
+ * idx_heads is 1 or Hkv (see Layouts); rows must hold distinct block ids that
+ * are not forced. */
+LSRM_API lsrm_status lsrm_nsa_select_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, int32_t idx_heads, float* o_slc, float* lse,
+                                 void* ws, void* stream);
+
+/* S5 window branch (LSRM page, sequence-parallel paragraph: window attention
+ * runs locally inside whole blocks).  W(t) = { u in beta(t) : r(t) - w/2 <=
+ * r(u) <= r(t) + w/2 - 1 }, r = position inside the block. */
+LSRM_API lsrm_status lsrm_nsa_window_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                                 const void* v, float* o_win, float* lse, void* ws, void* stream);
+
+/* S6 gated combine (LSRM page, gate equations; Speed3R page 2.1 gated
+ * aggregation): out = g_cmp o_cmp + g_slc o_slc (+ g_win o_win), bf16 out. */
+LSRM_API lsrm_status lsrm_nsa_gate_combine(const lsrm_nsa_desc* desc, const float* o_cmp, const float* o_slc,
+                                  const float* o_win_or_null, const void* gates, void* out, void* stream);
+
+/* S3+S4+S5+S6 fused: the three attention branches and the gated combine in one
+ * kernel (one CTA per query block, KV group and 128-row chunk), given the bf16
+ * block means kc/vc (lsrm_nsa_compress) and the routing indices (idx_heads 1 or
+ * Hkv; route_all = 1 selects every block and ignores idx).  Writes bf16 out and,
+ * when lse_or_null is given, the per-branch LSE [N][Hq][n_gates].  For pooled_q
+ * this call is not available (use lsrm_nsa_forward). */
+LSRM_API lsrm_status lsrm_nsa_attend(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                                     const void* v, const void* kc, const void* vc, const void* gates,
+                                     const int32_t* idx, int32_t idx_heads, int32_t route_all, void* out,
+                                     float* lse_or_null, void* ws, void* stream);
+
+/* S7 the fused layer forward: compression, routing (route_mode), then the three
+ * branches and the gated combine in one attention kernel whose epilogue writes
+ * out.  route_mode: LSRM_ROUTE_GIVEN reads idx_inout as [B][Hkv][top_k];
+ * LSRM_ROUTE_SCORE writes it as [B][Hkv][top_k]; LSRM_ROUTE_GEOMETRIC (coords
+ * required) writes [B][top_k]; LSRM_ROUTE_ALL needs top_k == B and selects every
+ * block (idx_inout may be NULL).  With a NULL idx_inout the indices live in the
+ * workspace.  For pooled_q the routing is the Speed3R rule and idx_inout is
+ * [B][Hq][top_k].
+ * lse_or_null receives fp32 [N][Hq][n_gates] per-branch LSE (needed by the
+ * backward). */
+LSRM_API lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                             const void* v, const void* gates, const int32_t* coords_or_null, int32_t route_mode,
+                             void* out, int32_t* idx_inout, float* lse_or_null, void* ws, void* stream);
+
+/* S10 backward of the LSRM layer (pooled_q = 0) with routing indices fixed:
+ * dq, dgates [N][Hq][.], dk, dv [N][Hkv][d] (bf16) of L = sum(out * dout),
+ * through the gated sum, the three softmax branches and the block mean.
+ * lse is the forward's per-branch LSE.  idx_heads as in lsrm_nsa_select_attn. */
+LSRM_API lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
+                              const void* v, const void* gates, const int32_t* idx, int32_t idx_heads,
+                              const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
+                              void* ws, void* stream);
+
+/* Read (synchronising `stream`) and clear the device status word of the workspace. */
+LSRM_API lsrm_status lsrm_nsa_last_device_status(void* ws, void* stream);
+
+/* Static text for a status code. */
+LSRM_API const char* lsrm_status_string(lsrm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LSRM_NSA_H */
