@@ -1,0 +1,533 @@
+// S3-S7 attention on the 5th-generation tensor cores: TMA -> shared memory, tcgen05.mma
+// with accumulators in tensor memory, one softmax thread per query row.
+//
+// Work unit: one CTA = one (query block a, KV group g, pair of 128-row M tiles).  A query
+// row is a (token, head) pair of block a whose head reads KV group g; rows are token-major
+// so an M tile is 128/G tokens x G heads and its Q rows arrive with one 3D TMA box.
+// All rows of the unit share one key stream, so every K/V tile is loaded once per CTA and
+// used by both M tiles:
+//   compressed branch: the B block means of group g (LSRM page, 方法: compressed block
+//     features give global coarse context; Speed3R page 2.1 compression branch);
+//   selected branch: the tokens of the routed (and forced) blocks, one 64-row slot per
+//     block (LSRM page: selected active blocks give local fine detail);
+//   window branch: the query's own block, band r(t)-w/2 .. r(t)+w/2-1 (LSRM page,
+//     sequence-parallel paragraph: window attention runs locally inside blocks).
+// The gated sum of the branch outputs (LSRM page, gate equations) happens in the epilogue.
+//
+// Roles (320 threads): warp 0 issues TMA loads; warp 1 owns tensor memory and issues the
+// MMAs (S = Q K^T from shared memory, O += P V with P read from tensor memory); warps
+// 2-5 and 6-9 are two softmax warpgroups, one per M tile, so one tile's exponentials
+// overlap the other tile's MMAs.  Every wait is bounded (see tc::mbar_wait).
+//
+// Tensor memory per M tile (256 columns): S [kKeys fp32] | P [kKeys/2, bf16 pairs] | O [D].
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "tc_ptx.cuh"
+
+namespace lsrm {
+
+using namespace tc;
+
+constexpr int kTcThreads = 320;
+constexpr int kTcMaxSel = 1024;
+
+template <int D>
+struct TcCfg {
+  static constexpr int kRows = 128;
+  static constexpr int kSlots = D == 32 ? 2 : 1;  // 64-key slots per chunk
+  static constexpr int kKeys = 64 * kSlots;       // keys per chunk = N of S = Q K^T
+  static constexpr int kStages = 4;
+  static constexpr int kRowBytes = D * 2;
+  static constexpr uint32_t kLayout = D == 32 ? kLayoutSW64 : kLayoutSW128;
+  static constexpr uint32_t kAtomBytes = 8 * kRowBytes;  // 8 rows of one swizzle atom
+  static constexpr int kQBytes = kRows * kRowBytes;
+  static constexpr int kSlotBytes = 64 * kRowBytes;
+  static constexpr int kKVBytes = kKeys * kRowBytes;
+  static constexpr int kColS = 0, kColP = kKeys, kColO = kKeys + kKeys / 2;
+  static constexpr int kColsPerTile = 256;
+  static constexpr uint32_t kIdescQK = idesc_bf16(128, kKeys, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
+  static_assert(kColO + D <= kColsPerTile, "tensor memory budget");
+};
+
+template <int D>
+struct TcSmem {
+  using C = TcCfg<D>;
+  uint8_t q[2][C::kQBytes];
+  uint8_t k[C::kStages][C::kKVBytes];
+  uint8_t v[C::kStages][C::kKVBytes];
+  uint64_t q_full[2], kv_full[C::kStages], kv_empty[C::kStages], s_full[2], p_full[2], pv_done[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_sel;
+  int sel_start[kTcMaxSel];
+  int sel_n[kTcMaxSel];
+};
+
+struct TcParams {
+  const int32_t* off;
+  const uint16_t* gates;
+  const int32_t* idx;
+  const int32_t* forced;
+  uint16_t* out;
+  float* obranch;
+  float* lse;
+  uint32_t* status;
+  int N, B, Hq, Hkv, G, top_k, idx_heads, n_forced, window, n_gates, route_all, branches, lse_stride, lse_first;
+  float scale_log2;
+};
+
+enum : int { TC_CMP = 1, TC_SLC = 2, TC_WIN = 4 };
+
+// chunk sequence shared by the three roles: [cmp chunks][slc chunks][win chunk]
+struct Chunks {
+  int n_cmp, n_slc, n_win, total;
+  __device__ __forceinline__ int branch(int c, int& local) const {
+    if (c < n_cmp) { local = c; return 0; }
+    if (c < n_cmp + n_slc) { local = c - n_cmp; return 1; }
+    local = 0;
+    return 2;
+  }
+  __device__ __forceinline__ bool first_of_branch(int c) const {
+    return c == 0 || c == n_cmp || c == n_cmp + n_slc;
+  }
+};
+
+template <int D>
+__device__ __forceinline__ void slot_info(const TcSmem<D>& S, const TcParams& p, int br, int local, int slot,
+                                          int t0, int n_a, int& start, int& nvalid) {
+  using C = TcCfg<D>;
+  if (br == 0) {
+    start = local * C::kKeys + slot * 64;
+    nvalid = min(64, max(0, p.B - start));
+  } else if (br == 1) {
+    const int i = local * C::kSlots + slot;
+    if (p.route_all) {
+      if (i < p.B) { start = p.off[i]; nvalid = p.off[i + 1] - start; }
+      else { start = t0; nvalid = 0; }
+    } else if (i < S.n_sel) {
+      start = S.sel_start[i];
+      nvalid = S.sel_n[i];
+    } else {
+      start = t0;
+      nvalid = 0;
+    }
+  } else {
+    start = t0;
+    nvalid = slot == 0 ? n_a : 0;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
+                   const __grid_constant__ CUtensorMap vcmap, const TcParams p) {
+  using C = TcCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  TcSmem<D>& S = *reinterpret_cast<TcSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, g = blockIdx.y, a = blockIdx.z;
+  const int t0 = p.off[a], n_a = p.off[a + 1] - t0;
+  const int rows_total = n_a * p.G;
+  const int tile0 = pair * 2;
+  if (tile0 * 128 >= rows_total) return;  // the whole CTA leaves before any setup
+  const int tokens_per_tile = 128 / p.G;
+
+  if (threadIdx.x == 0) {
+    S.abort = 0;
+    int n = 0;
+    if ((p.branches & TC_SLC) && !p.route_all) {
+      const int32_t* r = p.idx + ((size_t)a * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.top_k;
+      for (int i = 0; i < p.n_forced + p.top_k && n < kTcMaxSel; ++i) {
+        const int j = i < p.n_forced ? p.forced[i] : r[i - p.n_forced];
+        if (j < 0 || j >= p.B) { raise_status(p.status, LSRM_ERR_BOUNDS); continue; }
+        S.sel_start[n] = p.off[j];
+        S.sel_n[n] = p.off[j + 1] - p.off[j];
+        ++n;
+      }
+    }
+    S.n_sel = n;
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&S.q_full[t], 1);
+      mbar_init(&S.s_full[t], 1);
+      mbar_init(&S.p_full[t], 128);
+      mbar_init(&S.pv_done[t], 1);
+    }
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    mbar_init(&S.drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  Chunks cs;
+  cs.n_cmp = (p.branches & TC_CMP) ? (p.B + C::kKeys - 1) / C::kKeys : 0;
+  const int n_sel = (p.branches & TC_SLC) ? (p.route_all ? p.B : S.n_sel) : 0;
+  cs.n_slc = (n_sel + C::kSlots - 1) / C::kSlots;
+  cs.n_win = ((p.branches & TC_WIN) && p.window > 0) ? 1 : 0;
+  cs.total = cs.n_cmp + cs.n_slc + cs.n_win;
+  volatile int* abort = &S.abort;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && cs.total > 0) {
+      tma_prefetch_desc(&qmap);
+      for (int t = 0; t < 2; ++t) {
+        mbar_arrive_expect_tx(&S.q_full[t], C::kQBytes);
+        tma_load_3d(S.q[t], &qmap, &S.q_full[t], 0, g * p.G, t0 + (tile0 + t) * tokens_per_tile);
+      }
+      int issued = 0;
+      for (int c = 0; c < cs.total; ++c) {
+        const int st = c % C::kStages;
+        if (c >= C::kStages && !mbar_wait(&S.kv_empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
+        int local;
+        const int br = cs.branch(c, local);
+        mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
+        for (int s = 0; s < C::kSlots; ++s) {
+          int start, nvalid;
+          slot_info<D>(S, p, br, local, s, t0, n_a, start, nvalid);
+          const CUtensorMap* km = br == 0 ? &kcmap : &kmap;
+          const CUtensorMap* vm = br == 0 ? &vcmap : &vmap;
+          tma_load_3d(S.k[st] + s * C::kSlotBytes, km, &S.kv_full[st], 0, g, start);
+          tma_load_3d(S.v[st] + s * C::kSlotBytes, vm, &S.kv_full[st], 0, g, start);
+        }
+        issued = c + 1;
+      }
+      if (*abort) {
+        // let the copies already issued land before the CTA's shared memory goes away
+        for (int c = max(0, issued - C::kStages); c < issued; ++c) {
+          volatile int no_abort = 0;
+          mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, &no_abort, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && cs.total > 0) {
+      bool ok = mbar_wait(&S.q_full[0], 0, abort, p.status) && mbar_wait(&S.q_full[1], 0, abort, p.status);
+      tc_fence_after();
+      const uint32_t qaddr[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
+      auto issue_qk = [&](int t, int st) {
+        const uint32_t d = tmem + t * C::kColsPerTile + C::kColS;
+        const uint32_t kaddr = smem_u32(S.k[st]);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t ad = smem_desc(qaddr[t] + k * 32, 16, C::kAtomBytes, C::kLayout);
+          const uint64_t bd = smem_desc(kaddr + k * 32, 16, C::kAtomBytes, C::kLayout);
+          mma_ss(d, ad, bd, C::kIdescQK, k > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int c) {
+        const int st = c % C::kStages;
+        const uint32_t d = tmem + t * C::kColsPerTile + C::kColO;
+        const uint32_t vaddr = smem_u32(S.v[st]);
+        const bool first = cs.first_of_branch(c);
+#pragma unroll
+        for (int kk = 0; kk < C::kKeys / 16; ++kk) {
+          const uint32_t at = tmem + t * C::kColsPerTile + C::kColP + kk * 8;
+          const uint64_t bd = smem_desc(vaddr + kk * 16 * C::kRowBytes, C::kKVBytes, C::kAtomBytes, C::kLayout);
+          mma_ts(d, at, bd, C::kIdescPV, (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      for (int c = 0; ok && c < cs.total; ++c) {
+        const int st = c % C::kStages;
+        if (!mbar_wait(&S.kv_full[st], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t) {
+          if (c > 0) {
+            if (!mbar_wait(&S.p_full[t], (c - 1) & 1, abort, p.status)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, c - 1);
+            mma_commit(&S.pv_done[t]);
+          }
+          issue_qk(t, st);
+          mma_commit(&S.s_full[t]);
+        }
+        if (!ok) break;
+        if (c > 0) mma_commit(&S.kv_empty[(c - 1) % C::kStages]);
+      }
+      for (int t = 0; ok && t < 2; ++t) {
+        if (!mbar_wait(&S.p_full[t], (cs.total - 1) & 1, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(t, cs.total - 1);
+        mma_commit(&S.pv_done[t]);
+      }
+      // every MMA issued so far must finish (and every arrive it owes must land) before the
+      // CTA can release tensor and shared memory, on the normal path and after an abort alike
+      mma_commit(&S.drain);
+      volatile int no_abort = 0;
+      mbar_wait(&S.drain, 0, &no_abort, nullptr);
+    }
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int t = (warp - 2) >> 2;               // M tile of this warpgroup
+    const int quarter = warp & 3;                // tensor-memory lane quarter this warp may access
+    const int row = quarter * 32 + lane;         // row of the M tile = TMEM lane
+    const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + t * C::kColsPerTile;
+    const int R = (tile0 + t) * 128 + row;
+    const bool valid = R < rows_total;
+    const int tok_local = R / p.G;
+    const int tok = t0 + (valid ? tok_local : 0);
+    const int head = g * p.G + R % p.G;
+    const size_t orow = (size_t)tok * p.Hq + head;
+    float gate[3] = {0.f, 0.f, 0.f};
+    if (p.out != nullptr && valid)
+      for (int b = 0; b < p.n_gates; ++b) gate[b] = bf16_to_f32(p.gates[orow * p.n_gates + b]);
+    float out_acc[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) out_acc[i] = 0.f;
+    float m = -INFINITY, l = 0.f;
+
+    auto finalize = [&](int br, float mb, float lb) {
+      uint32_t o[D];
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) tmem_ld32(tbase + C::kColO + 32 * i, o + 32 * i);
+      tmem_ld_wait();
+      const float inv = lb > 0.f ? 1.f / lb : 0.f;
+      if (p.out != nullptr) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) out_acc[i] = fmaf(gate[br] * inv, __uint_as_float(o[i]), out_acc[i]);
+      }
+      if (p.obranch != nullptr && valid) {
+        float4* dst = reinterpret_cast<float4*>(p.obranch + orow * D);
+#pragma unroll
+        for (int i = 0; i < D / 4; ++i)
+          dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                               __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+      }
+      if (p.lse != nullptr && valid) {
+        int slot = p.lse_first;
+        if (p.branches & TC_CMP) slot += (br > 0);
+        if ((p.branches & TC_SLC) && br > 1) slot += 1;
+        p.lse[orow * p.lse_stride + slot] = lb > 0.f ? (mb + __log2f(lb)) * 0.6931471805599453f : -INFINITY;
+      }
+    };
+
+    int prev_br = -1;
+    bool ok = true;
+    const int wlo = tok_local - p.window / 2, whi = tok_local + p.window / 2 - 1;
+    // waits are made warp-uniform: the tensor-memory accesses after them are .sync.aligned
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const bool w = mbar_wait(bar, parity, abort, p.status);
+      return __all_sync(0xffffffffu, w);
+    };
+    for (int c = 0; c < cs.total; ++c) {
+      if (!wait_all(&S.s_full[t], c & 1)) { ok = false; break; }
+      tc_fence_after();
+      int local;
+      const int br = cs.branch(c, local);
+      const bool first = cs.first_of_branch(c);
+      int nv[C::kSlots];
+      bool need_mask = br == 2;
+#pragma unroll
+      for (int s = 0; s < C::kSlots; ++s) {
+        int start;
+        slot_info<D>(S, p, br, local, s, t0, n_a, start, nv[s]);
+        need_mask |= nv[s] < 64;
+      }
+      // key j of the chunk: slot j/64, row j%64 of that slot
+      auto logit = [&](uint32_t raw, int j) -> float {
+        if (need_mask) {
+          const int kr = j & 63;
+          bool kv = kr < nv[j >> 6];
+          if (br == 2) kv = kv && kr >= wlo && kr <= whi;
+          if (!kv) return -INFINITY;
+        }
+        return __uint_as_float(raw) * p.scale_log2;
+      };
+      // pass 1: chunk max (log2 units), 32 columns at a time
+      float mc = -INFINITY;
+#pragma unroll
+      for (int qd = 0; qd < C::kKeys / 32; ++qd) {
+        uint32_t r[32];
+        tmem_ld32(tbase + C::kColS + 32 * qd, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mc = fmaxf(mc, logit(r[i], 32 * qd + i));
+      }
+      const float m_prev = m, l_prev = l;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (first) {
+        m = mc;
+        l = 0.f;
+      } else if (mc > m + 8.f) {  // move the reference only when it would grow by more than 2^8
+        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mc);
+        m = mc;
+        l *= alpha;
+        rescale = true;
+      }
+      const float mref = m == -INFINITY ? 0.f : m;
+      // the previous P V must be done before P is overwritten and before O is read
+      if (c > 0) {
+        if (!wait_all(&S.pv_done[t], (c - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (first) {
+          finalize(prev_br, m_prev, l_prev);
+        } else if (__any_sync(0xffffffffu, rescale)) {  // rows that keep their reference use alpha = 1
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) {
+            uint32_t o[32];
+            tmem_ld32(tbase + C::kColO + 32 * i, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tbase + C::kColO + 32 * i, o);
+          }
+        }
+      }
+      // pass 2: P = exp2(x - m) as bf16 pairs, 32 columns of S -> 16 columns of P
+      float ls = 0.f;
+#pragma unroll
+      for (int qd = 0; qd < C::kKeys / 32; ++qd) {
+        uint32_t r[32];
+        tmem_ld32(tbase + C::kColS + 32 * qd, r);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(logit(r[2 * i], 32 * qd + 2 * i) - mref);
+          const float p1 = fast_exp2(logit(r[2 * i + 1], 32 * qd + 2 * i + 1) - mref);
+          ls += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tbase + C::kColP + 16 * qd, pk);
+      }
+      l += ls;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&S.p_full[t]);
+      prev_br = br;
+    }
+    if (ok && cs.total > 0) {
+      if (wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
+        tc_fence_after();
+        finalize(prev_br, m, l);
+        if (p.out != nullptr && valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i) {
+            uint4 u;
+            u.x = pack_bf16x2(out_acc[8 * i + 0], out_acc[8 * i + 1]);
+            u.y = pack_bf16x2(out_acc[8 * i + 2], out_acc[8 * i + 3]);
+            u.z = pack_bf16x2(out_acc[8 * i + 4], out_acc[8 * i + 5]);
+            u.w = pack_bf16x2(out_acc[8 * i + 6], out_acc[8 * i + 7]);
+            dst[i] = u;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---- host side ------------------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 3D bf16 map over a [rows][heads][D] tensor with a (D, box_heads, box_rows) box
+bool make_map(CUtensorMap* map, const void* base, int D, int heads, long long rows, int box_heads, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr || base == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle swz = D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q, const void* k, const void* v,
+                        const void* kc, const void* vc, cudaStream_t stream) {
+  CUtensorMap qm, km, vm, kcm, vcm;
+  const void* kk = k ? k : kc;
+  const void* vv = v ? v : vc;
+  const void* kkc = kc ? kc : k;
+  const void* vvc = vc ? vc : v;
+  if (!make_map(&qm, q, D, d.n_q_heads, d.n_tokens, p.G, 128 / p.G)) return LSRM_ERR_CUDA;
+  if (!make_map(&km, kk, D, d.n_kv_heads, k ? d.n_tokens : d.n_blocks, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&vm, vv, D, d.n_kv_heads, v ? d.n_tokens : d.n_blocks, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&kcm, kkc, D, d.n_kv_heads, kc ? d.n_blocks : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&vcm, vvc, D, d.n_kv_heads, vc ? d.n_blocks : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
+  const size_t smem = sizeof(TcSmem<D>) + 1024;
+  if (cudaFuncSetAttribute(nsa_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LSRM_ERR_CUDA;
+  const int tiles = (d.max_block_len * p.G + 127) / 128;
+  dim3 grid((unsigned)((tiles + 1) / 2), (unsigned)d.n_kv_heads, (unsigned)d.n_blocks);
+  nsa_attn_tc_kernel<D><<<grid, kTcThreads, smem, stream>>>(qm, km, vm, kcm, vcm, p);
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
+}  // namespace
+
+lsrm_status launch_attn_tc(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
+                           const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
+                           int route_all, int branches, void* out, float* obranch, float* lse, int lse_stride,
+                           int lse_first, uint32_t* status, cudaStream_t stream) {
+  const int G = d.n_q_heads / d.n_kv_heads;
+  if (128 % G != 0) return LSRM_ERR_UNSUPPORTED;
+  if (d.n_forced + d.top_k > kTcMaxSel || d.n_blocks > 65535) return LSRM_ERR_UNSUPPORTED;
+  TcParams p{};
+  p.off = off;
+  p.gates = (const uint16_t*)gates;
+  p.idx = idx;
+  p.forced = d.forced_blocks;
+  p.out = (uint16_t*)out;
+  p.obranch = obranch;
+  p.lse = lse;
+  p.status = status;
+  p.N = (int)d.n_tokens;
+  p.B = d.n_blocks;
+  p.Hq = d.n_q_heads;
+  p.Hkv = d.n_kv_heads;
+  p.G = G;
+  p.top_k = d.top_k;
+  p.idx_heads = idx_heads;
+  p.n_forced = d.n_forced;
+  p.window = d.window;
+  p.n_gates = d.n_gates;
+  p.route_all = route_all;
+  p.branches = branches;
+  p.lse_stride = lse_stride;
+  p.lse_first = lse_first;
+  const float tau = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim);
+  p.scale_log2 = tau * 1.4426950408889634f;
+  if (d.head_dim == 32) return launch_tc_d<32>(d, p, q, k, v, kc, vc, stream);
+  if (d.head_dim == 64) return launch_tc_d<64>(d, p, q, k, v, kc, vc, stream);
+  return LSRM_ERR_UNSUPPORTED;
+}
+
+}  // namespace lsrm
