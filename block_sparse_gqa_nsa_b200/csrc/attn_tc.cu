@@ -493,7 +493,7 @@ lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q
 
 }  // namespace
 
-lsrm_status launch_attn_tc(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
+lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                            const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                            int route_all, int branches, void* out, float* obranch, float* lse, int lse_stride,
                            int lse_first, uint32_t* status, cudaStream_t stream) {
