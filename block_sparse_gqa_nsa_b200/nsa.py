@@ -27,7 +27,7 @@ ROUTE_GIVEN, ROUTE_SCORE, ROUTE_GEOMETRIC, ROUTE_ALL = 0, 1, 2, 3
 
 # every symbol include/lsrm_nsa.h declares
 EXPORTS = ("lsrm_nsa_workspace_size", "lsrm_nsa_workspace_init", "lsrm_nsa_compress", "lsrm_route_score_topk",
-           "lsrm_route_geometric", "lsrm_route_pooled_topk", "lsrm_nsa_cmp_attn", "lsrm_nsa_select_attn",
+           "lsrm_route_geometric", "lsrm_route_geometric_noalloc", "lsrm_route_pooled_topk", "lsrm_nsa_cmp_attn", "lsrm_nsa_select_attn",
            "lsrm_nsa_window_attn", "lsrm_nsa_gate_combine", "lsrm_nsa_attend", "lsrm_nsa_forward", "lsrm_nsa_backward",
            "lsrm_nsa_last_device_status", "lsrm_status_string")
 
@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsrm_nsa_compress": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_route_score_topk": ([D, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_route_geometric": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
+        "lsrm_route_geometric_noalloc": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_route_pooled_topk": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_cmp_attn": ([D, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_select_attn": ([D, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp], ctypes.c_int),
@@ -162,6 +163,17 @@ def lsrm_route_score_topk(desc, off, q, kc32, idx, score=None, ws=None, stream=N
 def lsrm_route_geometric(desc, off, coords, idx, ws, stream=None):
     _check(off, torch.int32, "off"); _check(coords, torch.int32, "coords"); _check(idx, torch.int32, "idx")
     _call("lsrm_route_geometric", ctypes.byref(desc), _ptr(off), _ptr(coords), _ptr(idx), _ptr(ws),
+          _stream(stream))
+
+
+def lsrm_route_geometric_noalloc(desc, off, coords, idx, status=None, stream=None):
+    """Geometric routing without a workspace, for callers that cannot allocate device memory
+    (its scratch is a fixed array inside the library; at most 16384 blocks; calls that
+    overlap on the GPU race).  `status` is an optional device uint32 tensor that receives
+    the bounds bit."""
+    _check(off, torch.int32, "off"); _check(coords, torch.int32, "coords"); _check(idx, torch.int32, "idx")
+    _check(status, torch.int32, "status")
+    _call("lsrm_route_geometric_noalloc", ctypes.byref(desc), _ptr(off), _ptr(coords), _ptr(idx), _ptr(status),
           _stream(stream))
 
 

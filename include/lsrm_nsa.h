@@ -120,6 +120,24 @@ LSRM_API lsrm_status lsrm_route_score_topk(const lsrm_nsa_desc* desc, const int3
 LSRM_API lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords,
                                  int32_t* idx, void* ws, void* stream);
 
+/* Geometric routing that allocates nothing and takes no workspace, for callers that may
+ * not allocate device memory at call time and have none to lend (for example a plugin in
+ * a host framework whose memory pool owns the whole GPU, or a loop whose policy forbids
+ * allocation after start-up).  The pages have no counterpart of this call; it computes
+ * exactly what lsrm_route_geometric computes.  Its centroid scratch is a fixed array in
+ * the library's own device memory (192 KiB, held on every GPU that loads the library until
+ * the process exits), so n_blocks may be at most 16384; larger descriptors are rejected
+ * with LSRM_ERR_WORKSPACE.  The first call on each device looks up that array's device
+ * address (with the device current); make that first call before any stream capture.
+ * Every call shares the one array: calls that may overlap on the GPU (different streams,
+ * or different host threads on one device) race and must be serialised by the caller.
+ * status_or_null (device uint32, may be NULL) receives LSRM_ERR_BOUNDS as bit
+ * (1 << (LSRM_ERR_BOUNDS - 1)) OR-ed in when a coordinate lies outside [-2^29, 2^29];
+ * the caller clears it. */
+LSRM_API lsrm_status lsrm_route_geometric_noalloc(const lsrm_nsa_desc* desc, const int32_t* off,
+                                                  const int32_t* coords, int32_t* idx, uint32_t* status_or_null,
+                                                  void* stream);
+
 /* Speed3R routing (Speed3R page 2.1 selection branch, 2.2 forced frame-0 and
  * camera blocks): per block a and head h, the top_k blocks j outside the forced
  * set by (tau * qc[a,h] . kc[j,h] desc, j asc), computed from the bf16 pooled
