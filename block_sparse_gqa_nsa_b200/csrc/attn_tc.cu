@@ -23,29 +23,39 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "tc_ptx.cuh"
 
 namespace lsrm {
 
 using namespace tc;
 
+// One pair in kPolyMod of the exponentials goes through poly_exp2 on the FMA pipe instead of
+// MUFU (whose 16 ex2 per clock per SM bound the kernel at d = 32); 0 keeps all on MUFU.
+#ifndef LSRM_POLY_MOD
+#define LSRM_POLY_MOD 0
+#endif
+constexpr int kPolyMod = LSRM_POLY_MOD;
+
 constexpr int kTcThreads = 320;
-constexpr int kTcMaxSel = 1024;
+constexpr int kTcMaxSel = 256;
 
 template <int D>
 struct TcCfg {
   static constexpr int kRows = 128;
-  static constexpr int kSlots = D == 32 ? 2 : 1;  // 64-key slots per chunk
-  static constexpr int kKeys = 64 * kSlots;       // keys per chunk = N of S = Q K^T
-  static constexpr int kStages = 4;
+  static constexpr int kKeys = 64;                 // keys per chunk = N of S = Q K^T (one block)
+  static constexpr int kStages = 4;                // K/V ring
+  static constexpr int kCtasPerSm = D == 32 ? 2 : 1;
+  static constexpr int kTmemCols = D == 32 ? 256 : 512;   // per CTA (power of two)
+  static constexpr int kColsPerTile = kTmemCols / 2;
   static constexpr int kRowBytes = D * 2;
   static constexpr uint32_t kLayout = D == 32 ? kLayoutSW64 : kLayoutSW128;
   static constexpr uint32_t kAtomBytes = 8 * kRowBytes;  // 8 rows of one swizzle atom
   static constexpr int kQBytes = kRows * kRowBytes;
-  static constexpr int kSlotBytes = 64 * kRowBytes;
   static constexpr int kKVBytes = kKeys * kRowBytes;
+  // tensor memory per tile: S (fp32 scores) | P (bf16 pairs) | O
   static constexpr int kColS = 0, kColP = kKeys, kColO = kKeys + kKeys / 2;
-  static constexpr int kColsPerTile = 256;
   static constexpr uint32_t kIdescQK = idesc_bf16(128, kKeys, false);
   static constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
   static_assert(kColO + D <= kColsPerTile, "tensor memory budget");
@@ -57,7 +67,9 @@ struct TcSmem {
   uint8_t q[2][C::kQBytes];
   uint8_t k[C::kStages][C::kKVBytes];
   uint8_t v[C::kStages][C::kKVBytes];
-  uint64_t q_full[2], kv_full[C::kStages], kv_empty[C::kStages], s_full[2], p_full[2], pv_done[2], drain;
+  float acc[2][D][128];  // gated output sum per tile, column-major so a warp's rows are one bank row
+  uint64_t q_full[2], kv_full[C::kStages], kv_empty[C::kStages];
+  uint64_t s_full[2], p_full[2], pv_done[2], drain;
   uint32_t tmem_base;
   int abort;
   int n_sel;
@@ -80,7 +92,7 @@ struct TcParams {
 
 enum : int { TC_CMP = 1, TC_SLC = 2, TC_WIN = 4 };
 
-// chunk sequence shared by the three roles: [cmp chunks][slc chunks][win chunk]
+// chunk sequence shared by the three roles: [cmp chunks][slc chunks][win chunk], 64 keys each
 struct Chunks {
   int n_cmp, n_slc, n_win, total;
   __device__ __forceinline__ int branch(int c, int& local) const {
@@ -94,33 +106,29 @@ struct Chunks {
   }
 };
 
+// first key row (block-mean index or token index) and number of valid keys of chunk (br, local)
 template <int D>
-__device__ __forceinline__ void slot_info(const TcSmem<D>& S, const TcParams& p, int br, int local, int slot,
-                                          int t0, int n_a, int& start, int& nvalid) {
-  using C = TcCfg<D>;
+__device__ __forceinline__ void chunk_keys(const TcSmem<D>& S, const TcParams& p, int br, int local, int t0,
+                                           int n_a, int& start, int& nvalid) {
   if (br == 0) {
-    start = local * C::kKeys + slot * 64;
-    nvalid = min(64, max(0, p.B - start));
+    start = local * 64;
+    nvalid = min(64, p.B - start);
   } else if (br == 1) {
-    const int i = local * C::kSlots + slot;
     if (p.route_all) {
-      if (i < p.B) { start = p.off[i]; nvalid = p.off[i + 1] - start; }
-      else { start = t0; nvalid = 0; }
-    } else if (i < S.n_sel) {
-      start = S.sel_start[i];
-      nvalid = S.sel_n[i];
+      start = p.off[local];
+      nvalid = p.off[local + 1] - start;
     } else {
-      start = t0;
-      nvalid = 0;
+      start = S.sel_start[local];
+      nvalid = S.sel_n[local];
     }
   } else {
     start = t0;
-    nvalid = slot == 0 ? n_a : 0;
+    nvalid = n_a;
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kCtasPerSm)
 nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
                    const __grid_constant__ CUtensorMap vcmap, const TcParams p) {
@@ -164,7 +172,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&S.tmem_base, 512);
+    tmem_alloc(&S.tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -174,8 +182,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 
   Chunks cs;
   cs.n_cmp = (p.branches & TC_CMP) ? (p.B + C::kKeys - 1) / C::kKeys : 0;
-  const int n_sel = (p.branches & TC_SLC) ? (p.route_all ? p.B : S.n_sel) : 0;
-  cs.n_slc = (n_sel + C::kSlots - 1) / C::kSlots;
+  cs.n_slc = (p.branches & TC_SLC) ? (p.route_all ? p.B : S.n_sel) : 0;
   cs.n_win = ((p.branches & TC_WIN) && p.window > 0) ? 1 : 0;
   cs.total = cs.n_cmp + cs.n_slc + cs.n_win;
   volatile int* abort = &S.abort;
@@ -192,17 +199,12 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       for (int c = 0; c < cs.total; ++c) {
         const int st = c % C::kStages;
         if (c >= C::kStages && !mbar_wait(&S.kv_empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
-        int local;
+        int local, start, nvalid;
         const int br = cs.branch(c, local);
+        chunk_keys<D>(S, p, br, local, t0, n_a, start, nvalid);
         mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
-        for (int s = 0; s < C::kSlots; ++s) {
-          int start, nvalid;
-          slot_info<D>(S, p, br, local, s, t0, n_a, start, nvalid);
-          const CUtensorMap* km = br == 0 ? &kcmap : &kmap;
-          const CUtensorMap* vm = br == 0 ? &vcmap : &vmap;
-          tma_load_3d(S.k[st] + s * C::kSlotBytes, km, &S.kv_full[st], 0, g, start);
-          tma_load_3d(S.v[st] + s * C::kSlotBytes, vm, &S.kv_full[st], 0, g, start);
-        }
+        tma_load_3d(S.k[st], br == 0 ? &kcmap : &kmap, &S.kv_full[st], 0, g, start);
+        tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
         issued = c + 1;
       }
       if (*abort) {
@@ -219,9 +221,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       bool ok = mbar_wait(&S.q_full[0], 0, abort, p.status) && mbar_wait(&S.q_full[1], 0, abort, p.status);
       tc_fence_after();
       const uint32_t qaddr[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
-      auto issue_qk = [&](int t, int st) {
+      auto issue_qk = [&](int t, int c) {
         const uint32_t d = tmem + t * C::kColsPerTile + C::kColS;
-        const uint32_t kaddr = smem_u32(S.k[st]);
+        const uint32_t kaddr = smem_u32(S.k[c % C::kStages]);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint64_t ad = smem_desc(qaddr[t] + k * 32, 16, C::kAtomBytes, C::kLayout);
@@ -230,9 +232,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         }
       };
       auto issue_pv = [&](int t, int c) {
-        const int st = c % C::kStages;
         const uint32_t d = tmem + t * C::kColsPerTile + C::kColO;
-        const uint32_t vaddr = smem_u32(S.v[st]);
+        const uint32_t vaddr = smem_u32(S.v[c % C::kStages]);
         const bool first = cs.first_of_branch(c);
 #pragma unroll
         for (int kk = 0; kk < C::kKeys / 16; ++kk) {
@@ -242,8 +243,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         }
       };
       for (int c = 0; ok && c < cs.total; ++c) {
-        const int st = c % C::kStages;
-        if (!mbar_wait(&S.kv_full[st], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
           if (c > 0) {
@@ -252,7 +252,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             issue_pv(t, c - 1);
             mma_commit(&S.pv_done[t]);
           }
-          issue_qk(t, st);
+          issue_qk(t, c);  // S of tile t was released with P(c - 1)
           mma_commit(&S.s_full[t]);
         }
         if (!ok) break;
@@ -282,30 +282,31 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     const int tok = t0 + (valid ? tok_local : 0);
     const int head = g * p.G + R % p.G;
     const size_t orow = (size_t)tok * p.Hq + head;
-    float gate[3] = {0.f, 0.f, 0.f};
-    if (p.out != nullptr && valid)
-      for (int b = 0; b < p.n_gates; ++b) gate[b] = bf16_to_f32(p.gates[orow * p.n_gates + b]);
-    float out_acc[D];
+    float* acc = &S.acc[t][0][row];  // acc[i * 128] = output column i of this row
 #pragma unroll
-    for (int i = 0; i < D; ++i) out_acc[i] = 0.f;
-    float m = -INFINITY, l = 0.f;
+    for (int i = 0; i < D; ++i) acc[i * 128] = 0.f;
+    float m = -INFINITY;  // reference of the current branch, log2 units
+    float l = 0.f;        // row sum of P for the current branch
 
     auto finalize = [&](int br, float mb, float lb) {
-      uint32_t o[D];
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) tmem_ld32(tbase + C::kColO + 32 * i, o + 32 * i);
-      tmem_ld_wait();
       const float inv = lb > 0.f ? 1.f / lb : 0.f;
-      if (p.out != nullptr) {
+      const float gi = (p.out != nullptr && valid) ? bf16_to_f32(p.gates[orow * p.n_gates + br]) * inv : 0.f;
 #pragma unroll
-        for (int i = 0; i < D; ++i) out_acc[i] = fmaf(gate[br] * inv, __uint_as_float(o[i]), out_acc[i]);
-      }
-      if (p.obranch != nullptr && valid) {
-        float4* dst = reinterpret_cast<float4*>(p.obranch + orow * D);
+      for (int i = 0; i < D / 32; ++i) {
+        uint32_t o[32];
+        tmem_ld32(tbase + C::kColO + 32 * i, o);
+        tmem_ld_wait();
+        if (p.out != nullptr) {
 #pragma unroll
-        for (int i = 0; i < D / 4; ++i)
-          dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                               __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          for (int e = 0; e < 32; ++e) acc[(32 * i + e) * 128] = fmaf(gi, __uint_as_float(o[e]), acc[(32 * i + e) * 128]);
+        }
+        if (p.obranch != nullptr && valid) {
+          float4* dst = reinterpret_cast<float4*>(p.obranch + orow * D + 32 * i);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                 __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+        }
       }
       if (p.lse != nullptr && valid) {
         int slot = p.lse_first;
@@ -315,68 +316,109 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       }
     };
 
-    int prev_br = -1;
-    bool ok = true;
-    const int wlo = tok_local - p.window / 2, whi = tok_local + p.window / 2 - 1;
     // waits are made warp-uniform: the tensor-memory accesses after them are .sync.aligned
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       const bool w = mbar_wait(bar, parity, abort, p.status);
       return __all_sync(0xffffffffu, w);
     };
-    for (int c = 0; c < cs.total; ++c) {
-      if (!wait_all(&S.s_full[t], c & 1)) { ok = false; break; }
-      tc_fence_after();
-      int local;
-      const int br = cs.branch(c, local);
-      const bool first = cs.first_of_branch(c);
-      int nv[C::kSlots];
-      bool need_mask = br == 2;
+    const int wlo = tok_local - p.window / 2, whi = tok_local + p.window / 2 - 1;
+    const float sc = p.scale_log2;
+    int br = 0, nv = 0;
+    // raw score of key j of the chunk, or -inf where masked (short block or outside the window band)
+    auto masked = [&](uint32_t raw, int j) -> float {
+      bool kv = j < nv;
+      if (br == 2) kv = kv && j >= wlo && j <= whi;
+      return kv ? __uint_as_float(raw) : -INFINITY;
+    };
+    // max of the chunk's raw scores (the scale is positive, so it commutes with the max)
+    auto chunk_max_t = [&](auto need_mask_tag) -> float {
+      constexpr bool need_mask = decltype(need_mask_tag)::value;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int s = 0; s < C::kSlots; ++s) {
-        int start;
-        slot_info<D>(S, p, br, local, s, t0, n_a, start, nv[s]);
-        need_mask |= nv[s] < 64;
-      }
-      // key j of the chunk: slot j/64, row j%64 of that slot
-      auto logit = [&](uint32_t raw, int j) -> float {
-        if (need_mask) {
-          const int kr = j & 63;
-          bool kv = kr < nv[j >> 6];
-          if (br == 2) kv = kv && kr >= wlo && kr <= whi;
-          if (!kv) return -INFINITY;
-        }
-        return __uint_as_float(raw) * p.scale_log2;
-      };
-      // pass 1: chunk max (log2 units), 32 columns at a time
-      float mc = -INFINITY;
-#pragma unroll
-      for (int qd = 0; qd < C::kKeys / 32; ++qd) {
+      for (int h = 0; h < 2; ++h) {
         uint32_t r[32];
-        tmem_ld32(tbase + C::kColS + 32 * qd, r);
+        tmem_ld32(tbase + C::kColS + 32 * h, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mc = fmaxf(mc, logit(r[i], 32 * qd + i));
+        for (int i = 0; i < 32; i += 2) {
+          const float s0 = need_mask ? masked(r[i], 32 * h + i) : __uint_as_float(r[i]);
+          const float s1 = need_mask ? masked(r[i + 1], 32 * h + i + 1) : __uint_as_float(r[i + 1]);
+          mx[(i >> 1) & 3] = fmax3(mx[(i >> 1) & 3], s0, s1);
+        }
       }
-      const float m_prev = m, l_prev = l;
-      float alpha = 1.f;
-      bool rescale = false;
+      return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    };
+    // P = exp2(s * scale - mref) as bf16 pairs into tensor memory, 32 keys at a time; returns the
+    // chunk's raw max and its sum of P in *lsum
+    auto exp_pass_t = [&](float mref, float* lsum, auto need_mask_tag) -> float {
+      constexpr bool need_mask = decltype(need_mask_tag)::value;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      const float nm = -mref;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[32];
+        tmem_ld32(tbase + C::kColS + 32 * h, r);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = 32 * h + 2 * i;
+          const float s0 = need_mask ? masked(r[2 * i], j) : __uint_as_float(r[2 * i]);
+          const float s1 = need_mask ? masked(r[2 * i + 1], j + 1) : __uint_as_float(r[2 * i + 1]);
+          mx[i & 3] = fmax3(mx[i & 3], s0, s1);
+          const float x0 = fmaf(s0, sc, nm), x1 = fmaf(s1, sc, nm);
+          float p0, p1;
+          if (kPolyMod > 0 && i % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
+            p0 = poly_exp2(x0);
+            p1 = poly_exp2(x1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          ls[i & 3] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tbase + C::kColP + 16 * h, pk);
+      }
+      *lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    };
+    // masking is decided once per chunk: two straight-line instantiations, no per-key branch
+    auto chunk_max = [&](bool need_mask) -> float {
+      return need_mask ? chunk_max_t(std::true_type{}) : chunk_max_t(std::false_type{});
+    };
+    auto exp_pass = [&](bool need_mask, float mref, float* lsum) -> float {
+      return need_mask ? exp_pass_t(mref, lsum, std::true_type{}) : exp_pass_t(mref, lsum, std::false_type{});
+    };
+
+    int prev_br = -1;
+    bool ok = true;
+    for (int c = 0; c < cs.total; ++c) {
+      if (!wait_all(&S.s_full[t], c & 1)) { ok = false; break; }
+      // P V of the previous chunk must be done before P is overwritten and O is read
+      if (c > 0 && !wait_all(&S.pv_done[t], (c - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      int local, start;
+      br = cs.branch(c, local);
+      const bool first = cs.first_of_branch(c);
+      chunk_keys<D>(S, p, br, local, t0, n_a, start, nv);
+      const bool need_mask = br == 2 || nv < 64;
+      float lsum;
       if (first) {
-        m = mc;
-        l = 0.f;
-      } else if (mc > m + 8.f) {  // move the reference only when it would grow by more than 2^8
-        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mc);
-        m = mc;
-        l *= alpha;
-        rescale = true;
-      }
-      const float mref = m == -INFINITY ? 0.f : m;
-      // the previous P V must be done before P is overwritten and before O is read
-      if (c > 0) {
-        if (!wait_all(&S.pv_done[t], (c - 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        if (first) {
-          finalize(prev_br, m_prev, l_prev);
-        } else if (__any_sync(0xffffffffu, rescale)) {  // rows that keep their reference use alpha = 1
+        if (c > 0) finalize(prev_br, m, l);
+        const float mraw = chunk_max(need_mask);
+        m = mraw == -INFINITY ? -INFINITY : mraw * sc;
+        exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
+        l = lsum;
+      } else {
+        const float mraw = exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
+        // move the reference only when the row max would exceed it by more than 2^8
+        const float cand = mraw == -INFINITY ? -INFINITY : mraw * sc;
+        const bool grow = cand > m + 8.f;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float mn = grow ? cand : m;
+          const float alpha = grow ? (m == -INFINITY ? 0.f : fast_exp2(m - mn)) : 1.f;
 #pragma unroll
           for (int i = 0; i < D / 32; ++i) {
             uint32_t o[32];
@@ -386,46 +428,30 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st32(tbase + C::kColO + 32 * i, o);
           }
+          l *= alpha;
+          m = mn;
+          exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
         }
+        l += lsum;
       }
-      // pass 2: P = exp2(x - m) as bf16 pairs, 32 columns of S -> 16 columns of P
-      float ls = 0.f;
-#pragma unroll
-      for (int qd = 0; qd < C::kKeys / 32; ++qd) {
-        uint32_t r[32];
-        tmem_ld32(tbase + C::kColS + 32 * qd, r);
-        tmem_ld_wait();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(logit(r[2 * i], 32 * qd + 2 * i) - mref);
-          const float p1 = fast_exp2(logit(r[2 * i + 1], 32 * qd + 2 * i + 1) - mref);
-          ls += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tbase + C::kColP + 16 * qd, pk);
-      }
-      l += ls;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&S.p_full[t]);
       prev_br = br;
     }
-    if (ok && cs.total > 0) {
-      if (wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
-        tc_fence_after();
-        finalize(prev_br, m, l);
-        if (p.out != nullptr && valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
+    if (ok && cs.total > 0 && wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
+      tc_fence_after();
+      finalize(prev_br, m, l);
+      if (p.out != nullptr && valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
 #pragma unroll
-          for (int i = 0; i < D / 8; ++i) {
-            uint4 u;
-            u.x = pack_bf16x2(out_acc[8 * i + 0], out_acc[8 * i + 1]);
-            u.y = pack_bf16x2(out_acc[8 * i + 2], out_acc[8 * i + 3]);
-            u.z = pack_bf16x2(out_acc[8 * i + 4], out_acc[8 * i + 5]);
-            u.w = pack_bf16x2(out_acc[8 * i + 6], out_acc[8 * i + 7]);
-            dst[i] = u;
-          }
+        for (int i = 0; i < D / 8; ++i) {
+          uint4 u;
+          u.x = pack_bf16x2(acc[(8 * i + 0) * 128], acc[(8 * i + 1) * 128]);
+          u.y = pack_bf16x2(acc[(8 * i + 2) * 128], acc[(8 * i + 3) * 128]);
+          u.z = pack_bf16x2(acc[(8 * i + 4) * 128], acc[(8 * i + 5) * 128]);
+          u.w = pack_bf16x2(acc[(8 * i + 6) * 128], acc[(8 * i + 7) * 128]);
+          dst[i] = u;
         }
       }
     }
@@ -435,7 +461,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -499,7 +525,7 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
                            int lse_first, uint32_t* status, cudaStream_t stream) {
   const int G = d.n_q_heads / d.n_kv_heads;
   if (128 % G != 0) return LSRM_ERR_UNSUPPORTED;
-  if (d.n_forced + d.top_k > kTcMaxSel || d.n_blocks > 65535) return LSRM_ERR_UNSUPPORTED;
+  if ((!route_all && d.n_forced + d.top_k > kTcMaxSel) || d.n_blocks > 65535) return LSRM_ERR_UNSUPPORTED;
   TcParams p{};
   p.off = off;
   p.gates = (const uint16_t*)gates;
