@@ -348,28 +348,26 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       }
       return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
     };
-    // P = exp2(s * scale - mref) as bf16 pairs into tensor memory, 32 keys at a time; returns the
-    // chunk's raw max and its sum of P in *lsum
+    // P = exp2(s * scale - mref) as bf16 pairs into tensor memory; returns the chunk's raw max and
+    // its sum of P in *lsum.  S is read 16 columns at a time, each load issued before the previous
+    // quarter is processed so the tensor-memory latency overlaps the exponentials.
     auto exp_pass_t = [&](float mref, float* lsum, auto need_mask_tag) -> float {
       constexpr bool need_mask = decltype(need_mask_tag)::value;
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
       const float nm = -mref;
+      uint32_t ra[16], rb[16];
+      auto quarter = [&](const uint32_t* r, int qd) {
+        uint32_t pk[8];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t r[32];
-        tmem_ld32(tbase + C::kColS + 32 * h, r);
-        tmem_ld_wait();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j = 32 * h + 2 * i;
+        for (int i = 0; i < 8; ++i) {
+          const int j = 16 * qd + 2 * i;
           const float s0 = need_mask ? masked(r[2 * i], j) : __uint_as_float(r[2 * i]);
           const float s1 = need_mask ? masked(r[2 * i + 1], j + 1) : __uint_as_float(r[2 * i + 1]);
           mx[i & 3] = fmax3(mx[i & 3], s0, s1);
           const float x0 = fmaf(s0, sc, nm), x1 = fmaf(s1, sc, nm);
           float p0, p1;
-          if (kPolyMod > 0 && i % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
+          if (kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
             p0 = poly_exp2(x0);
             p1 = poly_exp2(x1);
           } else {
@@ -379,7 +377,17 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           ls[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tbase + C::kColP + 16 * h, pk);
+        tmem_st8(tbase + C::kColP + 8 * qd, pk);
+      };
+      tmem_ld16(tbase + C::kColS, ra);
+      tmem_ld_wait();
+#pragma unroll
+      for (int qd = 0; qd < C::kKeys / 16; ++qd) {
+        uint32_t* cur = (qd & 1) ? rb : ra;
+        uint32_t* nxt = (qd & 1) ? ra : rb;
+        if (qd + 1 < C::kKeys / 16) tmem_ld16(tbase + C::kColS + 16 * (qd + 1), nxt);
+        quarter(cur, qd);
+        if (qd + 1 < C::kKeys / 16) tmem_ld_wait();
       }
       *lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
