@@ -23,6 +23,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <climits>
 #include <type_traits>
 
 #include "tc_ptx.cuh"
@@ -88,6 +89,16 @@ struct TcParams {
   uint32_t* status;
   int N, B, Hq, Hkv, G, top_k, idx_heads, n_forced, window, n_gates, route_all, branches, lse_stride, lse_first;
   float scale_log2;
+  // compressed-branch key count (block means, or gathered forced tokens); n_ckeys_dev overrides it
+  int n_ckeys;
+  const int* n_ckeys_dev;
+  // query blocks of a fixed size instead of `off` (dense passes over pooled queries or all tokens)
+  int uniform_block;
+  // streaming top-k of the compressed-branch logits (pooled-query routing, d = 64 only):
+  // topk_idx [rows][topk_heads][topk_k]; blocks whose bit is set in forced_bits are skipped
+  int32_t* topk_idx;
+  int topk_k;
+  const uint32_t* forced_bits;
 };
 
 enum : int { TC_CMP = 1, TC_SLC = 2, TC_WIN = 4 };
@@ -109,10 +120,10 @@ struct Chunks {
 // first key row (block-mean index or token index) and number of valid keys of chunk (br, local)
 template <int D>
 __device__ __forceinline__ void chunk_keys(const TcSmem<D>& S, const TcParams& p, int br, int local, int t0,
-                                           int n_a, int& start, int& nvalid) {
+                                           int n_a, int n_ckeys, int& start, int& nvalid) {
   if (br == 0) {
     start = local * 64;
-    nvalid = min(64, p.B - start);
+    nvalid = min(64, n_ckeys - start);
   } else if (br == 1) {
     if (p.route_all) {
       start = p.off[local];
@@ -138,7 +149,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   TcSmem<D>& S = *reinterpret_cast<TcSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, g = blockIdx.y, a = blockIdx.z;
-  const int t0 = p.off[a], n_a = p.off[a + 1] - t0;
+  const int t0 = p.uniform_block ? a * p.uniform_block : p.off[a];
+  const int n_a = p.uniform_block ? min(p.uniform_block, p.N - t0) : p.off[a + 1] - t0;
   const int rows_total = n_a * p.G;
   const int tile0 = pair * 2;
   if (tile0 * 128 >= rows_total) return;  // the whole CTA leaves before any setup
@@ -181,7 +193,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   const uint32_t tmem = S.tmem_base;
 
   Chunks cs;
-  cs.n_cmp = (p.branches & TC_CMP) ? (p.B + C::kKeys - 1) / C::kKeys : 0;
+  const int n_ckeys = p.n_ckeys_dev != nullptr ? *p.n_ckeys_dev : p.n_ckeys;
+  cs.n_cmp = (p.branches & TC_CMP) ? (n_ckeys + C::kKeys - 1) / C::kKeys : 0;
   cs.n_slc = (p.branches & TC_SLC) ? (p.route_all ? p.B : S.n_sel) : 0;
   cs.n_win = ((p.branches & TC_WIN) && p.window > 0) ? 1 : 0;
   cs.total = cs.n_cmp + cs.n_slc + cs.n_win;
@@ -201,7 +214,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (c >= C::kStages && !mbar_wait(&S.kv_empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
         int local, start, nvalid;
         const int br = cs.branch(c, local);
-        chunk_keys<D>(S, p, br, local, t0, n_a, start, nvalid);
+        chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nvalid);
         mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
         tma_load_3d(S.k[st], br == 0 ? &kcmap : &kmap, &S.kv_full[st], 0, g, start);
         tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
@@ -330,6 +343,45 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       if (br == 2) kv = kv && j >= wlo && j <= whi;
       return kv ? __uint_as_float(raw) : -INFINITY;
     };
+    // ---- streaming top-k of the compressed-branch logits (pooled-query routing) ----
+    // A 32-entry min-heap per row, kept in this row's column of the (otherwise unused) output
+    // accumulator: values in acc[0..31], block ids in acc[32..63].  The root is the worst entry
+    // in the order (logit desc, block asc), so ties evict the larger block id first; keys arrive
+    // in increasing block order, so a candidate enters only when strictly above the root.
+    const bool topk_on = (D == 64) && p.topk_idx != nullptr;
+    float thr = -INFINITY;
+    int key_base = 0;        // block id of key 0 of the current chunk
+    uint64_t fmask = 0;      // forced blocks among the chunk's 64 keys
+    auto hv = [&](int i) -> float& { return acc[i * 128]; };
+    auto hj = [&](int i) -> int& { return reinterpret_cast<int&>(acc[(32 + i) * 128]); };
+    auto worse = [&](float va, int ja, float vb, int jb) { return va < vb || (va == vb && ja > jb); };
+    auto topk_consider = [&](float sv, int j) {
+      if (sv > thr && !((fmask >> j) & 1ull)) {
+        const int jg = key_base + j;
+        int i = 0;
+        while (true) {
+          const int l = 2 * i + 1, r = l + 1;
+          if (l >= 32) break;
+          int c = l;
+          if (r < 32 && worse(hv(r), hj(r), hv(l), hj(l))) c = r;
+          if (!worse(hv(c), hj(c), sv, jg)) break;
+          hv(i) = hv(c);
+          hj(i) = hj(c);
+          i = c;
+        }
+        hv(i) = sv;
+        hj(i) = jg;
+        thr = hv(0);
+      }
+    };
+    if (topk_on) {
+#pragma unroll 1
+      for (int i = 0; i < 32; ++i) {
+        hv(i) = -INFINITY;
+        hj(i) = INT_MAX;
+      }
+    }
+
     // max of the chunk's raw scores (the scale is positive, so it commutes with the max)
     auto chunk_max_t = [&](auto need_mask_tag) -> float {
       constexpr bool need_mask = decltype(need_mask_tag)::value;
@@ -351,8 +403,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     // P = exp2(s * scale - mref) as bf16 pairs into tensor memory; returns the chunk's raw max and
     // its sum of P in *lsum.  S is read 16 columns at a time, each load issued before the previous
     // quarter is processed so the tensor-memory latency overlaps the exponentials.
-    auto exp_pass_t = [&](float mref, float* lsum, auto need_mask_tag) -> float {
+    auto exp_pass_t = [&](float mref, float* lsum, auto need_mask_tag, auto topk_tag) -> float {
       constexpr bool need_mask = decltype(need_mask_tag)::value;
+      constexpr bool topk = decltype(topk_tag)::value && D == 64;
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
       const float nm = -mref;
@@ -365,6 +418,10 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           const float s0 = need_mask ? masked(r[2 * i], j) : __uint_as_float(r[2 * i]);
           const float s1 = need_mask ? masked(r[2 * i + 1], j + 1) : __uint_as_float(r[2 * i + 1]);
           mx[i & 3] = fmax3(mx[i & 3], s0, s1);
+          if constexpr (topk) {
+            topk_consider(s0, j);
+            topk_consider(s1, j + 1);
+          }
           const float x0 = fmaf(s0, sc, nm), x1 = fmaf(s1, sc, nm);
           float p0, p1;
           if (kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
@@ -397,7 +454,11 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       return need_mask ? chunk_max_t(std::true_type{}) : chunk_max_t(std::false_type{});
     };
     auto exp_pass = [&](bool need_mask, float mref, float* lsum) -> float {
-      return need_mask ? exp_pass_t(mref, lsum, std::true_type{}) : exp_pass_t(mref, lsum, std::false_type{});
+      if (topk_on && br == 0)
+        return need_mask ? exp_pass_t(mref, lsum, std::true_type{}, std::true_type{})
+                         : exp_pass_t(mref, lsum, std::false_type{}, std::true_type{});
+      return need_mask ? exp_pass_t(mref, lsum, std::true_type{}, std::false_type{})
+                       : exp_pass_t(mref, lsum, std::false_type{}, std::false_type{});
     };
 
     int prev_br = -1;
@@ -410,8 +471,13 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       int local, start;
       br = cs.branch(c, local);
       const bool first = cs.first_of_branch(c);
-      chunk_keys<D>(S, p, br, local, t0, n_a, start, nv);
+      chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nv);
       const bool need_mask = br == 2 || nv < 64;
+      if (topk_on && br == 0) {
+        key_base = local * 64;
+        const uint32_t w0 = p.forced_bits[key_base >> 5], w1 = p.forced_bits[(key_base >> 5) + 1];
+        fmask = (uint64_t)w0 | ((uint64_t)w1 << 32);
+      }
       float lsum;
       if (first) {
         if (c > 0) finalize(prev_br, m, l);
@@ -446,6 +512,27 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       tc_fence_before();
       mbar_arrive(&S.p_full[t]);
       prev_br = br;
+    }
+    if (cs.total == 0 && valid) {  // no keys at all (e.g. an empty forced set): defined outputs
+      if (p.obranch != nullptr)
+        for (int i = 0; i < D; ++i) p.obranch[orow * D + i] = 0.f;
+      if (p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first] = -INFINITY;
+    }
+    if (ok && topk_on && valid) {
+      // emit the row's top-k in order (logit desc, block asc); missing entries are -1
+      int32_t* dst = p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k;
+      uint32_t taken = 0;
+#pragma unroll 1
+      for (int k = 0; k < p.topk_k; ++k) {
+        int best = -1;
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i) {
+          if ((taken >> i) & 1u) continue;
+          if (best < 0 || worse(hv(best), hj(best), hv(i), hj(i))) best = i;
+        }
+        taken |= 1u << best;
+        dst[k] = hj(best) == INT_MAX ? -1 : hj(best);
+      }
     }
     if (ok && cs.total > 0 && wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
       tc_fence_after();
@@ -504,17 +591,17 @@ bool make_map(CUtensorMap* map, const void* base, int D, int heads, long long ro
 
 template <int D>
 lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q, const void* k, const void* v,
-                        const void* kc, const void* vc, cudaStream_t stream) {
+                        const void* kc, const void* vc, long long kc_rows, cudaStream_t stream) {
   CUtensorMap qm, km, vm, kcm, vcm;
   const void* kk = k ? k : kc;
   const void* vv = v ? v : vc;
   const void* kkc = kc ? kc : k;
   const void* vvc = vc ? vc : v;
   if (!make_map(&qm, q, D, d.n_q_heads, d.n_tokens, p.G, 128 / p.G)) return LSRM_ERR_CUDA;
-  if (!make_map(&km, kk, D, d.n_kv_heads, k ? d.n_tokens : d.n_blocks, 1, 64)) return LSRM_ERR_CUDA;
-  if (!make_map(&vm, vv, D, d.n_kv_heads, v ? d.n_tokens : d.n_blocks, 1, 64)) return LSRM_ERR_CUDA;
-  if (!make_map(&kcm, kkc, D, d.n_kv_heads, kc ? d.n_blocks : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
-  if (!make_map(&vcm, vvc, D, d.n_kv_heads, vc ? d.n_blocks : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&km, kk, D, d.n_kv_heads, k ? d.n_tokens : kc_rows, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&vm, vv, D, d.n_kv_heads, v ? d.n_tokens : kc_rows, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&kcm, kkc, D, d.n_kv_heads, kc ? kc_rows : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&vcm, vvc, D, d.n_kv_heads, vc ? kc_rows : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
   const size_t smem = sizeof(TcSmem<D>) + 1024;
   if (cudaFuncSetAttribute(nsa_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -559,8 +646,51 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
   p.lse_first = lse_first;
   const float tau = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim);
   p.scale_log2 = tau * 1.4426950408889634f;
-  if (d.head_dim == 32) return launch_tc_d<32>(d, p, q, k, v, kc, vc, stream);
-  if (d.head_dim == 64) return launch_tc_d<64>(d, p, q, k, v, kc, vc, stream);
+  p.n_ckeys = d.n_blocks;
+  if (d.head_dim == 32) return launch_tc_d<32>(d, p, q, k, v, kc, vc, d.n_blocks, stream);
+  if (d.head_dim == 64) return launch_tc_d<64>(d, p, q, k, v, kc, vc, d.n_blocks, stream);
+  return LSRM_ERR_UNSUPPORTED;
+}
+
+// Dense multi-head attention of n_q query rows (q [n_q][H][D]) against n_ckeys rows of
+// (kc, vc) ([kc_rows][H][D]), in fixed groups of 256 query rows: the pooled-query compressed
+// branch (optionally with the streaming top-k that routes it) and the forced-block part of the
+// pooled-query selected branch.  Writes fp32 obranch [n_q][H][D] and the natural-log lse [n_q][H].
+lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
+                              long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
+                              float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
+                              uint32_t* status, cudaStream_t stream) {
+  if (topk_idx != nullptr && (D != 64 || topk_k < 1 || topk_k > 32 || forced_bits == nullptr))
+    return LSRM_ERR_UNSUPPORTED;
+  if ((n_q + 255) / 256 > 65535 || n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
+  lsrm_nsa_desc d{};
+  d.n_tokens = n_q;
+  d.n_blocks = (int32_t)((n_q + 255) / 256);  // query groups (grid z)
+  d.max_block_len = 256;
+  d.n_q_heads = H;
+  d.n_kv_heads = H;
+  d.head_dim = D;
+  TcParams p{};
+  p.status = status;
+  p.obranch = obranch;
+  p.lse = lse;
+  p.N = (int)n_q;
+  p.B = n_ckeys;
+  p.Hq = H;
+  p.Hkv = H;
+  p.G = 1;
+  p.n_gates = 1;
+  p.branches = TC_CMP;
+  p.lse_stride = 1;
+  p.scale_log2 = tau * 1.4426950408889634f;
+  p.n_ckeys = n_ckeys;
+  p.n_ckeys_dev = n_ckeys_dev;
+  p.uniform_block = 256;
+  p.topk_idx = topk_idx;
+  p.topk_k = topk_k;
+  p.forced_bits = forced_bits;
+  if (D == 32) return launch_tc_d<32>(d, p, q, nullptr, nullptr, kc, vc, kc_rows, stream);
+  if (D == 64) return launch_tc_d<64>(d, p, q, nullptr, nullptr, kc, vc, kc_rows, stream);
   return LSRM_ERR_UNSUPPORTED;
 }
 

@@ -14,21 +14,25 @@ lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, c
                                    int32_t* idx, uint32_t* status, cudaStream_t s);
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
                                int32_t* idx, float* score, uint32_t* status, cudaStream_t s);
-lsrm_status launch_route_pooled(const lsrm_nsa_desc& d, const void* qc, const void* kc, int32_t* idx,
-                                uint32_t* status, cudaStream_t s);
 lsrm_status launch_gate_combine(const lsrm_nsa_desc& d, const float* oc, const float* os, const float* ow,
                                 const void* gates, void* out, cudaStream_t s);
 lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                         const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                         int route_all, int branches, void* out, float* obranch, float* lse, int lse_stride,
                         int lse_first, uint32_t* status, cudaStream_t stream);
-lsrm_status launch_pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, const void* vc, float* o_blk,
-                              float* lse_blk, cudaStream_t s);
+lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
+                              long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
+                              float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
+                              uint32_t* status, cudaStream_t stream);
 lsrm_status launch_pooled_broadcast(const lsrm_nsa_desc& d, const int32_t* off, const float* o_blk,
                                     const float* lse_blk, float* o_cmp, float* lse, cudaStream_t s);
-lsrm_status launch_attn_pooled_fused(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
-                                     const void* v, const void* gates, const int32_t* idx, const float* o_blk,
-                                     void* out, float* lse, uint32_t* status, cudaStream_t stream);
+lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, const void* k, const void* v,
+                                  uint32_t* bits, int* pre, int* total, void* kf, void* vf, uint32_t* status,
+                                  cudaStream_t s);
+lsrm_status launch_speed3r_routed(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
+                                  const void* v, const void* gates, const int32_t* idx, const float* o_forced,
+                                  const float* lse_forced, const float* o_blk, const float* lse_blk, void* out,
+                                  float* lse_out, uint32_t* status, cudaStream_t s);
 lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
@@ -74,6 +78,30 @@ T* wsp(void* ws, size_t off) {
 }
 
 uint32_t* status_of(void* ws) { return wsp<uint32_t>(ws, 0); }
+
+float tau_of(const lsrm_nsa_desc& d) { return d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim); }
+
+// pooled compressed branch over all B block means, per head (and, with idx, the Speed3R routing:
+// top_k blocks by pooled logit outside the forced set); o_blk / lse_blk go to the workspace
+lsrm_status pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, const void* vc, int32_t* idx,
+                       void* ws, cudaStream_t s) {
+  const Workspace w = workspace_layout(d);
+  uint32_t* bits = wsp<uint32_t>(ws, w.fbits);
+  float* o_blk = wsp<float>(ws, w.obranch);
+  float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
+  if (idx != nullptr) {
+    if (d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
+    if (cudaMemsetAsync(bits, 0, ((size_t)d.n_blocks / 32 + 2) * 4, s) != cudaSuccess) return LSRM_ERR_CUDA;
+    if (d.n_forced > 0) {
+      // bits only (the prefix/gather outputs of this call are not needed here)
+      lsrm_status st = launch_speed3r_forced(d, nullptr, nullptr, nullptr, bits, nullptr, nullptr, nullptr, nullptr,
+                                             status_of(ws), s);
+      if (st != LSRM_OK) return st;
+    }
+  }
+  return launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc, kc, vc, d.n_blocks, d.n_blocks, nullptr,
+                           tau_of(d), o_blk, l_blk, idx, idx ? d.top_k : 0, idx ? bits : nullptr, status_of(ws), s);
+}
 
 #define LSRM_TRY(x)                         \
   do {                                      \
@@ -132,7 +160,9 @@ lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, co
   LSRM_TRY(check_desc(desc));
   LSRM_TRY(check_ws(desc, ws));
   if (!desc->pooled_q || qc == nullptr || kc == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
-  return launch_route_pooled(*desc, qc, kc, idx, status_of(ws), (cudaStream_t)stream);
+  // the routing pass is the pooled compressed branch with its top-k; values are not needed, so the
+  // keys stand in for them and the branch output stays in the workspace
+  return pooled_cmp(*desc, qc, kc, kc, idx, ws, (cudaStream_t)stream);
 }
 
 lsrm_status lsrm_nsa_cmp_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* kc,
@@ -145,7 +175,7 @@ lsrm_status lsrm_nsa_cmp_attn(const lsrm_nsa_desc* desc, const int32_t* off, con
     const Workspace w = workspace_layout(*desc);
     float* o_blk = wsp<float>(ws, w.obranch);
     float* l_blk = o_blk + (size_t)desc->n_blocks * desc->n_q_heads * desc->head_dim;
-    LSRM_TRY(launch_pooled_cmp(*desc, q, kc, vc, o_blk, l_blk, (cudaStream_t)stream));
+    LSRM_TRY(pooled_cmp(*desc, q, kc, vc, nullptr, ws, (cudaStream_t)stream));
     return launch_pooled_broadcast(*desc, off, o_blk, l_blk, o_cmp, lse, (cudaStream_t)stream);
   }
   return launch_attn(*desc, off, q, nullptr, nullptr, kc, vc, nullptr, nullptr, 1, 0, BR_CMP, nullptr, o_cmp, lse,
@@ -220,16 +250,30 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
   int32_t* idx = idx_inout != nullptr ? idx_inout : wsp<int32_t>(ws, w.idx);
 
   if (d.pooled_q) {
+    // Speed3R: pooled Q/K/V; pooled compressed branch + routing; forced part of the selected
+    // branch (dense, tensor cores); routed part merged with it, plus the gated combine
     if (route_mode != LSRM_ROUTE_SCORE && route_mode != LSRM_ROUTE_GIVEN) return LSRM_ERR_INVALID_ARG;
     if (route_mode == LSRM_ROUTE_GIVEN && idx_inout == nullptr) return LSRM_ERR_INVALID_ARG;
-    float* qc32 = wsp<float>(ws, w.qc32);
+    if (d.head_dim != 64 || d.max_block_len > 16) return LSRM_ERR_UNSUPPORTED;
     void* qc16 = wsp<void>(ws, w.qc16);
-    LSRM_TRY(launch_compress(d, off, q, k, v, nullptr, kc16, nullptr, vc16, qc32, qc16, s));
-    if (route_mode == LSRM_ROUTE_SCORE) LSRM_TRY(launch_route_pooled(d, qc16, kc16, idx, status_of(ws), s));
+    LSRM_TRY(launch_compress(d, off, q, k, v, nullptr, kc16, nullptr, vc16, wsp<float>(ws, w.qc32), qc16, s));
+    int* ftotal = wsp<int>(ws, w.ftotal);
+    LSRM_TRY(launch_speed3r_forced(d, off, k, v, wsp<uint32_t>(ws, w.fbits), wsp<int>(ws, w.fpre), ftotal,
+                                   wsp<void>(ws, w.kf), wsp<void>(ws, w.vf), status_of(ws), s));
     float* o_blk = wsp<float>(ws, w.obranch);
     float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
-    LSRM_TRY(launch_pooled_cmp(d, qc16, kc16, vc16, o_blk, l_blk, s));
-    return launch_attn_pooled_fused(d, off, q, k, v, gates, idx, o_blk, out, lse_or_null, status_of(ws), s);
+    const bool route = route_mode == LSRM_ROUTE_SCORE;
+    if (route && d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
+    LSRM_TRY(launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc16, kc16, vc16, d.n_blocks, d.n_blocks,
+                               nullptr, tau_of(d), o_blk, l_blk, route ? idx : nullptr, route ? d.top_k : 0,
+                               route ? wsp<uint32_t>(ws, w.fbits) : nullptr, status_of(ws), s));
+    float* ofrc = wsp<float>(ws, w.ofrc);
+    float* lfrc = wsp<float>(ws, w.lfrc);
+    const long long cap = (long long)(d.n_forced > 0 ? d.n_forced : 1) * d.max_block_len;
+    LSRM_TRY(launch_attn_dense(d.head_dim, d.n_tokens, d.n_q_heads, q, wsp<void>(ws, w.kf), wsp<void>(ws, w.vf),
+                               cap, 0, ftotal, tau_of(d), ofrc, lfrc, nullptr, 0, nullptr, status_of(ws), s));
+    return launch_speed3r_routed(d, off, q, k, v, gates, idx, ofrc, lfrc, o_blk, l_blk, out, lse_or_null,
+                                 status_of(ws), s);
   }
 
   LSRM_TRY(launch_compress(d, off, nullptr, k, v, route_mode == LSRM_ROUTE_SCORE ? kc32 : nullptr, kc16, nullptr,

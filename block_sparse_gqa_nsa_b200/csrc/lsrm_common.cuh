@@ -19,7 +19,11 @@ __device__ __forceinline__ void raise_status(uint32_t* status, lsrm_status s) {
 
 // ---- workspace layout ----------------------------------------------------------------------------
 struct Workspace {
-  size_t status, kc32, vc32, kc16, vc16, qc32, qc16, centroids, idx, obranch, bwd, total;
+  size_t status, kc32, vc32, kc16, vc16, qc32, qc16, centroids, idx, obranch, bwd;
+  // pooled-query (Speed3R) path: forced-block bitmap, prefix and total, gathered forced K / V,
+  // and the forced part of the selected branch per token
+  size_t fbits, fpre, ftotal, kf, vf, ofrc, lfrc;
+  size_t total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -45,6 +49,15 @@ inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   w.obranch = o;   o = align256(o + (d.pooled_q ? B * Hq * (D + 1) * 4 : 0));
   // backward scratch: dKbar/dVbar fp32 [B][Hkv][d] x2, per-row D terms fp32 [N][Hq][3]
   w.bwd = o;       o = align256(o + (d.pooled_q ? 0 : (2 * B * Hkv * D * 4 + N * Hq * 3 * 4)));
+  const size_t nf = d.pooled_q ? (size_t)(d.n_forced > 0 ? d.n_forced : 0) : 0;
+  const size_t nf_tok = nf * (size_t)d.max_block_len;
+  w.fbits = o;     o = align256(o + (d.pooled_q ? (B / 32 + 2) * 4 : 0));
+  w.fpre = o;      o = align256(o + (d.pooled_q ? (nf + 1) * 4 : 0));
+  w.ftotal = o;    o = align256(o + (d.pooled_q ? 16 : 0));
+  w.kf = o;        o = align256(o + nf_tok * Hkv * D * 2);
+  w.vf = o;        o = align256(o + nf_tok * Hkv * D * 2);
+  w.ofrc = o;      o = align256(o + (d.pooled_q ? N * Hq * D * 4 : 0));
+  w.lfrc = o;      o = align256(o + (d.pooled_q ? N * Hq * 4 : 0));
   w.total = o;
   return w;
 }

@@ -287,3 +287,86 @@ def test_fused_forward_dense_equals_dense_gqa_sampled():
     idx = np.tile(np.arange(w.n_blocks, dtype=np.int32), (w.n_blocks, 1))
     ref = O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, qblocks=qb)
     assert_close(to_np(out)[rows_for(w.off, qb)], ref, "out")
+
+
+# ------------------------------------------------------------------------------------------------
+# S9 Speed3R pooled-query variant
+# ------------------------------------------------------------------------------------------------
+
+def check_pooled_routing(gpu_idx, w, qblocks, k):
+    """Validity of Speed3R routing: k distinct, non-forced blocks, each with an oracle pooled logit
+    within 1e-3 of the k-th best; where the oracle gap exceeds 1e-3 the sets must agree."""
+    D = oracle_desc(w, top_k=k)
+    qc = O.compress(D, w.off, w.q, w.n_q_heads)
+    kc = O.compress(D, w.off, w.k, w.n_kv_heads)
+    _, logits = O.route_pooled(D, qc, kc, w.forced, qblocks=qblocks, want_logits=True)
+    forced = set(w.forced.tolist())
+    for i, a in enumerate(qblocks):
+        for h in range(w.n_q_heads):
+            chosen = gpu_idx[a, h].tolist()
+            assert len(set(chosen)) == k and not (set(chosen) & forced), (a, h)
+            lg = logits[i, h].copy()
+            lg[list(forced)] = -np.inf
+            order = np.lexsort((np.arange(w.n_blocks), -lg))
+            sk = lg[order[k - 1]]
+            assert np.all(lg[chosen] >= sk - GAP), (a, h)
+            if k < len(order) and sk - lg[order[k]] > GAP:
+                assert set(chosen) == set(order[:k].tolist()), (a, h)
+
+
+@pytest.mark.parametrize("n_frames", [3, 6])
+def test_speed3r_forward_small(n_frames):
+    w = make_workload("speed3r_small", n_frames=n_frames)
+    c = DeviceCase(w)
+    idx = c.empty(w.n_blocks, w.n_q_heads, w.top_k, dtype=torch.int32)
+    out = c.empty(w.n_tokens, w.n_q_heads, w.head_dim, dtype=torch.bfloat16)
+    lse = c.empty(w.n_tokens, w.n_q_heads, 2)
+    nsa.lsrm_nsa_forward(c.desc, c.off, c.q, c.k, c.v, c.gates, None, nsa.ROUTE_SCORE, out, idx, lse, c.ws)
+    assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
+    gidx = to_np(idx)
+    check_pooled_routing(gidx, w, np.arange(w.n_blocks, dtype=np.int32), w.top_k)
+    D = oracle_desc(w)
+    ref, br, rl = O.forward(D, w.off, w.q, w.k, w.v, w.gates, gidx, forced=w.forced, want_branches=True)
+    assert_close(to_np(out), ref, "out")
+    assert np.abs(to_np(lse) - rl).max() < 2e-3
+    # one-hot gates: each branch on its own
+    for b in range(2):
+        g = np.zeros_like(w.gates)
+        g[..., b] = f32_to_bf16_bits(np.array([1.0], np.float32))[0]
+        nsa.lsrm_nsa_forward(c.desc, c.off, c.q, c.k, c.v, bf16_tensor(g), None, nsa.ROUTE_GIVEN, out, idx, None,
+                             c.ws)
+        assert_close(to_np(out), br[:, :, b], f"branch{b}")
+
+
+def test_speed3r_pooled_routing_and_compressed_branch_calls():
+    w = make_workload("speed3r_small", n_frames=5)
+    c = DeviceCase(w)
+    B, H, d = w.n_blocks, w.n_q_heads, w.head_dim
+    qc, kc, vc = (c.empty(B, H, d, dtype=torch.bfloat16) for _ in range(3))
+    nsa.lsrm_nsa_compress(c.desc, c.off, c.q, c.k, c.v, None, kc, None, vc, None, qc, ws=c.ws)
+    idx = c.empty(B, H, w.top_k, dtype=torch.int32)
+    nsa.lsrm_route_pooled_topk(c.desc, qc, kc, idx, c.ws)
+    check_pooled_routing(to_np(idx), w, np.arange(B, dtype=np.int32), w.top_k)
+    o, lse = c.empty(w.n_tokens, H, d), c.empty(w.n_tokens, H)
+    nsa.lsrm_nsa_cmp_attn(c.desc, c.off, qc, kc, vc, o, lse, c.ws)
+    D = oracle_desc(w)
+    ro, rl = O.cmp_attn(D, w.off, w.q, O.compress(D, w.off, w.k, H), O.compress(D, w.off, w.v, H),
+                        qc=O.compress(D, w.off, w.q, H))
+    assert_close(to_np(o), ro, "cmp")
+    assert np.abs(to_np(lse) - rl).max() < 2e-3
+    assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
+
+
+def test_speed3r_full_size_sampled():
+    w = make_workload("speed3r")
+    c = DeviceCase(w)
+    idx = c.empty(w.n_blocks, w.n_q_heads, w.top_k, dtype=torch.int32)
+    out = c.empty(w.n_tokens, w.n_q_heads, w.head_dim, dtype=torch.bfloat16)
+    nsa.lsrm_nsa_forward(c.desc, c.off, c.q, c.k, c.v, c.gates, None, nsa.ROUTE_SCORE, out, idx, None, c.ws)
+    assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
+    gidx = to_np(idx)
+    rng = np.random.default_rng(1)
+    qb = np.sort(np.r_[rng.choice(w.n_blocks, 3, replace=False), [0, 101, w.n_blocks - 1]]).astype(np.int32)
+    check_pooled_routing(gidx, w, qb, w.top_k)
+    ref = O.forward(oracle_desc(w), w.off, w.q, w.k, w.v, w.gates, gidx, forced=w.forced, qblocks=qb)
+    assert_close(to_np(out)[rows_for(w.off, qb)], ref, "out")
