@@ -1,0 +1,757 @@
+// S10 backward of the LSRM layer with the routing indices fixed.
+//
+// L = sum(out * dout) with out = sum_b g_b o_b (LSRM page, gate equations), o_b the softmax
+// attention of branch b (compressed block means, selected blocks, in-block window).  With the
+// forward's per-branch LSE, P_b = exp(tau q.k - lse_b) and, per branch:
+//   dgates_b = <dO, o_b>,  G_b = g_b dO,  Delta_b = <G_b, o_b> = g_b dgates_b,
+//   dS = P (G_b V^T - Delta_b),  dQ += tau dS K,  dK += tau dS^T Q,  dV += P^T G_b,
+// and the compressed keys/values are block means, so every token of block j receives
+// dKbar_j / n_j (and dVbar_j / n_j).
+//
+// Kernels (mma.sync m16n8k16 bf16 -> fp32; every sum in a fixed order, no float atomics):
+//   bwd_query:   one CTA per (query block, KV group, 128 rows): o_b recomputed -> dgates, Delta;
+//                then dQ from a second pass over each branch's keys.
+//   bwd_kv_local: one CTA per (key block, KV group): dK, dV of the block's tokens from the
+//                selected branch (query blocks that routed to it, in ascending order, from an
+//                inverse routing list) and from the window branch (its own block).
+//   bwd_kv_cmp:  one CTA per (64 block means, KV group, query split): partial dKbar, dVbar.
+//   bwd_finish:  dK = local part + (sum of the splits' dKbar of the token's block) / n_block.
+// The key-side passes compute S^T and dP^T (keys x query rows) directly, so P^T and dS^T are
+// already in the A-operand layout of the dV and dK products.
+#include "lsrm_common.cuh"
+
+namespace lsrm {
+
+constexpr int kBqThreads = 256;   // 8 warps x 16 query rows
+constexpr int kBkThreads = 128;   // 4 warps x 16 keys
+
+template <int D>
+__device__ __forceinline__ uint32_t bswz(int row, int ch) {
+  if (D == 32) return (uint32_t)(row * 64 + ((ch ^ ((row >> 1) & 3)) << 4));
+  return (uint32_t)(row * 128 + ((ch ^ (row & 7)) << 4));
+}
+
+struct BwdParams {
+  const int32_t* off;
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const uint16_t* kc;     // bf16 block means [B][Hkv][D]
+  const uint16_t* vc;
+  const uint16_t* gates;  // [N][Hq][NG]
+  const int32_t* idx;     // [B][idx_heads][top_k]
+  const float* lse;       // [N][Hq][NG] natural log
+  const uint16_t* dout;   // [N][Hq][D]
+  uint16_t* dq;
+  uint16_t* dgates;
+  float* delta;           // [N][Hq][NG]
+  float* dk_tok;          // [N][Hkv][D] selected + window part
+  float* dv_tok;
+  float* dkc_part;        // [splits][B][Hkv][D]
+  float* dvc_part;
+  const int* inv_start;   // [n_lists + 1]
+  const int* inv_list;    // query blocks routed to each key block, ascending per list
+  uint16_t* dk;
+  uint16_t* dv;
+  uint32_t* status;
+  long long N;
+  int B, Hq, Hkv, G, NG, top_k, idx_heads, window, n_lists;
+  float tau, scale_log2;
+};
+
+// ------------------------------------------------------------------------------------------------
+// query pass
+// ------------------------------------------------------------------------------------------------
+template <int D>
+struct BqSmem {
+  uint16_t q[128 * D];
+  uint16_t go[128 * D];   // dO rows
+  uint16_t kb[2][64 * D];
+  uint16_t vb[2][64 * D];
+  int32_t sel[256];
+  int32_t pre[257];
+  int32_t n_sel;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBqThreads) bwd_query_kernel(const BwdParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  BqSmem<D>& S = *reinterpret_cast<BqSmem<D>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int chunk_id = blockIdx.x, g = blockIdx.y, a = blockIdx.z;
+  const int t0 = p.off[a], n_a = p.off[a + 1] - t0;
+  const int rows_total = n_a * p.G;
+  const int row0 = chunk_id * 128;
+  if (row0 >= rows_total) return;
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  constexpr int KT = D / 16, NT = D / 8;
+
+  if (tid == 0) {
+    int n = 0, tot = 0;
+    const int32_t* r = p.idx + ((size_t)a * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.top_k;
+    for (int i = 0; i < p.top_k && n < 256; ++i) {
+      const int j = r[i];
+      if (j < 0 || j >= p.B) { raise_status(p.status, LSRM_ERR_BOUNDS); continue; }
+      S.sel[n] = j;
+      S.pre[n] = tot;
+      tot += p.off[j + 1] - p.off[j];
+      ++n;
+    }
+    S.pre[n] = tot;
+    S.n_sel = n;
+  }
+  for (int e = tid; e < 128 * CPR; e += kBqThreads) {
+    const int r = e / CPR, ch = e % CPR;
+    const int rr = row0 + r;
+    const bool ok = rr < rows_total;
+    const int t = t0 + (ok ? rr / p.G : 0), h = g * p.G + (ok ? rr % p.G : 0);
+    const size_t src = ((size_t)t * p.Hq + h) * D + ch * 8;
+    cp_async16(reinterpret_cast<unsigned char*>(S.q) + bswz<D>(r, ch), p.q + src, ok);
+    cp_async16(reinterpret_cast<unsigned char*>(S.go) + bswz<D>(r, ch), p.dout + src, ok);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  const int gq = lane >> 2, cq = lane & 3;
+  int tokl[2], head[2];
+  bool rvalid[2];
+  size_t orow[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int rr = row0 + warp * 16 + gq + 8 * i;
+    rvalid[i] = rr < rows_total;
+    tokl[i] = rvalid[i] ? rr / p.G : 0;
+    head[i] = g * p.G + (rvalid[i] ? rr % p.G : 0);
+    orow[i] = (size_t)(t0 + tokl[i]) * p.Hq + head[i];
+  }
+  uint32_t qa[KT][4], ga[KT][4];  // Q and dO A-fragments of the warp's 16 rows
+#pragma unroll
+  for (int kt = 0; kt < KT; ++kt) {
+    const int r = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int ch = kt * 2 + (lane >> 4);
+    ldmatrix_x4(qa[kt][0], qa[kt][1], qa[kt][2], qa[kt][3], smem_u32(S.q) + bswz<D>(r, ch));
+    ldmatrix_x4(ga[kt][0], ga[kt][1], ga[kt][2], ga[kt][3], smem_u32(S.go) + bswz<D>(r, ch));
+  }
+  const int n_sel_tok = S.pre[S.n_sel];
+  float dq[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dq[n][e] = 0.f;
+
+  for (int br = 0; br < p.NG; ++br) {
+    if (br == 2 && p.window <= 0) {
+      if (cq == 0)
+        for (int i = 0; i < 2; ++i)
+          if (rvalid[i]) {
+            p.dgates[orow[i] * p.NG + 2] = 0;
+            p.delta[orow[i] * p.NG + 2] = 0.f;
+          }
+      continue;
+    }
+    const int total = br == 0 ? p.B : (br == 1 ? n_sel_tok : n_a);
+    const int n_chunks = (total + 63) / 64;
+    float lse2[2], gate[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      lse2[i] = rvalid[i] ? p.lse[orow[i] * p.NG + br] * 1.4426950408889634f : 0.f;
+      gate[i] = rvalid[i] ? bf16_to_f32(p.gates[orow[i] * p.NG + br]) : 0.f;
+    }
+    // G_b = g_b * dO as A-fragments (rows gq and gq + 8 of the warp tile)
+    uint32_t gb[KT][4];
+#pragma unroll
+    for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float sc = gate[e & 1];
+        const uint32_t u = ga[kt][e];
+        gb[kt][e] = pack_bf16x2(__uint_as_float(u << 16) * sc, __uint_as_float(u & 0xFFFF0000u) * sc);
+      }
+    auto load_chunk = [&](int c, int buf) {
+      for (int e = tid; e < 64 * CPR; e += kBqThreads) {
+        const int kk = e / CPR, ch = e % CPR;
+        const int pos = c * 64 + kk;
+        const bool ok = pos < total;
+        const uint16_t *ks, *vs;
+        if (br == 0) {
+          const size_t base = ((size_t)(ok ? pos : 0) * p.Hkv + g) * D + ch * 8;
+          ks = p.kc + base;
+          vs = p.vc + base;
+        } else {
+          long long u = t0;
+          if (ok) {
+            if (br == 2) {
+              u = t0 + pos;
+            } else {
+              int lo = 0, hi = S.n_sel - 1;
+              while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (S.pre[mid] <= pos) lo = mid; else hi = mid - 1;
+              }
+              u = p.off[S.sel[lo]] + (pos - S.pre[lo]);
+            }
+          }
+          const size_t base = ((size_t)u * p.Hkv + g) * D + ch * 8;
+          ks = p.k + base;
+          vs = p.v + base;
+        }
+        cp_async16(reinterpret_cast<unsigned char*>(S.kb[buf]) + bswz<D>(kk, ch), ks, ok);
+        cp_async16(reinterpret_cast<unsigned char*>(S.vb[buf]) + bswz<D>(kk, ch), vs, ok);
+      }
+      cp_async_commit();
+    };
+    // S = Q K^T of the warp's rows against 64 keys; P = exp(S tau - lse) with masking
+    auto scores = [&](uint32_t sk, int c, float (&s)[8][4]) {
+#pragma unroll
+      for (int n = 0; n < 8; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
+#pragma unroll
+      for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t b0, b1, b2, b3;
+          const int key = np * 16 + (lane >> 4) * 8 + (lane & 7);
+          const int ch = kt * 2 + ((lane >> 3) & 1);
+          ldmatrix_x4(b0, b1, b2, b3, sk + bswz<D>(key, ch));
+          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+          mma_bf16_16816(s[2 * np], qa[kt], bb0);
+          mma_bf16_16816(s[2 * np + 1], qa[kt], bb1);
+        }
+#pragma unroll
+      for (int n = 0; n < 8; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = e >> 1;
+          const int key = n * 8 + 2 * cq + (e & 1);
+          const int pos = c * 64 + key;
+          bool ok = pos < total && rvalid[i];
+          if (br == 2) ok = ok && pos >= tokl[i] - p.window / 2 && pos <= tokl[i] + p.window / 2 - 1;
+          s[n][e] = ok ? fast_exp2(s[n][e] * p.scale_log2 - lse2[i]) : 0.f;
+        }
+    };
+    // ---- pass A: o_b = P V ----
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
+    if (n_chunks > 0) load_chunk(0, 0);
+    for (int c = 0; c < n_chunks; ++c) {
+      const int buf = c & 1;
+      if (c + 1 < n_chunks) { load_chunk(c + 1, buf ^ 1); cp_async_wait<1>(); } else { cp_async_wait<0>(); }
+      __syncthreads();
+      float s[8][4];
+      scores(smem_u32(S.kb[buf]), c, s);
+      uint32_t pa[4][4];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(s[n][0], s[n][1]);
+        pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(s[n][2], s[n][3]);
+      }
+      const uint32_t sv = smem_u32(S.vb[buf]);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int dn = 0; dn < D / 16; ++dn) {
+          uint32_t b0, b1, b2, b3;
+          const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+          const int ch = dn * 2 + (lane >> 4);
+          ldmatrix_x4_trans(b0, b1, b2, b3, sv + bswz<D>(key, ch));
+          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+          mma_bf16_16816(o[2 * dn], pa[kk], bb0);
+          mma_bf16_16816(o[2 * dn + 1], pa[kk], bb1);
+        }
+      __syncthreads();
+    }
+    // dgates_b = <dO, o_b>, Delta_b = g_b dgates_b (dO read back from shared memory)
+    float dg[2] = {0.f, 0.f};
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = warp * 16 + gq + 8 * i, col = n * 8 + 2 * cq;
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const unsigned char*>(S.go) +
+                                                              bswz<D>(r, col / 8) + (col % 8) * 2);
+        dg[i] += __uint_as_float(u << 16) * o[n][2 * i] + __uint_as_float(u & 0xFFFF0000u) * o[n][2 * i + 1];
+      }
+    float dlt[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      dg[i] += __shfl_xor_sync(0xffffffffu, dg[i], 1);
+      dg[i] += __shfl_xor_sync(0xffffffffu, dg[i], 2);
+      dlt[i] = gate[i] * dg[i];
+      if (rvalid[i] && cq == 0) {
+        p.dgates[orow[i] * p.NG + br] = __bfloat16_as_ushort(__float2bfloat16_rn(dg[i]));
+        p.delta[orow[i] * p.NG + br] = dlt[i];
+      }
+    }
+    // ---- pass B: dS = P (G_b V^T - Delta), dQ += tau dS K ----
+    if (n_chunks > 0) load_chunk(0, 0);
+    for (int c = 0; c < n_chunks; ++c) {
+      const int buf = c & 1;
+      if (c + 1 < n_chunks) { load_chunk(c + 1, buf ^ 1); cp_async_wait<1>(); } else { cp_async_wait<0>(); }
+      __syncthreads();
+      float s[8][4];
+      scores(smem_u32(S.kb[buf]), c, s);
+      float dp[8][4];
+#pragma unroll
+      for (int n = 0; n < 8; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dp[n][e] = 0.f;
+      const uint32_t sv = smem_u32(S.vb[buf]);
+#pragma unroll
+      for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t b0, b1, b2, b3;
+          const int key = np * 16 + (lane >> 4) * 8 + (lane & 7);
+          const int ch = kt * 2 + ((lane >> 3) & 1);
+          ldmatrix_x4(b0, b1, b2, b3, sv + bswz<D>(key, ch));
+          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+          mma_bf16_16816(dp[2 * np], gb[kt], bb0);
+          mma_bf16_16816(dp[2 * np + 1], gb[kt], bb1);
+        }
+      uint32_t da[4][4];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        float ds[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ds[e] = s[n][e] * (dp[n][e] - dlt[e >> 1]);
+        da[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(ds[0], ds[1]);
+        da[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+      }
+      const uint32_t sk = smem_u32(S.kb[buf]);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int dn = 0; dn < D / 16; ++dn) {
+          uint32_t b0, b1, b2, b3;
+          const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+          const int ch = dn * 2 + (lane >> 4);
+          ldmatrix_x4_trans(b0, b1, b2, b3, sk + bswz<D>(key, ch));
+          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
+          mma_bf16_16816(dq[2 * dn], da[kk], bb0);
+          mma_bf16_16816(dq[2 * dn + 1], da[kk], bb1);
+        }
+      __syncthreads();
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+      if (rvalid[i])
+        *reinterpret_cast<uint32_t*>(p.dq + orow[i] * D + n * 8 + 2 * cq) =
+            pack_bf16x2(p.tau * dq[n][2 * i], p.tau * dq[n][2 * i + 1]);
+}
+
+// ------------------------------------------------------------------------------------------------
+// key passes: S^T = K Q^T, dP^T = V G^T for 64 keys (4 warps x 16) against query rows staged
+// 64 at a time and consumed in 16-row sub-tiles
+// ------------------------------------------------------------------------------------------------
+constexpr int kBkRows = 64;
+
+template <int D>
+struct BkSmem {
+  uint16_t kt[64 * D];
+  uint16_t vt[64 * D];
+  uint16_t q[kBkRows * D];
+  uint16_t g[kBkRows * D];  // G_b = g_b dO rows
+  float lse2[kBkRows];      // log2-unit LSE of the rows
+  float dlt[kBkRows];
+  int tok[kBkRows];         // query token position inside its block (window mask), -1 = invalid row
+};
+
+// A fragments of the warp's 16 keys (K and V)
+template <int D>
+__device__ __forceinline__ void bk_key_frags(const BkSmem<D>& S, int warp, int lane, uint32_t (&ka)[D / 16][4],
+                                             uint32_t (&va)[D / 16][4]) {
+#pragma unroll
+  for (int kt = 0; kt < D / 16; ++kt) {
+    const int r = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int ch = kt * 2 + (lane >> 4);
+    ldmatrix_x4(ka[kt][0], ka[kt][1], ka[kt][2], ka[kt][3], smem_u32(S.kt) + bswz<D>(r, ch));
+    ldmatrix_x4(va[kt][0], va[kt][1], va[kt][2], va[kt][3], smem_u32(S.vt) + bswz<D>(r, ch));
+  }
+}
+
+// accumulate the staged rows [sub*16, sub*16+16) into the warp's dK / dV (16 keys x D)
+template <int D, bool kWindow>
+__device__ __forceinline__ void bk_tile(const BkSmem<D>& S, int sub, int lane, int key_valid, const int (&key_pos)[2],
+                                        int window, float scale_log2, const uint32_t (&ka)[D / 16][4],
+                                        const uint32_t (&va)[D / 16][4], float (&dk)[D / 8][4],
+                                        float (&dv)[D / 8][4]) {
+  constexpr int KT = D / 16;
+  const int gq = lane >> 2, cq = lane & 3;
+  const int rb = sub * 16;
+  float st[2][4], dpt[2][4];  // [row n-tile][frag]: rows = keys gq, gq+8; cols = query rows 8 n + 2 cq (+1)
+#pragma unroll
+  for (int n = 0; n < 2; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) { st[n][e] = 0.f; dpt[n][e] = 0.f; }
+#pragma unroll
+  for (int kt = 0; kt < KT; ++kt) {
+    uint32_t b0, b1, b2, b3;
+    const int r = rb + (lane >> 4) * 8 + (lane & 7);
+    const int ch = kt * 2 + ((lane >> 3) & 1);
+    ldmatrix_x4(b0, b1, b2, b3, smem_u32(S.q) + bswz<D>(r, ch));
+    const uint32_t q0[2] = {b0, b1}, q1[2] = {b2, b3};
+    mma_bf16_16816(st[0], ka[kt], q0);
+    mma_bf16_16816(st[1], ka[kt], q1);
+    ldmatrix_x4(b0, b1, b2, b3, smem_u32(S.g) + bswz<D>(r, ch));
+    const uint32_t g0[2] = {b0, b1}, g1[2] = {b2, b3};
+    mma_bf16_16816(dpt[0], va[kt], g0);
+    mma_bf16_16816(dpt[1], va[kt], g1);
+  }
+  // P^T and dS^T (keys x rows), masked
+  uint32_t pa[4], da[4];
+#pragma unroll
+  for (int n = 0; n < 2; ++n) {
+    float pv[4], dv4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int krow = gq + 8 * (e >> 1);             // key of the warp tile
+      const int qrow = rb + n * 8 + 2 * cq + (e & 1);  // staged query row
+      const int r = S.tok[qrow];
+      bool ok = krow < key_valid && r >= 0;
+      if (kWindow) {
+        const int u = key_pos[e >> 1];
+        ok = ok && u >= r - window / 2 && u <= r + window / 2 - 1;
+      }
+      const float pp = ok ? fast_exp2(st[n][e] * scale_log2 - S.lse2[qrow]) : 0.f;
+      pv[e] = pp;
+      dv4[e] = pp * (dpt[n][e] - S.dlt[qrow]);
+    }
+    pa[n * 2 + 0] = pack_bf16x2(pv[0], pv[1]);
+    pa[n * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+    da[n * 2 + 0] = pack_bf16x2(dv4[0], dv4[1]);
+    da[n * 2 + 1] = pack_bf16x2(dv4[2], dv4[3]);
+  }
+  // dV += P^T G, dK += dS^T Q (B operands: staged rows of G / Q, transposed loads)
+#pragma unroll
+  for (int dn = 0; dn < D / 16; ++dn) {
+    uint32_t b0, b1, b2, b3;
+    const int r = rb + ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int ch = dn * 2 + (lane >> 4);
+    ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(S.g) + bswz<D>(r, ch));
+    const uint32_t g0[2] = {b0, b1}, g1[2] = {b2, b3};
+    mma_bf16_16816(dv[2 * dn], pa, g0);
+    mma_bf16_16816(dv[2 * dn + 1], pa, g1);
+    ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(S.q) + bswz<D>(r, ch));
+    const uint32_t q0[2] = {b0, b1}, q1[2] = {b2, b3};
+    mma_bf16_16816(dk[2 * dn], da, q0);
+    mma_bf16_16816(dk[2 * dn + 1], da, q1);
+  }
+}
+
+// stage kBkRows query rows (row0.. of the token range starting at t_base) of group g for branch br;
+// G_b = g_b dO is formed here, rounded to bf16
+template <int D>
+__device__ __forceinline__ void bk_stage_rows(BkSmem<D>& S, const BwdParams& p, int g, int br, int row0,
+                                              int rows_total, long long t_base, int tid) {
+  constexpr int CPR = D / 8;
+  for (int e = tid; e < kBkRows * CPR; e += kBkThreads) {
+    const int r = e / CPR, ch = e % CPR;
+    const int rr = row0 + r;
+    const bool ok = rr < rows_total;
+    const long long t = t_base + (ok ? rr / p.G : 0);
+    const int h = g * p.G + (ok ? rr % p.G : 0);
+    const size_t src = ((size_t)t * p.Hq + h) * D + ch * 8;
+    cp_async16(reinterpret_cast<unsigned char*>(S.q) + bswz<D>(r, ch), p.q + src, ok);
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (ok) {
+      const float gt = bf16_to_f32(p.gates[((size_t)t * p.Hq + h) * p.NG + br]);
+      const uint4 dd = *reinterpret_cast<const uint4*>(p.dout + src);
+      const uint32_t w[4] = {dd.x, dd.y, dd.z, dd.w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o4[i] = pack_bf16x2(__uint_as_float(w[i] << 16) * gt, __uint_as_float(w[i] & 0xFFFF0000u) * gt);
+      u = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.g) + bswz<D>(r, ch)) = u;
+  }
+  for (int r = tid; r < kBkRows; r += kBkThreads) {
+    const int rr = row0 + r;
+    if (rr < rows_total) {
+      const long long t = t_base + rr / p.G;
+      const int h = g * p.G + rr % p.G;
+      const size_t row = (size_t)t * p.Hq + h;
+      S.lse2[r] = p.lse[row * p.NG + br] * 1.4426950408889634f;
+      S.dlt[r] = p.delta[row * p.NG + br];
+      S.tok[r] = rr / p.G;
+    } else {
+      S.lse2[r] = 0.f;
+      S.dlt[r] = 0.f;
+      S.tok[r] = -1;
+    }
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+}
+
+template <int D>
+__device__ __forceinline__ void bk_load_keys(BkSmem<D>& S, const uint16_t* k, const uint16_t* v, long long first,
+                                             int n_keys, int Hkv, int g, int tid) {
+  constexpr int CPR = D / 8;
+  for (int e = tid; e < 64 * CPR; e += kBkThreads) {
+    const int r = e / CPR, ch = e % CPR;
+    const bool ok = r < n_keys;
+    const size_t src = ((size_t)(first + (ok ? r : 0)) * Hkv + g) * D + ch * 8;
+    cp_async16(reinterpret_cast<unsigned char*>(S.kt) + bswz<D>(r, ch), k + src, ok);
+    cp_async16(reinterpret_cast<unsigned char*>(S.vt) + bswz<D>(r, ch), v + src, ok);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+}
+
+// store the warp's 16 rows of dK (scaled by tau) and dV as fp32 into [row][Hkv][D] at dst_row0
+template <int D>
+__device__ __forceinline__ void bk_store(float* dkp, float* dvp, size_t dst_row0, int n_keys, int warp, int lane,
+                                         int Hkv, int g, float tau, const float (&dk)[D / 8][4],
+                                         const float (&dv)[D / 8][4]) {
+  const int gq = lane >> 2, cq = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int kr = warp * 16 + gq + 8 * i;
+    if (kr >= n_keys) continue;
+    const size_t row = ((dst_row0 + kr) * Hkv + g) * D;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      *reinterpret_cast<float2*>(dkp + row + n * 8 + 2 * cq) = make_float2(tau * dk[n][2 * i], tau * dk[n][2 * i + 1]);
+      *reinterpret_cast<float2*>(dvp + row + n * 8 + 2 * cq) = make_float2(dv[n][2 * i], dv[n][2 * i + 1]);
+    }
+  }
+}
+
+// selected + window parts of dK, dV for the tokens of key block j, group g
+template <int D>
+__global__ void __launch_bounds__(kBkThreads) bwd_kv_local_kernel(const BwdParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  BkSmem<D>& S = *reinterpret_cast<BkSmem<D>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j = blockIdx.x, g = blockIdx.y;
+  const int u0 = p.off[j], n_j = min(64, p.off[j + 1] - u0);
+  bk_load_keys<D>(S, p.k, p.v, u0, n_j, p.Hkv, g, tid);
+  __syncthreads();
+  uint32_t ka[D / 16][4], va[D / 16][4];
+  bk_key_frags<D>(S, warp, lane, ka, va);
+  const int key_valid = n_j - warp * 16;  // valid keys among this warp's 16
+  const int gq = lane >> 2;
+  const int key_pos[2] = {warp * 16 + gq, warp * 16 + gq + 8};
+  float dk[D / 8][4], dv[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) { dk[n][e] = 0.f; dv[n][e] = 0.f; }
+  // selected branch: every query block whose routed set contains j, in ascending order; the
+  // last pass is the window branch of block j itself
+  const int list = p.idx_heads == 1 ? j : j * p.Hkv + g;
+  const int l0 = p.inv_start[list], l1 = p.inv_start[list + 1];
+  const int l_end = p.window > 0 ? l1 + 1 : l1;
+  for (int li = l0; li < l_end; ++li) {
+    const bool window = li == l1;
+    const int a = window ? j : p.inv_list[li];
+    const int br = window ? 2 : 1;
+    const int t_base = p.off[a], rows_total = (p.off[a + 1] - t_base) * p.G;
+    for (int row0 = 0; row0 < rows_total; row0 += kBkRows) {
+      __syncthreads();
+      bk_stage_rows<D>(S, p, g, br, row0, rows_total, t_base, tid);
+      __syncthreads();
+      const int subs = min(4, (rows_total - row0 + 15) / 16);
+      for (int sub = 0; sub < subs; ++sub) {
+        if (window)
+          bk_tile<D, true>(S, sub, lane, key_valid, key_pos, p.window, p.scale_log2, ka, va, dk, dv);
+        else
+          bk_tile<D, false>(S, sub, lane, key_valid, key_pos, p.window, p.scale_log2, ka, va, dk, dv);
+      }
+    }
+  }
+  bk_store<D>(p.dk_tok, p.dv_tok, (size_t)u0, n_j, warp, lane, p.Hkv, g, p.tau, dk, dv);
+}
+
+// compressed part: partial dKbar / dVbar of 64 block means of group g over one split of the query tokens
+template <int D>
+__global__ void __launch_bounds__(kBkThreads) bwd_kv_cmp_kernel(const BwdParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  BkSmem<D>& S = *reinterpret_cast<BkSmem<D>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int jc = blockIdx.x, g = blockIdx.y, split = blockIdx.z;
+  const int j0 = jc * 64, n_j = min(64, p.B - j0);
+  bk_load_keys<D>(S, p.kc, p.vc, j0, n_j, p.Hkv, g, tid);
+  __syncthreads();
+  uint32_t ka[D / 16][4], va[D / 16][4];
+  bk_key_frags<D>(S, warp, lane, ka, va);
+  const int key_valid = n_j - warp * 16;
+  const int key_pos[2] = {0, 0};
+  float dk[D / 8][4], dv[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) { dk[n][e] = 0.f; dv[n][e] = 0.f; }
+  // this split's query tokens (all heads of group g), rows token-major with G rows per token
+  const long long t_lo = p.N * split / kBwdSplits, t_hi = p.N * (split + 1) / kBwdSplits;
+  const int rows_total = (int)((t_hi - t_lo) * p.G);
+  for (int row0 = 0; row0 < rows_total; row0 += kBkRows) {
+    __syncthreads();
+    bk_stage_rows<D>(S, p, g, 0, row0, rows_total, t_lo, tid);
+    __syncthreads();
+    const int subs = min(4, (rows_total - row0 + 15) / 16);
+    for (int sub = 0; sub < subs; ++sub)
+      bk_tile<D, false>(S, sub, lane, key_valid, key_pos, 0, p.scale_log2, ka, va, dk, dv);
+  }
+  bk_store<D>(p.dkc_part, p.dvc_part, (size_t)split * p.B + j0, n_j, warp, lane, p.Hkv, g, p.tau, dk, dv);
+}
+
+// dK = local part + (sum over splits of dKbar of the token's block) / n_block, as bf16
+__global__ void bwd_finish_kernel(const BwdParams p, int D) {
+  const int b = blockIdx.x;
+  const int u0 = p.off[b], n = p.off[b + 1] - u0;
+  const int HD = p.Hkv * D;
+  const float inv = n > 0 ? 1.f / (float)n : 0.f;
+  for (int e = threadIdx.x; e < HD; e += blockDim.x) {
+    float sk = 0.f, sv = 0.f;
+    for (int s = 0; s < kBwdSplits; ++s) {
+      sk += p.dkc_part[((size_t)s * p.B + b) * HD + e];
+      sv += p.dvc_part[((size_t)s * p.B + b) * HD + e];
+    }
+    for (int r = 0; r < n; ++r) {
+      const size_t i = (size_t)(u0 + r) * HD + e;
+      p.dk[i] = __bfloat16_as_ushort(__float2bfloat16_rn(p.dk_tok[i] + sk * inv));
+      p.dv[i] = __bfloat16_as_ushort(__float2bfloat16_rn(p.dv_tok[i] + sv * inv));
+    }
+  }
+}
+
+// ---- inverse routing lists: for each key block (and group), the query blocks that selected it ----
+__global__ void inv_count_kernel(const int32_t* __restrict__ idx, int B, int ih, int k, int* count,
+                                 uint32_t* status) {
+  const long long n = (long long)B * ih * k;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const int gg = (int)((e / k) % ih);
+    const int j = idx[e];
+    if (j < 0 || j >= B) { raise_status(status, LSRM_ERR_BOUNDS); continue; }
+    atomicAdd(count + (size_t)j * ih + gg, 1);
+  }
+}
+// exclusive scan of the list counts by one CTA of kScanThreads: each thread scans a contiguous
+// slice, the slice totals are scanned in shared memory, then every slice is written
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) inv_scan_kernel(const int* count, int n, int* start) {
+  __shared__ int part[kScanThreads];
+  const int per = (n + kScanThreads - 1) / kScanThreads;
+  const int lo = min(n, threadIdx.x * per), hi = min(n, lo + per);
+  int s = 0;
+  for (int i = lo; i < hi; ++i) s += count[i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int i = 0; i < kScanThreads; ++i) { const int c = part[i]; part[i] = acc; acc += c; }
+    start[n] = acc;
+  }
+  __syncthreads();
+  int acc = part[threadIdx.x];
+  for (int i = lo; i < hi; ++i) { start[i] = acc; acc += count[i]; }
+}
+__global__ void inv_fill_kernel(const int32_t* __restrict__ idx, int B, int ih, int k, const int* start,
+                                int* cursor, int* list) {
+  const long long n = (long long)B * ih * k;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const int a = (int)(e / ((long long)ih * k)), gg = (int)((e / k) % ih);
+    const int j = idx[e];
+    if (j < 0 || j >= B) continue;
+    const int li = j * ih + gg;
+    list[start[li] + atomicAdd(cursor + li, 1)] = a;
+  }
+}
+// sort every list ascending (fixed summation order); lists are short, insertion sort per thread
+__global__ void inv_sort_kernel(const int* start, int n_lists, int* list) {
+  for (int li = blockIdx.x * blockDim.x + threadIdx.x; li < n_lists; li += gridDim.x * blockDim.x) {
+    const int s = start[li], e = start[li + 1];
+    for (int i = s + 1; i < e; ++i) {
+      const int x = list[i];
+      int j = i - 1;
+      while (j >= s && list[j] > x) { list[j + 1] = list[j]; --j; }
+      list[j + 1] = x;
+    }
+  }
+}
+
+template <int D>
+static lsrm_status launch_backward_d(const lsrm_nsa_desc& d, const BwdParams& p, int idx_heads, cudaStream_t s) {
+  const int G = p.G;
+  const int chunks = (d.max_block_len * G + 127) / 128;
+  size_t sm = sizeof(BqSmem<D>);
+  if (cudaFuncSetAttribute(bwd_query_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+    return LSRM_ERR_CUDA;
+  bwd_query_kernel<D><<<dim3(chunks, d.n_kv_heads, d.n_blocks), kBqThreads, sm, s>>>(p);
+  sm = sizeof(BkSmem<D>);
+  bwd_kv_local_kernel<D><<<dim3(d.n_blocks, d.n_kv_heads), kBkThreads, sm, s>>>(p);
+  bwd_kv_cmp_kernel<D><<<dim3((d.n_blocks + 63) / 64, d.n_kv_heads, kBwdSplits), kBkThreads, sm, s>>>(p);
+  bwd_finish_kernel<<<d.n_blocks, 256, 0, s>>>(p, D);
+  (void)idx_heads;
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
+lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
+                            const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
+                            unsigned char* ws_bwd, uint32_t* status, cudaStream_t s) {
+  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.n_blocks > 65535) return LSRM_ERR_UNSUPPORTED;
+  const BwdWs w = bwd_layout(d, idx_heads);
+  BwdParams p{};
+  p.off = off;
+  p.q = (const uint16_t*)q;
+  p.k = (const uint16_t*)k;
+  p.v = (const uint16_t*)v;
+  p.kc = (const uint16_t*)kc;
+  p.vc = (const uint16_t*)vc;
+  p.gates = (const uint16_t*)gates;
+  p.idx = idx;
+  p.lse = lse;
+  p.dout = (const uint16_t*)dout;
+  p.dq = (uint16_t*)dq;
+  p.dgates = (uint16_t*)dgates;
+  p.delta = reinterpret_cast<float*>(ws_bwd + w.delta);
+  p.dk_tok = reinterpret_cast<float*>(ws_bwd + w.dk_tok);
+  p.dv_tok = reinterpret_cast<float*>(ws_bwd + w.dv_tok);
+  p.dkc_part = reinterpret_cast<float*>(ws_bwd + w.dkc);
+  p.dvc_part = reinterpret_cast<float*>(ws_bwd + w.dvc);
+  p.inv_start = reinterpret_cast<const int*>(ws_bwd + w.inv_start);
+  p.inv_list = reinterpret_cast<const int*>(ws_bwd + w.inv_list);
+  p.dk = (uint16_t*)dk;
+  p.dv = (uint16_t*)dv;
+  p.status = status;
+  p.N = d.n_tokens;
+  p.B = d.n_blocks;
+  p.Hq = d.n_q_heads;
+  p.Hkv = d.n_kv_heads;
+  p.G = d.n_q_heads / d.n_kv_heads;
+  p.NG = d.n_gates;
+  p.top_k = d.top_k;
+  p.idx_heads = idx_heads;
+  p.window = d.n_gates == 3 ? d.window : 0;
+  p.n_lists = d.n_blocks * idx_heads;
+  p.tau = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim);
+  p.scale_log2 = p.tau * 1.4426950408889634f;
+  // inverse routing lists
+  int* count = reinterpret_cast<int*>(ws_bwd + w.inv_count);
+  int* cursor = reinterpret_cast<int*>(ws_bwd + w.inv_cursor);
+  int* start = reinterpret_cast<int*>(ws_bwd + w.inv_start);
+  int* list = reinterpret_cast<int*>(ws_bwd + w.inv_list);
+  if (cudaMemsetAsync(count, 0, (size_t)p.n_lists * 4, s) != cudaSuccess) return LSRM_ERR_CUDA;
+  if (cudaMemsetAsync(cursor, 0, (size_t)p.n_lists * 4, s) != cudaSuccess) return LSRM_ERR_CUDA;
+  const int grid = 148 * 4;
+  inv_count_kernel<<<grid, 256, 0, s>>>(idx, d.n_blocks, idx_heads, d.top_k, count, status);
+  inv_scan_kernel<<<1, kScanThreads, 0, s>>>(count, p.n_lists, start);
+  inv_fill_kernel<<<grid, 256, 0, s>>>(idx, d.n_blocks, idx_heads, d.top_k, start, cursor, list);
+  inv_sort_kernel<<<(p.n_lists + 127) / 128, 128, 0, s>>>(start, p.n_lists, list);
+  if (d.head_dim == 32) return launch_backward_d<32>(d, p, idx_heads, s);
+  if (d.head_dim == 64) return launch_backward_d<64>(d, p, idx_heads, s);
+  return LSRM_ERR_UNSUPPORTED;
+}
+
+}  // namespace lsrm

@@ -28,6 +28,31 @@ struct Workspace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// backward scratch (inside the workspace's backward region): per-row Delta terms, fp32 selected +
+// window parts of dK / dV, per-split compressed-branch partials, and the inverse routing lists
+constexpr int kBwdSplits = 32;  // query splits of the compressed-key pass
+struct BwdWs {
+  size_t delta, dk_tok, dv_tok, dkc, dvc, inv_count, inv_cursor, inv_start, inv_list, total;
+};
+inline BwdWs bwd_layout(const lsrm_nsa_desc& d, int idx_heads) {
+  BwdWs w{};
+  size_t o = 0;
+  const size_t N = (size_t)d.n_tokens, B = (size_t)d.n_blocks, Hq = (size_t)d.n_q_heads, Hkv = (size_t)d.n_kv_heads;
+  const size_t D = (size_t)d.head_dim, nl = B * (size_t)idx_heads, NG = (size_t)(d.n_gates > 0 ? d.n_gates : 0);
+  const size_t K = (size_t)(d.top_k > 0 ? d.top_k : 0);
+  w.delta = o;      o = align256(o + N * Hq * NG * 4);
+  w.dk_tok = o;     o = align256(o + N * Hkv * D * 4);
+  w.dv_tok = o;     o = align256(o + N * Hkv * D * 4);
+  w.dkc = o;        o = align256(o + (size_t)kBwdSplits * B * Hkv * D * 4);
+  w.dvc = o;        o = align256(o + (size_t)kBwdSplits * B * Hkv * D * 4);
+  w.inv_count = o;  o = align256(o + nl * 4);
+  w.inv_cursor = o; o = align256(o + nl * 4);
+  w.inv_start = o;  o = align256(o + (nl + 1) * 4);
+  w.inv_list = o;   o = align256(o + nl * K * 4);
+  w.total = o;
+  return w;
+}
+
 inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   Workspace w{};
   size_t o = 0;
@@ -47,8 +72,8 @@ inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   w.idx = o;       o = align256(o + B * ih * (size_t)(d.top_k > 0 ? d.top_k : 1) * 4);
   // pooled compressed-branch output [B][Hq][d] fp32 (Speed3R) + its LSE [B][Hq]
   w.obranch = o;   o = align256(o + (d.pooled_q ? B * Hq * (D + 1) * 4 : 0));
-  // backward scratch: dKbar/dVbar fp32 [B][Hkv][d] x2, per-row D terms fp32 [N][Hq][3]
-  w.bwd = o;       o = align256(o + (d.pooled_q ? 0 : (2 * B * Hkv * D * 4 + N * Hq * 3 * 4)));
+  // backward scratch, sized for per-group routing lists (the larger case)
+  w.bwd = o;       o = align256(o + (d.pooled_q ? 0 : bwd_layout(d, d.n_kv_heads > 0 ? d.n_kv_heads : 1).total));
   const size_t nf = d.pooled_q ? (size_t)(d.n_forced > 0 ? d.n_forced : 0) : 0;
   const size_t nf_tok = nf * (size_t)d.max_block_len;
   w.fbits = o;     o = align256(o + (d.pooled_q ? (B / 32 + 2) * 4 : 0));

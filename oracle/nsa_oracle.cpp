@@ -406,10 +406,14 @@ int impl_forward(const Desc* D, const int32_t* off, const T* q, const T* k, cons
 // Outputs cover all tokens: dq [N][Hq][d], dk, dv [N][Hkv][d], dgates [N][Hq][n_gates].
 // nthreads > 1 splits the query blocks across threads; each thread keeps its own
 // key-side accumulators, which are summed in thread order.
+// With a query-block list (n_qb, qblocks), only those query blocks contribute: dq and dgates of
+// their rows are the full gradients, dk and dv hold the listed blocks' contributions alone, and
+// the other rows of dq and dgates are left untouched.
 template <typename T>
 int impl_backward(const Desc* D, const int32_t* off, const T* q, const T* k, const T* v,
                     const T* gates, const int32_t* idx, int32_t idx_heads, const T* dout,
-                    double* dq, double* dk, double* dv, double* dgates, int32_t nthreads) {
+                    double* dq, double* dk, double* dv, double* dgates, int32_t n_qb,
+                    const int32_t* qblocks, int32_t nthreads) {
   if (D->pooled_q) return 1;
   const int32_t B = D->n_blocks, Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim, NG = D->n_gates;
   const int32_t G = Hq / Hkv, K = D->top_k, w = D->window;
@@ -428,7 +432,9 @@ int impl_backward(const Desc* D, const int32_t* off, const T* q, const T* k, con
   auto work = [&](int tid) {
     std::vector<double> qv((size_t)d), go((size_t)d), ob((size_t)d), dqv((size_t)d);
     std::vector<double> s, p;
-    for (int32_t a = tid; a < B; a += nthreads) {
+    const int32_t nq = qblocks ? n_qb : B;
+    for (int32_t qi = tid; qi < nq; qi += nthreads) {
+      const int32_t a = qblocks ? qblocks[qi] : qi;
       // per group: token ids of the selected set
       std::vector<std::vector<int64_t>> sel((size_t)Hkv);
       for (int32_t g = 0; g < Hkv; ++g) {
@@ -618,13 +624,17 @@ int oracle_forward_f64(const Desc* D, const int32_t* off, const double* q, const
 }
 int oracle_backward(const Desc* D, const int32_t* off, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     const uint16_t* gates, const int32_t* idx, int32_t idx_heads, const uint16_t* dout, double* dq,
-                    double* dk, double* dv, double* dgates, int32_t nthreads) {
-  return impl_backward<uint16_t>(D, off, q, k, v, gates, idx, idx_heads, dout, dq, dk, dv, dgates, nthreads);
+                    double* dk, double* dv, double* dgates, int32_t n_qb, const int32_t* qblocks,
+                    int32_t nthreads) {
+  return impl_backward<uint16_t>(D, off, q, k, v, gates, idx, idx_heads, dout, dq, dk, dv, dgates, n_qb, qblocks,
+                                 nthreads);
 }
 int oracle_backward_f64(const Desc* D, const int32_t* off, const double* q, const double* k, const double* v,
                         const double* gates, const int32_t* idx, int32_t idx_heads, const double* dout, double* dq,
-                        double* dk, double* dv, double* dgates, int32_t nthreads) {
-  return impl_backward<double>(D, off, q, k, v, gates, idx, idx_heads, dout, dq, dk, dv, dgates, nthreads);
+                        double* dk, double* dv, double* dgates, int32_t n_qb, const int32_t* qblocks,
+                        int32_t nthreads) {
+  return impl_backward<double>(D, off, q, k, v, gates, idx, idx_heads, dout, dq, dk, dv, dgates, n_qb, qblocks,
+                               nthreads);
 }
 double oracle_loss_f64(const Desc* D, const int32_t* off, const double* q, const double* k, const double* v,
                        const double* gates, const int32_t* idx, int32_t idx_heads, const double* dout) {

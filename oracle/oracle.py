@@ -62,8 +62,8 @@ def _L():
             "oracle_window_attn": [P, vp, vp, vp, vp, i32, vp, vp, vp],
             "oracle_forward": [P, vp, vp, vp, vp, vp, vp, i32, i32, vp, i32, vp, vp, vp, vp],
             "oracle_forward_f64": [P, vp, vp, vp, vp, vp, vp, i32, i32, vp, i32, vp, vp, vp, vp],
-            "oracle_backward": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32],
-            "oracle_backward_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32],
+            "oracle_backward": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, vp, i32],
+            "oracle_backward_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, vp, i32],
             "oracle_loss_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp],
         }
         for name, args in sig.items():
@@ -208,7 +208,7 @@ def forward_f64(D, off, q, k, v, gates, idx, forced=None, qblocks=None, want_bra
                     want_branches)
 
 
-def _backward(fn, dtype, D, off, q, k, v, gates, idx, dout, nthreads):
+def _backward(fn, dtype, D, off, q, k, v, gates, idx, dout, nthreads, qblocks=None):
     off = _c(off, np.int32)
     q, k, v, gates, dout = _inputs(dtype, q, k, v, gates, dout)
     idx = _c(idx, np.int32)
@@ -218,20 +218,24 @@ def _backward(fn, dtype, D, off, q, k, v, gates, idx, dout, nthreads):
     dk = np.zeros((N, D.n_kv_heads, D.head_dim))
     dv = np.zeros((N, D.n_kv_heads, D.head_dim))
     dg = np.zeros((N, D.n_q_heads, D.n_gates))
+    qb = None if qblocks is None else _c(qblocks, np.int32)
+    n_qb = 0 if qb is None else len(qb)
     rc = fn(ctypes.byref(D), _p(off), _p(q), _p(k), _p(v), _p(gates), _p(idx), idx_heads, _p(dout), _p(dq),
-            _p(dk), _p(dv), _p(dg), int(nthreads))
+            _p(dk), _p(dv), _p(dg), n_qb, _p(qb), int(nthreads))
     if rc != 0:
         raise ValueError("oracle backward: unsupported configuration")
     return dq, dk, dv, dg
 
 
-def backward(D, off, q, k, v, gates, idx, dout, nthreads=1):
-    """(dq, dk, dv, dgates) of L = sum(O * dO) over all tokens, routing indices fixed."""
-    return _backward(_L().oracle_backward, np.uint16, D, off, q, k, v, gates, idx, dout, nthreads)
+def backward(D, off, q, k, v, gates, idx, dout, nthreads=1, qblocks=None):
+    """(dq, dk, dv, dgates) of L = sum(O * dO) over all tokens, routing indices fixed.
+    With qblocks only those query blocks contribute: dq and dgates of their rows are exact,
+    dk and dv are the listed blocks' share, other rows of dq and dgates stay zero."""
+    return _backward(_L().oracle_backward, np.uint16, D, off, q, k, v, gates, idx, dout, nthreads, qblocks)
 
 
-def backward_f64(D, off, q, k, v, gates, idx, dout, nthreads=1):
-    return _backward(_L().oracle_backward_f64, np.float64, D, off, q, k, v, gates, idx, dout, nthreads)
+def backward_f64(D, off, q, k, v, gates, idx, dout, nthreads=1, qblocks=None):
+    return _backward(_L().oracle_backward_f64, np.float64, D, off, q, k, v, gates, idx, dout, nthreads, qblocks)
 
 
 def loss_f64(D, off, q, k, v, gates, idx, dout) -> float:

@@ -72,3 +72,9 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.bfloat16:
         return t.float().cpu().numpy()
     return t.cpu().numpy()
+
+
+def assert_grad_close(got, ref, what=""):
+    """Gradient bounds: max-abs 1e-2 scaled by max(1, max|ref|), relative L2 5e-3."""
+    ref = np.asarray(ref, dtype=np.float64)
+    return assert_close(got, ref, what, max_abs=MAX_ABS * max(1.0, float(np.abs(ref).max())), rel=REL_L2)

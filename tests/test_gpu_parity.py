@@ -12,7 +12,7 @@ import torch
 import oracle as O
 from block_sparse_gqa_nsa_b200 import nsa
 from block_sparse_gqa_nsa_b200.build import build
-from nsa_case import DeviceCase, oracle_desc, assert_close, rows_for, to_np, i32, bf16_tensor
+from nsa_case import DeviceCase, oracle_desc, assert_close, assert_grad_close, rows_for, to_np, i32, bf16_tensor
 from workloads import make_workload
 from workloads.nsa_workloads import f32_to_bf16_bits
 
@@ -370,3 +370,124 @@ def test_speed3r_full_size_sampled():
     check_pooled_routing(gidx, w, qb, w.top_k)
     ref = O.forward(oracle_desc(w), w.off, w.q, w.k, w.v, w.gates, gidx, forced=w.forced, qblocks=qb)
     assert_close(to_np(out)[rows_for(w.off, qb)], ref, "out")
+
+
+# ------------------------------------------------------------------------------------------------
+# S10 backward (routing indices fixed; gradients of L = sum(out * dO))
+# ------------------------------------------------------------------------------------------------
+
+def _dout(w, seed=7):
+    from workloads.nsa_workloads import normal_bf16
+    return w.dout if w.dout is not None else normal_bf16(seed, 5, w.q.shape, 1.0)
+
+
+def _gpu_backward(c: DeviceCase, idx_t, idx_heads, lse, dout_t):
+    w = c.w
+    bf = torch.bfloat16
+    dq = c.empty(w.n_tokens, w.n_q_heads, w.head_dim, dtype=bf)
+    dk = c.empty(w.n_tokens, w.n_kv_heads, w.head_dim, dtype=bf)
+    dv = c.empty(w.n_tokens, w.n_kv_heads, w.head_dim, dtype=bf)
+    dg = c.empty(w.n_tokens, w.n_q_heads, w.n_gates, dtype=bf)
+    nsa.lsrm_nsa_backward(c.desc, c.off, c.q, c.k, c.v, c.gates, idx_t, idx_heads, lse, dout_t, dq, dk, dv, dg, c.ws)
+    assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
+    return dq, dk, dv, dg
+
+
+def _check_grads(got, ref, rows=None):
+    for name, g, r in zip(("dq", "dk", "dv", "dgates"), got, ref):
+        g = to_np(g)
+        if rows is not None and name in ("dq", "dgates"):
+            g, r = g[rows], r[rows]
+        assert_grad_close(g, r, name)
+
+
+@pytest.mark.parametrize("name,kw,mode", [
+    ("backward_small", {}, "geom"),
+    ("ragged_geo", {}, "geom"),
+    ("tiny", {}, "score"),
+    ("tiny", {"head_dim": 64}, "score"),
+    ("tiny_geo", {"window": 0}, "geom"),
+    ("tiny_geo", {"window": 2}, "geom"),
+    ("ragged_geo", {"top_k": 1}, "geom"),
+])
+def test_backward_matches_oracle(name, kw, mode):
+    w = make_workload(name, **kw)
+    c = DeviceCase(w)
+    out, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC if mode == "geom" else nsa.ROUTE_SCORE)
+    heads = 1 if mode == "geom" else w.n_kv_heads
+    gidx = to_np(idx).reshape(w.n_blocks, heads, w.top_k)
+    dout = _dout(w)
+    got = _gpu_backward(c, idx, heads, lse, bf16_tensor(dout))
+    ref_idx = gidx[:, 0, :] if heads == 1 else gidx
+    ref = O.backward(oracle_desc(w), w.off, w.q, w.k, w.v, w.gates, ref_idx, dout, nthreads=8)
+    _check_grads(got, ref)
+
+
+def test_backward_is_deterministic():
+    w = make_workload("backward_small")
+    c = DeviceCase(w)
+    _, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC)
+    dout = bf16_tensor(_dout(w))
+    a = _gpu_backward(c, idx, 1, lse, dout)
+    b = _gpu_backward(c, idx, 1, lse, dout)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+
+
+def test_backward_compressed_only_gates_spread_block_gradient():
+    # with the selected and window gates at zero only the block means receive gradient, so every
+    # token of a block gets the same dK and dV
+    w = make_workload("ragged_geo")
+    g = w.gates.copy()
+    g[..., 1:] = 0
+    w.gates = g
+    c = DeviceCase(w)
+    _, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC)
+    dq, dk, dv, dg = _gpu_backward(c, idx, 1, lse, bf16_tensor(_dout(w)))
+    dk, dv = to_np(dk), to_np(dv)
+    for b in range(w.n_blocks):
+        blk = slice(w.off[b], w.off[b + 1])
+        assert np.array_equal(dk[blk], np.broadcast_to(dk[w.off[b]], dk[blk].shape))
+        assert np.array_equal(dv[blk], np.broadcast_to(dv[w.off[b]], dv[blk].shape))
+
+
+def test_backward_sparse_stage_full_size():
+    """The backward workload (sparse stage, 121 344 tokens, dO ~ N(0, 1)) at full size:
+    sampled query blocks exactly against the oracle restricted to them, key-side sums against
+    identities that hold at any size, and sampled key blocks with the compressed gate at zero
+    against the oracle over the query blocks that reach them."""
+    w = make_workload("backward")
+    c = DeviceCase(w)
+    _, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC)
+    gidx = to_np(idx).reshape(w.n_blocks, w.top_k)
+    dout_t = bf16_tensor(w.dout)
+    dq, dk, dv, dg = _gpu_backward(c, idx, 1, lse, dout_t)
+    D = oracle_desc(w)
+    rng = np.random.default_rng(2)
+    qb = np.sort(np.r_[rng.choice(w.n_blocks, 2, replace=False), [w.n_blocks - 1]]).astype(np.int32)
+    ref = O.backward(D, w.off, w.q, w.k, w.v, w.gates, gidx, w.dout, nthreads=len(qb), qblocks=qb)
+    rows = rows_for(w.off, qb)
+    assert_grad_close(to_np(dq)[rows], ref[0][rows], "dq")
+    assert_grad_close(to_np(dg)[rows], ref[3][rows], "dgates")
+    # sum_u dV[u, g] = sum over the group's rows of sum_b g_b dO (every branch's P sums to one);
+    # sum_u dK[u, g] = 0 (every row of dS sums to zero)
+    G = w.n_q_heads // w.n_kv_heads
+    gsum = to_np(c.gates).sum(-1, keepdims=True) * to_np(dout_t)
+    want_dv = gsum.reshape(w.n_tokens, w.n_kv_heads, G, w.head_dim).sum((0, 2))
+    got_dv = to_np(dv).astype(np.float64).sum(0)
+    assert np.abs(got_dv - want_dv).max() <= 1e-2 * np.abs(want_dv).max()
+    dk64 = to_np(dk).astype(np.float64)
+    assert np.abs(dk64.sum(0)).max() <= 1e-3 * np.abs(dk64).sum(0).max()
+    # key blocks with the compressed gate at zero: dK, dV of block j come only from the query
+    # blocks that routed to it and from j itself
+    g = w.gates.copy()
+    g[..., 0] = 0
+    w.gates = g
+    c.gates = bf16_tensor(g)
+    dq, dk, dv, dg = _gpu_backward(c, idx, 1, lse, dout_t)
+    for j in rng.choice(w.n_blocks, 2, replace=False):
+        src = np.unique(np.r_[np.nonzero((gidx == j).any(1))[0], [j]]).astype(np.int32)
+        ref = O.backward(D, w.off, w.q, w.k, w.v, g, gidx, w.dout, nthreads=6, qblocks=src)
+        blk = slice(w.off[j], w.off[j + 1])
+        assert_grad_close(to_np(dk)[blk], ref[1][blk], f"dk block {j}")
+        assert_grad_close(to_np(dv)[blk], ref[2][blk], f"dv block {j}")

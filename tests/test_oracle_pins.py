@@ -447,3 +447,20 @@ def test_backward_threads_agree_with_single_thread():
     b = O.backward(D, w.off, w.q, w.k, w.v, w.gates, idx, dout, nthreads=3)
     for x, y in zip(a, b):
         assert np.abs(x - y).max() < 1e-12 * max(1.0, np.abs(x).max())
+
+
+def test_backward_query_block_lists_partition_the_gradient():
+    # restricting the backward to a list of query blocks splits it by linearity: the key-side
+    # gradients of a partition of the blocks add up to the full ones, and the query-side rows of
+    # each listed block are the full rows
+    D, off, qf, kf, vf, gf, idx, dout = _fd_case(5)
+    full = O.backward_f64(D, off, qf, kf, vf, gf, idx, dout)
+    part_a = O.backward_f64(D, off, qf, kf, vf, gf, idx, dout, qblocks=np.array([0, 2], np.int32))
+    part_b = O.backward_f64(D, off, qf, kf, vf, gf, idx, dout, qblocks=np.array([1, 3], np.int32))
+    for i in (1, 2):  # dk, dv
+        assert np.abs(part_a[i] + part_b[i] - full[i]).max() < 1e-13 * max(1.0, np.abs(full[i]).max())
+    for i in (0, 3):  # dq, dgates
+        for b, part in ((0, part_a), (2, part_a), (1, part_b), (3, part_b)):
+            blk = slice(off[b], off[b + 1])
+            assert np.array_equal(part[i][blk], full[i][blk])
+        assert not part_a[i][off[1]:off[2]].any()
