@@ -43,14 +43,17 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-sample-blocks", type=int, default=24,
-                    help="query blocks of the oracle's bounded CPU sample")
+    ap.add_argument("--cpu-sample-blocks", type=int, default=None,
+                    help="query blocks of the oracle's bounded CPU sample (default 64 forward, 8 backward: "
+                         "10-20 s of one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward"],
+                    help="sparse: the layer forward (the default line); backward: its gradients")
     return ap.parse_args()
 
 
@@ -76,6 +79,40 @@ def algorithmic_flops(w, idx: np.ndarray) -> dict:
     return {"cmp": f * cmp, "slc": f * slc, "win": f * win, "total": f * (cmp + slc + win)}
 
 
+def backward_flops(fwd: dict) -> dict:
+    """Algorithmic backward FLOPs over the same attended (row, key) pairs: the score recompute
+    (2d), dV (2d), dP (2d), dQ (2d) and dK (2d), i.e. 2.5x the forward's 4d per pair."""
+    return {k: 2.5 * v for k, v in fwd.items()}
+
+
+KERNEL_SOURCES = {"attn": ["attn_tc.cu", "tc_ptx.cuh", "lsrm_common.cuh"],
+                  "bwd": ["backward.cu", "lsrm_common.cuh"]}
+
+
+def kernel_source_hash(which: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[which]:
+        with open(os.path.join(ROOT, "block_sparse_gqa_nsa_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(which: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the kernel
+    sources as they are now (else None)."""
+    import re
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    pat = re.compile(rf"^\|\s*{which}\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|", re.M)
+    with open(path) as f:
+        m = pat.search(f.read())
+    if m is None or m.group(2) != kernel_source_hash(which):
+        return None
+    return float(m.group(1))
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -98,6 +135,10 @@ class ClockSampler:
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
+        # start timing only once nvidia-smi is producing samples
+        t0 = time.time()
+        while self.p is not None and time.time() - t0 < 5.0 and os.path.getsize(self.f.name) == 0:
+            time.sleep(0.05)
 
     def stop(self) -> dict:
         if self.p is None:
@@ -322,16 +363,225 @@ def run_ours(args):
                 "flops_per_step": flops,
                 "kernel_ms": {"fused_attention": attn_avg, "compress_and_route": sum(pre_ms) / len(pre_ms)},
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                             "frac": achieved / peak, "traffic": None,
+                             "frac": achieved / peak, "traffic": profiled_traffic("attn"),
                              "kernel": "nsa_attn (fused cmp+slc+win attention, gated combine)",
                              "peak_source": f"{src} bf16_tflops (burst)"},
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clocks, "e2e": e2e}
         if not args.no_cpu_baseline and world == 1:
-            tok, dt = oracle_sample(w, idx.cpu().numpy(), args.cpu_sample_blocks, 7)
+            n_blk = args.cpu_sample_blocks or 64
+            tok, dt = oracle_sample(w, idx.cpu().numpy(), n_blk, 7)
             line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"{args.cpu_sample_blocks} seeded query blocks ({tok} tokens) "
+                                    "sample": f"{n_blk} seeded query blocks ({tok} tokens) "
                                               f"of the same workload, fp64, 1 thread, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# the backward workload: gradients of the same layer, routing indices fixed from its forward
+# ------------------------------------------------------------------------------------------------
+BWD_METRIC = "sparse-attn bwd tokens/s and effective TFLOP/s vs B200 bf16 tensor peak"
+BWD_WORKLOAD = "lsrm_sparse_stage_backward_dO_normal"
+
+
+def oracle_backward_sample(w, idx, n_blocks: int, seed: int):
+    """Time the fp64 oracle backward restricted to a seeded sample of query blocks (1 thread)."""
+    import oracle as O
+    D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window,
+                   n_gates=w.n_gates)
+    rng = np.random.default_rng(seed)
+    qb = np.sort(rng.choice(w.n_blocks, size=n_blocks, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    O.backward(D, w.off, w.q, w.k, w.v, w.gates, idx, w.dout, nthreads=1, qblocks=qb)
+    dt = time.perf_counter() - t0
+    return int((w.off[qb + 1] - w.off[qb]).sum()), dt
+
+
+def bwd_config(w, world, seed, extra=None):
+    c = {"workload": BWD_WORKLOAD, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
+         "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "top_k": w.top_k,
+         "window": w.window, "route": "geometric (indices fixed from the forward)",
+         "parallelism": f"replicas{world}" if world > 1 else "single", "seed": seed}
+    c.update(extra or {})
+    return c
+
+
+def run_backward_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    from workloads import make_workload
+    import oracle as O
+    w = make_workload("backward", seed=args.seed)
+    D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window)
+    idx, _ = O.route_geometric(D, w.off, w.coords)
+    for s in range(args.warmup):
+        oracle_backward_sample(w, idx, 1, 1000 + s)
+    tok, tsum = 0, 0.0
+    for s in range(args.steps):
+        t, dt = oracle_backward_sample(w, idx, 1, s)
+        tok += t
+        tsum += dt
+    value = tok / tsum
+    line = {"metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * tsum / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": bwd_config(w, 1, args.seed, {"sample": "1 seeded query block per step"}),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "1 query block (64 tokens) per step, fp64, 1 thread"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_backward(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+
+    from block_sparse_gqa_nsa_b200 import nsa
+    from block_sparse_gqa_nsa_b200.build import build
+    from workloads import make_workload
+
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    nsa.load_library()
+
+    w = make_workload("backward", seed=args.seed)
+    N, B, Hq, Hkv, d, k = w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    h_in = {"q": bf(w.q), "k": bf(w.k), "v": bf(w.v), "gates": bf(w.gates), "dout": bf(w.dout),
+            "off": torch.from_numpy(w.off.astype(np.int32)), "coords": torch.from_numpy(w.coords.astype(np.int32))}
+    x = {n: t.to(dev) for n, t in h_in.items()}
+    desc = nsa.make_desc(N, B, w.max_block_len, Hq, Hkv, d, k, w.window, 0.0, False, w.n_gates)
+    ws = nsa.workspace(desc, dev)
+    bf16 = torch.bfloat16
+    out = torch.empty(N, Hq, d, dtype=bf16, device=dev)
+    idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
+    lse = torch.empty(N, Hq, w.n_gates, dtype=torch.float32, device=dev)
+    nsa.lsrm_nsa_forward(desc, x["off"], x["q"], x["k"], x["v"], x["gates"], x["coords"], nsa.ROUTE_GEOMETRIC,
+                         out, idx, lse, ws)
+    grads = {"dq": torch.empty(N, Hq, d, dtype=bf16, device=dev), "dk": torch.empty(N, Hkv, d, dtype=bf16, device=dev),
+             "dv": torch.empty(N, Hkv, d, dtype=bf16, device=dev),
+             "dgates": torch.empty(N, Hq, w.n_gates, dtype=bf16, device=dev)}
+    stream = torch.cuda.current_stream(dev)
+
+    def step(t=x, g=grads, ix=idx, ls=lse):
+        nsa.lsrm_nsa_backward(desc, t["off"], t["q"], t["k"], t["v"], t["gates"], ix, 1, ls, t["dout"], g["dq"],
+                              g["dk"], g["dv"], g["dgates"], ws)
+
+    # compress, then the inverse routing lists (count, scan, fill, sort), then the query, local-key,
+    # compressed-key and finishing kernels
+    launches_per_step = 9
+    for _ in range(max(3, args.warmup)):
+        step()
+    st = nsa.lsrm_nsa_last_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    flops = backward_flops(algorithmic_flops(w, idx.view(B, k).cpu().numpy()))
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    tt = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    total_ms = float(tt.item())
+    call_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    value = world * N * args.steps / (total_ms / 1000.0)
+
+    e2e = None
+    if not args.no_e2e:
+        h_idx = idx.cpu().pin_memory()
+        h_lse = lse.cpu().pin_memory()
+        p_in = {n: t.pin_memory() for n, t in h_in.items() if n != "coords"}
+        d_in = {n: torch.empty_like(x[n]) for n in p_in}
+        d_idx, d_lse = torch.empty_like(idx), torch.empty_like(lse)
+        p_out = {n: torch.empty(g.shape, dtype=g.dtype).pin_memory() for n, g in grads.items()}
+        d_out = {n: torch.empty_like(g) for n, g in grads.items()}
+
+        def e2e_step():
+            for n in p_in:
+                d_in[n].copy_(p_in[n], non_blocking=True)
+            d_idx.copy_(h_idx, non_blocking=True)
+            d_lse.copy_(h_lse, non_blocking=True)
+            step(d_in, d_out, d_idx, d_lse)
+            for n in p_out:
+                p_out[n].copy_(d_out[n], non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(t.numel() * t.element_size() for t in p_in.values()) + \
+            h_idx.numel() * h_idx.element_size() + h_lse.numel() * h_lse.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in p_out.values())
+        e2e = {"value": world * N * args.steps / (float(te.item()) / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        for n in grads:
+            if not torch.equal(p_out[n].view(torch.int16), grads[n].view(torch.int16).cpu()):
+                raise RuntimeError(f"end-to-end {n} differs from the device-resident run")
+
+    if rank == 0:
+        peaks, src = measured_peaks()
+        achieved = flops["total"] / (call_ms / 1000.0) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        line = {"metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": bwd_config(w, world, args.seed,
+                                     {"l2": "inputs larger than L2 (q, dO, dq 249 MB each per step)"}),
+                "flops_per_step": flops,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                             "frac": achieved / peak, "traffic": profiled_traffic("bwd"),
+                             "kernel": "lsrm_nsa_backward (all launches of one call)",
+                             "peak_source": f"{src} bf16_tflops (burst)"},
+                "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "e2e": e2e}
+        if not args.no_cpu_baseline and world == 1:
+            n_blk = args.cpu_sample_blocks or 8
+            tok, dt = oracle_backward_sample(w, idx.view(B, k).cpu().numpy(), n_blk, 7)
+            line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"{n_blk} seeded query blocks ({tok} tokens) of the same workload, "
+                                              f"fp64 backward, 1 thread, {dt:.1f} s"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -341,6 +591,8 @@ def run_ours(args):
 
 def main():
     args = parse()
+    if args.workload == "backward":
+        return run_backward_reference(args) if args.impl == "reference" else run_backward(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
