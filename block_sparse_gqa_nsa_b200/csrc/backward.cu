@@ -19,10 +19,11 @@
 // The key-side passes compute S^T and dP^T (keys x query rows) directly, so P^T and dS^T are
 // already in the A-operand layout of the dV and dK products.
 #include "lsrm_common.cuh"
+#include "tc_ptx.cuh"
+#include "tma_map.cuh"
 
 namespace lsrm {
 
-constexpr int kBqThreads = 256;   // 8 warps x 16 query rows
 constexpr int kBkThreads = 128;   // 4 warps x 16 keys
 
 template <int D>
@@ -60,291 +61,364 @@ struct BwdParams {
 };
 
 // ------------------------------------------------------------------------------------------------
-// query pass
+// query pass on the tensor cores: per 128-row tile and branch, pass A recomputes o_b = P V
+// (P = exp(tau q.k - lse_b), normalised by the saved LSE) to get dgates_b and Delta_b; pass B
+// forms dS = P (g_b dO V^T - Delta_b) and accumulates dQ_b = dS K.
+//   TMEM (256 columns): S [0, 64) | dP [64, 128) | P or dS as bf16 pairs [128, 160) | O or dQ_b
+//   warp 0 TMA (Q and dO tiles once, then K/V chunks: every branch is streamed twice),
+//   warp 1 MMA issuer, warps 2-9 element-wise: two warps per TMEM lane quarter, each taking
+//   32 of a chunk's 64 keys (no online softmax here: the LSE is known, so the halves are
+//   independent).
 // ------------------------------------------------------------------------------------------------
+constexpr int kBqtThreads = 320;
+constexpr int kBqtMaxSel = 256;
+
 template <int D>
-struct BqSmem {
-  uint16_t q[128 * D];
-  uint16_t go[128 * D];   // dO rows
-  uint16_t kb[2][64 * D];
-  uint16_t vb[2][64 * D];
-  int32_t sel[256];
-  int32_t pre[257];
-  int32_t n_sel;
+struct BqtCfg {
+  static constexpr int kKeys = 64;
+  static constexpr int kStages = D == 32 ? 4 : 3;
+  static constexpr int kCtasPerSm = D == 32 ? 2 : 1;
+  static constexpr int kTmemCols = 256;
+  static constexpr int kColS = 0, kColDP = 64, kColP = 128, kColO = 160;
+  static constexpr int kRowBytes = D * 2;
+  static constexpr uint32_t kLayout = D == 32 ? tc::kLayoutSW64 : tc::kLayoutSW128;
+  static constexpr uint32_t kAtomBytes = 8 * kRowBytes;
+  static constexpr int kQBytes = 128 * kRowBytes;
+  static constexpr int kKVBytes = kKeys * kRowBytes;
+  static constexpr uint32_t kIdescNK = tc::idesc_bf16(128, kKeys, false);  // [rows x keys] from K-major B
+  static constexpr uint32_t kIdescND = tc::idesc_bf16(128, D, true);       // [rows x D] from MN-major B
+  static_assert(kColO + D <= kTmemCols, "tensor memory budget");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBqThreads) bwd_query_kernel(const BwdParams p) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  BqSmem<D>& S = *reinterpret_cast<BqSmem<D>*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int chunk_id = blockIdx.x, g = blockIdx.y, a = blockIdx.z;
+struct BqtSmem {
+  using C = BqtCfg<D>;
+  uint8_t q[C::kQBytes];
+  uint8_t go[C::kQBytes];  // dO rows of the tile
+  uint8_t k[C::kStages][C::kKVBytes];
+  uint8_t v[C::kStages][C::kKVBytes];
+  float acc[D][128];       // dQ of the tile, column-major
+  uint64_t q_full, kv_full[C::kStages], kv_empty[C::kStages], s_full, p_full, pv_done, drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_sel;
+  int sel_start[kBqtMaxSel];
+  int sel_n[kBqtMaxSel];
+};
+
+// chunk order: for each branch with keys, its chunks twice (pass A, then pass B)
+struct BqtSeq {
+  int n[3];
+  int total;
+  __device__ __forceinline__ void decode(int c, int& br, int& pass, int& local, bool& first, bool& last) const {
+    br = 0;
+    while (c >= 2 * n[br]) { c -= 2 * n[br]; ++br; }
+    pass = c >= n[br];
+    local = c - pass * n[br];
+    first = local == 0;
+    last = local == n[br] - 1;
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBqtThreads, BqtCfg<D>::kCtasPerSm)
+bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap,
+                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                    const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap vcmap,
+                    const BwdParams p) {
+  using namespace tc;
+  using C = BqtCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  BqtSmem<D>& S = *reinterpret_cast<BqtSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, g = blockIdx.y, a = blockIdx.z;
   const int t0 = p.off[a], n_a = p.off[a + 1] - t0;
   const int rows_total = n_a * p.G;
-  const int row0 = chunk_id * 128;
-  if (row0 >= rows_total) return;
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
-  constexpr int KT = D / 16, NT = D / 8;
+  if (tile * 128 >= rows_total) return;
+  const int tokens_per_tile = 128 / p.G;
 
-  if (tid == 0) {
-    int n = 0, tot = 0;
+  if (threadIdx.x == 0) {
+    S.abort = 0;
+    int n = 0;
     const int32_t* r = p.idx + ((size_t)a * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.top_k;
-    for (int i = 0; i < p.top_k && n < 256; ++i) {
+    for (int i = 0; i < p.top_k && n < kBqtMaxSel; ++i) {
       const int j = r[i];
       if (j < 0 || j >= p.B) { raise_status(p.status, LSRM_ERR_BOUNDS); continue; }
-      S.sel[n] = j;
-      S.pre[n] = tot;
-      tot += p.off[j + 1] - p.off[j];
+      int len = p.off[j + 1] - p.off[j];
+      if (len > C::kKeys) { raise_status(p.status, LSRM_ERR_BOUNDS); len = C::kKeys; }
+      S.sel_start[n] = p.off[j];
+      S.sel_n[n] = len;
       ++n;
     }
-    S.pre[n] = tot;
     S.n_sel = n;
+    mbar_init(&S.q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    mbar_init(&S.s_full, 1);
+    mbar_init(&S.p_full, 256);
+    mbar_init(&S.pv_done, 1);
+    mbar_init(&S.drain, 1);
+    fence_mbar_init();
   }
-  for (int e = tid; e < 128 * CPR; e += kBqThreads) {
-    const int r = e / CPR, ch = e % CPR;
-    const int rr = row0 + r;
-    const bool ok = rr < rows_total;
-    const int t = t0 + (ok ? rr / p.G : 0), h = g * p.G + (ok ? rr % p.G : 0);
-    const size_t src = ((size_t)t * p.Hq + h) * D + ch * 8;
-    cp_async16(reinterpret_cast<unsigned char*>(S.q) + bswz<D>(r, ch), p.q + src, ok);
-    cp_async16(reinterpret_cast<unsigned char*>(S.go) + bswz<D>(r, ch), p.dout + src, ok);
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, C::kTmemCols);
+    tmem_relinquish();
   }
-  cp_async_commit();
-  cp_async_wait<0>();
+  tc_fence_before();
   __syncthreads();
-
-  const int gq = lane >> 2, cq = lane & 3;
-  int tokl[2], head[2];
-  bool rvalid[2];
-  size_t orow[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int rr = row0 + warp * 16 + gq + 8 * i;
-    rvalid[i] = rr < rows_total;
-    tokl[i] = rvalid[i] ? rr / p.G : 0;
-    head[i] = g * p.G + (rvalid[i] ? rr % p.G : 0);
-    orow[i] = (size_t)(t0 + tokl[i]) * p.Hq + head[i];
-  }
-  uint32_t qa[KT][4], ga[KT][4];  // Q and dO A-fragments of the warp's 16 rows
-#pragma unroll
-  for (int kt = 0; kt < KT; ++kt) {
-    const int r = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-    const int ch = kt * 2 + (lane >> 4);
-    ldmatrix_x4(qa[kt][0], qa[kt][1], qa[kt][2], qa[kt][3], smem_u32(S.q) + bswz<D>(r, ch));
-    ldmatrix_x4(ga[kt][0], ga[kt][1], ga[kt][2], ga[kt][3], smem_u32(S.go) + bswz<D>(r, ch));
-  }
-  const int n_sel_tok = S.pre[S.n_sel];
-  float dq[NT][4];
-#pragma unroll
-  for (int n = 0; n < NT; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dq[n][e] = 0.f;
-
-  for (int br = 0; br < p.NG; ++br) {
-    if (br == 2 && p.window <= 0) {
-      if (cq == 0)
-        for (int i = 0; i < 2; ++i)
-          if (rvalid[i]) {
-            p.dgates[orow[i] * p.NG + 2] = 0;
-            p.delta[orow[i] * p.NG + 2] = 0.f;
-          }
-      continue;
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  BqtSeq seq;
+  seq.n[0] = (p.B + C::kKeys - 1) / C::kKeys;
+  seq.n[1] = S.n_sel;
+  seq.n[2] = (p.NG == 3 && p.window > 0) ? 1 : 0;
+  seq.total = 2 * (seq.n[0] + seq.n[1] + seq.n[2]);
+  volatile int* abort = &S.abort;
+  auto chunk_start = [&](int br, int local, int& start, int& nv) {
+    if (br == 0) {
+      start = local * C::kKeys;
+      nv = min(C::kKeys, p.B - start);
+    } else if (br == 1) {
+      start = S.sel_start[local];
+      nv = S.sel_n[local];
+    } else {
+      start = t0;
+      nv = min(C::kKeys, n_a);
     }
-    const int total = br == 0 ? p.B : (br == 1 ? n_sel_tok : n_a);
-    const int n_chunks = (total + 63) / 64;
-    float lse2[2], gate[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      lse2[i] = rvalid[i] ? p.lse[orow[i] * p.NG + br] * 1.4426950408889634f : 0.f;
-      gate[i] = rvalid[i] ? bf16_to_f32(p.gates[orow[i] * p.NG + br]) : 0.f;
-    }
-    // G_b = g_b * dO as A-fragments (rows gq and gq + 8 of the warp tile)
-    uint32_t gb[KT][4];
-#pragma unroll
-    for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float sc = gate[e & 1];
-        const uint32_t u = ga[kt][e];
-        gb[kt][e] = pack_bf16x2(__uint_as_float(u << 16) * sc, __uint_as_float(u & 0xFFFF0000u) * sc);
+  };
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && seq.total > 0) {
+      mbar_arrive_expect_tx(&S.q_full, 2 * C::kQBytes);
+      tma_load_3d(S.q, &qmap, &S.q_full, 0, g * p.G, t0 + tile * tokens_per_tile);
+      tma_load_3d(S.go, &omap, &S.q_full, 0, g * p.G, t0 + tile * tokens_per_tile);
+      int issued = 0;
+      for (int c = 0; c < seq.total; ++c) {
+        const int st = c % C::kStages;
+        if (c >= C::kStages && !mbar_wait(&S.kv_empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
+        int br, pass, local, start, nv;
+        bool first, last;
+        seq.decode(c, br, pass, local, first, last);
+        chunk_start(br, local, start, nv);
+        mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
+        tma_load_3d(S.k[st], br == 0 ? &kcmap : &kmap, &S.kv_full[st], 0, g, start);
+        tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
+        issued = c + 1;
       }
-    auto load_chunk = [&](int c, int buf) {
-      for (int e = tid; e < 64 * CPR; e += kBqThreads) {
-        const int kk = e / CPR, ch = e % CPR;
-        const int pos = c * 64 + kk;
-        const bool ok = pos < total;
-        const uint16_t *ks, *vs;
-        if (br == 0) {
-          const size_t base = ((size_t)(ok ? pos : 0) * p.Hkv + g) * D + ch * 8;
-          ks = p.kc + base;
-          vs = p.vc + base;
-        } else {
-          long long u = t0;
-          if (ok) {
-            if (br == 2) {
-              u = t0 + pos;
-            } else {
-              int lo = 0, hi = S.n_sel - 1;
-              while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (S.pre[mid] <= pos) lo = mid; else hi = mid - 1;
+      if (*abort) {
+        volatile int no_abort = 0;
+        mbar_wait(&S.q_full, 0, &no_abort, nullptr);
+        for (int c = max(0, issued - C::kStages); c < issued; ++c)
+          mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, &no_abort, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && seq.total > 0) {
+      bool ok = mbar_wait(&S.q_full, 0, abort, p.status);
+      const uint32_t qaddr = smem_u32(S.q), oaddr = smem_u32(S.go);
+      // pass A: S = Q K^T;  pass B: S = Q K^T and dP = dO V^T  (both [128 x 64], K-major B)
+      auto first_stage = [&](int c, int pass) {
+        const uint32_t kaddr = smem_u32(S.k[c % C::kStages]), vaddr = smem_u32(S.v[c % C::kStages]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          mma_ss(tmem + C::kColS, smem_desc(qaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
+                 smem_desc(kaddr + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNK, kk > 0 ? 1u : 0u);
+        }
+        if (pass) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            mma_ss(tmem + C::kColDP, smem_desc(oaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
+                   smem_desc(vaddr + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNK, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(&S.s_full);
+      };
+      // pass A: O += P V;  pass B: dQ_b += dS K  (A from tensor memory, MN-major B)
+      auto second_stage = [&](int c, int pass, bool first) {
+        const uint32_t baddr = smem_u32(pass ? S.k[c % C::kStages] : S.v[c % C::kStages]);
+#pragma unroll
+        for (int kk = 0; kk < C::kKeys / 16; ++kk) {
+          const uint64_t bd = smem_desc(baddr + kk * 16 * C::kRowBytes, C::kKVBytes, C::kAtomBytes, C::kLayout);
+          mma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, bd, C::kIdescND, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(&S.pv_done);
+        mma_commit(&S.kv_empty[c % C::kStages]);
+      };
+      int prev_pass = 0;
+      bool prev_first = false;
+      for (int c = 0; ok && c < seq.total; ++c) {
+        if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        int br, pass, local;
+        bool first, last;
+        seq.decode(c, br, pass, local, first, last);
+        if (c > 0) {
+          // the element-wise warps are done with S, dP and P(c - 1)
+          if (!mbar_wait(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+          second_stage(c - 1, prev_pass, prev_first);
+        }
+        tc_fence_after();
+        first_stage(c, pass);
+        prev_pass = pass;
+        prev_first = first;
+      }
+      if (ok && mbar_wait(&S.p_full, (seq.total - 1) & 1, abort, p.status)) {
+        tc_fence_after();
+        second_stage(seq.total - 1, prev_pass, prev_first);
+      }
+      mma_commit(&S.drain);
+      volatile int no_abort = 0;
+      mbar_wait(&S.drain, 0, &no_abort, nullptr);
+    }
+  } else {
+    // ---------------- element-wise warps ----------------
+    const int h = (warp - 2) >> 2;        // key half: keys [32 h, 32 h + 32) of every chunk
+    const int quarter = warp & 3;         // tensor-memory lane quarter
+    const int row = quarter * 32 + lane;
+    const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int R = tile * 128 + row;
+    const bool valid = R < rows_total;
+    const int tok_local = R / p.G;
+    const size_t orow = (size_t)(t0 + (valid ? tok_local : 0)) * p.Hq + g * p.G + R % p.G;
+    const int wlo = tok_local - p.window / 2, whi = tok_local + p.window / 2 - 1;
+    const float sc = p.scale_log2;
+    float lse2[3] = {0.f, 0.f, 0.f}, gate[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+    for (int b = 0; b < 3; ++b) {
+      if (valid && b < p.NG) {
+        lse2[b] = p.lse[orow * p.NG + b] * 1.4426950408889634f;
+        gate[b] = bf16_to_f32(p.gates[orow * p.NG + b]);
+      }
+    }
+    float* acc = &S.acc[0][row];
+    if (h == 0) {
+#pragma unroll
+      for (int i = 0; i < D; ++i) acc[i * 128] = 0.f;
+      for (int b = 0; b < p.NG; ++b)
+        if (seq.n[b] == 0 && valid) {  // a branch without keys has no gradient
+          p.dgates[orow * p.NG + b] = 0;
+          p.delta[orow * p.NG + b] = 0.f;
+        }
+    }
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const bool w = mbar_wait(bar, parity, abort, p.status);
+      return __all_sync(0xffffffffu, w);
+    };
+    // one pv_done phase per chunk; while chunk c is worked on it has completed c - 1 or c phases
+    int pv_seen = 0;
+    auto pv_wait_through = [&](int j) -> bool {
+      while (pv_seen <= j) {
+        if (!wait_all(&S.pv_done, pv_seen & 1)) return false;
+        ++pv_seen;
+      }
+      tc_fence_after();
+      return true;
+    };
+    auto swz = [](int r, int ch) -> uint32_t {
+      if (D == 32) return (uint32_t)(r * 64 + ((ch ^ ((r >> 1) & 3)) << 4));
+      return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
+    };
+    float delta = 0.f;
+    for (int c = 0; c < seq.total; ++c) {
+      int br, pass, local, start, nv;
+      bool first, last;
+      seq.decode(c, br, pass, local, first, last);
+      chunk_start(br, local, start, nv);
+      if (!wait_all(&S.s_full, c & 1)) break;
+      tc_fence_after();
+      if (!pv_wait_through(c - 1)) break;  // the P / dS columns are free again
+      const float l2 = br == 0 ? lse2[0] : (br == 1 ? lse2[1] : lse2[2]);
+      const float gb = br == 0 ? gate[0] : (br == 1 ? gate[1] : gate[2]);
+      const bool need_mask = br == 2 || nv < 32 * (h + 1);
+      uint32_t s[32], dp[32];
+      tmem_ld32(tbase + C::kColS + 32 * h, s);
+      if (pass) tmem_ld32(tbase + C::kColDP + 32 * h, dp);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float v2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int j = 32 * h + 2 * i + e;
+          bool kv = true;
+          if (need_mask) {
+            kv = j < nv;
+            if (br == 2) kv = kv && j >= wlo && j <= whi;
+          }
+          const float pr = kv ? fast_exp2(fmaf(__uint_as_float(s[2 * i + e]), sc, -l2)) : 0.f;
+          v2[e] = pass ? pr * fmaf(gb, __uint_as_float(dp[2 * i + e]), -delta) : pr;
+        }
+        pk[i] = pack_bf16x2(v2[0], v2[1]);
+      }
+      tmem_st16(tbase + C::kColP + 16 * h, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&S.p_full);
+      if (last) {
+        if (!pv_wait_through(c)) break;
+        if (pass == 0) {
+          // o_b is final: dgates_b = <dO, o_b>, Delta_b = g_b dgates_b
+          float dg = 0.f;
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) {
+            uint32_t o[32];
+            tmem_ld32(tbase + C::kColO + 32 * i, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint4 u = *reinterpret_cast<const uint4*>(S.go + swz(row, 4 * i + ch));
+              const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                dg = fmaf(__uint_as_float(w4[e] << 16), __uint_as_float(o[8 * ch + 2 * e]), dg);
+                dg = fmaf(__uint_as_float(w4[e] & 0xFFFF0000u), __uint_as_float(o[8 * ch + 2 * e + 1]), dg);
               }
-              u = p.off[S.sel[lo]] + (pos - S.pre[lo]);
             }
           }
-          const size_t base = ((size_t)u * p.Hkv + g) * D + ch * 8;
-          ks = p.k + base;
-          vs = p.v + base;
+          delta = gb * dg;
+          if (h == 0 && valid) {
+            p.dgates[orow * p.NG + br] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
+            p.delta[orow * p.NG + br] = delta;
+          }
+        } else if (h == 0) {
+          // dQ_b is final: add tau dQ_b to the tile's dQ
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) {
+            uint32_t o[32];
+            tmem_ld32(tbase + C::kColO + 32 * i, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[(32 * i + e) * 128] = fmaf(p.tau, __uint_as_float(o[e]), acc[(32 * i + e) * 128]);
+          }
         }
-        cp_async16(reinterpret_cast<unsigned char*>(S.kb[buf]) + bswz<D>(kk, ch), ks, ok);
-        cp_async16(reinterpret_cast<unsigned char*>(S.vb[buf]) + bswz<D>(kk, ch), vs, ok);
-      }
-      cp_async_commit();
-    };
-    // S = Q K^T of the warp's rows against 64 keys; P = exp(S tau - lse) with masking
-    auto scores = [&](uint32_t sk, int c, float (&s)[8][4]) {
-#pragma unroll
-      for (int n = 0; n < 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
-#pragma unroll
-      for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b0, b1, b2, b3;
-          const int key = np * 16 + (lane >> 4) * 8 + (lane & 7);
-          const int ch = kt * 2 + ((lane >> 3) & 1);
-          ldmatrix_x4(b0, b1, b2, b3, sk + bswz<D>(key, ch));
-          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
-          mma_bf16_16816(s[2 * np], qa[kt], bb0);
-          mma_bf16_16816(s[2 * np + 1], qa[kt], bb1);
-        }
-#pragma unroll
-      for (int n = 0; n < 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = e >> 1;
-          const int key = n * 8 + 2 * cq + (e & 1);
-          const int pos = c * 64 + key;
-          bool ok = pos < total && rvalid[i];
-          if (br == 2) ok = ok && pos >= tokl[i] - p.window / 2 && pos <= tokl[i] + p.window / 2 - 1;
-          s[n][e] = ok ? fast_exp2(s[n][e] * p.scale_log2 - lse2[i]) : 0.f;
-        }
-    };
-    // ---- pass A: o_b = P V ----
-    float o[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
-    if (n_chunks > 0) load_chunk(0, 0);
-    for (int c = 0; c < n_chunks; ++c) {
-      const int buf = c & 1;
-      if (c + 1 < n_chunks) { load_chunk(c + 1, buf ^ 1); cp_async_wait<1>(); } else { cp_async_wait<0>(); }
-      __syncthreads();
-      float s[8][4];
-      scores(smem_u32(S.kb[buf]), c, s);
-      uint32_t pa[4][4];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(s[n][0], s[n][1]);
-        pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(s[n][2], s[n][3]);
-      }
-      const uint32_t sv = smem_u32(S.vb[buf]);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int dn = 0; dn < D / 16; ++dn) {
-          uint32_t b0, b1, b2, b3;
-          const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-          const int ch = dn * 2 + (lane >> 4);
-          ldmatrix_x4_trans(b0, b1, b2, b3, sv + bswz<D>(key, ch));
-          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
-          mma_bf16_16816(o[2 * dn], pa[kk], bb0);
-          mma_bf16_16816(o[2 * dn + 1], pa[kk], bb1);
-        }
-      __syncthreads();
-    }
-    // dgates_b = <dO, o_b>, Delta_b = g_b dgates_b (dO read back from shared memory)
-    float dg[2] = {0.f, 0.f};
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = warp * 16 + gq + 8 * i, col = n * 8 + 2 * cq;
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const unsigned char*>(S.go) +
-                                                              bswz<D>(r, col / 8) + (col % 8) * 2);
-        dg[i] += __uint_as_float(u << 16) * o[n][2 * i] + __uint_as_float(u & 0xFFFF0000u) * o[n][2 * i + 1];
-      }
-    float dlt[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      dg[i] += __shfl_xor_sync(0xffffffffu, dg[i], 1);
-      dg[i] += __shfl_xor_sync(0xffffffffu, dg[i], 2);
-      dlt[i] = gate[i] * dg[i];
-      if (rvalid[i] && cq == 0) {
-        p.dgates[orow[i] * p.NG + br] = __bfloat16_as_ushort(__float2bfloat16_rn(dg[i]));
-        p.delta[orow[i] * p.NG + br] = dlt[i];
       }
     }
-    // ---- pass B: dS = P (G_b V^T - Delta), dQ += tau dS K ----
-    if (n_chunks > 0) load_chunk(0, 0);
-    for (int c = 0; c < n_chunks; ++c) {
-      const int buf = c & 1;
-      if (c + 1 < n_chunks) { load_chunk(c + 1, buf ^ 1); cp_async_wait<1>(); } else { cp_async_wait<0>(); }
-      __syncthreads();
-      float s[8][4];
-      scores(smem_u32(S.kb[buf]), c, s);
-      float dp[8][4];
+    if (h == 0 && valid) {
+      uint4* dst = reinterpret_cast<uint4*>(p.dq + orow * D);
 #pragma unroll
-      for (int n = 0; n < 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dp[n][e] = 0.f;
-      const uint32_t sv = smem_u32(S.vb[buf]);
-#pragma unroll
-      for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b0, b1, b2, b3;
-          const int key = np * 16 + (lane >> 4) * 8 + (lane & 7);
-          const int ch = kt * 2 + ((lane >> 3) & 1);
-          ldmatrix_x4(b0, b1, b2, b3, sv + bswz<D>(key, ch));
-          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
-          mma_bf16_16816(dp[2 * np], gb[kt], bb0);
-          mma_bf16_16816(dp[2 * np + 1], gb[kt], bb1);
-        }
-      uint32_t da[4][4];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        float ds[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) ds[e] = s[n][e] * (dp[n][e] - dlt[e >> 1]);
-        da[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(ds[0], ds[1]);
-        da[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+      for (int i = 0; i < D / 8; ++i) {
+        uint4 u;
+        u.x = pack_bf16x2(acc[(8 * i + 0) * 128], acc[(8 * i + 1) * 128]);
+        u.y = pack_bf16x2(acc[(8 * i + 2) * 128], acc[(8 * i + 3) * 128]);
+        u.z = pack_bf16x2(acc[(8 * i + 4) * 128], acc[(8 * i + 5) * 128]);
+        u.w = pack_bf16x2(acc[(8 * i + 6) * 128], acc[(8 * i + 7) * 128]);
+        dst[i] = u;
       }
-      const uint32_t sk = smem_u32(S.kb[buf]);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int dn = 0; dn < D / 16; ++dn) {
-          uint32_t b0, b1, b2, b3;
-          const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-          const int ch = dn * 2 + (lane >> 4);
-          ldmatrix_x4_trans(b0, b1, b2, b3, sk + bswz<D>(key, ch));
-          const uint32_t bb0[2] = {b0, b1}, bb1[2] = {b2, b3};
-          mma_bf16_16816(dq[2 * dn], da[kk], bb0);
-          mma_bf16_16816(dq[2 * dn + 1], da[kk], bb1);
-        }
-      __syncthreads();
     }
   }
-#pragma unroll
-  for (int n = 0; n < NT; ++n)
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-      if (rvalid[i])
-        *reinterpret_cast<uint32_t*>(p.dq + orow[i] * D + n * 8 + 2 * cq) =
-            pack_bf16x2(p.tau * dq[n][2 * i], p.tau * dq[n][2 * i + 1]);
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -683,11 +757,19 @@ __global__ void inv_sort_kernel(const int* start, int n_lists, int* list) {
 template <int D>
 static lsrm_status launch_backward_d(const lsrm_nsa_desc& d, const BwdParams& p, int idx_heads, cudaStream_t s) {
   const int G = p.G;
-  const int chunks = (d.max_block_len * G + 127) / 128;
-  size_t sm = sizeof(BqSmem<D>);
-  if (cudaFuncSetAttribute(bwd_query_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+  const int tiles = (d.max_block_len * G + 127) / 128;
+  CUtensorMap qm, om, km, vm, kcm, vcm;
+  if (!make_map(&qm, p.q, D, d.n_q_heads, d.n_tokens, G, 128 / G) ||
+      !make_map(&om, p.dout, D, d.n_q_heads, d.n_tokens, G, 128 / G) ||
+      !make_map(&km, p.k, D, d.n_kv_heads, d.n_tokens, 1, 64) || !make_map(&vm, p.v, D, d.n_kv_heads, d.n_tokens, 1, 64) ||
+      !make_map(&kcm, p.kc, D, d.n_kv_heads, d.n_blocks, 1, 64) ||
+      !make_map(&vcm, p.vc, D, d.n_kv_heads, d.n_blocks, 1, 64))
     return LSRM_ERR_CUDA;
-  bwd_query_kernel<D><<<dim3(chunks, d.n_kv_heads, d.n_blocks), kBqThreads, sm, s>>>(p);
+  size_t sm = sizeof(BqtSmem<D>) + 1024;
+  if (cudaFuncSetAttribute(bwd_query_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+      cudaSuccess)
+    return LSRM_ERR_CUDA;
+  bwd_query_tc_kernel<D><<<dim3(tiles, d.n_kv_heads, d.n_blocks), kBqtThreads, sm, s>>>(qm, om, km, vm, kcm, vcm, p);
   sm = sizeof(BkSmem<D>);
   bwd_kv_local_kernel<D><<<dim3(d.n_blocks, d.n_kv_heads), kBkThreads, sm, s>>>(p);
   bwd_kv_cmp_kernel<D><<<dim3((d.n_blocks + 63) / 64, d.n_kv_heads, kBwdSplits), kBkThreads, sm, s>>>(p);
@@ -700,7 +782,8 @@ lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const vo
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
                             unsigned char* ws_bwd, uint32_t* status, cudaStream_t s) {
-  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.n_blocks > 65535) return LSRM_ERR_UNSUPPORTED;
+  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.n_blocks > 65535 || 128 % (d.n_q_heads / d.n_kv_heads) != 0)
+    return LSRM_ERR_UNSUPPORTED;
   const BwdWs w = bwd_layout(d, idx_heads);
   BwdParams p{};
   p.off = off;
