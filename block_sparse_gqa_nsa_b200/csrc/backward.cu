@@ -18,6 +18,8 @@
 //   bwd_finish:  dK = local part + (sum of the splits' dKbar of the token's block) / n_block.
 // The key-side passes compute S^T and dP^T (keys x query rows) directly, so P^T and dS^T are
 // already in the A-operand layout of the dV and dK products.
+#include <type_traits>
+
 #include "lsrm_common.cuh"
 #include "tc_ptx.cuh"
 #include "tma_map.cuh"
@@ -323,6 +325,43 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       if (D == 32) return (uint32_t)(r * 64 + ((ch ^ ((r >> 1) & 3)) << 4));
       return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
     };
+    // P (pass A) or dS (pass B) of this half's 32 keys as bf16 pairs; S and dP are read 16
+    // columns at a time, the next quarter's loads issued before the current one is processed
+    auto chunk_pass = [&](auto mask_tag, auto pass_tag, int nv, int br, float l2, float gb, float dlt) {
+      constexpr bool kMask = decltype(mask_tag)::value;
+      constexpr bool kPassB = decltype(pass_tag)::value;
+      uint32_t sa[16], sb[16], da[16], db[16];
+      auto quarter_pass = [&](const uint32_t* sr, const uint32_t* dr, int qd) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float v2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 32 * h + 16 * qd + 2 * i + e;
+            bool kv = true;
+            if constexpr (kMask) {
+              kv = j < nv;
+              if (br == 2) kv = kv && j >= wlo && j <= whi;
+            }
+            float pr = fast_exp2(fmaf(__uint_as_float(sr[2 * i + e]), sc, -l2));
+            if constexpr (kMask) pr = kv ? pr : 0.f;
+            if constexpr (kPassB) pr *= fmaf(gb, __uint_as_float(dr[2 * i + e]), -dlt);
+            v2[e] = pr;
+          }
+          pk[i] = pack_bf16x2(v2[0], v2[1]);
+        }
+        tmem_st8(tbase + C::kColP + 16 * h + 8 * qd, pk);
+      };
+      tmem_ld16(tbase + C::kColS + 32 * h, sa);
+      if constexpr (kPassB) tmem_ld16(tbase + C::kColDP + 32 * h, da);
+      tmem_ld_wait();
+      tmem_ld16(tbase + C::kColS + 32 * h + 16, sb);
+      if constexpr (kPassB) tmem_ld16(tbase + C::kColDP + 32 * h + 16, db);
+      quarter_pass(sa, da, 0);
+      tmem_ld_wait();
+      quarter_pass(sb, db, 1);
+    };
     float delta = 0.f;
     for (int c = 0; c < seq.total; ++c) {
       int br, pass, local, start, nv;
@@ -335,28 +374,13 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       const float l2 = br == 0 ? lse2[0] : (br == 1 ? lse2[1] : lse2[2]);
       const float gb = br == 0 ? gate[0] : (br == 1 ? gate[1] : gate[2]);
       const bool need_mask = br == 2 || nv < 32 * (h + 1);
-      uint32_t s[32], dp[32];
-      tmem_ld32(tbase + C::kColS + 32 * h, s);
-      if (pass) tmem_ld32(tbase + C::kColDP + 32 * h, dp);
-      tmem_ld_wait();
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float v2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = 32 * h + 2 * i + e;
-          bool kv = true;
-          if (need_mask) {
-            kv = j < nv;
-            if (br == 2) kv = kv && j >= wlo && j <= whi;
-          }
-          const float pr = kv ? fast_exp2(fmaf(__uint_as_float(s[2 * i + e]), sc, -l2)) : 0.f;
-          v2[e] = pass ? pr * fmaf(gb, __uint_as_float(dp[2 * i + e]), -delta) : pr;
-        }
-        pk[i] = pack_bf16x2(v2[0], v2[1]);
+      if (need_mask) {
+        if (pass) chunk_pass(std::true_type{}, std::true_type{}, nv, br, l2, gb, delta);
+        else chunk_pass(std::true_type{}, std::false_type{}, nv, br, l2, gb, delta);
+      } else {
+        if (pass) chunk_pass(std::false_type{}, std::true_type{}, nv, br, l2, gb, delta);
+        else chunk_pass(std::false_type{}, std::false_type{}, nv, br, l2, gb, delta);
       }
-      tmem_st16(tbase + C::kColP + 16 * h, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&S.p_full);
