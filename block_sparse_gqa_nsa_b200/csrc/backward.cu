@@ -26,7 +26,6 @@
 
 namespace lsrm {
 
-constexpr int kBkThreads = 128;   // 4 warps x 16 keys
 
 template <int D>
 __device__ __forceinline__ uint32_t bswz(int row, int ch) {
@@ -446,261 +445,358 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
 }
 
 // ------------------------------------------------------------------------------------------------
-// key passes: S^T = K Q^T, dP^T = V G^T for 64 keys (4 warps x 16) against query rows staged
-// 64 at a time and consumed in 16-row sub-tiles
+// key passes on the tensor cores.  The keys are the M dimension: a CTA holds a 128-row key tile
+// (128 block means for the compressed branch; one block's <= 64 tokens, padded, for the selected
+// and window branches) and streams the query rows that attend to it in chunks of 64:
+//   S^T = K Q^T and dP^T = V dO^T  ([128 x 64], K-major operands from shared memory)
+//   P^T = exp(tau S^T - lse) per query row, Pg = P^T g, dS^T = P^T (g dP^T - Delta)
+//   dV += Pg dO and dK += dS^T Q   ([128 x D], A from tensor memory, MN-major B)
+// The per-row constants (lse in log2 units, gate, Delta, token position) of each chunk are
+// staged next to its Q and dO tiles by the producer warp.
+//   compressed: CTA = (128 block means, group, query split), rows = the split's tokens x G heads
+//   local:      CTA = (key block j, group), rows = the query blocks that routed to j (ascending,
+//               selected branch), then block j itself (window branch)
+// TMEM: S^T [0, 64) | dP^T [64, 128) | Pg [128, 160) | dS^T [160, 192) | dV | dK
 // ------------------------------------------------------------------------------------------------
-constexpr int kBkRows = 64;
+constexpr int kKvThreads = 320;
 
 template <int D>
-struct BkSmem {
-  uint16_t kt[64 * D];
-  uint16_t vt[64 * D];
-  uint16_t q[kBkRows * D];
-  uint16_t g[kBkRows * D];  // G_b = g_b dO rows
-  float lse2[kBkRows];      // log2-unit LSE of the rows
-  float dlt[kBkRows];
-  int tok[kBkRows];         // query token position inside its block (window mask), -1 = invalid row
+struct KvCfg {
+  static constexpr int kRowsPerChunk = 64;
+  static constexpr int kStages = 4;
+  static constexpr int kTmemCols = D == 32 ? 256 : 512;
+  static constexpr int kCtasPerSm = D == 32 ? 2 : 1;
+  static constexpr int kColS = 0, kColDP = 64, kColPg = 128, kColDS = 160, kColDV = 192, kColDK = 192 + D;
+  static constexpr int kRowBytes = D * 2;
+  static constexpr uint32_t kLayout = D == 32 ? tc::kLayoutSW64 : tc::kLayoutSW128;
+  static constexpr uint32_t kAtomBytes = 8 * kRowBytes;
+  static constexpr int kKeyBytes = 128 * kRowBytes;
+  static constexpr int kChunkBytes = kRowsPerChunk * kRowBytes;
+  static constexpr uint32_t kIdescNR = tc::idesc_bf16(128, kRowsPerChunk, false);  // [keys x rows]
+  static constexpr uint32_t kIdescND = tc::idesc_bf16(128, D, true);               // [keys x D]
+  static_assert(kColDK + D <= kTmemCols, "tensor memory budget");
 };
 
-// A fragments of the warp's 16 keys (K and V)
 template <int D>
-__device__ __forceinline__ void bk_key_frags(const BkSmem<D>& S, int warp, int lane, uint32_t (&ka)[D / 16][4],
-                                             uint32_t (&va)[D / 16][4]) {
-#pragma unroll
-  for (int kt = 0; kt < D / 16; ++kt) {
-    const int r = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-    const int ch = kt * 2 + (lane >> 4);
-    ldmatrix_x4(ka[kt][0], ka[kt][1], ka[kt][2], ka[kt][3], smem_u32(S.kt) + bswz<D>(r, ch));
-    ldmatrix_x4(va[kt][0], va[kt][1], va[kt][2], va[kt][3], smem_u32(S.vt) + bswz<D>(r, ch));
-  }
-}
+struct KvSmem {
+  using C = KvCfg<D>;
+  uint8_t kt[C::kKeyBytes];  // key tile (K), 128 rows
+  uint8_t vt[C::kKeyBytes];  // key tile (V)
+  uint8_t q[C::kStages][C::kChunkBytes];
+  uint8_t go[C::kStages][C::kChunkBytes];  // dO rows
+  float4 rv[C::kStages][64];               // per query row: lse (log2), gate, Delta, token position
+  int br[C::kStages];                      // branch of the chunk in each stage
+  uint64_t key_full, full[C::kStages], empty[C::kStages], s_full, p_full, pv_done, drain;
+  uint32_t tmem_base;
+  int abort;
+  int total;
+};
 
-// accumulate the staged rows [sub*16, sub*16+16) into the warp's dK / dV (16 keys x D)
-template <int D, bool kWindow>
-__device__ __forceinline__ void bk_tile(const BkSmem<D>& S, int sub, int lane, int key_valid, const int (&key_pos)[2],
-                                        int window, float scale_log2, const uint32_t (&ka)[D / 16][4],
-                                        const uint32_t (&va)[D / 16][4], float (&dk)[D / 8][4],
-                                        float (&dv)[D / 8][4]) {
-  constexpr int KT = D / 16;
-  const int gq = lane >> 2, cq = lane & 3;
-  const int rb = sub * 16;
-  float st[2][4], dpt[2][4];  // [row n-tile][frag]: rows = keys gq, gq+8; cols = query rows 8 n + 2 cq (+1)
-#pragma unroll
-  for (int n = 0; n < 2; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) { st[n][e] = 0.f; dpt[n][e] = 0.f; }
-#pragma unroll
-  for (int kt = 0; kt < KT; ++kt) {
-    uint32_t b0, b1, b2, b3;
-    const int r = rb + (lane >> 4) * 8 + (lane & 7);
-    const int ch = kt * 2 + ((lane >> 3) & 1);
-    ldmatrix_x4(b0, b1, b2, b3, smem_u32(S.q) + bswz<D>(r, ch));
-    const uint32_t q0[2] = {b0, b1}, q1[2] = {b2, b3};
-    mma_bf16_16816(st[0], ka[kt], q0);
-    mma_bf16_16816(st[1], ka[kt], q1);
-    ldmatrix_x4(b0, b1, b2, b3, smem_u32(S.g) + bswz<D>(r, ch));
-    const uint32_t g0[2] = {b0, b1}, g1[2] = {b2, b3};
-    mma_bf16_16816(dpt[0], va[kt], g0);
-    mma_bf16_16816(dpt[1], va[kt], g1);
-  }
-  // P^T and dS^T (keys x rows), masked
-  uint32_t pa[4], da[4];
-#pragma unroll
-  for (int n = 0; n < 2; ++n) {
-    float pv[4], dv4[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int krow = gq + 8 * (e >> 1);             // key of the warp tile
-      const int qrow = rb + n * 8 + 2 * cq + (e & 1);  // staged query row
-      const int r = S.tok[qrow];
-      bool ok = krow < key_valid && r >= 0;
-      if (kWindow) {
-        const int u = key_pos[e >> 1];
-        ok = ok && u >= r - window / 2 && u <= r + window / 2 - 1;
-      }
-      const float pp = ok ? fast_exp2(st[n][e] * scale_log2 - S.lse2[qrow]) : 0.f;
-      pv[e] = pp;
-      dv4[e] = pp * (dpt[n][e] - S.dlt[qrow]);
-    }
-    pa[n * 2 + 0] = pack_bf16x2(pv[0], pv[1]);
-    pa[n * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-    da[n * 2 + 0] = pack_bf16x2(dv4[0], dv4[1]);
-    da[n * 2 + 1] = pack_bf16x2(dv4[2], dv4[3]);
-  }
-  // dV += P^T G, dK += dS^T Q (B operands: staged rows of G / Q, transposed loads)
-#pragma unroll
-  for (int dn = 0; dn < D / 16; ++dn) {
-    uint32_t b0, b1, b2, b3;
-    const int r = rb + ((lane >> 3) & 1) * 8 + (lane & 7);
-    const int ch = dn * 2 + (lane >> 4);
-    ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(S.g) + bswz<D>(r, ch));
-    const uint32_t g0[2] = {b0, b1}, g1[2] = {b2, b3};
-    mma_bf16_16816(dv[2 * dn], pa, g0);
-    mma_bf16_16816(dv[2 * dn + 1], pa, g1);
-    ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(S.q) + bswz<D>(r, ch));
-    const uint32_t q0[2] = {b0, b1}, q1[2] = {b2, b3};
-    mma_bf16_16816(dk[2 * dn], da, q0);
-    mma_bf16_16816(dk[2 * dn + 1], da, q1);
-  }
-}
+// walks the query-row chunks of a key tile in order
+struct KvCursor {
+  int e = 0, r0 = 0;  // entry (query block or split), first row of the chunk within it
+};
 
-// stage kBkRows query rows (row0.. of the token range starting at t_base) of group g for branch br;
-// G_b = g_b dO is formed here, rounded to bf16
-template <int D>
-__device__ __forceinline__ void bk_stage_rows(BkSmem<D>& S, const BwdParams& p, int g, int br, int row0,
-                                              int rows_total, long long t_base, int tid) {
-  constexpr int CPR = D / 8;
-  for (int e = tid; e < kBkRows * CPR; e += kBkThreads) {
-    const int r = e / CPR, ch = e % CPR;
-    const int rr = row0 + r;
-    const bool ok = rr < rows_total;
-    const long long t = t_base + (ok ? rr / p.G : 0);
-    const int h = g * p.G + (ok ? rr % p.G : 0);
-    const size_t src = ((size_t)t * p.Hq + h) * D + ch * 8;
-    cp_async16(reinterpret_cast<unsigned char*>(S.q) + bswz<D>(r, ch), p.q + src, ok);
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (ok) {
-      const float gt = bf16_to_f32(p.gates[((size_t)t * p.Hq + h) * p.NG + br]);
-      const uint4 dd = *reinterpret_cast<const uint4*>(p.dout + src);
-      const uint32_t w[4] = {dd.x, dd.y, dd.z, dd.w};
-      uint32_t o4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        o4[i] = pack_bf16x2(__uint_as_float(w[i] << 16) * gt, __uint_as_float(w[i] & 0xFFFF0000u) * gt);
-      u = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-    }
-    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.g) + bswz<D>(r, ch)) = u;
-  }
-  for (int r = tid; r < kBkRows; r += kBkThreads) {
-    const int rr = row0 + r;
-    if (rr < rows_total) {
-      const long long t = t_base + rr / p.G;
-      const int h = g * p.G + rr % p.G;
-      const size_t row = (size_t)t * p.Hq + h;
-      S.lse2[r] = p.lse[row * p.NG + br] * 1.4426950408889634f;
-      S.dlt[r] = p.delta[row * p.NG + br];
-      S.tok[r] = rr / p.G;
-    } else {
-      S.lse2[r] = 0.f;
-      S.dlt[r] = 0.f;
-      S.tok[r] = -1;
-    }
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-}
-
-template <int D>
-__device__ __forceinline__ void bk_load_keys(BkSmem<D>& S, const uint16_t* k, const uint16_t* v, long long first,
-                                             int n_keys, int Hkv, int g, int tid) {
-  constexpr int CPR = D / 8;
-  for (int e = tid; e < 64 * CPR; e += kBkThreads) {
-    const int r = e / CPR, ch = e % CPR;
-    const bool ok = r < n_keys;
-    const size_t src = ((size_t)(first + (ok ? r : 0)) * Hkv + g) * D + ch * 8;
-    cp_async16(reinterpret_cast<unsigned char*>(S.kt) + bswz<D>(r, ch), k + src, ok);
-    cp_async16(reinterpret_cast<unsigned char*>(S.vt) + bswz<D>(r, ch), v + src, ok);
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-}
-
-// store the warp's 16 rows of dK (scaled by tau) and dV as fp32 into [row][Hkv][D] at dst_row0
-template <int D>
-__device__ __forceinline__ void bk_store(float* dkp, float* dvp, size_t dst_row0, int n_keys, int warp, int lane,
-                                         int Hkv, int g, float tau, const float (&dk)[D / 8][4],
-                                         const float (&dv)[D / 8][4]) {
-  const int gq = lane >> 2, cq = lane & 3;
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int kr = warp * 16 + gq + 8 * i;
-    if (kr >= n_keys) continue;
-    const size_t row = ((dst_row0 + kr) * Hkv + g) * D;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      *reinterpret_cast<float2*>(dkp + row + n * 8 + 2 * cq) = make_float2(tau * dk[n][2 * i], tau * dk[n][2 * i + 1]);
-      *reinterpret_cast<float2*>(dvp + row + n * 8 + 2 * cq) = make_float2(dv[n][2 * i], dv[n][2 * i + 1]);
-    }
-  }
-}
-
-// selected + window parts of dK, dV for the tokens of key block j, group g
-template <int D>
-__global__ void __launch_bounds__(kBkThreads) bwd_kv_local_kernel(const BwdParams p) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  BkSmem<D>& S = *reinterpret_cast<BkSmem<D>*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int j = blockIdx.x, g = blockIdx.y;
-  const int u0 = p.off[j], n_j = min(64, p.off[j + 1] - u0);
-  bk_load_keys<D>(S, p.k, p.v, u0, n_j, p.Hkv, g, tid);
-  __syncthreads();
-  uint32_t ka[D / 16][4], va[D / 16][4];
-  bk_key_frags<D>(S, warp, lane, ka, va);
-  const int key_valid = n_j - warp * 16;  // valid keys among this warp's 16
-  const int gq = lane >> 2;
-  const int key_pos[2] = {warp * 16 + gq, warp * 16 + gq + 8};
-  float dk[D / 8][4], dv[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) { dk[n][e] = 0.f; dv[n][e] = 0.f; }
-  // selected branch: every query block whose routed set contains j, in ascending order; the
-  // last pass is the window branch of block j itself
-  const int list = p.idx_heads == 1 ? j : j * p.Hkv + g;
-  const int l0 = p.inv_start[list], l1 = p.inv_start[list + 1];
-  const int l_end = p.window > 0 ? l1 + 1 : l1;
-  for (int li = l0; li < l_end; ++li) {
-    const bool window = li == l1;
-    const int a = window ? j : p.inv_list[li];
-    const int br = window ? 2 : 1;
-    const int t_base = p.off[a], rows_total = (p.off[a + 1] - t_base) * p.G;
-    for (int row0 = 0; row0 < rows_total; row0 += kBkRows) {
-      __syncthreads();
-      bk_stage_rows<D>(S, p, g, br, row0, rows_total, t_base, tid);
-      __syncthreads();
-      const int subs = min(4, (rows_total - row0 + 15) / 16);
-      for (int sub = 0; sub < subs; ++sub) {
-        if (window)
-          bk_tile<D, true>(S, sub, lane, key_valid, key_pos, p.window, p.scale_log2, ka, va, dk, dv);
-        else
-          bk_tile<D, false>(S, sub, lane, key_valid, key_pos, p.window, p.scale_log2, ka, va, dk, dv);
-      }
-    }
-  }
-  bk_store<D>(p.dk_tok, p.dv_tok, (size_t)u0, n_j, warp, lane, p.Hkv, g, p.tau, dk, dv);
-}
-
-// compressed part: partial dKbar / dVbar of 64 block means of group g over one split of the query tokens
-template <int D>
-__global__ void __launch_bounds__(kBkThreads) bwd_kv_cmp_kernel(const BwdParams p) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  BkSmem<D>& S = *reinterpret_cast<BkSmem<D>*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int jc = blockIdx.x, g = blockIdx.y, split = blockIdx.z;
-  const int j0 = jc * 64, n_j = min(64, p.B - j0);
-  bk_load_keys<D>(S, p.kc, p.vc, j0, n_j, p.Hkv, g, tid);
-  __syncthreads();
-  uint32_t ka[D / 16][4], va[D / 16][4];
-  bk_key_frags<D>(S, warp, lane, ka, va);
-  const int key_valid = n_j - warp * 16;
-  const int key_pos[2] = {0, 0};
-  float dk[D / 8][4], dv[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) { dk[n][e] = 0.f; dv[n][e] = 0.f; }
-  // this split's query tokens (all heads of group g), rows token-major with G rows per token
+template <int D, bool kLocal>
+__global__ void __launch_bounds__(kKvThreads, KvCfg<D>::kCtasPerSm)
+bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                 const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap,
+                 const BwdParams p) {
+  using namespace tc;
+  using C = KvCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  KvSmem<D>& S = *reinterpret_cast<KvSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.y;
+  // the key tile
+  const int j = blockIdx.x;
+  const int key0 = kLocal ? p.off[j] : j * 128;
+  const int n_keys = kLocal ? min(64, p.off[j + 1] - key0) : min(128, p.B - key0);
+  // the query-row entries: one token range (compressed), or the routed query blocks then j itself
+  const int split = blockIdx.z;
   const long long t_lo = p.N * split / kBwdSplits, t_hi = p.N * (split + 1) / kBwdSplits;
-  const int rows_total = (int)((t_hi - t_lo) * p.G);
-  for (int row0 = 0; row0 < rows_total; row0 += kBkRows) {
-    __syncthreads();
-    bk_stage_rows<D>(S, p, g, 0, row0, rows_total, t_lo, tid);
-    __syncthreads();
-    const int subs = min(4, (rows_total - row0 + 15) / 16);
-    for (int sub = 0; sub < subs; ++sub)
-      bk_tile<D, false>(S, sub, lane, key_valid, key_pos, 0, p.scale_log2, ka, va, dk, dv);
+  int l0 = 0, n_sel_e = 0;
+  if (kLocal) {
+    const int list = p.idx_heads == 1 ? j : j * p.Hkv + g;
+    l0 = p.inv_start[list];
+    n_sel_e = p.inv_start[list + 1] - l0;
   }
-  bk_store<D>(p.dkc_part, p.dvc_part, (size_t)split * p.B + j0, n_j, warp, lane, p.Hkv, g, p.tau, dk, dv);
+  const int n_entries = kLocal ? n_sel_e + (p.window > 0 ? 1 : 0) : 1;
+  // entry e: branch, first token, rows (tokens x G)
+  auto entry = [&](int e, int& br, int& t0a, int& rows) {
+    if (!kLocal) {
+      br = 0;
+      t0a = (int)t_lo;
+      rows = (int)(t_hi - t_lo) * p.G;
+    } else {
+      const int a = e < n_sel_e ? p.inv_list[l0 + e] : j;
+      br = e < n_sel_e ? 1 : 2;
+      t0a = p.off[a];
+      rows = (p.off[a + 1] - t0a) * p.G;
+    }
+  };
+  auto skip_empty = [&](KvCursor& cu) {
+    int br, t0a, rows;
+    while (cu.e < n_entries) {
+      entry(cu.e, br, t0a, rows);
+      if (cu.r0 < rows) break;
+      ++cu.e;
+      cu.r0 = 0;
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    S.abort = 0;
+    int total = 0;
+    for (int e = 0; e < n_entries; ++e) {
+      int br, t0a, rows;
+      entry(e, br, t0a, rows);
+      total += (rows + C::kRowsPerChunk - 1) / C::kRowsPerChunk;
+    }
+    S.total = n_keys > 0 ? total : 0;
+    mbar_init(&S.key_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&S.full[s], 1 + 32);  // the TMA byte count, and every producer lane's row constants
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.s_full, 1);
+    mbar_init(&S.p_full, kLocal ? 128 : 256);  // local tiles have 64 keys: lane quarters 0 and 1
+    mbar_init(&S.pv_done, 1);
+    mbar_init(&S.drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  const int total = S.total;
+  volatile int* abort = &S.abort;
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const bool w = mbar_wait(bar, parity, abort, p.status);
+    return __all_sync(0xffffffffu, w);
+  };
+
+  if (warp == 0) {
+    // ---------------- producer warp: key tile once, then Q / dO chunks with their row constants ----------------
+    if (total > 0) {
+      if (lane == 0) {
+        const int key_rows = kLocal ? 64 : 128;
+        mbar_arrive_expect_tx(&S.key_full, 2 * key_rows * C::kRowBytes);
+        tma_load_3d(S.kt, &kmap, &S.key_full, 0, g, key0);
+        tma_load_3d(S.vt, &vmap, &S.key_full, 0, g, key0);
+      }
+      KvCursor cu;
+      skip_empty(cu);
+      int issued = 0;
+      for (int c = 0; c < total; ++c) {
+        const int st = c % C::kStages;
+        if (c >= C::kStages && !wait_all(&S.empty[st], ((c / C::kStages) + 1) & 1)) break;
+        int br, t0a, rows;
+        entry(cu.e, br, t0a, rows);
+        const int rows_valid = min(C::kRowsPerChunk, rows - cu.r0);
+        const int t_first = t0a + cu.r0 / p.G;
+        if (lane == 0) {
+          S.br[st] = br;
+          mbar_arrive_expect_tx(&S.full[st], 2 * C::kChunkBytes);
+          tma_load_3d(S.q[st], &qmap, &S.full[st], 0, g * p.G, t_first);
+          tma_load_3d(S.go[st], &omap, &S.full[st], 0, g * p.G, t_first);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int rr = lane + 32 * k;
+          float4 v = make_float4(INFINITY, 0.f, 0.f, __int_as_float(INT_MIN / 2));
+          if (rr < rows_valid) {
+            const int t = t_first + rr / p.G;
+            const size_t orow = (size_t)t * p.Hq + g * p.G + rr % p.G;
+            v = make_float4(p.lse[orow * p.NG + br] * 1.4426950408889634f, bf16_to_f32(p.gates[orow * p.NG + br]),
+                            p.delta[orow * p.NG + br], __int_as_float(t - t0a));
+          }
+          S.rv[st][rr] = v;
+        }
+        mbar_arrive(&S.full[st]);
+        issued = c + 1;
+        cu.r0 += C::kRowsPerChunk;
+        skip_empty(cu);
+      }
+      if (lane == 0 && *abort) {
+        volatile int no_abort = 0;
+        mbar_wait(&S.key_full, 0, &no_abort, nullptr);
+        for (int c = max(0, issued - C::kStages); c < issued; ++c)
+          mbar_wait(&S.full[c % C::kStages], (c / C::kStages) & 1, &no_abort, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && total > 0) {
+      bool ok = mbar_wait(&S.key_full, 0, abort, p.status);
+      const uint32_t kaddr = smem_u32(S.kt), vaddr = smem_u32(S.vt);
+      auto first_stage = [&](int c) {
+        const int st = c % C::kStages;
+        const uint32_t qa = smem_u32(S.q[st]), oa = smem_u32(S.go[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::kColS, smem_desc(kaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
+                 smem_desc(qa + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNR, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::kColDP, smem_desc(vaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
+                 smem_desc(oa + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNR, kk > 0 ? 1u : 0u);
+        mma_commit(&S.s_full);
+      };
+      auto second_stage = [&](int c) {
+        const int st = c % C::kStages;
+        const uint32_t qa = smem_u32(S.q[st]), oa = smem_u32(S.go[st]);
+#pragma unroll
+        for (int kk = 0; kk < C::kRowsPerChunk / 16; ++kk) {
+          const uint32_t acc = (c == 0 && kk == 0) ? 0u : 1u;
+          mma_ts(tmem + C::kColDV, tmem + C::kColPg + 8 * kk,
+                 smem_desc(oa + kk * 16 * C::kRowBytes, C::kChunkBytes, C::kAtomBytes, C::kLayout), C::kIdescND, acc);
+          mma_ts(tmem + C::kColDK, tmem + C::kColDS + 8 * kk,
+                 smem_desc(qa + kk * 16 * C::kRowBytes, C::kChunkBytes, C::kAtomBytes, C::kLayout), C::kIdescND, acc);
+        }
+        mma_commit(&S.pv_done);
+        mma_commit(&S.empty[st]);
+      };
+      for (int c = 0; ok && c < total; ++c) {
+        if (!mbar_wait(&S.full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        if (c > 0) {
+          if (!mbar_wait(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+          second_stage(c - 1);
+        }
+        tc_fence_after();
+        first_stage(c);
+      }
+      if (ok && mbar_wait(&S.p_full, (total - 1) & 1, abort, p.status)) {
+        tc_fence_after();
+        second_stage(total - 1);
+      }
+      mma_commit(&S.drain);
+      volatile int no_abort = 0;
+      mbar_wait(&S.drain, 0, &no_abort, nullptr);
+    }
+  } else {
+    // ---------------- element-wise warps: one thread per key, 32 of the chunk's 64 rows ----------------
+    const int h = (warp - 2) >> 2;  // row half: rows [32 h, 32 h + 32) of every chunk
+    const int quarter = warp & 3;
+    const int key = quarter * 32 + lane;  // key of the tile = TMEM lane
+    const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
+    const bool active = !kLocal || quarter < 2;
+    const float sc = p.scale_log2;
+    const int wh = p.window / 2;
+    int pv_seen = 0;
+    auto pv_wait_through = [&](int jj) -> bool {
+      while (pv_seen <= jj) {
+        if (!wait_all(&S.pv_done, pv_seen & 1)) return false;
+        ++pv_seen;
+      }
+      tc_fence_after();
+      return true;
+    };
+    auto chunk_pass = [&](int st, auto window_tag) {
+      constexpr bool kWindow = decltype(window_tag)::value;
+      uint32_t sa[16], sb[16], da[16], db[16];
+      auto quarter_pass = [&](const uint32_t* sr, const uint32_t* dr, int qd) {
+        uint32_t pg[8], ds[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float a2[2], b2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 rv = S.rv[st][32 * h + 16 * qd + 2 * i + e];
+            float pr = fast_exp2(fmaf(__uint_as_float(sr[2 * i + e]), sc, -rv.x));
+            if constexpr (kWindow) {
+              const int tp = __float_as_int(rv.w);
+              pr = (key >= tp - wh && key <= tp + wh - 1) ? pr : 0.f;
+            }
+            a2[e] = pr * rv.y;
+            b2[e] = pr * fmaf(rv.y, __uint_as_float(dr[2 * i + e]), -rv.z);
+          }
+          pg[i] = pack_bf16x2(a2[0], a2[1]);
+          ds[i] = pack_bf16x2(b2[0], b2[1]);
+        }
+        tmem_st8(tbase + C::kColPg + 16 * h + 8 * qd, pg);
+        tmem_st8(tbase + C::kColDS + 16 * h + 8 * qd, ds);
+      };
+      tmem_ld16(tbase + C::kColS + 32 * h, sa);
+      tmem_ld16(tbase + C::kColDP + 32 * h, da);
+      tmem_ld_wait();
+      tmem_ld16(tbase + C::kColS + 32 * h + 16, sb);
+      tmem_ld16(tbase + C::kColDP + 32 * h + 16, db);
+      quarter_pass(sa, da, 0);
+      tmem_ld_wait();
+      quarter_pass(sb, db, 1);
+    };
+    bool ok = active;
+    for (int c = 0; ok && c < total; ++c) {
+      if (!wait_all(&S.s_full, c & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (!pv_wait_through(c - 1)) { ok = false; break; }  // Pg and dS columns are free again
+      const int st = c % C::kStages;
+      if (kLocal && S.br[st] == 2) chunk_pass(st, std::true_type{});
+      else chunk_pass(st, std::false_type{});
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&S.p_full);
+    }
+    if (active && h == 0) {
+      float* dkp;
+      float* dvp;
+      size_t rowi;
+      if (kLocal) {
+        dkp = p.dk_tok;
+        dvp = p.dv_tok;
+        rowi = ((size_t)(key0 + key) * p.Hkv + g) * D;
+      } else {
+        dkp = p.dkc_part;
+        dvp = p.dvc_part;
+        rowi = (((size_t)split * p.B + key0 + key) * p.Hkv + g) * D;
+      }
+      const bool store = key < n_keys;
+      if (total == 0) {
+        if (store)
+          for (int i = 0; i < D; ++i) {
+            dkp[rowi + i] = 0.f;
+            dvp[rowi + i] = 0.f;
+          }
+      } else if (ok && pv_wait_through(total - 1)) {  // warp-uniform: the loads are .sync.aligned
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) {
+          uint32_t o[32];
+          tmem_ld32(tbase + C::kColDK + 32 * i, o);
+          tmem_ld_wait();
+          if (store) {
+            float4* dst = reinterpret_cast<float4*>(dkp + rowi + 32 * i);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(p.tau * __uint_as_float(o[4 * e]), p.tau * __uint_as_float(o[4 * e + 1]),
+                                   p.tau * __uint_as_float(o[4 * e + 2]), p.tau * __uint_as_float(o[4 * e + 3]));
+          }
+          tmem_ld32(tbase + C::kColDV + 32 * i, o);
+          tmem_ld_wait();
+          if (store) {
+            float4* dsv = reinterpret_cast<float4*>(dvp + rowi + 32 * i);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dsv[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                   __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
 
 // dK = local part + (sum over splits of dKbar of the token's block) / n_block, as bf16
@@ -794,9 +890,22 @@ static lsrm_status launch_backward_d(const lsrm_nsa_desc& d, const BwdParams& p,
       cudaSuccess)
     return LSRM_ERR_CUDA;
   bwd_query_tc_kernel<D><<<dim3(tiles, d.n_kv_heads, d.n_blocks), kBqtThreads, sm, s>>>(qm, om, km, vm, kcm, vcm, p);
-  sm = sizeof(BkSmem<D>);
-  bwd_kv_local_kernel<D><<<dim3(d.n_blocks, d.n_kv_heads), kBkThreads, sm, s>>>(p);
-  bwd_kv_cmp_kernel<D><<<dim3((d.n_blocks + 63) / 64, d.n_kv_heads, kBwdSplits), kBkThreads, sm, s>>>(p);
+  CUtensorMap k64, v64, kc128, vc128, q64, o64;
+  if (!make_map(&k64, p.k, D, d.n_kv_heads, d.n_tokens, 1, 64) || !make_map(&v64, p.v, D, d.n_kv_heads, d.n_tokens, 1, 64) ||
+      !make_map(&kc128, p.kc, D, d.n_kv_heads, d.n_blocks, 1, 128) ||
+      !make_map(&vc128, p.vc, D, d.n_kv_heads, d.n_blocks, 1, 128) ||
+      !make_map(&q64, p.q, D, d.n_q_heads, d.n_tokens, G, 64 / G) ||
+      !make_map(&o64, p.dout, D, d.n_q_heads, d.n_tokens, G, 64 / G))
+    return LSRM_ERR_CUDA;
+  sm = sizeof(KvSmem<D>) + 1024;
+  if (cudaFuncSetAttribute(bwd_kv_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bwd_kv_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+          cudaSuccess)
+    return LSRM_ERR_CUDA;
+  bwd_kv_tc_kernel<D, true><<<dim3(d.n_blocks, d.n_kv_heads, 1), kKvThreads, sm, s>>>(k64, v64, q64, o64, p);
+  bwd_kv_tc_kernel<D, false><<<dim3((d.n_blocks + 127) / 128, d.n_kv_heads, kBwdSplits), kKvThreads, sm, s>>>(
+      kc128, vc128, q64, o64, p);
   bwd_finish_kernel<<<d.n_blocks, 256, 0, s>>>(p, D);
   (void)idx_heads;
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
@@ -806,7 +915,7 @@ lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const vo
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
                             unsigned char* ws_bwd, uint32_t* status, cudaStream_t s) {
-  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.n_blocks > 65535 || 128 % (d.n_q_heads / d.n_kv_heads) != 0)
+  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.n_blocks > 65535 || 64 % (d.n_q_heads / d.n_kv_heads) != 0)
     return LSRM_ERR_UNSUPPORTED;
   const BwdWs w = bwd_layout(d, idx_heads);
   BwdParams p{};
