@@ -48,7 +48,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-sample-blocks", type=int, default=None,
-                    help="query blocks of the oracle's bounded CPU sample (default 64 forward, 8 backward: "
+                    help="query blocks of the oracle's bounded CPU sample (default 64 forward, 24 backward: "
                          "10-20 s of one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -85,8 +85,8 @@ def backward_flops(fwd: dict) -> dict:
     return {k: 2.5 * v for k, v in fwd.items()}
 
 
-KERNEL_SOURCES = {"attn": ["attn_tc.cu", "tc_ptx.cuh", "lsrm_common.cuh"],
-                  "bwd": ["backward.cu", "lsrm_common.cuh"]}
+KERNEL_SOURCES = {"attn": ["attn_tc.cu", "tc_ptx.cuh", "tma_map.cuh", "lsrm_common.cuh"],
+                  "bwd": ["backward.cu", "tc_ptx.cuh", "tma_map.cuh", "lsrm_common.cuh"]}
 
 
 def kernel_source_hash(which: str) -> str:
@@ -577,7 +577,7 @@ def run_backward(args):
                              "peak_source": f"{src} bf16_tflops (burst)"},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "e2e": e2e}
         if not args.no_cpu_baseline and world == 1:
-            n_blk = args.cpu_sample_blocks or 8
+            n_blk = args.cpu_sample_blocks or 24
             tok, dt = oracle_backward_sample(w, idx.view(B, k).cpu().numpy(), n_blk, 7)
             line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                     "sample": f"{n_blk} seeded query blocks ({tok} tokens) of the same workload, "
