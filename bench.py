@@ -113,6 +113,22 @@ def profiled_traffic(which: str):
     return float(m.group(1))
 
 
+def max_over_ranks(ms: float, device, world: int) -> float:
+    """The slowest rank's time: every rank contributes its device-measured milliseconds and all
+    receive the maximum (one all-reduce; a no-op on one rank)."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(world: int, units_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job units per second: every rank processes units_per_rank per step (replicas)."""
+    return world * units_per_rank * steps / (max_ms / 1000.0)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -302,12 +318,9 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
     pre_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev, world)
     ms_per_step = total_ms / args.steps
-    value = world * N * args.steps / (total_ms / 1000.0)
+    value = throughput(world, N, args.steps, total_ms)
 
     # end to end through lsrm_nsa_forward with pinned host buffers
     e2e = None
@@ -337,12 +350,10 @@ def run_ours(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te = max_over_ranks(e0.elapsed_time(e1), dev, world)
         h2d = sum(src.numel() * src.element_size() for _, src in ins)
         d2h = p_out.numel() * p_out.element_size()
-        e2e = {"value": world * N * args.steps / (float(te.item()) / 1000.0), "unit": "tokens/s",
+        e2e = {"value": throughput(world, N, args.steps, te), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
         if not np.array_equal(p_out.view(torch.int16).numpy(), out.view(torch.int16).cpu().numpy()):
             raise RuntimeError("end-to-end output differs from the device-resident run")
@@ -512,12 +523,9 @@ def run_backward(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
-    tt = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    total_ms = float(tt.item())
+    total_ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
     call_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    value = world * N * args.steps / (total_ms / 1000.0)
+    value = throughput(world, N, args.steps, total_ms)
 
     e2e = None
     if not args.no_e2e:
@@ -549,13 +557,11 @@ def run_backward(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te = max_over_ranks(e0.elapsed_time(e1), dev, world)
         h2d = sum(t.numel() * t.element_size() for t in p_in.values()) + \
             h_idx.numel() * h_idx.element_size() + h_lse.numel() * h_lse.element_size()
         d2h = sum(t.numel() * t.element_size() for t in p_out.values())
-        e2e = {"value": world * N * args.steps / (float(te.item()) / 1000.0), "unit": "tokens/s",
+        e2e = {"value": throughput(world, N, args.steps, te), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
         for n in grads:
             if not torch.equal(p_out[n].view(torch.int16), grads[n].view(torch.int16).cpu()):
