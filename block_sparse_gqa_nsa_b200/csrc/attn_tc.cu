@@ -235,26 +235,27 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       bool ok = mbar_wait(&S.q_full[0], 0, abort, p.status) && mbar_wait(&S.q_full[1], 0, abort, p.status);
       tc_fence_after();
       const uint32_t qaddr[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
+      // shared-memory descriptors are computed once; a byte offset moves the start-address
+      // field (address / 16, bits 0..13; shared addresses stay below 2^18) by offset / 16
+      const uint64_t qdesc[2] = {smem_desc(qaddr[0], 16, C::kAtomBytes, C::kLayout),
+                                 smem_desc(qaddr[1], 16, C::kAtomBytes, C::kLayout)};
+      const uint64_t kdesc = smem_desc(smem_u32(S.k[0]), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t vdesc = smem_desc(smem_u32(S.v[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
+      constexpr uint32_t kStageStep = C::kKVBytes >> 4;
       auto issue_qk = [&](int t, int c) {
         const uint32_t d = tmem + t * C::kColsPerTile + C::kColS;
-        const uint32_t kaddr = smem_u32(S.k[c % C::kStages]);
+        const uint64_t bd = kdesc + (uint64_t)((c % C::kStages) * kStageStep);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t ad = smem_desc(qaddr[t] + k * 32, 16, C::kAtomBytes, C::kLayout);
-          const uint64_t bd = smem_desc(kaddr + k * 32, 16, C::kAtomBytes, C::kLayout);
-          mma_ss(d, ad, bd, C::kIdescQK, k > 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < D / 16; ++k) mma_ss(d, qdesc[t] + 2 * k, bd + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
       };
       auto issue_pv = [&](int t, int c) {
         const uint32_t d = tmem + t * C::kColsPerTile + C::kColO;
-        const uint32_t vaddr = smem_u32(S.v[c % C::kStages]);
+        const uint64_t bd = vdesc + (uint64_t)((c % C::kStages) * kStageStep);
         const bool first = cs.first_of_branch(c);
 #pragma unroll
-        for (int kk = 0; kk < C::kKeys / 16; ++kk) {
-          const uint32_t at = tmem + t * C::kColsPerTile + C::kColP + kk * 8;
-          const uint64_t bd = smem_desc(vaddr + kk * 16 * C::kRowBytes, C::kKVBytes, C::kAtomBytes, C::kLayout);
-          mma_ts(d, at, bd, C::kIdescPV, (first && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < C::kKeys / 16; ++kk)
+          mma_ts(d, tmem + t * C::kColsPerTile + C::kColP + kk * 8, bd + kk * (16 * C::kRowBytes >> 4), C::kIdescPV,
+                 (first && kk == 0) ? 0u : 1u);
       };
       for (int c = 0; ok && c < cs.total; ++c) {
         if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }

@@ -221,32 +221,34 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     // ---------------- MMA issuer ----------------
     if (lane == 0 && seq.total > 0) {
       bool ok = mbar_wait(&S.q_full, 0, abort, p.status);
-      const uint32_t qaddr = smem_u32(S.q), oaddr = smem_u32(S.go);
+      // descriptors computed once; a byte offset moves the start-address field by offset / 16
+      const uint64_t qd = smem_desc(smem_u32(S.q), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t od = smem_desc(smem_u32(S.go), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t kd_k = smem_desc(smem_u32(S.k[0]), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t vd_k = smem_desc(smem_u32(S.v[0]), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t kd_mn = smem_desc(smem_u32(S.k[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
+      const uint64_t vd_mn = smem_desc(smem_u32(S.v[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
+      constexpr uint32_t kStep = C::kKVBytes >> 4, kRow16 = (16 * C::kRowBytes) >> 4;
       // pass A: S = Q K^T;  pass B: S = Q K^T and dP = dO V^T  (both [128 x 64], K-major B)
       auto first_stage = [&](int c, int pass) {
-        const uint32_t kaddr = smem_u32(S.k[c % C::kStages]), vaddr = smem_u32(S.v[c % C::kStages]);
+        const uint64_t so = (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          mma_ss(tmem + C::kColS, smem_desc(qaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
-                 smem_desc(kaddr + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNK, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::kColS, qd + 2 * kk, kd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
         if (pass) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            mma_ss(tmem + C::kColDP, smem_desc(oaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
-                   smem_desc(vaddr + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNK, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + C::kColDP, od + 2 * kk, vd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
         }
         mma_commit(&S.s_full);
       };
       // pass A: O += P V;  pass B: dQ_b += dS K  (A from tensor memory, MN-major B)
       auto second_stage = [&](int c, int pass, bool first) {
-        const uint32_t baddr = smem_u32(pass ? S.k[c % C::kStages] : S.v[c % C::kStages]);
+        const uint64_t bd = (pass ? kd_mn : vd_mn) + (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
-        for (int kk = 0; kk < C::kKeys / 16; ++kk) {
-          const uint64_t bd = smem_desc(baddr + kk * 16 * C::kRowBytes, C::kKVBytes, C::kAtomBytes, C::kLayout);
-          mma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, bd, C::kIdescND, (first && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < C::kKeys / 16; ++kk)
+          mma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, bd + kk * kRow16, C::kIdescND,
+                 (first && kk == 0) ? 0u : 1u);
         mma_commit(&S.pv_done);
         mma_commit(&S.kv_empty[c % C::kStages]);
       };
@@ -634,30 +636,32 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     // ---------------- MMA issuer ----------------
     if (lane == 0 && total > 0) {
       bool ok = mbar_wait(&S.key_full, 0, abort, p.status);
-      const uint32_t kaddr = smem_u32(S.kt), vaddr = smem_u32(S.vt);
+      // descriptors computed once; a byte offset moves the start-address field by offset / 16
+      const uint64_t ktd = smem_desc(smem_u32(S.kt), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t vtd = smem_desc(smem_u32(S.vt), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t qd_k = smem_desc(smem_u32(S.q[0]), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t od_k = smem_desc(smem_u32(S.go[0]), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t qd_mn = smem_desc(smem_u32(S.q[0]), C::kChunkBytes, C::kAtomBytes, C::kLayout);
+      const uint64_t od_mn = smem_desc(smem_u32(S.go[0]), C::kChunkBytes, C::kAtomBytes, C::kLayout);
+      constexpr uint32_t kStep = C::kChunkBytes >> 4, kRow16 = (16 * C::kRowBytes) >> 4;
       auto first_stage = [&](int c) {
-        const int st = c % C::kStages;
-        const uint32_t qa = smem_u32(S.q[st]), oa = smem_u32(S.go[st]);
+        const uint64_t so = (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::kColS, smem_desc(kaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
-                 smem_desc(qa + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNR, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + C::kColS, ktd + 2 * kk, qd_k + so + 2 * kk, C::kIdescNR, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::kColDP, smem_desc(vaddr + kk * 32, 16, C::kAtomBytes, C::kLayout),
-                 smem_desc(oa + kk * 32, 16, C::kAtomBytes, C::kLayout), C::kIdescNR, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + C::kColDP, vtd + 2 * kk, od_k + so + 2 * kk, C::kIdescNR, kk > 0 ? 1u : 0u);
         mma_commit(&S.s_full);
       };
       auto second_stage = [&](int c) {
         const int st = c % C::kStages;
-        const uint32_t qa = smem_u32(S.q[st]), oa = smem_u32(S.go[st]);
+        const uint64_t so = (uint64_t)(st * kStep);
 #pragma unroll
         for (int kk = 0; kk < C::kRowsPerChunk / 16; ++kk) {
           const uint32_t acc = (c == 0 && kk == 0) ? 0u : 1u;
-          mma_ts(tmem + C::kColDV, tmem + C::kColPg + 8 * kk,
-                 smem_desc(oa + kk * 16 * C::kRowBytes, C::kChunkBytes, C::kAtomBytes, C::kLayout), C::kIdescND, acc);
-          mma_ts(tmem + C::kColDK, tmem + C::kColDS + 8 * kk,
-                 smem_desc(qa + kk * 16 * C::kRowBytes, C::kChunkBytes, C::kAtomBytes, C::kLayout), C::kIdescND, acc);
+          mma_ts(tmem + C::kColDV, tmem + C::kColPg + 8 * kk, od_mn + so + kk * kRow16, C::kIdescND, acc);
+          mma_ts(tmem + C::kColDK, tmem + C::kColDS + 8 * kk, qd_mn + so + kk * kRow16, C::kIdescND, acc);
         }
         mma_commit(&S.pv_done);
         mma_commit(&S.empty[st]);
