@@ -129,6 +129,55 @@ def throughput(world: int, units_per_rank: int, steps: int, max_ms: float) -> fl
     return world * units_per_rank * steps / (max_ms / 1000.0)
 
 
+def pipelined_e2e(dev, world: int, steps: int, warmup: int, h_in: dict, outs_like: dict, compute):
+    """End-to-end steps through the public API with the host copies inside the timed region:
+    step i's inputs go host -> device on one stream, its compute runs on the current stream and
+    its result comes back on a third, with two sets of device buffers, so the copies of
+    neighbouring steps overlap the compute (and each other: the link is full duplex).
+    Returns (max-over-ranks milliseconds for `steps` steps, the last step's host outputs)."""
+    import torch
+    import torch.distributed as dist
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    comp_s = torch.cuda.current_stream(dev)
+    d_in = [{n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in h_in.items()} for _ in range(2)]
+    d_out = [{n: torch.empty_like(t) for n, t in outs_like.items()} for _ in range(2)]
+    p_out = [{n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in outs_like.items()} for _ in range(2)]
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                h2d_s.wait_event(comp_done[b])  # step i - 2 has consumed buffer b's inputs
+            with torch.cuda.stream(h2d_s):
+                for name, t in h_in.items():
+                    d_in[b][name].copy_(t, non_blocking=True)
+            h2d_done[b].record(h2d_s)
+            comp_s.wait_event(h2d_done[b])
+            if i >= 2:
+                comp_s.wait_event(d2h_done[b])  # step i - 2's result has left buffer b
+            compute(d_in[b], d_out[b], comp_s)
+            comp_done[b].record(comp_s)
+            d2h_s.wait_event(comp_done[b])
+            with torch.cuda.stream(d2h_s):
+                for name, t in d_out[b].items():
+                    p_out[b][name].copy_(t, non_blocking=True)
+            d2h_done[b].record(d2h_s)
+
+    run(max(3, warmup))
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(h2d_s)
+    run(steps)
+    end.record(d2h_s)
+    torch.cuda.synchronize(dev)
+    return max_over_ranks(start.elapsed_time(end), dev, world), p_out[(steps - 1) & 1]
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -325,37 +374,20 @@ def run_ours(args):
     # end to end through lsrm_nsa_forward with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        p_q, p_k, p_v, p_g = h_q.pin_memory(), h_k.pin_memory(), h_v.pin_memory(), h_g.pin_memory()
-        p_off, p_c = h_off.pin_memory(), h_coords.pin_memory()
-        p_out = torch.empty(N, Hq, d, dtype=torch.bfloat16).pin_memory()
-        d_q, d_k, d_v, d_g = torch.empty_like(q), torch.empty_like(kk), torch.empty_like(v), torch.empty_like(gates)
-        d_off, d_c = torch.empty_like(off), torch.empty_like(coords)
-        d_out = torch.empty_like(out)
-        ins = ((d_q, p_q), (d_k, p_k), (d_v, p_v), (d_g, p_g), (d_off, p_off), (d_c, p_c))
+        h_in = {"q": h_q.pin_memory(), "k": h_k.pin_memory(), "v": h_v.pin_memory(), "gates": h_g.pin_memory(),
+                "off": h_off.pin_memory(), "coords": h_coords.pin_memory()}
 
-        def e2e_step():
-            for dst, src in ins:
-                dst.copy_(src, non_blocking=True)
-            nsa.lsrm_nsa_forward(desc, d_off, d_q, d_k, d_v, d_g, d_c, nsa.ROUTE_GEOMETRIC, d_out, None, None, ws)
-            p_out.copy_(d_out, non_blocking=True)
+        def fwd(di, do, st):
+            nsa.lsrm_nsa_forward(desc, di["off"], di["q"], di["k"], di["v"], di["gates"], di["coords"],
+                                 nsa.ROUTE_GEOMETRIC, do["out"], None, None, ws, stream=st)
 
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        te = max_over_ranks(e0.elapsed_time(e1), dev, world)
-        h2d = sum(src.numel() * src.element_size() for _, src in ins)
-        d2h = p_out.numel() * p_out.element_size()
+        te, last = pipelined_e2e(dev, world, args.steps, args.warmup, h_in, {"out": out}, fwd)
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = out.numel() * out.element_size()
         e2e = {"value": throughput(world, N, args.steps, te), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
-        if not np.array_equal(p_out.view(torch.int16).numpy(), out.view(torch.int16).cpu().numpy()):
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "overlap": "H2D, compute and D2H of neighbouring steps on three streams"}
+        if not torch.equal(last["out"].view(torch.int16), out.view(torch.int16).cpu()):
             raise RuntimeError("end-to-end output differs from the device-resident run")
 
     if rank == 0:
@@ -529,42 +561,22 @@ def run_backward(args):
 
     e2e = None
     if not args.no_e2e:
-        h_idx = idx.cpu().pin_memory()
-        h_lse = lse.cpu().pin_memory()
-        p_in = {n: t.pin_memory() for n, t in h_in.items() if n != "coords"}
-        d_in = {n: torch.empty_like(x[n]) for n in p_in}
-        d_idx, d_lse = torch.empty_like(idx), torch.empty_like(lse)
-        p_out = {n: torch.empty(g.shape, dtype=g.dtype).pin_memory() for n, g in grads.items()}
-        d_out = {n: torch.empty_like(g) for n, g in grads.items()}
+        h_in = {n: t.pin_memory() for n, t in h_in.items() if n != "coords"}
+        h_in["idx"] = idx.cpu().pin_memory()
+        h_in["lse"] = lse.cpu().pin_memory()
 
-        def e2e_step():
-            for n in p_in:
-                d_in[n].copy_(p_in[n], non_blocking=True)
-            d_idx.copy_(h_idx, non_blocking=True)
-            d_lse.copy_(h_lse, non_blocking=True)
-            step(d_in, d_out, d_idx, d_lse)
-            for n in p_out:
-                p_out[n].copy_(d_out[n], non_blocking=True)
+        def bwd(di, do, st):
+            nsa.lsrm_nsa_backward(desc, di["off"], di["q"], di["k"], di["v"], di["gates"], di["idx"], 1, di["lse"],
+                                  di["dout"], do["dq"], do["dk"], do["dv"], do["dgates"], ws, stream=st)
 
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        te = max_over_ranks(e0.elapsed_time(e1), dev, world)
-        h2d = sum(t.numel() * t.element_size() for t in p_in.values()) + \
-            h_idx.numel() * h_idx.element_size() + h_lse.numel() * h_lse.element_size()
-        d2h = sum(t.numel() * t.element_size() for t in p_out.values())
+        te, last = pipelined_e2e(dev, world, args.steps, args.warmup, h_in, grads, bwd)
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in grads.values())
         e2e = {"value": throughput(world, N, args.steps, te), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "overlap": "H2D, compute and D2H of neighbouring steps on three streams"}
         for n in grads:
-            if not torch.equal(p_out[n].view(torch.int16), grads[n].view(torch.int16).cpu()):
+            if not torch.equal(last[n].view(torch.int16), grads[n].view(torch.int16).cpu()):
                 raise RuntimeError(f"end-to-end {n} differs from the device-resident run")
 
     if rank == 0:
