@@ -52,8 +52,9 @@ def parse():
                          "10-20 s of one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward"],
-                    help="sparse: the layer forward (the default line); backward: its gradients")
+    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r"],
+                    help="sparse: the layer forward (the default line); backward: its gradients; dense: the "
+                         "dense-stage shape with every block selected; speed3r: the pooled-query variant")
     return ap.parse_args()
 
 
@@ -607,10 +608,204 @@ def run_backward(args):
     return 0
 
 
+# ------------------------------------------------------------------------------------------------
+# the other forward workloads: the dense-stage shape (every block selected) and the Speed3R variant
+# ------------------------------------------------------------------------------------------------
+EXTRA = {
+    "dense": ("sparse-attn fwd tokens/s, dense-stage shape (k = B)", "lsrm_dense_stage_all_blocks"),
+    "speed3r": ("sparse-attn fwd tokens/s, Speed3R pooled-query variant", "speed3r_512_frames_top32_forced"),
+}
+
+
+def speed3r_flops(w, idx: np.ndarray) -> dict:
+    """4 d per attended (query, key): pooled queries against every block mean (one query per
+    block and head), and every token against its block's forced and routed tokens."""
+    n = np.diff(w.off.astype(np.int64))
+    B, H, d = w.n_blocks, w.n_q_heads, w.head_dim
+    cmp = B * B * H
+    forced_tok = int(n[w.forced].sum())
+    routed_tok = n[np.clip(idx, 0, B - 1)].sum(axis=-1)  # [B][H]
+    slc = float((n[:, None] * (forced_tok + routed_tok)).sum())
+    f = 4 * d
+    return {"cmp": f * cmp, "slc": f * slc, "total": f * (cmp + slc)}
+
+
+def run_extra(args):
+    import torch
+    metric, workload = EXTRA[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_extra_reference(args, metric, workload)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    from block_sparse_gqa_nsa_b200 import nsa
+    from block_sparse_gqa_nsa_b200.build import build
+    from workloads import make_workload
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    nsa.load_library()
+    w = make_workload(args.workload, seed=args.seed)
+    N, B, Hq, Hkv, d, k = w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, kk, v, gates = bf(w.q), bf(w.k), bf(w.v), bf(w.gates)
+    off = torch.from_numpy(w.off.astype(np.int32)).to(dev)
+    forced = torch.from_numpy(w.forced.astype(np.int32)).to(dev) if len(w.forced) else None
+    desc = nsa.make_desc(N, B, w.max_block_len, Hq, Hkv, d, k, w.window, 0.0, w.pooled_q, w.n_gates, forced)
+    ws = nsa.workspace(desc, dev)
+    out = torch.empty(N, Hq, d, dtype=torch.bfloat16, device=dev)
+    if args.workload == "speed3r":
+        idx = torch.empty(B, Hq, k, dtype=torch.int32, device=dev)
+
+        def step():
+            nsa.lsrm_nsa_forward(desc, off, q, kk, v, gates, None, nsa.ROUTE_SCORE, out, idx, None, ws)
+        # compress (Q, K, V), forced bitmap / prefix / gather, pooled compressed pass with the
+        # streaming top-k, forced-token pass, routed part with the merge and gated combine
+        launches_per_step = 7
+    else:
+        idx = None
+
+        def step():
+            nsa.lsrm_nsa_forward(desc, off, q, kk, v, gates, None, nsa.ROUTE_ALL, out, None, None, ws)
+        launches_per_step = 2  # compress, fused attention over every block
+    for _ in range(max(3, args.warmup)):
+        step()
+    st = nsa.lsrm_nsa_last_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    if args.workload == "speed3r":
+        flops = speed3r_flops(w, idx.cpu().numpy())
+    else:
+        flops = algorithmic_flops(w, np.tile(np.arange(B, dtype=np.int32), (B, 1)))
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
+    ms = total_ms / args.steps
+    if rank == 0:
+        peaks, src = measured_peaks()
+        achieved = flops["total"] / (ms / 1000.0) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        line = {"metric": metric, "value": throughput(world, N, args.steps, total_ms), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": workload, "n_tokens": N, "n_blocks": B, "heads": f"{Hq}q/{Hkv}kv",
+                           "head_dim": d, "top_k": k, "window": w.window, "n_forced": int(len(w.forced)),
+                           "parallelism": f"replicas{world}" if world > 1 else "single", "seed": args.seed,
+                           "l2": "inputs larger than L2"},
+                "flops_per_step": flops,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                             "frac": achieved / peak, "traffic": None,
+                             "kernel": "lsrm_nsa_forward (all launches of one call)",
+                             "peak_source": f"{src} bf16_tflops (burst)"},
+                "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+        if not args.no_cpu_baseline and world == 1:
+            n_blk = args.cpu_sample_blocks or 4
+            tok, dt = extra_oracle_sample(w, idx.cpu().numpy() if idx is not None else None, n_blk, 7)
+            line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"{n_blk} seeded query blocks ({tok} tokens) of the same workload, "
+                                              f"fp64, 1 thread, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def extra_oracle_sample(w, idx, n_blocks: int, seed: int):
+    """The fp64 oracle forward on a seeded sample of query blocks (1 thread); the Speed3R sample
+    uses routing indices given (the GPU's, or the oracle's own in the reference arm)."""
+    import oracle as O
+    D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window,
+                   n_gates=w.n_gates, pooled_q=w.pooled_q)
+    rng = np.random.default_rng(seed)
+    qb = np.sort(rng.choice(w.n_blocks, size=n_blocks, replace=False)).astype(np.int32)
+    if idx is None:
+        idx = np.tile(np.arange(w.n_blocks, dtype=np.int32), (w.n_blocks, 1))
+    t0 = time.perf_counter()
+    if w.pooled_q:
+        O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, forced=w.forced, qblocks=qb)
+    else:
+        O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, qblocks=qb)
+    dt = time.perf_counter() - t0
+    return int((w.off[qb + 1] - w.off[qb]).sum()), dt
+
+
+def run_extra_reference(args, metric, workload):
+    from workloads import make_workload
+    import oracle as O
+    w = make_workload(args.workload, seed=args.seed)
+    D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window,
+                   n_gates=w.n_gates, pooled_q=w.pooled_q)
+    qc = kc = None
+    if w.pooled_q:
+        qc = O.compress(D, w.off, w.q, w.n_q_heads)
+        kc = O.compress(D, w.off, w.k, w.n_kv_heads)
+    all_idx = np.tile(np.arange(w.n_blocks, dtype=np.int32), (w.n_blocks, 1))
+
+    def one(seed):
+        # one seeded query block: (Speed3R: its routing by the oracle, then) the layer forward
+        qb = np.array([np.random.default_rng(seed).integers(w.n_blocks)], dtype=np.int32)
+        t0 = time.perf_counter()
+        if w.pooled_q:
+            rows, _ = O.route_pooled(D, qc, kc, w.forced, qblocks=qb)
+            idx = np.zeros((w.n_blocks, w.n_q_heads, w.top_k), dtype=np.int32)
+            idx[qb] = rows
+            O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, forced=w.forced, qblocks=qb)
+        else:
+            O.forward(D, w.off, w.q, w.k, w.v, w.gates, all_idx, qblocks=qb)
+        return int((w.off[qb + 1] - w.off[qb]).sum()), time.perf_counter() - t0
+
+    for s in range(args.warmup):
+        one(1000 + s)
+    tok, tsum = 0, 0.0
+    for s in range(args.steps):
+        t, dt = one(s)
+        tok += t
+        tsum += dt
+    value = tok / tsum
+    line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * tsum / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
+                       "sample": "1 seeded query block per step"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "1 query block per step, fp64, 1 thread"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.workload == "backward":
         return run_backward_reference(args) if args.impl == "reference" else run_backward(args)
+    if args.workload in EXTRA:
+        return run_extra(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
