@@ -47,7 +47,8 @@ template <int D>
 struct TcCfg {
   static constexpr int kRows = 128;
   static constexpr int kKeys = 64;                 // keys per chunk = N of S = Q K^T (one block)
-  static constexpr int kStages = 4;                // K/V ring
+  static constexpr int kStages = D == 32 ? 4 : 3;  // K/V ring
+  static constexpr int kCand = D == 64 ? 32 : 1;   // streaming top-k candidate buffer per row
   static constexpr int kCtasPerSm = D == 32 ? 2 : 1;
   static constexpr int kTmemCols = D == 32 ? 256 : 512;   // per CTA (power of two)
   static constexpr int kColsPerTile = kTmemCols / 2;
@@ -69,7 +70,8 @@ struct TcSmem {
   uint8_t q[2][C::kQBytes];
   uint8_t k[C::kStages][C::kKVBytes];
   uint8_t v[C::kStages][C::kKVBytes];
-  float acc[2][D][128];  // gated output sum per tile, column-major so a warp's rows are one bank row
+  float acc[2][D][128];  // gated sum per tile, column-major so a warp's rows are one bank row
+  float cand[2][2 * C::kCand][128];  // top-k candidates per row: values, then block ids
   uint64_t q_full[2], kv_full[C::kStages], kv_empty[C::kStages];
   uint64_t s_full[2], p_full[2], pv_done[2], drain;
   uint32_t tmem_base;
@@ -350,31 +352,49 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     // accumulator: values in acc[0..31], block ids in acc[32..63].  The root is the worst entry
     // in the order (logit desc, block asc), so ties evict the larger block id first; keys arrive
     // in increasing block order, so a candidate enters only when strictly above the root.
+    // Scores above the (possibly stale) root are first appended to a per-row candidate buffer;
+    // the warp merges its rows' buffers together, re-testing every candidate in key order
+    // against the live root, which makes the same decisions as inserting key by key while
+    // keeping the divergent heap work out of the per-key loop.  Forced blocks are dropped here.
     const bool topk_on = (D == 64) && p.topk_idx != nullptr;
     float thr = -INFINITY;
-    int key_base = 0;        // block id of key 0 of the current chunk
-    uint64_t fmask = 0;      // forced blocks among the chunk's 64 keys
+    int key_base = 0;  // block id of key 0 of the current chunk
+    int ncand = 0;     // this row's buffered candidates
+    float* cbuf = &S.cand[t][0][row];
     auto hv = [&](int i) -> float& { return acc[i * 128]; };
     auto hj = [&](int i) -> int& { return reinterpret_cast<int&>(acc[(32 + i) * 128]); };
     auto worse = [&](float va, int ja, float vb, int jb) { return va < vb || (va == vb && ja > jb); };
-    auto topk_consider = [&](float sv, int j) {
-      if (sv > thr && !((fmask >> j) & 1ull)) {
-        const int jg = key_base + j;
-        int i = 0;
-        while (true) {
-          const int l = 2 * i + 1, r = l + 1;
-          if (l >= 32) break;
-          int c = l;
-          if (r < 32 && worse(hv(r), hj(r), hv(l), hj(l))) c = r;
-          if (!worse(hv(c), hj(c), sv, jg)) break;
-          hv(i) = hv(c);
-          hj(i) = hj(c);
-          i = c;
-        }
-        hv(i) = sv;
-        hj(i) = jg;
-        thr = hv(0);
+    auto heap_insert = [&](float sv, int jg) {
+      int i = 0;
+      while (true) {
+        const int lc = 2 * i + 1, rc = lc + 1;
+        if (lc >= 32) break;
+        int cc = lc;
+        if (rc < 32 && worse(hv(rc), hj(rc), hv(lc), hj(lc))) cc = rc;
+        if (!worse(hv(cc), hj(cc), sv, jg)) break;
+        hv(i) = hv(cc);
+        hj(i) = hj(cc);
+        i = cc;
       }
+      hv(i) = sv;
+      hj(i) = jg;
+      thr = hv(0);
+    };
+    auto topk_append = [&](float sv, int j) {
+      if (sv > thr) {
+        cbuf[ncand * 128] = sv;
+        reinterpret_cast<int&>(cbuf[(C::kCand + ncand) * 128]) = key_base + j;
+        ++ncand;
+      }
+    };
+    auto topk_flush = [&]() {
+#pragma unroll 1
+      for (int e = 0; e < ncand; ++e) {
+        const float sv = cbuf[e * 128];
+        const int jg = reinterpret_cast<const int&>(cbuf[(C::kCand + e) * 128]);
+        if (sv > thr && !((p.forced_bits[jg >> 5] >> (jg & 31)) & 1u)) heap_insert(sv, jg);
+      }
+      ncand = 0;
     };
     if (topk_on) {
 #pragma unroll 1
@@ -421,8 +441,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           const float s1 = need_mask ? masked(r[2 * i + 1], j + 1) : __uint_as_float(r[2 * i + 1]);
           mx[i & 3] = fmax3(mx[i & 3], s0, s1);
           if constexpr (topk) {
-            topk_consider(s0, j);
-            topk_consider(s1, j + 1);
+            topk_append(s0, j);
+            topk_append(s1, j + 1);
           }
           const float x0 = fmaf(s0, sc, nm), x1 = fmaf(s1, sc, nm);
           float p0, p1;
@@ -437,6 +457,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st8(tbase + C::kColP + 8 * qd, pk);
+        if constexpr (topk) {  // a quarter appends at most 16 candidates per row
+          if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_flush();
+        }
       };
       tmem_ld16(tbase + C::kColS, ra);
       tmem_ld_wait();
@@ -455,8 +478,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     auto chunk_max = [&](bool need_mask) -> float {
       return need_mask ? chunk_max_t(std::true_type{}) : chunk_max_t(std::false_type{});
     };
-    auto exp_pass = [&](bool need_mask, float mref, float* lsum) -> float {
-      if (topk_on && br == 0)
+    auto exp_pass = [&](bool need_mask, float mref, float* lsum, bool offer = true) -> float {
+      if (topk_on && br == 0 && offer)
         return need_mask ? exp_pass_t(mref, lsum, std::true_type{}, std::true_type{})
                          : exp_pass_t(mref, lsum, std::false_type{}, std::true_type{});
       return need_mask ? exp_pass_t(mref, lsum, std::true_type{}, std::false_type{})
@@ -475,11 +498,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       const bool first = cs.first_of_branch(c);
       chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nv);
       const bool need_mask = br == 2 || nv < 64;
-      if (topk_on && br == 0) {
-        key_base = local * 64;
-        const uint32_t w0 = p.forced_bits[key_base >> 5], w1 = p.forced_bits[(key_base >> 5) + 1];
-        fmask = (uint64_t)w0 | ((uint64_t)w1 << 32);
-      }
+      if (topk_on && br == 0) key_base = local * 64;
       float lsum;
       if (first) {
         if (c > 0) finalize(prev_br, m, l);
@@ -506,7 +525,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           }
           l *= alpha;
           m = mn;
-          exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
+          exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum, false);  // candidates were taken
         }
         l += lsum;
       }
@@ -520,6 +539,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         for (int i = 0; i < D; ++i) p.obranch[orow * D + i] = 0.f;
       if (p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first] = -INFINITY;
     }
+    if (ok && topk_on) topk_flush();
     if (ok && topk_on && valid) {
       // emit the row's top-k in order (logit desc, block asc); missing entries are -1
       int32_t* dst = p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k;
