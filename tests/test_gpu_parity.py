@@ -293,12 +293,18 @@ def test_fused_forward_dense_equals_dense_gqa_sampled():
 # S9 Speed3R pooled-query variant
 # ------------------------------------------------------------------------------------------------
 
-def check_pooled_routing(gpu_idx, w, qblocks, k):
+def check_pooled_routing(gpu_idx, w, qblocks, k, operands_bf16=False):
     """Validity of Speed3R routing: k distinct, non-forced blocks, each with an oracle pooled logit
-    within 1e-3 of the k-th best; where the oracle gap exceeds 1e-3 the sets must agree."""
+    within 1e-3 of the k-th best; where the oracle gap exceeds 1e-3 the sets must agree.
+    With operands_bf16 the oracle ranks with the pooled Q and K rounded to bf16, the precision the
+    kernel's MMA operands have (the top-k is an integer decision taken from those products)."""
     D = oracle_desc(w, top_k=k)
     qc = O.compress(D, w.off, w.q, w.n_q_heads)
     kc = O.compress(D, w.off, w.k, w.n_kv_heads)
+    if operands_bf16:
+        from workloads.nsa_workloads import bf16_bits_to_f32
+        qc = bf16_bits_to_f32(f32_to_bf16_bits(qc.astype(np.float32))).astype(np.float64)
+        kc = bf16_bits_to_f32(f32_to_bf16_bits(kc.astype(np.float32))).astype(np.float64)
     _, logits = O.route_pooled(D, qc, kc, w.forced, qblocks=qblocks, want_logits=True)
     forced = set(w.forced.tolist())
     for i, a in enumerate(qblocks):
@@ -491,3 +497,53 @@ def test_backward_sparse_stage_full_size():
         blk = slice(w.off[j], w.off[j + 1])
         assert_grad_close(to_np(dk)[blk], ref[1][blk], f"dk block {j}")
         assert_grad_close(to_np(dv)[blk], ref[2][blk], f"dv block {j}")
+
+
+# ------------------------------------------------------------------------------------------------
+# the online softmax's reference move (a later chunk's max exceeds the running reference by more
+# than 2^8): one block's keys are scaled up so its scores jump late in the key stream
+# ------------------------------------------------------------------------------------------------
+
+def _set_block_keys(w, block, value):
+    """Every key of `block` becomes `value` in every component: its scores (and its block mean's)
+    reach many times the others' in log2 units, so the running reference has to move."""
+    k = w.k.copy()
+    k[w.off[block]:w.off[block + 1]] = f32_to_bf16_bits(np.array([value], np.float32))[0]
+    w.k = k
+
+
+def test_fused_forward_reference_moves_late_in_the_stream():
+    w = make_workload("dense")      # 320 blocks: five compressed chunks, 320 selected chunks
+    _set_block_keys(w, 300, 50.0)   # block 300: late in both the compressed and selected streams
+    D = oracle_desc(w)
+    qb = np.array([0, 150, 300], dtype=np.int32)
+    idx = np.tile(np.arange(w.n_blocks, dtype=np.int32), (w.n_blocks, 1))
+    for b in range(3):  # every branch on its own
+        one = np.zeros_like(w.gates)
+        one[..., b] = f32_to_bf16_bits(np.array([1.0], np.float32))[0]
+        w.gates = one
+        c = DeviceCase(w)
+        o1, _, _ = _forward(c, nsa.ROUTE_ALL)
+        ref = O.forward(D, w.off, w.q, w.k, w.v, one, idx, qblocks=qb)
+        assert_close(to_np(o1)[rows_for(w.off, qb)], ref, f"branch{b}")
+
+
+def test_speed3r_routing_with_a_late_dominant_block():
+    w = make_workload("speed3r_small", n_frames=6)
+    target = w.n_blocks - 3                      # a late, non-forced block
+    assert target not in set(w.forced.tolist())
+    _set_block_keys(w, target, 400.0)
+    c = DeviceCase(w)
+    idx = c.empty(w.n_blocks, w.n_q_heads, w.top_k, dtype=torch.int32)
+    out = c.empty(w.n_tokens, w.n_q_heads, w.head_dim, dtype=torch.bfloat16)
+    nsa.lsrm_nsa_forward(c.desc, c.off, c.q, c.k, c.v, c.gates, None, nsa.ROUTE_SCORE, out, idx, None, c.ws)
+    assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
+    gidx = to_np(idx)
+    for row in gidx.reshape(-1, w.top_k):
+        assert len(set(row.tolist())) == w.top_k  # distinct: no candidate offered twice
+    qb = np.arange(w.n_blocks, dtype=np.int32)
+    # the dominant block's logits are ~400x the others': bf16 rounding of the pooled queries moves
+    # them by more than the 1e-3 gap rule, so the ranking is checked at the operands' precision
+    check_pooled_routing(gidx, w, qb, w.top_k, operands_bf16=True)
+    ref = O.forward(oracle_desc(w), w.off, w.q, w.k, w.v, w.gates, gidx, forced=w.forced)
+    assert_close(to_np(out), ref, "out")
