@@ -103,12 +103,61 @@ geo_topk_kernel(const int32_t* __restrict__ cen, int32_t B, int32_t k, int32_t* 
   }
 }
 
+// One CTA per query block for B <= kRouteThreads * kGeoPer: each thread computes its candidates'
+// distances once and keeps them in registers; every round takes the best candidate strictly after
+// the previous round's (key, index) with one block barrier (the per-warp winners alternate
+// between two shared buffers, and every thread reduces the eight winners itself).
+constexpr int kGeoPer = 8;
+__global__ void __launch_bounds__(kRouteThreads)
+geo_topk_reg_kernel(const int32_t* __restrict__ cen, int32_t B, int32_t k, int32_t* __restrict__ idx) {
+  __shared__ DistKey s_warp[2][kRouteThreads / 32];
+  const int a = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long ax = cen[a * 3 + 0], ay = cen[a * 3 + 1], az = cen[a * 3 + 2];
+  long long dist[kGeoPer];
+#pragma unroll
+  for (int i = 0; i < kGeoPer; ++i) {
+    const int j = tid + i * kRouteThreads;
+    if (j < B) {
+      const long long dx = cen[j * 3 + 0] - ax, dy = cen[j * 3 + 1] - ay, dz = cen[j * 3 + 2] - az;
+      dist[i] = dx * dx + dy * dy + dz * dz;
+    } else {
+      dist[i] = LLONG_MAX;
+    }
+  }
+  DistKey last{-1, -1};
+  for (int r = 0; r < k; ++r) {
+    DistKey best{LLONG_MAX, INT_MAX};
+#pragma unroll
+    for (int i = 0; i < kGeoPer; ++i) {
+      const int j = tid + i * kRouteThreads;
+      const DistKey cand{dist[i], j};
+      if (j < B && key_less(last, cand) && key_less(cand, best)) best = cand;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      DistKey other{__shfl_xor_sync(0xffffffffu, best.d, o), __shfl_xor_sync(0xffffffffu, best.j, o)};
+      if (key_less(other, best)) best = other;
+    }
+    if (lane == 0) s_warp[r & 1][warp] = best;
+    __syncthreads();
+    DistKey b = s_warp[r & 1][0];
+#pragma unroll
+    for (int w = 1; w < kRouteThreads / 32; ++w)
+      if (key_less(s_warp[r & 1][w], b)) b = s_warp[r & 1][w];
+    if (tid == 0) idx[(size_t)a * k + r] = b.j;
+    last = b;
+  }
+}
+
 lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, const int32_t* coords, int32_t* cen,
                                    int32_t* idx, uint32_t* status, cudaStream_t stream) {
   const int B = d.n_blocks;
   centroid_kernel<<<(B * 32 + 255) / 256, 256, 0, stream>>>(off, coords, B, cen, status);
   const size_t smem = (size_t)B * 3 * sizeof(int32_t);
-  if (smem <= 48 * 1024) {
+  if (B <= kRouteThreads * kGeoPer) {
+    geo_topk_reg_kernel<<<B, kRouteThreads, 0, stream>>>(cen, B, d.top_k, idx);
+  } else if (smem <= 48 * 1024) {
     geo_topk_kernel<true><<<B, kRouteThreads, smem, stream>>>(cen, B, d.top_k, idx);
   } else {
     geo_topk_kernel<false><<<B, kRouteThreads, 0, stream>>>(cen, B, d.top_k, idx);
