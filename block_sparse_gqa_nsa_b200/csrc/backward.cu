@@ -46,7 +46,7 @@ struct BwdParams {
   const uint16_t* dout;   // [N][Hq][D]
   uint16_t* dq;
   uint16_t* dgates;
-  float* delta;           // [N][Hq][NG]
+  float4* rowc;           // [NG][N][Hq]: lse (log2 units), gate, Delta, token position (int bits)
   float* dk_tok;          // [N][Hkv][D] selected + window part
   float* dv_tok;
   float* dkc_part;        // [splits][B][Hkv][D]
@@ -305,7 +305,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       for (int b = 0; b < p.NG; ++b)
         if (seq.n[b] == 0 && valid) {  // a branch without keys has no gradient
           p.dgates[orow * p.NG + b] = 0;
-          p.delta[orow * p.NG + b] = 0.f;
+          p.rowc[((size_t)b * p.N + t0 + tok_local) * p.Hq + g * p.G + R % p.G] =
+              make_float4(INFINITY, 0.f, 0.f, __int_as_float(tok_local));
         }
     }
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -409,7 +410,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           delta = gb * dg;
           if (h == 0 && valid) {
             p.dgates[orow * p.NG + br] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
-            p.delta[orow * p.NG + br] = delta;
+            p.rowc[((size_t)br * p.N + t0 + tok_local) * p.Hq + g * p.G + R % p.G] =
+                make_float4(l2, gb, delta, __int_as_float(tok_local));
           }
         } else if (h == 0) {
           // dQ_b is final: add tau dQ_b to the tile's dQ
@@ -453,8 +455,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
 //   S^T = K Q^T and dP^T = V dO^T  ([128 x 64], K-major operands from shared memory)
 //   P^T = exp(tau S^T - lse) per query row, Pg = P^T g, dS^T = P^T (g dP^T - Delta)
 //   dV += Pg dO and dK += dS^T Q   ([128 x D], A from tensor memory, MN-major B)
-// The per-row constants (lse in log2 units, gate, Delta, token position) of each chunk are
-// staged next to its Q and dO tiles by the producer warp.
+// The per-row constants of each chunk (LSE in log2 units, gate, Delta, token position, written
+// by the query pass as one float4 per branch, token and head) arrive by TMA with its Q and dO.
 //   compressed: CTA = (128 block means, group, query split), rows = the split's tokens x G heads
 //   local:      CTA = (key block j, group), rows = the query blocks that routed to j (ascending,
 //               selected branch), then block j itself (window branch)
@@ -488,6 +490,7 @@ struct KvSmem {
   uint8_t go[C::kStages][C::kChunkBytes];  // dO rows
   float4 rv[C::kStages][64];               // per query row: lse (log2), gate, Delta, token position
   int br[C::kStages];                      // branch of the chunk in each stage
+  int nrows[C::kStages];                   // valid rows of the chunk in each stage
   uint64_t key_full, full[C::kStages], empty[C::kStages], s_full, p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort;
@@ -503,7 +506,7 @@ template <int D, bool kLocal>
 __global__ void __launch_bounds__(kKvThreads, KvCfg<D>::kCtasPerSm)
 bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                  const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap,
-                 const BwdParams p) {
+                 const __grid_constant__ CUtensorMap rmap, const BwdParams p) {
   using namespace tc;
   using C = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -559,7 +562,7 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     S.total = n_keys > 0 ? total : 0;
     mbar_init(&S.key_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&S.full[s], 1 + 32);  // the TMA byte count, and every producer lane's row constants
+      mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
     }
     mbar_init(&S.s_full, 1);
@@ -584,48 +587,32 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   };
 
   if (warp == 0) {
-    // ---------------- producer warp: key tile once, then Q / dO chunks with their row constants ----------------
-    if (total > 0) {
-      if (lane == 0) {
-        const int key_rows = kLocal ? 64 : 128;
-        mbar_arrive_expect_tx(&S.key_full, 2 * key_rows * C::kRowBytes);
-        tma_load_3d(S.kt, &kmap, &S.key_full, 0, g, key0);
-        tma_load_3d(S.vt, &vmap, &S.key_full, 0, g, key0);
-      }
+    // ---------------- producer: key tile once, then Q / dO chunks with their row constants ----------------
+    if (lane == 0 && total > 0) {
+      const int key_rows = kLocal ? 64 : 128;
+      mbar_arrive_expect_tx(&S.key_full, 2 * key_rows * C::kRowBytes);
+      tma_load_3d(S.kt, &kmap, &S.key_full, 0, g, key0);
+      tma_load_3d(S.vt, &vmap, &S.key_full, 0, g, key0);
       KvCursor cu;
       skip_empty(cu);
       int issued = 0;
       for (int c = 0; c < total; ++c) {
         const int st = c % C::kStages;
-        if (c >= C::kStages && !wait_all(&S.empty[st], ((c / C::kStages) + 1) & 1)) break;
+        if (c >= C::kStages && !mbar_wait(&S.empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
         int br, t0a, rows;
         entry(cu.e, br, t0a, rows);
-        const int rows_valid = min(C::kRowsPerChunk, rows - cu.r0);
         const int t_first = t0a + cu.r0 / p.G;
-        if (lane == 0) {
-          S.br[st] = br;
-          mbar_arrive_expect_tx(&S.full[st], 2 * C::kChunkBytes);
-          tma_load_3d(S.q[st], &qmap, &S.full[st], 0, g * p.G, t_first);
-          tma_load_3d(S.go[st], &omap, &S.full[st], 0, g * p.G, t_first);
-        }
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int rr = lane + 32 * k;
-          float4 v = make_float4(INFINITY, 0.f, 0.f, __int_as_float(INT_MIN / 2));
-          if (rr < rows_valid) {
-            const int t = t_first + rr / p.G;
-            const size_t orow = (size_t)t * p.Hq + g * p.G + rr % p.G;
-            v = make_float4(p.lse[orow * p.NG + br] * 1.4426950408889634f, bf16_to_f32(p.gates[orow * p.NG + br]),
-                            p.delta[orow * p.NG + br], __int_as_float(t - t0a));
-          }
-          S.rv[st][rr] = v;
-        }
-        mbar_arrive(&S.full[st]);
+        S.br[st] = br;
+        S.nrows[st] = min(C::kRowsPerChunk, rows - cu.r0);
+        mbar_arrive_expect_tx(&S.full[st], 2 * C::kChunkBytes + C::kRowsPerChunk * 16);
+        tma_load_3d(S.q[st], &qmap, &S.full[st], 0, g * p.G, t_first);
+        tma_load_3d(S.go[st], &omap, &S.full[st], 0, g * p.G, t_first);
+        tma_load_3d(S.rv[st], &rmap, &S.full[st], 0, g * p.G, br * p.N + t_first);
         issued = c + 1;
         cu.r0 += C::kRowsPerChunk;
         skip_empty(cu);
       }
-      if (lane == 0 && *abort) {
+      if (*abort) {
         volatile int no_abort = 0;
         mbar_wait(&S.key_full, 0, &no_abort, nullptr);
         for (int c = max(0, issued - C::kStages); c < issued; ++c)
@@ -702,8 +689,10 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       tc_fence_after();
       return true;
     };
-    auto chunk_pass = [&](int st, auto window_tag) {
+    auto chunk_pass = [&](int st, auto window_tag, auto mask_tag) {
       constexpr bool kWindow = decltype(window_tag)::value;
+      constexpr bool kMask = decltype(mask_tag)::value;  // rows past the chunk's valid rows
+      const int nrows = S.nrows[st];
       uint32_t sa[16], sb[16], da[16], db[16];
       auto quarter_pass = [&](const uint32_t* sr, const uint32_t* dr, int qd) {
         uint32_t pg[8], ds[8];
@@ -712,12 +701,14 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
           float a2[2], b2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float4 rv = S.rv[st][32 * h + 16 * qd + 2 * i + e];
+            const int r = 32 * h + 16 * qd + 2 * i + e;
+            const float4 rv = S.rv[st][r];
             float pr = fast_exp2(fmaf(__uint_as_float(sr[2 * i + e]), sc, -rv.x));
             if constexpr (kWindow) {
               const int tp = __float_as_int(rv.w);
               pr = (key >= tp - wh && key <= tp + wh - 1) ? pr : 0.f;
             }
+            if constexpr (kMask) pr = r < nrows ? pr : 0.f;
             a2[e] = pr * rv.y;
             b2[e] = pr * fmaf(rv.y, __uint_as_float(dr[2 * i + e]), -rv.z);
           }
@@ -742,8 +733,14 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       tc_fence_after();
       if (!pv_wait_through(c - 1)) { ok = false; break; }  // Pg and dS columns are free again
       const int st = c % C::kStages;
-      if (kLocal && S.br[st] == 2) chunk_pass(st, std::true_type{});
-      else chunk_pass(st, std::false_type{});
+      const bool partial = S.nrows[st] < C::kRowsPerChunk;
+      if (kLocal && S.br[st] == 2) {
+        if (partial) chunk_pass(st, std::true_type{}, std::true_type{});
+        else chunk_pass(st, std::true_type{}, std::false_type{});
+      } else {
+        if (partial) chunk_pass(st, std::false_type{}, std::true_type{});
+        else chunk_pass(st, std::false_type{}, std::false_type{});
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&S.p_full);
@@ -907,9 +904,11 @@ static lsrm_status launch_backward_d(const lsrm_nsa_desc& d, const BwdParams& p,
       cudaFuncSetAttribute(bwd_kv_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
           cudaSuccess)
     return LSRM_ERR_CUDA;
-  bwd_kv_tc_kernel<D, true><<<dim3(d.n_blocks, d.n_kv_heads, 1), kKvThreads, sm, s>>>(k64, v64, q64, o64, p);
+  CUtensorMap rmap;
+  if (!make_map_rows(&rmap, p.rowc, d.n_q_heads, (long long)p.NG * d.n_tokens, G, 64 / G)) return LSRM_ERR_CUDA;
+  bwd_kv_tc_kernel<D, true><<<dim3(d.n_blocks, d.n_kv_heads, 1), kKvThreads, sm, s>>>(k64, v64, q64, o64, rmap, p);
   bwd_kv_tc_kernel<D, false><<<dim3((d.n_blocks + 127) / 128, d.n_kv_heads, kBwdSplits), kKvThreads, sm, s>>>(
-      kc128, vc128, q64, o64, p);
+      kc128, vc128, q64, o64, rmap, p);
   bwd_finish_kernel<<<d.n_blocks, 256, 0, s>>>(p, D);
   (void)idx_heads;
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
@@ -935,7 +934,7 @@ lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const vo
   p.dout = (const uint16_t*)dout;
   p.dq = (uint16_t*)dq;
   p.dgates = (uint16_t*)dgates;
-  p.delta = reinterpret_cast<float*>(ws_bwd + w.delta);
+  p.rowc = reinterpret_cast<float4*>(ws_bwd + w.rowc);
   p.dk_tok = reinterpret_cast<float*>(ws_bwd + w.dk_tok);
   p.dv_tok = reinterpret_cast<float*>(ws_bwd + w.dv_tok);
   p.dkc_part = reinterpret_cast<float*>(ws_bwd + w.dkc);

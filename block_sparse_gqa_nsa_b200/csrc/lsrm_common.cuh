@@ -28,11 +28,12 @@ struct Workspace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// backward scratch (inside the workspace's backward region): per-row Delta terms, fp32 selected +
-// window parts of dK / dV, per-split compressed-branch partials, and the inverse routing lists
+// backward scratch (inside the workspace's backward region): per-row constants of every branch
+// (LSE in log2 units, gate, Delta, token position in its block), fp32 selected + window parts of
+// dK / dV, per-split compressed-branch partials, and the inverse routing lists
 constexpr int kBwdSplits = 32;  // query splits of the compressed-key pass
 struct BwdWs {
-  size_t delta, dk_tok, dv_tok, dkc, dvc, inv_count, inv_cursor, inv_start, inv_list, total;
+  size_t rowc, dk_tok, dv_tok, dkc, dvc, inv_count, inv_cursor, inv_start, inv_list, total;
 };
 inline BwdWs bwd_layout(const lsrm_nsa_desc& d, int idx_heads) {
   BwdWs w{};
@@ -40,7 +41,7 @@ inline BwdWs bwd_layout(const lsrm_nsa_desc& d, int idx_heads) {
   const size_t N = (size_t)d.n_tokens, B = (size_t)d.n_blocks, Hq = (size_t)d.n_q_heads, Hkv = (size_t)d.n_kv_heads;
   const size_t D = (size_t)d.head_dim, nl = B * (size_t)idx_heads, NG = (size_t)(d.n_gates > 0 ? d.n_gates : 0);
   const size_t K = (size_t)(d.top_k > 0 ? d.top_k : 0);
-  w.delta = o;      o = align256(o + N * Hq * NG * 4);
+  w.rowc = o;       o = align256(o + NG * N * Hq * 16);
   w.dk_tok = o;     o = align256(o + N * Hkv * D * 4);
   w.dv_tok = o;     o = align256(o + N * Hkv * D * 4);
   w.dkc = o;        o = align256(o + (size_t)kBwdSplits * B * Hkv * D * 4);

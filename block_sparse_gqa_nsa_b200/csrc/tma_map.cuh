@@ -35,4 +35,17 @@ inline bool make_map(CUtensorMap* map, const void* base, int D, int heads, long 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D map over float4 rows [rows][heads][4 floats] (no swizzle) with a (4, box_heads, box_rows) box
+inline bool make_map_rows(CUtensorMap* map, const void* base, int heads, long long rows, int box_heads, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr || base == nullptr) return false;
+  cuuint64_t dims[3] = {4, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {16, (cuuint64_t)heads * 16};
+  cuuint32_t box[3] = {4, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace lsrm
