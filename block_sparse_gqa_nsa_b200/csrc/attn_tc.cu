@@ -263,14 +263,18 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
+          // S(c) is issued ahead of P(c - 1) V: it overwrites only S, which the softmax released
+          // with P(c - 1), and the softmax waits for P(c - 1) V before it stores P(c)
           if (c > 0) {
             if (!mbar_wait(&S.p_full[t], (c - 1) & 1, abort, p.status)) { ok = false; break; }
             tc_fence_after();
+          }
+          issue_qk(t, c);
+          mma_commit(&S.s_full[t]);
+          if (c > 0) {
             issue_pv(t, c - 1);
             mma_commit(&S.pv_done[t]);
           }
-          issue_qk(t, c);  // S of tile t was released with P(c - 1)
-          mma_commit(&S.s_full[t]);
         }
         if (!ok) break;
         if (c > 0) mma_commit(&S.kv_empty[(c - 1) % C::kStages]);
@@ -422,6 +426,17 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       }
       return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
     };
+    // The previous chunk's P V is waited for as late as possible: before the first P store of a
+    // chunk, before O is read, and at the latest before P(c) is handed over.
+    int pv_wait_for = -1;
+    bool pv_ok = true;
+    auto wait_pv = [&]() {
+      if (pv_wait_for >= 0) {
+        pv_ok = wait_all(&S.pv_done[t], pv_wait_for & 1);
+        tc_fence_after();
+        pv_wait_for = -1;
+      }
+    };
     // P = exp2(s * scale - mref) as bf16 pairs into tensor memory; returns the chunk's raw max and
     // its sum of P in *lsum.  S is read 16 columns at a time, each load issued before the previous
     // quarter is processed so the tensor-memory latency overlaps the exponentials.
@@ -456,7 +471,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           ls[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st8(tbase + C::kColP + 8 * qd, pk);
+        if (qd == 0) wait_pv();
+        if (pv_ok) tmem_st8(tbase + C::kColP + 8 * qd, pk);
         if constexpr (topk) {  // a quarter appends at most 16 candidates per row
           if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_flush();
         }
@@ -490,9 +506,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     bool ok = true;
     for (int c = 0; c < cs.total; ++c) {
       if (!wait_all(&S.s_full[t], c & 1)) { ok = false; break; }
-      // P V of the previous chunk must be done before P is overwritten and O is read
-      if (c > 0 && !wait_all(&S.pv_done[t], (c - 1) & 1)) { ok = false; break; }
       tc_fence_after();
+      pv_wait_for = c - 1;  // P(c - 1) V must be done before P is overwritten and O is read
       int local, start;
       br = cs.branch(c, local);
       const bool first = cs.first_of_branch(c);
@@ -501,6 +516,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       if (topk_on && br == 0) key_base = local * 64;
       float lsum;
       if (first) {
+        wait_pv();
+        if (!pv_ok) { ok = false; break; }
         if (c > 0) finalize(prev_br, m, l);
         const float mraw = chunk_max(need_mask);
         m = mraw == -INFINITY ? -INFINITY : mraw * sc;
@@ -508,6 +525,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         l = lsum;
       } else {
         const float mraw = exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
+        if (!pv_ok) { ok = false; break; }
         // move the reference only when the row max would exceed it by more than 2^8
         const float cand = mraw == -INFINITY ? -INFINITY : mraw * sc;
         const bool grow = cand > m + 8.f;
@@ -529,6 +547,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         }
         l += lsum;
       }
+      wait_pv();  // chunks whose exponentials stored nothing still keep the phase order
+      if (!pv_ok) { ok = false; break; }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&S.p_full[t]);

@@ -262,11 +262,12 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         if (c > 0) {
           // the element-wise warps are done with S, dP and P(c - 1)
           if (!mbar_wait(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
-          tc_fence_after();
-          second_stage(c - 1, prev_pass, prev_first);
         }
         tc_fence_after();
+        // S(c) (and dP(c)) go ahead of the P(c - 1) product: they touch other columns, and the
+        // element-wise warps wait for that product before they store P(c)
         first_stage(c, pass);
+        if (c > 0) second_stage(c - 1, prev_pass, prev_first);
         prev_pass = pass;
         prev_first = first;
       }
@@ -329,6 +330,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     };
     // P (pass A) or dS (pass B) of this half's 32 keys as bf16 pairs; S and dP are read 16
     // columns at a time, the next quarter's loads issued before the current one is processed
+    int pv_before_store = -1;
+    bool pv_ok = true;
     auto chunk_pass = [&](auto mask_tag, auto pass_tag, int nv, int br, float l2, float gb, float dlt) {
       constexpr bool kMask = decltype(mask_tag)::value;
       constexpr bool kPassB = decltype(pass_tag)::value;
@@ -353,7 +356,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           }
           pk[i] = pack_bf16x2(v2[0], v2[1]);
         }
-        tmem_st8(tbase + C::kColP + 16 * h + 8 * qd, pk);
+        if (qd == 0) pv_ok = pv_wait_through(pv_before_store);
+        if (pv_ok) tmem_st8(tbase + C::kColP + 16 * h + 8 * qd, pk);
       };
       tmem_ld16(tbase + C::kColS + 32 * h, sa);
       if constexpr (kPassB) tmem_ld16(tbase + C::kColDP + 32 * h, da);
@@ -372,7 +376,7 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       chunk_start(br, local, start, nv);
       if (!wait_all(&S.s_full, c & 1)) break;
       tc_fence_after();
-      if (!pv_wait_through(c - 1)) break;  // the P / dS columns are free again
+      pv_before_store = c - 1;  // the P / dS columns are free once P(c - 1)'s product is done
       const float l2 = br == 0 ? lse2[0] : (br == 1 ? lse2[1] : lse2[2]);
       const float gb = br == 0 ? gate[0] : (br == 1 ? gate[1] : gate[2]);
       const bool need_mask = br == 2 || nv < 32 * (h + 1);
@@ -383,6 +387,7 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         if (pass) chunk_pass(std::false_type{}, std::true_type{}, nv, br, l2, gb, delta);
         else chunk_pass(std::false_type{}, std::false_type{}, nv, br, l2, gb, delta);
       }
+      if (!pv_ok) break;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&S.p_full);
@@ -657,11 +662,10 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         if (!mbar_wait(&S.full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         if (c > 0) {
           if (!mbar_wait(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
-          tc_fence_after();
-          second_stage(c - 1);
         }
         tc_fence_after();
-        first_stage(c);
+        first_stage(c);  // ahead of the products of chunk c - 1 (other columns; see the query pass)
+        if (c > 0) second_stage(c - 1);
       }
       if (ok && mbar_wait(&S.p_full, (total - 1) & 1, abort, p.status)) {
         tc_fence_after();
@@ -689,6 +693,8 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       tc_fence_after();
       return true;
     };
+    int kv_before_store = -1;
+    bool kv_ok = true;
     auto chunk_pass = [&](int st, auto window_tag, auto mask_tag) {
       constexpr bool kWindow = decltype(window_tag)::value;
       constexpr bool kMask = decltype(mask_tag)::value;  // rows past the chunk's valid rows
@@ -715,8 +721,11 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
           pg[i] = pack_bf16x2(a2[0], a2[1]);
           ds[i] = pack_bf16x2(b2[0], b2[1]);
         }
-        tmem_st8(tbase + C::kColPg + 16 * h + 8 * qd, pg);
-        tmem_st8(tbase + C::kColDS + 16 * h + 8 * qd, ds);
+        if (qd == 0) kv_ok = pv_wait_through(kv_before_store);
+        if (kv_ok) {
+          tmem_st8(tbase + C::kColPg + 16 * h + 8 * qd, pg);
+          tmem_st8(tbase + C::kColDS + 16 * h + 8 * qd, ds);
+        }
       };
       tmem_ld16(tbase + C::kColS + 32 * h, sa);
       tmem_ld16(tbase + C::kColDP + 32 * h, da);
@@ -731,7 +740,7 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     for (int c = 0; ok && c < total; ++c) {
       if (!wait_all(&S.s_full, c & 1)) { ok = false; break; }
       tc_fence_after();
-      if (!pv_wait_through(c - 1)) { ok = false; break; }  // Pg and dS columns are free again
+      kv_before_store = c - 1;  // Pg and dS are free once chunk c - 1's products are done
       const int st = c % C::kStages;
       const bool partial = S.nrows[st] < C::kRowsPerChunk;
       if (kLocal && S.br[st] == 2) {
@@ -741,6 +750,7 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         if (partial) chunk_pass(st, std::false_type{}, std::true_type{});
         else chunk_pass(st, std::false_type{}, std::false_type{});
       }
+      if (!kv_ok) { ok = false; break; }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&S.p_full);
