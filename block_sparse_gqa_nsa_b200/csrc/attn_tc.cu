@@ -449,16 +449,14 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       uint32_t ra[16], rb[16];
       auto quarter = [&](const uint32_t* r, int qd) {
         uint32_t pk[8];
+        float qmx = -INFINITY;  // the quarter's max (top-k gate)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int j = 16 * qd + 2 * i;
           const float s0 = need_mask ? masked(r[2 * i], j) : __uint_as_float(r[2 * i]);
           const float s1 = need_mask ? masked(r[2 * i + 1], j + 1) : __uint_as_float(r[2 * i + 1]);
           mx[i & 3] = fmax3(mx[i & 3], s0, s1);
-          if constexpr (topk) {
-            topk_append(s0, j);
-            topk_append(s1, j + 1);
-          }
+          if constexpr (topk) qmx = fmax3(qmx, s0, s1);
           const float x0 = fmaf(s0, sc, nm), x1 = fmaf(s1, sc, nm);
           float p0, p1;
           if (kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
@@ -473,8 +471,17 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         }
         if (qd == 0) wait_pv();
         if (pv_ok) tmem_st8(tbase + C::kColP + 8 * qd, pk);
-        if constexpr (topk) {  // a quarter appends at most 16 candidates per row
-          if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_flush();
+        if constexpr (topk) {
+          // only quarters where some row of the warp has a score above its root visit the keys
+          if (__any_sync(0xffffffffu, qmx > thr)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int j = 16 * qd + i;
+              topk_append(need_mask ? masked(r[i], j) : __uint_as_float(r[i]), j);
+            }
+            // a quarter appends at most 16 candidates per row
+            if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_flush();
+          }
         }
       };
       tmem_ld16(tbase + C::kColS, ra);
