@@ -8,15 +8,16 @@
 // and the compressed keys/values are block means, so every token of block j receives
 // dKbar_j / n_j (and dVbar_j / n_j).
 //
-// Kernels (mma.sync m16n8k16 bf16 -> fp32; every sum in a fixed order, no float atomics):
-//   bwd_query:   one CTA per (query block, KV group, 128 rows): o_b recomputed -> dgates, Delta;
-//                then dQ from a second pass over each branch's keys.
-//   bwd_kv_local: one CTA per (key block, KV group): dK, dV of the block's tokens from the
-//                selected branch (query blocks that routed to it, in ascending order, from an
-//                inverse routing list) and from the window branch (its own block).
-//   bwd_kv_cmp:  one CTA per (64 block means, KV group, query split): partial dKbar, dVbar.
-//   bwd_finish:  dK = local part + (sum of the splits' dKbar of the token's block) / n_block.
-// The key-side passes compute S^T and dP^T (keys x query rows) directly, so P^T and dS^T are
+// Kernels (tcgen05 MMAs, bf16 operands, fp32 accumulators in tensor memory; every sum in a fixed
+// order, no float atomics):
+//   bwd_query_tc:  one CTA per (128 query rows, KV group, query block): per branch, pass A sums
+//                  dgates_b = sum_u P_u dP_u, pass B accumulates dQ_b = dS K.
+//   bwd_kv_tc:     the keys as the M dimension: local (one key block, group: the selected branch
+//                  from the query blocks that routed to it, ascending, from inverse routing
+//                  lists, then the window branch of its own block) and compressed (128 block
+//                  means, group, query split: partial dKbar, dVbar).
+//   bwd_finish:    dK = local part + (sum of the splits' dKbar of the token's block) / n_block.
+// The key passes compute S^T and dP^T (keys x query rows) directly, so P^T g and dS^T are
 // already in the A-operand layout of the dV and dK products.
 #include <type_traits>
 
@@ -26,12 +27,6 @@
 
 namespace lsrm {
 
-
-template <int D>
-__device__ __forceinline__ uint32_t bswz(int row, int ch) {
-  if (D == 32) return (uint32_t)(row * 64 + ((ch ^ ((row >> 1) & 3)) << 4));
-  return (uint32_t)(row * 128 + ((ch ^ (row & 7)) << 4));
-}
 
 struct BwdParams {
   const int32_t* off;
@@ -62,10 +57,11 @@ struct BwdParams {
 };
 
 // ------------------------------------------------------------------------------------------------
-// query pass on the tensor cores: per 128-row tile and branch, pass A recomputes o_b = P V
-// (P = exp(tau q.k - lse_b), normalised by the saved LSE) to get dgates_b and Delta_b; pass B
-// forms dS = P (g_b dO V^T - Delta_b) and accumulates dQ_b = dS K.
-//   TMEM (256 columns): S [0, 64) | dP [64, 128) | P or dS as bf16 pairs [128, 160) | O or dQ_b
+// query pass on the tensor cores: per 128-row tile and branch, pass A forms S = Q K^T and
+// dP = dO V^T and sums dgates_b = <dO, o_b> = sum_u P_u dP_u in fp32 (P = exp(tau q.k - lse_b),
+// normalised by the saved LSE; no P V product is needed); pass B forms dS = P (g_b dP - Delta_b)
+// with Delta_b = g_b dgates_b and accumulates dQ_b = dS K.
+//   TMEM (256 columns): S [0, 64) | dP [64, 128) | dS as bf16 pairs [128, 160) | dQ_b
 //   warp 0 TMA (Q and dO tiles once, then K/V chunks: every branch is streamed twice),
 //   warp 1 MMA issuer, warps 2-9 element-wise: two warps per TMEM lane quarter, each taking
 //   32 of a chunk's 64 keys (no online softmax here: the LSE is known, so the halves are
@@ -99,7 +95,10 @@ struct BqtSmem {
   uint8_t k[C::kStages][C::kKVBytes];
   uint8_t v[C::kStages][C::kKVBytes];
   float acc[D][128];       // dQ of the tile, column-major
+  float xdg[128];          // half 1's partial dgates sum, handed to half 0
+  float dgs[128];          // the full sum, handed back
   uint64_t q_full, kv_full[C::kStages], kv_empty[C::kStages], s_full, p_full, pv_done, drain;
+  uint64_t xfer[4], back[4];  // pass-A end hand-over between the two warps that own 32 rows
   uint32_t tmem_base;
   int abort;
   int n_sel;
@@ -162,6 +161,10 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     mbar_init(&S.p_full, 256);
     mbar_init(&S.pv_done, 1);
     mbar_init(&S.drain, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&S.xfer[q], 32);
+      mbar_init(&S.back[q], 32);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -229,22 +232,22 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       const uint64_t kd_mn = smem_desc(smem_u32(S.k[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
       const uint64_t vd_mn = smem_desc(smem_u32(S.v[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
       constexpr uint32_t kStep = C::kKVBytes >> 4, kRow16 = (16 * C::kRowBytes) >> 4;
-      // pass A: S = Q K^T;  pass B: S = Q K^T and dP = dO V^T  (both [128 x 64], K-major B)
+      // both passes: S = Q K^T and dP = dO V^T  (both [128 x 64], K-major B); a pass-A chunk's
+      // K/V stage is free as soon as these complete
       auto first_stage = [&](int c, int pass) {
         const uint64_t so = (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + C::kColS, qd + 2 * kk, kd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
-        if (pass) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + C::kColDP, od + 2 * kk, vd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::kColDP, od + 2 * kk, vd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
         mma_commit(&S.s_full);
+        if (!pass) mma_commit(&S.kv_empty[c % C::kStages]);
       };
-      // pass A: O += P V;  pass B: dQ_b += dS K  (A from tensor memory, MN-major B)
-      auto second_stage = [&](int c, int pass, bool first) {
-        const uint64_t bd = (pass ? kd_mn : vd_mn) + (uint64_t)((c % C::kStages) * kStep);
+      // pass B only: dQ_b += dS K  (A from tensor memory, MN-major B)
+      auto second_stage = [&](int c, bool first) {
+        const uint64_t bd = kd_mn + (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
         for (int kk = 0; kk < C::kKeys / 16; ++kk)
           mma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, bd + kk * kRow16, C::kIdescND,
@@ -267,13 +270,13 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         // S(c) (and dP(c)) go ahead of the P(c - 1) product: they touch other columns, and the
         // element-wise warps wait for that product before they store P(c)
         first_stage(c, pass);
-        if (c > 0) second_stage(c - 1, prev_pass, prev_first);
+        if (c > 0 && prev_pass) second_stage(c - 1, prev_first);
         prev_pass = pass;
         prev_first = first;
       }
       if (ok && mbar_wait(&S.p_full, (seq.total - 1) & 1, abort, p.status)) {
         tc_fence_after();
-        second_stage(seq.total - 1, prev_pass, prev_first);
+        if (prev_pass) second_stage(seq.total - 1, prev_first);
       }
       mma_commit(&S.drain);
       volatile int no_abort = 0;
@@ -314,7 +317,9 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       const bool w = mbar_wait(bar, parity, abort, p.status);
       return __all_sync(0xffffffffu, w);
     };
-    // one pv_done phase per chunk; while chunk c is worked on it has completed c - 1 or c phases
+    // pv_done completes once per pass-B chunk (its dS K product).  While the k-th pass-B chunk is
+    // worked on it has completed k - 1 or k phases: that chunk's S was issued after the product of
+    // pass-B chunk k - 2 (or much later than it), and product k needs this chunk's dS
     int pv_seen = 0;
     auto pv_wait_through = [&](int j) -> bool {
       while (pv_seen <= j) {
@@ -324,20 +329,19 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       tc_fence_after();
       return true;
     };
-    auto swz = [](int r, int ch) -> uint32_t {
-      if (D == 32) return (uint32_t)(r * 64 + ((ch ^ ((r >> 1) & 3)) << 4));
-      return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
-    };
-    // P (pass A) or dS (pass B) of this half's 32 keys as bf16 pairs; S and dP are read 16
-    // columns at a time, the next quarter's loads issued before the current one is processed
+    // Pass A: this half's share of dgates_b = sum_u P_u dP_u over its 32 keys, in fp32.
+    // Pass B: dS of its 32 keys as bf16 pairs.  S and dP are read 16 columns at a time, the next
+    // quarter's loads issued before the current one is processed.
     int pv_before_store = -1;
     bool pv_ok = true;
+    float dg_part = 0.f;
     auto chunk_pass = [&](auto mask_tag, auto pass_tag, int nv, int br, float l2, float gb, float dlt) {
       constexpr bool kMask = decltype(mask_tag)::value;
       constexpr bool kPassB = decltype(pass_tag)::value;
       uint32_t sa[16], sb[16], da[16], db[16];
       auto quarter_pass = [&](const uint32_t* sr, const uint32_t* dr, int qd) {
         uint32_t pk[8];
+        float dgq = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           float v2[2];
@@ -351,24 +355,30 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
             }
             float pr = fast_exp2(fmaf(__uint_as_float(sr[2 * i + e]), sc, -l2));
             if constexpr (kMask) pr = kv ? pr : 0.f;
-            if constexpr (kPassB) pr *= fmaf(gb, __uint_as_float(dr[2 * i + e]), -dlt);
-            v2[e] = pr;
+            if constexpr (kPassB) v2[e] = pr * fmaf(gb, __uint_as_float(dr[2 * i + e]), -dlt);
+            else dgq = fmaf(pr, __uint_as_float(dr[2 * i + e]), dgq);
           }
-          pk[i] = pack_bf16x2(v2[0], v2[1]);
+          if constexpr (kPassB) pk[i] = pack_bf16x2(v2[0], v2[1]);
         }
-        if (qd == 0) pv_ok = pv_wait_through(pv_before_store);
-        if (pv_ok) tmem_st8(tbase + C::kColP + 16 * h + 8 * qd, pk);
+        if constexpr (kPassB) {
+          if (qd == 0) pv_ok = pv_wait_through(pv_before_store);
+          if (pv_ok) tmem_st8(tbase + C::kColP + 16 * h + 8 * qd, pk);
+        } else {
+          dg_part += dgq;
+        }
       };
       tmem_ld16(tbase + C::kColS + 32 * h, sa);
-      if constexpr (kPassB) tmem_ld16(tbase + C::kColDP + 32 * h, da);
+      tmem_ld16(tbase + C::kColDP + 32 * h, da);
       tmem_ld_wait();
       tmem_ld16(tbase + C::kColS + 32 * h + 16, sb);
-      if constexpr (kPassB) tmem_ld16(tbase + C::kColDP + 32 * h + 16, db);
+      tmem_ld16(tbase + C::kColDP + 32 * h + 16, db);
       quarter_pass(sa, da, 0);
       tmem_ld_wait();
       quarter_pass(sb, db, 1);
     };
     float delta = 0.f;
+    int nb = 0;      // pass-B chunks done
+    int merges = 0;  // pass-A ends done
     for (int c = 0; c < seq.total; ++c) {
       int br, pass, local, start, nv;
       bool first, last;
@@ -376,7 +386,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       chunk_start(br, local, start, nv);
       if (!wait_all(&S.s_full, c & 1)) break;
       tc_fence_after();
-      pv_before_store = c - 1;  // the P / dS columns are free once P(c - 1)'s product is done
+      pv_before_store = nb - 1;  // the dS columns are free once the previous dS K product is done
+      if (!pass && first) dg_part = 0.f;
       const float l2 = br == 0 ? lse2[0] : (br == 1 ? lse2[1] : lse2[2]);
       const float gb = br == 0 ? gate[0] : (br == 1 ? gate[1] : gate[2]);
       const bool need_mask = br == 2 || nv < 32 * (h + 1);
@@ -391,35 +402,33 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&S.p_full);
-      if (last) {
-        if (!pv_wait_through(c)) break;
-        if (pass == 0) {
-          // o_b is final: dgates_b = <dO, o_b>, Delta_b = g_b dgates_b
-          float dg = 0.f;
-#pragma unroll
-          for (int i = 0; i < D / 32; ++i) {
-            uint32_t o[32];
-            tmem_ld32(tbase + C::kColO + 32 * i, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-              const uint4 u = *reinterpret_cast<const uint4*>(S.go + swz(row, 4 * i + ch));
-              const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                dg = fmaf(__uint_as_float(w4[e] << 16), __uint_as_float(o[8 * ch + 2 * e]), dg);
-                dg = fmaf(__uint_as_float(w4[e] & 0xFFFF0000u), __uint_as_float(o[8 * ch + 2 * e + 1]), dg);
-              }
-            }
-          }
-          delta = gb * dg;
-          if (h == 0 && valid) {
-            p.dgates[orow * p.NG + br] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
-            p.rowc[((size_t)br * p.N + t0 + tok_local) * p.Hq + g * p.G + R % p.G] =
-                make_float4(l2, gb, delta, __int_as_float(tok_local));
-          }
-        } else if (h == 0) {
-          // dQ_b is final: add tau dQ_b to the tile's dQ
+      if (pass) ++nb;
+      if (!last) continue;
+      if (pass == 0) {
+        // dgates_b: the two halves' sums meet (half 1 hands over, half 0 adds and hands back)
+        const uint32_t par = merges & 1;
+        ++merges;
+        float dg;
+        if (h == 1) {
+          S.xdg[row] = dg_part;
+          mbar_arrive(&S.xfer[quarter]);
+          if (!wait_all(&S.back[quarter], par)) break;
+          dg = S.dgs[row];
+        } else {
+          if (!wait_all(&S.xfer[quarter], par)) break;
+          dg = dg_part + S.xdg[row];
+          S.dgs[row] = dg;
+          mbar_arrive(&S.back[quarter]);
+        }
+        delta = gb * dg;
+        if (h == 0 && valid) {
+          p.dgates[orow * p.NG + br] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
+          p.rowc[((size_t)br * p.N + t0 + tok_local) * p.Hq + g * p.G + R % p.G] =
+              make_float4(l2, gb, delta, __int_as_float(tok_local));
+        }
+      } else {
+        if (!pv_wait_through(nb - 1)) break;  // dQ_b is final
+        if (h == 0) {
 #pragma unroll
           for (int i = 0; i < D / 32; ++i) {
             uint32_t o[32];
