@@ -59,9 +59,12 @@ struct TcCfg {
   static constexpr int kKVBytes = kKeys * kRowBytes;
   // tensor memory per tile: S (fp32 scores) | P (bf16 pairs) | O
   static constexpr int kColS = 0, kColP = kKeys, kColO = kKeys + kKeys / 2;
+  // second score buffer of the bound pass (odd chunks), in columns no other role uses there
+  static constexpr int kColS2 = kColsPerTile - kKeys;
   static constexpr uint32_t kIdescQK = idesc_bf16(128, kKeys, false);
   static constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
   static_assert(kColO + D <= kColsPerTile, "tensor memory budget");
+  static_assert(kColS2 >= kKeys, "second score buffer overlaps the first");
 };
 
 template <int D>
@@ -74,6 +77,7 @@ struct TcSmem {
   float cand[2][2 * C::kCand][128];  // top-k candidates per row: values, then block ids
   uint64_t q_full[2], kv_full[C::kStages], kv_empty[C::kStages];
   uint64_t s_full[2], p_full[2], pv_done[2], drain;
+  uint64_t s_full2[2], p_full2[2];  // bound pass: the odd chunks' score buffer
   uint32_t tmem_base;
   int abort;
   int n_sel;
@@ -102,6 +106,10 @@ struct TcParams {
   int32_t* topk_idx;
   int topk_k;
   const uint32_t* forced_bits;
+  // per-row lower bound on the topk_k-th largest non-forced logit [rows][topk_heads]: the bound
+  // pass (bound_pass = 1: scores only, no softmax, no P V) writes it; the top-k pass reads it
+  float* topk_thr;
+  int bound_pass;
 };
 
 enum : int { TC_CMP = 1, TC_SLC = 2, TC_WIN = 4 };
@@ -141,6 +149,36 @@ __device__ __forceinline__ void chunk_keys(const TcSmem<D>& S, const TcParams& p
   }
 }
 
+// Streaming top-k merge: the n buffered candidates of one row (values at cand[e * 128], block ids
+// at cand[(cap + e) * 128]) enter, in order, the row's 32-entry min-heap (values at heap[i * 128],
+// ids at heap[(32 + i) * 128]; the root is the worst entry in the order (logit desc, block asc))
+// when strictly above the current root.  Returns the new root value.
+__device__ __noinline__ float topk_merge(float* heap, const float* cand, int n, int cap, float thr) {
+  auto hv = [&](int i) -> float& { return heap[i * 128]; };
+  auto hj = [&](int i) -> int& { return reinterpret_cast<int&>(heap[(32 + i) * 128]); };
+  auto worse = [](float va, int ja, float vb, int jb) { return va < vb || (va == vb && ja > jb); };
+  for (int e = 0; e < n; ++e) {
+    const float sv = cand[e * 128];
+    const int jg = reinterpret_cast<const int&>(cand[(cap + e) * 128]);
+    if (!(sv > thr)) continue;
+    int i = 0;
+    while (true) {
+      const int lc = 2 * i + 1, rc = lc + 1;
+      if (lc >= 32) break;
+      int cc = lc;
+      if (rc < 32 && worse(hv(rc), hj(rc), hv(lc), hj(lc))) cc = rc;
+      if (!worse(hv(cc), hj(cc), sv, jg)) break;
+      hv(i) = hv(cc);
+      hj(i) = hj(cc);
+      i = cc;
+    }
+    hv(i) = sv;
+    hj(i) = jg;
+    thr = hv(0);
+  }
+  return thr;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kCtasPerSm)
 nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -178,6 +216,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       mbar_init(&S.s_full[t], 1);
       mbar_init(&S.p_full[t], 128);
       mbar_init(&S.pv_done[t], 1);
+      mbar_init(&S.s_full2[t], 1);
+      mbar_init(&S.p_full2[t], 128);
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&S.kv_full[s], 1);
@@ -218,9 +258,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         int local, start, nvalid;
         const int br = cs.branch(c, local);
         chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nvalid);
-        mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
+        mbar_arrive_expect_tx(&S.kv_full[st], p.bound_pass ? C::kKVBytes : 2 * C::kKVBytes);
         tma_load_3d(S.k[st], br == 0 ? &kcmap : &kmap, &S.kv_full[st], 0, g, start);
-        tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
+        if (!p.bound_pass) tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
         issued = c + 1;
       }
       if (*abort) {
@@ -244,8 +284,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       const uint64_t kdesc = smem_desc(smem_u32(S.k[0]), 16, C::kAtomBytes, C::kLayout);
       const uint64_t vdesc = smem_desc(smem_u32(S.v[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
       constexpr uint32_t kStageStep = C::kKVBytes >> 4;
-      auto issue_qk = [&](int t, int c) {
-        const uint32_t d = tmem + t * C::kColsPerTile + C::kColS;
+      auto issue_qk = [&](int t, int c, int col) {
+        const uint32_t d = tmem + t * C::kColsPerTile + col;
         const uint64_t bd = kdesc + (uint64_t)((c % C::kStages) * kStageStep);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) mma_ss(d, qdesc[t] + 2 * k, bd + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
@@ -259,7 +299,28 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           mma_ts(d, tmem + t * C::kColsPerTile + C::kColP + kk * 8, bd + kk * (16 * C::kRowBytes >> 4), C::kIdescPV,
                  (first && kk == 0) ? 0u : 1u);
       };
-      for (int c = 0; ok && c < cs.total; ++c) {
+      // bound pass: scores only, double-buffered (even chunks in S, odd chunks in S2) so that the
+      // next chunk's MMAs run while the softmax warps reduce the current one; each buffer has its
+      // own full/free barrier pair, completed once per two chunks
+      for (int c = 0; ok && p.bound_pass && c < cs.total; ++c) {
+        if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const int b = c & 1;
+        for (int t = 0; t < 2; ++t) {
+          if (c >= 2) {
+            if (!mbar_wait(b ? &S.p_full2[t] : &S.p_full[t], ((c >> 1) - 1) & 1, abort, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          issue_qk(t, c, b ? C::kColS2 : C::kColS);
+          mma_commit(b ? &S.s_full2[t] : &S.s_full[t]);
+        }
+        if (!ok) break;
+        mma_commit(&S.kv_empty[c % C::kStages]);
+      }
+      for (int c = 0; ok && !p.bound_pass && c < cs.total; ++c) {
         if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
@@ -269,7 +330,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             if (!mbar_wait(&S.p_full[t], (c - 1) & 1, abort, p.status)) { ok = false; break; }
             tc_fence_after();
           }
-          issue_qk(t, c);
+          issue_qk(t, c, C::kColS);
           mma_commit(&S.s_full[t]);
           if (c > 0) {
             issue_pv(t, c - 1);
@@ -279,7 +340,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (!ok) break;
         if (c > 0) mma_commit(&S.kv_empty[(c - 1) % C::kStages]);
       }
-      for (int t = 0; ok && t < 2; ++t) {
+      for (int t = 0; ok && !p.bound_pass && t < 2; ++t) {
         if (!mbar_wait(&S.p_full[t], (cs.total - 1) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         issue_pv(t, cs.total - 1);
@@ -359,51 +420,40 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     // Scores above the (possibly stale) root are first appended to a per-row candidate buffer;
     // the warp merges its rows' buffers together, re-testing every candidate in key order
     // against the live root, which makes the same decisions as inserting key by key while
-    // keeping the divergent heap work out of the per-key loop.  Forced blocks are dropped here.
+    // keeping the divergent heap work out of the per-key loop.  Forced blocks never enter the
+    // buffer (a 64-bit mask per chunk from the forced-block bitmap).  The merge is one function
+    // outside the unrolled per-key code, which would otherwise carry a copy at every call site.
     const bool topk_on = (D == 64) && p.topk_idx != nullptr;
     float thr = -INFINITY;
     int key_base = 0;  // block id of key 0 of the current chunk
+    uint64_t fmask = 0;  // forced blocks among the chunk's 64 keys (never candidates)
     int ncand = 0;     // this row's buffered candidates
     float* cbuf = &S.cand[t][0][row];
     auto hv = [&](int i) -> float& { return acc[i * 128]; };
     auto hj = [&](int i) -> int& { return reinterpret_cast<int&>(acc[(32 + i) * 128]); };
     auto worse = [&](float va, int ja, float vb, int jb) { return va < vb || (va == vb && ja > jb); };
-    auto heap_insert = [&](float sv, int jg) {
-      int i = 0;
-      while (true) {
-        const int lc = 2 * i + 1, rc = lc + 1;
-        if (lc >= 32) break;
-        int cc = lc;
-        if (rc < 32 && worse(hv(rc), hj(rc), hv(lc), hj(lc))) cc = rc;
-        if (!worse(hv(cc), hj(cc), sv, jg)) break;
-        hv(i) = hv(cc);
-        hj(i) = hj(cc);
-        i = cc;
-      }
-      hv(i) = sv;
-      hj(i) = jg;
-      thr = hv(0);
-    };
     auto topk_append = [&](float sv, int j) {
-      if (sv > thr) {
+      if (sv > thr && !((fmask >> j) & 1ull)) {
         cbuf[ncand * 128] = sv;
         reinterpret_cast<int&>(cbuf[(C::kCand + ncand) * 128]) = key_base + j;
         ++ncand;
       }
     };
     auto topk_flush = [&]() {
-#pragma unroll 1
-      for (int e = 0; e < ncand; ++e) {
-        const float sv = cbuf[e * 128];
-        const int jg = reinterpret_cast<const int&>(cbuf[(C::kCand + e) * 128]);
-        if (sv > thr && !((p.forced_bits[jg >> 5] >> (jg & 31)) & 1u)) heap_insert(sv, jg);
-      }
+      thr = topk_merge(acc, cbuf, ncand, C::kCand, thr);
       ncand = 0;
     };
     if (topk_on) {
+      // With a lower bound b on the k-th largest non-forced logit, the heap starts full of
+      // placeholders just below b: every key at or above b gets in, no key below b can be among
+      // the k best (k keys at or above b exist), and the placeholders are all displaced.
+      if (p.topk_thr != nullptr && valid) {
+        const float b = p.topk_thr[(size_t)(t0 + R) * p.Hkv + g];
+        if (b > -INFINITY) thr = nextafterf(b, -INFINITY);
+      }
 #pragma unroll 1
       for (int i = 0; i < 32; ++i) {
-        hv(i) = -INFINITY;
+        hv(i) = thr;
         hj(i) = INT_MAX;
       }
     }
@@ -509,9 +559,72 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
                        : exp_pass_t(mref, lsum, std::false_type{}, std::false_type{});
     };
 
+    if (p.bound_pass) {
+      // ---- bound pass: per row, the max non-forced logit of each of 64 key groups (chunk c
+      // joins group c mod 64), then the topk_k-th largest group max.  Groups are disjoint, so
+      // at least topk_k distinct keys score at or above that value: a lower bound on the
+      // topk_k-th largest logit that needs no selection in the per-key loop.
+      float* gmax = acc;  // gmax[i * 128], i < 64 (the output accumulator is unused here)
+#pragma unroll 1
+      for (int i = 0; i < 64; ++i) gmax[i * 128] = -INFINITY;
+      auto bound_max_t = [&](uint32_t col, auto mask_tag) -> float {
+        constexpr bool need_mask = decltype(mask_tag)::value;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+          tmem_ld32(tbase + col + 32 * h, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float s0 = __uint_as_float(r[i]), s1 = __uint_as_float(r[i + 1]);
+            if (need_mask) {
+              const int j = 32 * h + i;
+              if (j >= nv || ((fmask >> j) & 1ull)) s0 = -INFINITY;
+              if (j + 1 >= nv || ((fmask >> (j + 1)) & 1ull)) s1 = -INFINITY;
+            }
+            mx[(i >> 1) & 3] = fmax3(mx[(i >> 1) & 3], s0, s1);
+          }
+        }
+        return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      };
+      bool okb = true;
+      for (int c = 0; c < cs.total; ++c) {
+        const int b = c & 1;
+        if (!wait_all(b ? &S.s_full2[t] : &S.s_full[t], (c >> 1) & 1)) { okb = false; break; }
+        tc_fence_after();
+        nv = min(64, n_ckeys - c * 64);
+        const uint32_t w0 = p.forced_bits[c * 2], w1 = p.forced_bits[c * 2 + 1];
+        fmask = (uint64_t)w0 | ((uint64_t)w1 << 32);
+        const uint32_t col = b ? C::kColS2 : C::kColS;
+        const float mx = (nv < 64 || fmask != 0) ? bound_max_t(col, std::true_type{})
+                                                 : bound_max_t(col, std::false_type{});
+        tc_fence_before();
+        mbar_arrive(b ? &S.p_full2[t] : &S.p_full[t]);
+        float& gv = gmax[(c & 63) * 128];
+        gv = fmaxf(gv, mx);
+      }
+      if (okb && valid) {
+        // the k-th largest of the 64 group maxima: the smallest value with fewer than k above it
+        float v[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) v[i] = gmax[i * 128];
+        float bound = INFINITY;
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i) {
+          const float vi = gmax[i * 128];
+          int above = 0;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) above += v[j] > vi ? 1 : 0;
+          if (above < p.topk_k) bound = fminf(bound, vi);
+        }
+        p.topk_thr[(size_t)(t0 + R) * p.Hkv + g] = bound;
+      }
+    }
+
     int prev_br = -1;
-    bool ok = true;
-    for (int c = 0; c < cs.total; ++c) {
+    bool ok = !p.bound_pass;
+    for (int c = 0; ok && c < cs.total; ++c) {
       if (!wait_all(&S.s_full[t], c & 1)) { ok = false; break; }
       tc_fence_after();
       pv_wait_for = c - 1;  // P(c - 1) V must be done before P is overwritten and O is read
@@ -520,7 +633,11 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       const bool first = cs.first_of_branch(c);
       chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nv);
       const bool need_mask = br == 2 || nv < 64;
-      if (topk_on && br == 0) key_base = local * 64;
+      if (topk_on && br == 0) {
+        key_base = local * 64;
+        const uint32_t w0 = p.forced_bits[key_base >> 5], w1 = p.forced_bits[(key_base >> 5) + 1];
+        fmask = (uint64_t)w0 | ((uint64_t)w1 << 32);
+      }
       float lsum;
       if (first) {
         wait_pv();
@@ -561,7 +678,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       mbar_arrive(&S.p_full[t]);
       prev_br = br;
     }
-    if (cs.total == 0 && valid) {  // no keys at all (e.g. an empty forced set): defined outputs
+    if (cs.total == 0 && valid && !p.bound_pass) {  // no keys at all (e.g. an empty forced set): defined outputs
       if (p.obranch != nullptr)
         for (int i = 0; i < D; ++i) p.obranch[orow * D + i] = 0.f;
       if (p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first] = -INFINITY;
@@ -679,10 +796,12 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
 // (kc, vc) ([kc_rows][H][D]), in fixed groups of 256 query rows: the pooled-query compressed
 // branch (optionally with the streaming top-k that routes it) and the forced-block part of the
 // pooled-query selected branch.  Writes fp32 obranch [n_q][H][D] and the natural-log lse [n_q][H].
+// With topk_thr ([n_q][H] fp32 scratch) the top-k pass is preceded by the bound pass, whose
+// per-row lower bound on the k-th logit lets the top-k pass skip almost every candidate.
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
-                              uint32_t* status, cudaStream_t stream) {
+                              float* topk_thr, uint32_t* status, cudaStream_t stream) {
   if (topk_idx != nullptr && (D != 64 || topk_k < 1 || topk_k > 32 || forced_bits == nullptr))
     return LSRM_ERR_UNSUPPORTED;
   if ((n_q + 255) / 256 > 65535 || n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
@@ -713,8 +832,19 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
   p.topk_k = topk_k;
   p.forced_bits = forced_bits;
   if (D == 32) return launch_tc_d<32>(d, p, q, nullptr, nullptr, kc, vc, kc_rows, stream);
-  if (D == 64) return launch_tc_d<64>(d, p, q, nullptr, nullptr, kc, vc, kc_rows, stream);
-  return LSRM_ERR_UNSUPPORTED;
+  if (D != 64) return LSRM_ERR_UNSUPPORTED;
+  if (topk_idx != nullptr && topk_thr != nullptr) {
+    TcParams pb = p;
+    pb.obranch = nullptr;
+    pb.lse = nullptr;
+    pb.topk_idx = nullptr;
+    pb.topk_thr = topk_thr;
+    pb.bound_pass = 1;
+    const lsrm_status st = launch_tc_d<64>(d, pb, q, nullptr, nullptr, kc, vc, kc_rows, stream);
+    if (st != LSRM_OK) return st;
+    p.topk_thr = topk_thr;
+  }
+  return launch_tc_d<64>(d, p, q, nullptr, nullptr, kc, vc, kc_rows, stream);
 }
 
 }  // namespace lsrm

@@ -23,7 +23,7 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
-                              uint32_t* status, cudaStream_t stream);
+                              float* topk_thr, uint32_t* status, cudaStream_t stream);
 lsrm_status launch_pooled_broadcast(const lsrm_nsa_desc& d, const int32_t* off, const float* o_blk,
                                     const float* lse_blk, float* o_cmp, float* lse, cudaStream_t s);
 lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, const void* k, const void* v,
@@ -100,7 +100,8 @@ lsrm_status pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, c
     }
   }
   return launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc, kc, vc, d.n_blocks, d.n_blocks, nullptr,
-                           tau_of(d), o_blk, l_blk, idx, idx ? d.top_k : 0, idx ? bits : nullptr, status_of(ws), s);
+                           tau_of(d), o_blk, l_blk, idx, idx ? d.top_k : 0, idx ? bits : nullptr,
+                           idx ? wsp<float>(ws, w.rthr) : nullptr, status_of(ws), s);
 }
 
 #define LSRM_TRY(x)                         \
@@ -266,12 +267,13 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
     if (route && d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
     LSRM_TRY(launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc16, kc16, vc16, d.n_blocks, d.n_blocks,
                                nullptr, tau_of(d), o_blk, l_blk, route ? idx : nullptr, route ? d.top_k : 0,
-                               route ? wsp<uint32_t>(ws, w.fbits) : nullptr, status_of(ws), s));
+                               route ? wsp<uint32_t>(ws, w.fbits) : nullptr, route ? wsp<float>(ws, w.rthr) : nullptr,
+                               status_of(ws), s));
     float* ofrc = wsp<float>(ws, w.ofrc);
     float* lfrc = wsp<float>(ws, w.lfrc);
     const long long cap = (long long)(d.n_forced > 0 ? d.n_forced : 1) * d.max_block_len;
     LSRM_TRY(launch_attn_dense(d.head_dim, d.n_tokens, d.n_q_heads, q, wsp<void>(ws, w.kf), wsp<void>(ws, w.vf),
-                               cap, 0, ftotal, tau_of(d), ofrc, lfrc, nullptr, 0, nullptr, status_of(ws), s));
+                               cap, 0, ftotal, tau_of(d), ofrc, lfrc, nullptr, 0, nullptr, nullptr, status_of(ws), s));
     return launch_speed3r_routed(d, off, q, k, v, gates, idx, ofrc, lfrc, o_blk, l_blk, out, lse_or_null,
                                  status_of(ws), s);
   }

@@ -23,6 +23,7 @@ struct Workspace {
   // pooled-query (Speed3R) path: forced-block bitmap, prefix and total, gathered forced K / V,
   // and the forced part of the selected branch per token
   size_t fbits, fpre, ftotal, kf, vf, ofrc, lfrc;
+  size_t rthr;  // per (block, head) lower bound on the k-th routing logit
   size_t total;
 };
 
@@ -84,6 +85,7 @@ inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   w.vf = o;        o = align256(o + nf_tok * Hkv * D * 2);
   w.ofrc = o;      o = align256(o + (d.pooled_q ? N * Hq * D * 4 : 0));
   w.lfrc = o;      o = align256(o + (d.pooled_q ? N * Hq * 4 : 0));
+  w.rthr = o;      o = align256(o + (d.pooled_q ? B * Hq * 4 : 0));
   w.total = o;
   return w;
 }

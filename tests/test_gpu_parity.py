@@ -549,6 +549,47 @@ def test_speed3r_routing_with_a_late_dominant_block():
     assert_close(to_np(out), ref, "out")
 
 
+def test_speed3r_routing_ties_break_by_block_id():
+    # Two classes of non-forced blocks with bit-identical pooled keys: even blocks share one key
+    # vector u, odd blocks the zero vector.  Every row then sees exactly equal logits inside each
+    # class, so its top-k is fixed by the order (logit desc, block asc) alone: the k smallest ids
+    # of the class whose logit is larger (with q.u clear of zero at operand precision).  Ties sit
+    # exactly at the k-th logit, which is where a lower bound on it must still let them through.
+    w = make_workload("speed3r_small", n_frames=6)
+    forced = set(w.forced.tolist())
+    rng = np.random.default_rng(7)
+    u = f32_to_bf16_bits(rng.standard_normal(w.head_dim).astype(np.float32))
+    k = w.k.copy()
+    for b in range(w.n_blocks):
+        if b in forced:
+            continue
+        k[w.off[b]:w.off[b + 1]] = u if b % 2 == 0 else 0
+    w.k = k
+    c = DeviceCase(w)
+    idx = c.empty(w.n_blocks, w.n_q_heads, w.top_k, dtype=torch.int32)
+    out = c.empty(w.n_tokens, w.n_q_heads, w.head_dim, dtype=torch.bfloat16)
+    nsa.lsrm_nsa_forward(c.desc, c.off, c.q, c.k, c.v, c.gates, None, nsa.ROUTE_SCORE, out, idx, None, c.ws)
+    assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
+    gidx = to_np(idx)
+    D = oracle_desc(w)
+    from workloads.nsa_workloads import bf16_bits_to_f32
+    qc = bf16_bits_to_f32(f32_to_bf16_bits(O.compress(D, w.off, w.q, w.n_q_heads).astype(np.float32)))
+    uf = bf16_bits_to_f32(u).astype(np.float64)
+    even = [b for b in range(0, w.n_blocks, 2) if b not in forced]
+    odd = [b for b in range(1, w.n_blocks, 2) if b not in forced]
+    assert len(even) >= w.top_k and len(odd) >= w.top_k
+    checked = 0
+    for a in range(w.n_blocks):
+        for h in range(w.n_q_heads):
+            lu = float(np.dot(qc[a, h].astype(np.float64), uf)) * w.scale
+            if abs(lu) < 1e-3:
+                continue
+            want = (even if lu > 0 else odd)[:w.top_k]
+            assert gidx[a, h].tolist() == want, (a, h, lu)
+            checked += 1
+    assert checked > 0.9 * w.n_blocks * w.n_q_heads
+
+
 def test_two_gate_layer_forward_and_backward():
     # n_gates = 2: compressed and selected branches only (no window), forward and backward
     w = make_workload("ragged_geo")
