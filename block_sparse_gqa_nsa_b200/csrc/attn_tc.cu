@@ -48,23 +48,34 @@ struct TcCfg {
   static constexpr int kRows = 128;
   static constexpr int kKeys = 64;                 // keys per chunk = N of S = Q K^T (one block)
   static constexpr int kStages = D == 32 ? 4 : 3;  // K/V ring
-  static constexpr int kCand = D == 64 ? 32 : 1;   // streaming top-k candidate buffer per row
+  // streaming top-k candidates per row: logits in the (then unused) output accumulator, block ids
+  // in the candidate array
+  static constexpr int kCand = D == 64 ? 64 : 1;
+  // bound pass: chunks of kBoundKeys keys (one N = 128 MMA per K step), two score buffers per
+  // tile, and a ring of 16 KB K slots laid over the K/V stages and the candidate-id array
+  static constexpr int kBoundKeys = 128;
+  static constexpr int kBoundBufs = 2;
+  static constexpr int kBoundStages = 6;
+  static constexpr uint32_t kIdescBound = idesc_bf16(128, kBoundKeys, false);
   static constexpr int kCtasPerSm = D == 32 ? 2 : 1;
   static constexpr int kTmemCols = D == 32 ? 256 : 512;   // per CTA (power of two)
   static constexpr int kColsPerTile = kTmemCols / 2;
   static constexpr int kRowBytes = D * 2;
+  static constexpr int kBoundSlotBytes = kBoundKeys * kRowBytes;
   static constexpr uint32_t kLayout = D == 32 ? kLayoutSW64 : kLayoutSW128;
   static constexpr uint32_t kAtomBytes = 8 * kRowBytes;  // 8 rows of one swizzle atom
   static constexpr int kQBytes = kRows * kRowBytes;
   static constexpr int kKVBytes = kKeys * kRowBytes;
   // tensor memory per tile: S (fp32 scores) | P (bf16 pairs) | O
   static constexpr int kColS = 0, kColP = kKeys, kColO = kKeys + kKeys / 2;
-  // second score buffer of the bound pass (odd chunks), in columns no other role uses there
-  static constexpr int kColS2 = kColsPerTile - kKeys;
+
   static constexpr uint32_t kIdescQK = idesc_bf16(128, kKeys, false);
   static constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
   static_assert(kColO + D <= kColsPerTile, "tensor memory budget");
-  static_assert(kColS2 >= kKeys, "second score buffer overlaps the first");
+  static_assert(kCand <= D, "candidate logits live in the output accumulator");
+  static_assert(kCand <= 64, "candidate ranks are counted in registers");
+  static_assert(D != 64 || kBoundBufs * kBoundKeys <= kColsPerTile, "bound-pass score buffers");
+  static_assert(D != 64 || 3 * kBoundSlotBytes <= 2 * kStages * kKVBytes, "bound-pass K slots over K/V");
 };
 
 template <int D>
@@ -74,16 +85,29 @@ struct TcSmem {
   uint8_t k[C::kStages][C::kKVBytes];
   uint8_t v[C::kStages][C::kKVBytes];
   float acc[2][D][128];  // gated sum per tile, column-major so a warp's rows are one bank row
-  float cand[2][2 * C::kCand][128];  // top-k candidates per row: values, then block ids
+  int cand_id[2][C::kCand][128];  // top-k candidate block ids per row (logits in acc)
   uint64_t q_full[2], kv_full[C::kStages], kv_empty[C::kStages];
   uint64_t s_full[2], p_full[2], pv_done[2], drain;
-  uint64_t s_full2[2], p_full2[2];  // bound pass: the odd chunks' score buffer
+  // bound pass: K ring, and per tile and score buffer a full (MMA) / free (softmax) pair
+  uint64_t kb_full[C::kBoundStages], kb_empty[C::kBoundStages];
+  uint64_t bs_full[2][C::kBoundBufs], bs_free[2][C::kBoundBufs];
   uint32_t tmem_base;
   int abort;
   int n_sel;
   int sel_start[kTcMaxSel];
   int sel_n[kTcMaxSel];
 };
+static_assert(sizeof(TcSmem<64>) + 1024 <= 227 * 1024, "shared memory per CTA (d = 64)");
+static_assert(sizeof(TcSmem<64>::cand_id) >= (TcCfg<64>::kBoundStages - 3) * TcCfg<64>::kBoundSlotBytes,
+              "bound-pass K slots over the candidate ids");
+// bound-pass K slot s: three over the K/V stages (contiguous), the rest over the candidate ids
+template <int D>
+__device__ __forceinline__ uint8_t* bound_slot(TcSmem<D>& S, int s) {
+  using C = TcCfg<D>;
+  return s < 3 ? S.k[0] + s * C::kBoundSlotBytes
+               : reinterpret_cast<uint8_t*>(&S.cand_id[0][0][0]) + (s - 3) * C::kBoundSlotBytes;
+}
+static_assert(2 * (sizeof(TcSmem<32>) + 1024) <= 228 * 1024, "shared memory per SM (d = 32, two CTAs)");
 
 struct TcParams {
   const int32_t* off;
@@ -149,34 +173,79 @@ __device__ __forceinline__ void chunk_keys(const TcSmem<D>& S, const TcParams& p
   }
 }
 
-// Streaming top-k merge: the n buffered candidates of one row (values at cand[e * 128], block ids
-// at cand[(cap + e) * 128]) enter, in order, the row's 32-entry min-heap (values at heap[i * 128],
-// ids at heap[(32 + i) * 128]; the root is the worst entry in the order (logit desc, block asc))
-// when strictly above the current root.  Returns the new root value.
-__device__ __noinline__ float topk_merge(float* heap, const float* cand, int n, int cap, float thr) {
-  auto hv = [&](int i) -> float& { return heap[i * 128]; };
-  auto hj = [&](int i) -> int& { return reinterpret_cast<int&>(heap[(32 + i) * 128]); };
-  auto worse = [](float va, int ja, float vb, int jb) { return va < vb || (va == vb && ja > jb); };
-  for (int e = 0; e < n; ++e) {
-    const float sv = cand[e * 128];
-    const int jg = reinterpret_cast<const int&>(cand[(cap + e) * 128]);
-    if (!(sv > thr)) continue;
-    int i = 0;
-    while (true) {
-      const int lc = 2 * i + 1, rc = lc + 1;
-      if (lc >= 32) break;
-      int cc = lc;
-      if (rc < 32 && worse(hv(rc), hj(rc), hv(lc), hj(lc))) cc = rc;
-      if (!worse(hv(cc), hj(cc), sv, jg)) break;
-      hv(i) = hv(cc);
-      hj(i) = hj(cc);
-      i = cc;
-    }
-    hv(i) = sv;
-    hj(i) = jg;
-    thr = hv(0);
+// Top-k over a row's buffered candidates (logits at val[i * 128], block ids at id[i * 128], in
+// arrival order, which is increasing block order).  The rank of entry i in the order (logit desc,
+// block asc) is the number of entries with a larger logit plus the earlier entries with an equal
+// one; ranks form a permutation of 0..n-1.
+constexpr int kMaxCand = 64;
+
+// exact rank from shared memory, ties included (the fallback when two logits are equal)
+__device__ __forceinline__ int cand_rank_exact(const float* val, int n, int i, float vi) {
+  int r = 0;
+  for (int j = 0; j < n; ++j) {
+    const float vj = val[j * 128];
+    r += (vj > vi || (vj == vi && j < i)) ? 1 : 0;
   }
-  return thr;
+  return r;
+}
+
+// Ranks of all n <= kMaxCand candidates, each logit counted against all the others held in
+// registers: f(i, r) is called with r = the number of strictly larger logits, which is the rank
+// when no two logits are equal.  That holds exactly when the counts sum to n (n - 1) / 2, and
+// the return value says so; otherwise the caller takes the exact tie-aware ranks.
+template <class F>
+__device__ __forceinline__ bool cand_ranks_fast(const float* val, int n, F f) {
+  float v[kMaxCand];
+#pragma unroll
+  for (int j = 0; j < kMaxCand; ++j) v[j] = j < n ? val[j * 128] : -INFINITY;
+  int sum = 0;
+  for (int i = 0; i < n; ++i) {
+    const float vi = val[i * 128];
+    int r = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxCand; ++j) r += v[j] > vi ? 1 : 0;
+    f(i, r);
+    sum += r;
+  }
+  return 2 * sum == n * (n - 1);
+}
+
+struct KeepBest {
+  int n;
+  float thr;
+};
+
+// Keep the k best of a row's n > k buffered candidates, in buffer order; the new gate is the k-th
+// best logit (a later key, from a larger block, has to beat it strictly).
+__device__ __noinline__ KeepBest topk_keep_best(float* val, int* id, int n, int k) {
+  uint64_t keep = 0;
+  if (!cand_ranks_fast(val, n, [&](int i, int r) { keep |= (uint64_t)(r < k) << i; })) {
+    keep = 0;
+    for (int i = 0; i < n; ++i) keep |= (uint64_t)(cand_rank_exact(val, n, i, val[i * 128]) < k) << i;
+  }
+  int m = 0;
+  float lo = INFINITY;
+  for (int i = 0; i < n; ++i) {
+    if (!((keep >> i) & 1ull)) continue;
+    const float v = val[i * 128];
+    val[m * 128] = v;
+    id[m * 128] = id[i * 128];
+    lo = fminf(lo, v);
+    ++m;
+  }
+  return KeepBest{m, lo};
+}
+
+// Emit the row's k best in order (logit desc, block asc); a row with fewer than k candidates pads
+// with -1.
+__device__ __noinline__ void topk_emit(const float* val, const int* id, int n, int k, int32_t* dst) {
+  if (!cand_ranks_fast(val, n, [&](int i, int r) { if (r < k) dst[r] = id[i * 128]; })) {
+    for (int i = 0; i < n; ++i) {
+      const int r = cand_rank_exact(val, n, i, val[i * 128]);
+      if (r < k) dst[r] = id[i * 128];
+    }
+  }
+  for (int r = n; r < k; ++r) dst[r] = -1;
 }
 
 template <int D>
@@ -216,8 +285,14 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       mbar_init(&S.s_full[t], 1);
       mbar_init(&S.p_full[t], 128);
       mbar_init(&S.pv_done[t], 1);
-      mbar_init(&S.s_full2[t], 1);
-      mbar_init(&S.p_full2[t], 128);
+      for (int b = 0; b < C::kBoundBufs; ++b) {
+        mbar_init(&S.bs_full[t][b], 1);
+        mbar_init(&S.bs_free[t][b], 128);
+      }
+    }
+    for (int s = 0; s < C::kBoundStages; ++s) {
+      mbar_init(&S.kb_full[s], 1);
+      mbar_init(&S.kb_empty[s], 1);
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&S.kv_full[s], 1);
@@ -252,29 +327,42 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         tma_load_3d(S.q[t], &qmap, &S.q_full[t], 0, g * p.G, t0 + (tile0 + t) * tokens_per_tile);
       }
       int issued = 0;
-      for (int c = 0; c < cs.total; ++c) {
+      // bound pass (compressed keys only): K alone, kBoundKeys rows per box
+      const int nb = p.bound_pass ? (n_ckeys + C::kBoundKeys - 1) / C::kBoundKeys : 0;
+      for (int c = 0; c < nb; ++c) {
+        const int st = c % C::kBoundStages;
+        if (c >= C::kBoundStages &&
+            !mbar_wait(&S.kb_empty[st], ((c / C::kBoundStages) + 1) & 1, abort, p.status))
+          break;
+        mbar_arrive_expect_tx(&S.kb_full[st], C::kBoundSlotBytes);
+        tma_load_3d(bound_slot(S, st), &kcmap, &S.kb_full[st], 0, g, c * C::kBoundKeys);
+        issued = c + 1;
+      }
+      for (int c = 0; !p.bound_pass && c < cs.total; ++c) {
         const int st = c % C::kStages;
         if (c >= C::kStages && !mbar_wait(&S.kv_empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
         int local, start, nvalid;
         const int br = cs.branch(c, local);
         chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nvalid);
-        mbar_arrive_expect_tx(&S.kv_full[st], p.bound_pass ? C::kKVBytes : 2 * C::kKVBytes);
+        mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
         tma_load_3d(S.k[st], br == 0 ? &kcmap : &kmap, &S.kv_full[st], 0, g, start);
-        if (!p.bound_pass) tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
+        tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
         issued = c + 1;
       }
       if (*abort) {
         // let the copies already issued land before the CTA's shared memory goes away
-        for (int c = max(0, issued - C::kStages); c < issued; ++c) {
+        const int ring = p.bound_pass ? C::kBoundStages : C::kStages;
+        for (int c = max(0, issued - ring); c < issued; ++c) {
           volatile int no_abort = 0;
-          mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, &no_abort, nullptr);
+          mbar_wait(p.bound_pass ? &S.kb_full[c % ring] : &S.kv_full[c % ring], (c / ring) & 1, &no_abort, nullptr);
         }
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0 && cs.total > 0) {
-      bool ok = mbar_wait(&S.q_full[0], 0, abort, p.status) && mbar_wait(&S.q_full[1], 0, abort, p.status);
+    // the whole warp runs the issue loop; one elected lane issues each instruction
+    if (cs.total > 0) {
+      bool ok = mbar_wait_w(&S.q_full[0], 0, abort, p.status) && mbar_wait_w(&S.q_full[1], 0, abort, p.status);
       tc_fence_after();
       const uint32_t qaddr[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
       // shared-memory descriptors are computed once; a byte offset moves the start-address
@@ -284,11 +372,11 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       const uint64_t kdesc = smem_desc(smem_u32(S.k[0]), 16, C::kAtomBytes, C::kLayout);
       const uint64_t vdesc = smem_desc(smem_u32(S.v[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
       constexpr uint32_t kStageStep = C::kKVBytes >> 4;
-      auto issue_qk = [&](int t, int c, int col) {
-        const uint32_t d = tmem + t * C::kColsPerTile + col;
+      auto issue_qk = [&](int t, int c) {
+        const uint32_t d = tmem + t * C::kColsPerTile + C::kColS;
         const uint64_t bd = kdesc + (uint64_t)((c % C::kStages) * kStageStep);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(d, qdesc[t] + 2 * k, bd + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
+        for (int k = 0; k < D / 16; ++k) mma_ss_w(d, qdesc[t] + 2 * k, bd + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
       };
       auto issue_pv = [&](int t, int c) {
         const uint32_t d = tmem + t * C::kColsPerTile + C::kColO;
@@ -296,59 +384,64 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         const bool first = cs.first_of_branch(c);
 #pragma unroll
         for (int kk = 0; kk < C::kKeys / 16; ++kk)
-          mma_ts(d, tmem + t * C::kColsPerTile + C::kColP + kk * 8, bd + kk * (16 * C::kRowBytes >> 4), C::kIdescPV,
+          mma_ts_w(d, tmem + t * C::kColsPerTile + C::kColP + kk * 8, bd + kk * (16 * C::kRowBytes >> 4), C::kIdescPV,
                  (first && kk == 0) ? 0u : 1u);
       };
-      // bound pass: scores only, double-buffered (even chunks in S, odd chunks in S2) so that the
-      // next chunk's MMAs run while the softmax warps reduce the current one; each buffer has its
-      // own full/free barrier pair, completed once per two chunks
-      for (int c = 0; ok && p.bound_pass && c < cs.total; ++c) {
-        if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+      // bound pass: scores only, N = kBoundKeys per MMA, into two score buffers per tile so that
+      // a tile's next chunk is computed while its warps reduce the current one; each buffer has
+      // its own full/free barrier pair, completed once per two chunks
+      const int nb = p.bound_pass ? (n_ckeys + C::kBoundKeys - 1) / C::kBoundKeys : 0;
+      for (int c = 0; ok && c < nb; ++c) {
+        const int st = c % C::kBoundStages;
+        if (!mbar_wait_w(&S.kb_full[st], (c / C::kBoundStages) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
-        const int b = c & 1;
+        const uint64_t bd = kdesc + (uint64_t)((smem_u32(bound_slot(S, st)) - smem_u32(S.k[0])) >> 4);
+        const int b = c % C::kBoundBufs;
         for (int t = 0; t < 2; ++t) {
-          if (c >= 2) {
-            if (!mbar_wait(b ? &S.p_full2[t] : &S.p_full[t], ((c >> 1) - 1) & 1, abort, p.status)) {
+          if (c >= C::kBoundBufs) {
+            if (!mbar_wait_w(&S.bs_free[t][b], ((c / C::kBoundBufs) + 1) & 1, abort, p.status)) {
               ok = false;
               break;
             }
             tc_fence_after();
           }
-          issue_qk(t, c, b ? C::kColS2 : C::kColS);
-          mma_commit(b ? &S.s_full2[t] : &S.s_full[t]);
+          const uint32_t d = tmem + t * C::kColsPerTile + b * C::kBoundKeys;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) mma_ss_w(d, qdesc[t] + 2 * k, bd + 2 * k, C::kIdescBound, k > 0 ? 1u : 0u);
+          mma_commit_w(&S.bs_full[t][b]);
         }
         if (!ok) break;
-        mma_commit(&S.kv_empty[c % C::kStages]);
+        mma_commit_w(&S.kb_empty[st]);
       }
       for (int c = 0; ok && !p.bound_pass && c < cs.total; ++c) {
-        if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_w(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
           // S(c) is issued ahead of P(c - 1) V: it overwrites only S, which the softmax released
           // with P(c - 1), and the softmax waits for P(c - 1) V before it stores P(c)
           if (c > 0) {
-            if (!mbar_wait(&S.p_full[t], (c - 1) & 1, abort, p.status)) { ok = false; break; }
+            if (!mbar_wait_w(&S.p_full[t], (c - 1) & 1, abort, p.status)) { ok = false; break; }
             tc_fence_after();
           }
-          issue_qk(t, c, C::kColS);
-          mma_commit(&S.s_full[t]);
+          issue_qk(t, c);
+          mma_commit_w(&S.s_full[t]);
           if (c > 0) {
             issue_pv(t, c - 1);
-            mma_commit(&S.pv_done[t]);
+            mma_commit_w(&S.pv_done[t]);
           }
         }
         if (!ok) break;
-        if (c > 0) mma_commit(&S.kv_empty[(c - 1) % C::kStages]);
+        if (c > 0) mma_commit_w(&S.kv_empty[(c - 1) % C::kStages]);
       }
       for (int t = 0; ok && !p.bound_pass && t < 2; ++t) {
-        if (!mbar_wait(&S.p_full[t], (cs.total - 1) & 1, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_w(&S.p_full[t], (cs.total - 1) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         issue_pv(t, cs.total - 1);
-        mma_commit(&S.pv_done[t]);
+        mma_commit_w(&S.pv_done[t]);
       }
       // every MMA issued so far must finish (and every arrive it owes must land) before the
       // CTA can release tensor and shared memory, on the normal path and after an abort alike
-      mma_commit(&S.drain);
+      mma_commit_w(&S.drain);
       volatile int no_abort = 0;
       mbar_wait(&S.drain, 0, &no_abort, nullptr);
     }
@@ -413,50 +506,45 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       return kv ? __uint_as_float(raw) : -INFINITY;
     };
     // ---- streaming top-k of the compressed-branch logits (pooled-query routing) ----
-    // A 32-entry min-heap per row, kept in this row's column of the (otherwise unused) output
-    // accumulator: values in acc[0..31], block ids in acc[32..63].  The root is the worst entry
-    // in the order (logit desc, block asc), so ties evict the larger block id first; keys arrive
-    // in increasing block order, so a candidate enters only when strictly above the root.
-    // Scores above the (possibly stale) root are first appended to a per-row candidate buffer;
-    // the warp merges its rows' buffers together, re-testing every candidate in key order
-    // against the live root, which makes the same decisions as inserting key by key while
-    // keeping the divergent heap work out of the per-key loop.  Forced blocks never enter the
-    // buffer (a 64-bit mask per chunk from the forced-block bitmap).  The merge is one function
-    // outside the unrolled per-key code, which would otherwise carry a copy at every call site.
+    // Every non-forced key whose logit is above the row's gate is appended, with its block id, to
+    // the row's candidate buffer (logits in this row's column of the otherwise unused output
+    // accumulator, ids in cand_id).  The gate starts just below a lower bound on the k-th largest
+    // non-forced logit (from the bound pass), so every key at or above the bound is a candidate and
+    // no key below it can be among the k best (k keys at or above it exist).  With that bound a
+    // row collects a few dozen candidates over the whole stream; should the buffer run short, the
+    // warp's rows keep their k best and the gate rises to the k-th of them.  The k best of the
+    // buffer are ranked at the end.
     const bool topk_on = (D == 64) && p.topk_idx != nullptr;
     float thr = -INFINITY;
-    int key_base = 0;  // block id of key 0 of the current chunk
+    int key_base = 0;    // block id of key 0 of the current chunk
     uint64_t fmask = 0;  // forced blocks among the chunk's 64 keys (never candidates)
-    int ncand = 0;     // this row's buffered candidates
-    float* cbuf = &S.cand[t][0][row];
-    auto hv = [&](int i) -> float& { return acc[i * 128]; };
-    auto hj = [&](int i) -> int& { return reinterpret_cast<int&>(acc[(32 + i) * 128]); };
-    auto worse = [&](float va, int ja, float vb, int jb) { return va < vb || (va == vb && ja > jb); };
+    int ncand = 0;       // this row's buffered candidates
+    float* cval = acc;
+    int* cid = &S.cand_id[t][0][row];
     auto topk_append = [&](float sv, int j) {
-      if (sv > thr && !((fmask >> j) & 1ull)) {
-        cbuf[ncand * 128] = sv;
-        reinterpret_cast<int&>(cbuf[(C::kCand + ncand) * 128]) = key_base + j;
+      if (sv > thr) {
+        cval[ncand * 128] = sv;
+        cid[ncand * 128] = key_base + j;
         ++ncand;
       }
     };
-    auto topk_flush = [&]() {
-      thr = topk_merge(acc, cbuf, ncand, C::kCand, thr);
-      ncand = 0;
+    auto topk_compact = [&]() {
+      if (ncand > p.topk_k) {
+        const KeepBest kb = topk_keep_best(cval, cid, ncand, p.topk_k);
+        ncand = kb.n;
+        thr = kb.thr;
+      }
     };
-    if (topk_on) {
-      // With a lower bound b on the k-th largest non-forced logit, the heap starts full of
-      // placeholders just below b: every key at or above b gets in, no key below b can be among
-      // the k best (k keys at or above b exist), and the placeholders are all displaced.
-      if (p.topk_thr != nullptr && valid) {
-        const float b = p.topk_thr[(size_t)(t0 + R) * p.Hkv + g];
-        if (b > -INFINITY) thr = nextafterf(b, -INFINITY);
-      }
-#pragma unroll 1
-      for (int i = 0; i < 32; ++i) {
-        hv(i) = thr;
-        hj(i) = INT_MAX;
-      }
+    if (topk_on && p.topk_thr != nullptr && valid) {
+      const float b = p.topk_thr[(size_t)(t0 + R) * p.Hkv + g];
+      if (b > -INFINITY) thr = nextafterf(b, -INFINITY);
     }
+    // forced blocks among compressed-key chunk c (bit j: block 64 c + j); the next chunk's mask
+    // is loaded one chunk ahead
+    auto load_fmask = [&](int c) -> uint64_t {
+      return (uint64_t)p.forced_bits[2 * c] | ((uint64_t)p.forced_bits[2 * c + 1] << 32);
+    };
+    uint64_t fmask_next = (topk_on && cs.n_cmp > 0) ? load_fmask(0) : 0ull;
 
     // max of the chunk's raw scores (the scale is positive, so it commutes with the max)
     auto chunk_max_t = [&](auto need_mask_tag) -> float {
@@ -499,14 +587,19 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       uint32_t ra[16], rb[16];
       auto quarter = [&](const uint32_t* r, int qd) {
         uint32_t pk[8];
-        float qmx = -INFINITY;  // the quarter's max (top-k gate)
+        // with the top-k on, the running max is kept per quarter (two chains), since the quarter's
+        // max is the top-k gate as well
+        float qm[2] = {-INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int j = 16 * qd + 2 * i;
           const float s0 = need_mask ? masked(r[2 * i], j) : __uint_as_float(r[2 * i]);
           const float s1 = need_mask ? masked(r[2 * i + 1], j + 1) : __uint_as_float(r[2 * i + 1]);
-          mx[i & 3] = fmax3(mx[i & 3], s0, s1);
-          if constexpr (topk) qmx = fmax3(qmx, s0, s1);
+          if constexpr (topk) {
+            qm[i & 1] = fmax3(qm[i & 1], s0, s1);
+          } else {
+            mx[i & 3] = fmax3(mx[i & 3], s0, s1);
+          }
           const float x0 = fmaf(s0, sc, nm), x1 = fmaf(s1, sc, nm);
           float p0, p1;
           if (kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
@@ -522,15 +615,28 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (qd == 0) wait_pv();
         if (pv_ok) tmem_st8(tbase + C::kColP + 8 * qd, pk);
         if constexpr (topk) {
-          // only quarters where some row of the warp has a score above its root visit the keys
-          if (__any_sync(0xffffffffu, qmx > thr)) {
+          float qmx = fmaxf(qm[0], qm[1]);
+          mx[qd] = fmaxf(mx[qd], qmx);
+          // forced blocks take part in the softmax but are never candidates: in the (few) quarters
+          // that hold one, they drop out of the gate and of the appends
+          const uint32_t qf = (uint32_t)(fmask >> (16 * qd)) & 0xffffu;
+          float sv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) sv[i] = need_mask ? masked(r[i], 16 * qd + i) : __uint_as_float(r[i]);
+          if (qf != 0u) {
+            qmx = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const int j = 16 * qd + i;
-              topk_append(need_mask ? masked(r[i], j) : __uint_as_float(r[i]), j);
+              if ((qf >> i) & 1u) sv[i] = -INFINITY;
+              qmx = fmaxf(qmx, sv[i]);
             }
+          }
+          // only quarters where some row of the warp has a key above its gate visit the keys
+          if (__any_sync(0xffffffffu, qmx > thr)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) topk_append(sv[i], 16 * qd + i);
             // a quarter appends at most 16 candidates per row
-            if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_flush();
+            if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_compact();
           }
         }
       };
@@ -560,47 +666,67 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     };
 
     if (p.bound_pass) {
-      // ---- bound pass: per row, the max non-forced logit of each of 64 key groups (chunk c
-      // joins group c mod 64), then the topk_k-th largest group max.  Groups are disjoint, so
+      // ---- bound pass: per row, the max non-forced logit of each of 64 key groups (chunk c of
+      // kBoundKeys keys joins group c mod 64), then the topk_k-th largest group max.  Groups are disjoint, so
       // at least topk_k distinct keys score at or above that value: a lower bound on the
       // topk_k-th largest logit that needs no selection in the per-key loop.
       float* gmax = acc;  // gmax[i * 128], i < 64 (the output accumulator is unused here)
 #pragma unroll 1
       for (int i = 0; i < 64; ++i) gmax[i * 128] = -INFINITY;
-      auto bound_max_t = [&](uint32_t col, auto mask_tag) -> float {
-        constexpr bool need_mask = decltype(mask_tag)::value;
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // max over 16 keys; forced keys (bits of qf) and keys past nv drop out
+      auto quarter_max = [&](const uint32_t* r, int j0, uint32_t qf, bool tail) -> float {
+        float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-          tmem_ld32(tbase + col + 32 * h, r);
-          tmem_ld_wait();
+        for (int i = 0; i < 16; i += 2) {
+          m0 = fmax3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+        }
+        if (qf != 0u || tail) {
+          m0 = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float s0 = __uint_as_float(r[i]), s1 = __uint_as_float(r[i + 1]);
-            if (need_mask) {
-              const int j = 32 * h + i;
-              if (j >= nv || ((fmask >> j) & 1ull)) s0 = -INFINITY;
-              if (j + 1 >= nv || ((fmask >> (j + 1)) & 1ull)) s1 = -INFINITY;
-            }
-            mx[(i >> 1) & 3] = fmax3(mx[(i >> 1) & 3], s0, s1);
+          for (int i = 0; i < 16; ++i) {
+            const bool drop = ((qf >> i) & 1u) || j0 + i >= nv;
+            m1 = fmaxf(m1, drop ? -INFINITY : __uint_as_float(r[i]));
           }
         }
-        return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        return fmaxf(m0, m1);
       };
+      // forced blocks among the chunk's kBoundKeys keys, one word per 32 keys (words past the
+      // last key are not read); the next chunk's words are loaded one chunk ahead
+      constexpr int kW = C::kBoundKeys / 32;
+      const int nb = (n_ckeys + C::kBoundKeys - 1) / C::kBoundKeys;
+      auto load_words = [&](int c, uint32_t* w) {
+#pragma unroll
+        for (int i = 0; i < kW; ++i) w[i] = (c * kW + i) * 32 < n_ckeys ? p.forced_bits[c * kW + i] : 0u;
+      };
+      uint32_t fw[kW], fw_next[kW];
+      if (nb > 0) load_words(0, fw_next);
       bool okb = true;
-      for (int c = 0; c < cs.total; ++c) {
-        const int b = c & 1;
-        if (!wait_all(b ? &S.s_full2[t] : &S.s_full[t], (c >> 1) & 1)) { okb = false; break; }
+      for (int c = 0; c < nb; ++c) {
+        const int b = c % C::kBoundBufs;
+#pragma unroll
+        for (int i = 0; i < kW; ++i) fw[i] = fw_next[i];
+        if (c + 1 < nb) load_words(c + 1, fw_next);
+        nv = min(C::kBoundKeys, n_ckeys - c * C::kBoundKeys);
+        const bool tail = nv < C::kBoundKeys;
+        if (!wait_all(&S.bs_full[t][b], (c / C::kBoundBufs) & 1)) { okb = false; break; }
         tc_fence_after();
-        nv = min(64, n_ckeys - c * 64);
-        const uint32_t w0 = p.forced_bits[c * 2], w1 = p.forced_bits[c * 2 + 1];
-        fmask = (uint64_t)w0 | ((uint64_t)w1 << 32);
-        const uint32_t col = b ? C::kColS2 : C::kColS;
-        const float mx = (nv < 64 || fmask != 0) ? bound_max_t(col, std::true_type{})
-                                                 : bound_max_t(col, std::false_type{});
+        // 32 columns at a time, each load issued before the previous block is reduced
+        const uint32_t col = tbase + b * C::kBoundKeys;
+        uint32_t ra[32], rb[32];
+        float mx = -INFINITY;
+        tmem_ld32(col, ra);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < kW; ++h) {
+          uint32_t* cur = (h & 1) ? rb : ra;
+          uint32_t* nxt = (h & 1) ? ra : rb;
+          if (h + 1 < kW) tmem_ld32(col + 32 * (h + 1), nxt);
+          mx = fmaxf(mx, fmaxf(quarter_max(cur, 32 * h, fw[h] & 0xffffu, tail),
+                               quarter_max(cur + 16, 32 * h + 16, fw[h] >> 16, tail)));
+          if (h + 1 < kW) tmem_ld_wait();
+        }
         tc_fence_before();
-        mbar_arrive(b ? &S.p_full2[t] : &S.p_full[t]);
+        mbar_arrive(&S.bs_free[t][b]);
         float& gv = gmax[(c & 63) * 128];
         gv = fmaxf(gv, mx);
       }
@@ -635,8 +761,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       const bool need_mask = br == 2 || nv < 64;
       if (topk_on && br == 0) {
         key_base = local * 64;
-        const uint32_t w0 = p.forced_bits[key_base >> 5], w1 = p.forced_bits[(key_base >> 5) + 1];
-        fmask = (uint64_t)w0 | ((uint64_t)w1 << 32);
+        fmask = fmask_next;
+        if (local + 1 < cs.n_cmp) fmask_next = load_fmask(local + 1);
       }
       float lsum;
       if (first) {
@@ -683,23 +809,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         for (int i = 0; i < D; ++i) p.obranch[orow * D + i] = 0.f;
       if (p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first] = -INFINITY;
     }
-    if (ok && topk_on) topk_flush();
-    if (ok && topk_on && valid) {
-      // emit the row's top-k in order (logit desc, block asc); missing entries are -1
-      int32_t* dst = p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k;
-      uint32_t taken = 0;
-#pragma unroll 1
-      for (int k = 0; k < p.topk_k; ++k) {
-        int best = -1;
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i) {
-          if ((taken >> i) & 1u) continue;
-          if (best < 0 || worse(hv(best), hj(best), hv(i), hj(i))) best = i;
-        }
-        taken |= 1u << best;
-        dst[k] = hj(best) == INT_MAX ? -1 : hj(best);
-      }
-    }
+    if (ok && topk_on && valid)
+      topk_emit(cval, cid, ncand, p.topk_k, p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k);
     if (ok && cs.total > 0 && wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
       tc_fence_after();
       finalize(prev_br, m, l);
@@ -740,7 +851,8 @@ lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q
   if (!make_map(&qm, q, D, d.n_q_heads, d.n_tokens, p.G, 128 / p.G)) return LSRM_ERR_CUDA;
   if (!make_map(&km, kk, D, d.n_kv_heads, k ? d.n_tokens : kc_rows, 1, 64)) return LSRM_ERR_CUDA;
   if (!make_map(&vm, vv, D, d.n_kv_heads, v ? d.n_tokens : kc_rows, 1, 64)) return LSRM_ERR_CUDA;
-  if (!make_map(&kcm, kkc, D, d.n_kv_heads, kc ? kc_rows : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
+  if (!make_map(&kcm, kkc, D, d.n_kv_heads, kc ? kc_rows : d.n_tokens, 1, p.bound_pass ? TcCfg<D>::kBoundKeys : 64))
+    return LSRM_ERR_CUDA;
   if (!make_map(&vcm, vvc, D, d.n_kv_heads, vc ? kc_rows : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
   const size_t smem = sizeof(TcSmem<D>) + 1024;
   if (cudaFuncSetAttribute(nsa_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

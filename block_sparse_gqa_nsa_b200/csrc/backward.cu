@@ -222,8 +222,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0 && seq.total > 0) {
-      bool ok = mbar_wait(&S.q_full, 0, abort, p.status);
+    if (seq.total > 0) {  // whole warp; one elected lane issues
+      bool ok = mbar_wait_w(&S.q_full, 0, abort, p.status);
       // descriptors computed once; a byte offset moves the start-address field by offset / 16
       const uint64_t qd = smem_desc(smem_u32(S.q), 16, C::kAtomBytes, C::kLayout);
       const uint64_t od = smem_desc(smem_u32(S.go), 16, C::kAtomBytes, C::kLayout);
@@ -238,33 +238,33 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         const uint64_t so = (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::kColS, qd + 2 * kk, kd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
+          mma_ss_w(tmem + C::kColS, qd + 2 * kk, kd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::kColDP, od + 2 * kk, vd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
-        mma_commit(&S.s_full);
-        if (!pass) mma_commit(&S.kv_empty[c % C::kStages]);
+          mma_ss_w(tmem + C::kColDP, od + 2 * kk, vd_k + so + 2 * kk, C::kIdescNK, kk > 0 ? 1u : 0u);
+        mma_commit_w(&S.s_full);
+        if (!pass) mma_commit_w(&S.kv_empty[c % C::kStages]);
       };
       // pass B only: dQ_b += dS K  (A from tensor memory, MN-major B)
       auto second_stage = [&](int c, bool first) {
         const uint64_t bd = kd_mn + (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
         for (int kk = 0; kk < C::kKeys / 16; ++kk)
-          mma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, bd + kk * kRow16, C::kIdescND,
+          mma_ts_w(tmem + C::kColO, tmem + C::kColP + kk * 8, bd + kk * kRow16, C::kIdescND,
                  (first && kk == 0) ? 0u : 1u);
-        mma_commit(&S.pv_done);
-        mma_commit(&S.kv_empty[c % C::kStages]);
+        mma_commit_w(&S.pv_done);
+        mma_commit_w(&S.kv_empty[c % C::kStages]);
       };
       int prev_pass = 0;
       bool prev_first = false;
       for (int c = 0; ok && c < seq.total; ++c) {
-        if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_w(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         int br, pass, local;
         bool first, last;
         seq.decode(c, br, pass, local, first, last);
         if (c > 0) {
           // the element-wise warps are done with S, dP and P(c - 1)
-          if (!mbar_wait(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait_w(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
         }
         tc_fence_after();
         // S(c) (and dP(c)) go ahead of the P(c - 1) product: they touch other columns, and the
@@ -274,11 +274,11 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         prev_pass = pass;
         prev_first = first;
       }
-      if (ok && mbar_wait(&S.p_full, (seq.total - 1) & 1, abort, p.status)) {
+      if (ok && mbar_wait_w(&S.p_full, (seq.total - 1) & 1, abort, p.status)) {
         tc_fence_after();
         if (prev_pass) second_stage(seq.total - 1, prev_first);
       }
-      mma_commit(&S.drain);
+      mma_commit_w(&S.drain);
       volatile int no_abort = 0;
       mbar_wait(&S.drain, 0, &no_abort, nullptr);
     }
@@ -635,8 +635,8 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0 && total > 0) {
-      bool ok = mbar_wait(&S.key_full, 0, abort, p.status);
+    if (total > 0) {  // whole warp; one elected lane issues
+      bool ok = mbar_wait_w(&S.key_full, 0, abort, p.status);
       // descriptors computed once; a byte offset moves the start-address field by offset / 16
       const uint64_t ktd = smem_desc(smem_u32(S.kt), 16, C::kAtomBytes, C::kLayout);
       const uint64_t vtd = smem_desc(smem_u32(S.vt), 16, C::kAtomBytes, C::kLayout);
@@ -649,11 +649,11 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         const uint64_t so = (uint64_t)((c % C::kStages) * kStep);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::kColS, ktd + 2 * kk, qd_k + so + 2 * kk, C::kIdescNR, kk > 0 ? 1u : 0u);
+          mma_ss_w(tmem + C::kColS, ktd + 2 * kk, qd_k + so + 2 * kk, C::kIdescNR, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::kColDP, vtd + 2 * kk, od_k + so + 2 * kk, C::kIdescNR, kk > 0 ? 1u : 0u);
-        mma_commit(&S.s_full);
+          mma_ss_w(tmem + C::kColDP, vtd + 2 * kk, od_k + so + 2 * kk, C::kIdescNR, kk > 0 ? 1u : 0u);
+        mma_commit_w(&S.s_full);
       };
       auto second_stage = [&](int c) {
         const int st = c % C::kStages;
@@ -661,26 +661,26 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
 #pragma unroll
         for (int kk = 0; kk < C::kRowsPerChunk / 16; ++kk) {
           const uint32_t acc = (c == 0 && kk == 0) ? 0u : 1u;
-          mma_ts(tmem + C::kColDV, tmem + C::kColPg + 8 * kk, od_mn + so + kk * kRow16, C::kIdescND, acc);
-          mma_ts(tmem + C::kColDK, tmem + C::kColDS + 8 * kk, qd_mn + so + kk * kRow16, C::kIdescND, acc);
+          mma_ts_w(tmem + C::kColDV, tmem + C::kColPg + 8 * kk, od_mn + so + kk * kRow16, C::kIdescND, acc);
+          mma_ts_w(tmem + C::kColDK, tmem + C::kColDS + 8 * kk, qd_mn + so + kk * kRow16, C::kIdescND, acc);
         }
-        mma_commit(&S.pv_done);
-        mma_commit(&S.empty[st]);
+        mma_commit_w(&S.pv_done);
+        mma_commit_w(&S.empty[st]);
       };
       for (int c = 0; ok && c < total; ++c) {
-        if (!mbar_wait(&S.full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_w(&S.full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         if (c > 0) {
-          if (!mbar_wait(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait_w(&S.p_full, (c - 1) & 1, abort, p.status)) { ok = false; break; }
         }
         tc_fence_after();
         first_stage(c);  // ahead of the products of chunk c - 1 (other columns; see the query pass)
         if (c > 0) second_stage(c - 1);
       }
-      if (ok && mbar_wait(&S.p_full, (total - 1) & 1, abort, p.status)) {
+      if (ok && mbar_wait_w(&S.p_full, (total - 1) & 1, abort, p.status)) {
         tc_fence_after();
         second_stage(total - 1);
       }
-      mma_commit(&S.drain);
+      mma_commit_w(&S.drain);
       volatile int no_abort = 0;
       mbar_wait(&S.drain, 0, &no_abort, nullptr);
     }
