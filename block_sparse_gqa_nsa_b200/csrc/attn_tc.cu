@@ -360,37 +360,20 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    // the whole warp runs the issue loop; one elected lane issues each instruction
-    if (cs.total > 0) {
+    if (p.bound_pass && cs.total > 0) {
+      // bound pass: the issuing thread is the bottleneck, so the whole warp runs the loop and one
+      // elected lane issues each instruction
       bool ok = mbar_wait_w(&S.q_full[0], 0, abort, p.status) && mbar_wait_w(&S.q_full[1], 0, abort, p.status);
       tc_fence_after();
-      const uint32_t qaddr[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
       // shared-memory descriptors are computed once; a byte offset moves the start-address
       // field (address / 16, bits 0..13; shared addresses stay below 2^18) by offset / 16
-      const uint64_t qdesc[2] = {smem_desc(qaddr[0], 16, C::kAtomBytes, C::kLayout),
-                                 smem_desc(qaddr[1], 16, C::kAtomBytes, C::kLayout)};
+      const uint64_t qdesc[2] = {smem_desc(smem_u32(S.q[0]), 16, C::kAtomBytes, C::kLayout),
+                                 smem_desc(smem_u32(S.q[1]), 16, C::kAtomBytes, C::kLayout)};
       const uint64_t kdesc = smem_desc(smem_u32(S.k[0]), 16, C::kAtomBytes, C::kLayout);
-      const uint64_t vdesc = smem_desc(smem_u32(S.v[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
-      constexpr uint32_t kStageStep = C::kKVBytes >> 4;
-      auto issue_qk = [&](int t, int c) {
-        const uint32_t d = tmem + t * C::kColsPerTile + C::kColS;
-        const uint64_t bd = kdesc + (uint64_t)((c % C::kStages) * kStageStep);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss_w(d, qdesc[t] + 2 * k, bd + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
-      };
-      auto issue_pv = [&](int t, int c) {
-        const uint32_t d = tmem + t * C::kColsPerTile + C::kColO;
-        const uint64_t bd = vdesc + (uint64_t)((c % C::kStages) * kStageStep);
-        const bool first = cs.first_of_branch(c);
-#pragma unroll
-        for (int kk = 0; kk < C::kKeys / 16; ++kk)
-          mma_ts_w(d, tmem + t * C::kColsPerTile + C::kColP + kk * 8, bd + kk * (16 * C::kRowBytes >> 4), C::kIdescPV,
-                 (first && kk == 0) ? 0u : 1u);
-      };
       // bound pass: scores only, N = kBoundKeys per MMA, into two score buffers per tile so that
       // a tile's next chunk is computed while its warps reduce the current one; each buffer has
       // its own full/free barrier pair, completed once per two chunks
-      const int nb = p.bound_pass ? (n_ckeys + C::kBoundKeys - 1) / C::kBoundKeys : 0;
+      const int nb = (n_ckeys + C::kBoundKeys - 1) / C::kBoundKeys;
       for (int c = 0; ok && c < nb; ++c) {
         const int st = c % C::kBoundStages;
         if (!mbar_wait_w(&S.kb_full[st], (c / C::kBoundStages) & 1, abort, p.status)) { ok = false; break; }
@@ -413,35 +396,65 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (!ok) break;
         mma_commit_w(&S.kb_empty[st]);
       }
-      for (int c = 0; ok && !p.bound_pass && c < cs.total; ++c) {
-        if (!mbar_wait_w(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
+      mma_commit_w(&S.drain);
+      volatile int no_abort = 0;
+      mbar_wait(&S.drain, 0, &no_abort, nullptr);
+    } else if (!p.bound_pass && lane == 0 && cs.total > 0) {
+      // attention passes: one thread issues (it mostly waits on the softmax warps)
+      bool ok = mbar_wait(&S.q_full[0], 0, abort, p.status) && mbar_wait(&S.q_full[1], 0, abort, p.status);
+      tc_fence_after();
+      const uint32_t qaddr[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
+      // shared-memory descriptors are computed once; a byte offset moves the start-address
+      // field (address / 16, bits 0..13; shared addresses stay below 2^18) by offset / 16
+      const uint64_t qdesc[2] = {smem_desc(qaddr[0], 16, C::kAtomBytes, C::kLayout),
+                                 smem_desc(qaddr[1], 16, C::kAtomBytes, C::kLayout)};
+      const uint64_t kdesc = smem_desc(smem_u32(S.k[0]), 16, C::kAtomBytes, C::kLayout);
+      const uint64_t vdesc = smem_desc(smem_u32(S.v[0]), C::kKVBytes, C::kAtomBytes, C::kLayout);
+      constexpr uint32_t kStageStep = C::kKVBytes >> 4;
+      auto issue_qk = [&](int t, int c) {
+        const uint32_t d = tmem + t * C::kColsPerTile + C::kColS;
+        const uint64_t bd = kdesc + (uint64_t)((c % C::kStages) * kStageStep);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) mma_ss(d, qdesc[t] + 2 * k, bd + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
+      };
+      auto issue_pv = [&](int t, int c) {
+        const uint32_t d = tmem + t * C::kColsPerTile + C::kColO;
+        const uint64_t bd = vdesc + (uint64_t)((c % C::kStages) * kStageStep);
+        const bool first = cs.first_of_branch(c);
+#pragma unroll
+        for (int kk = 0; kk < C::kKeys / 16; ++kk)
+          mma_ts(d, tmem + t * C::kColsPerTile + C::kColP + kk * 8, bd + kk * (16 * C::kRowBytes >> 4), C::kIdescPV,
+                 (first && kk == 0) ? 0u : 1u);
+      };
+      for (int c = 0; ok && c < cs.total; ++c) {
+        if (!mbar_wait(&S.kv_full[c % C::kStages], (c / C::kStages) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
           // S(c) is issued ahead of P(c - 1) V: it overwrites only S, which the softmax released
           // with P(c - 1), and the softmax waits for P(c - 1) V before it stores P(c)
           if (c > 0) {
-            if (!mbar_wait_w(&S.p_full[t], (c - 1) & 1, abort, p.status)) { ok = false; break; }
+            if (!mbar_wait(&S.p_full[t], (c - 1) & 1, abort, p.status)) { ok = false; break; }
             tc_fence_after();
           }
           issue_qk(t, c);
-          mma_commit_w(&S.s_full[t]);
+          mma_commit(&S.s_full[t]);
           if (c > 0) {
             issue_pv(t, c - 1);
-            mma_commit_w(&S.pv_done[t]);
+            mma_commit(&S.pv_done[t]);
           }
         }
         if (!ok) break;
-        if (c > 0) mma_commit_w(&S.kv_empty[(c - 1) % C::kStages]);
+        if (c > 0) mma_commit(&S.kv_empty[(c - 1) % C::kStages]);
       }
-      for (int t = 0; ok && !p.bound_pass && t < 2; ++t) {
-        if (!mbar_wait_w(&S.p_full[t], (cs.total - 1) & 1, abort, p.status)) { ok = false; break; }
+      for (int t = 0; ok && t < 2; ++t) {
+        if (!mbar_wait(&S.p_full[t], (cs.total - 1) & 1, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         issue_pv(t, cs.total - 1);
-        mma_commit_w(&S.pv_done[t]);
+        mma_commit(&S.pv_done[t]);
       }
       // every MMA issued so far must finish (and every arrive it owes must land) before the
       // CTA can release tensor and shared memory, on the normal path and after an abort alike
-      mma_commit_w(&S.drain);
+      mma_commit(&S.drain);
       volatile int no_abort = 0;
       mbar_wait(&S.drain, 0, &no_abort, nullptr);
     }
@@ -600,7 +613,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           } else {
             mx[i & 3] = fmax3(mx[i & 3], s0, s1);
           }
-          const float x0 = fmaf(s0, sc, nm), x1 = fmaf(s1, sc, nm);
+          float x0, x1;
+          ffma2(x0, x1, s0, s1, sc, nm);  // one packed FMA for the pair
           float p0, p1;
           if (kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
             p0 = poly_exp2(x0);
@@ -609,7 +623,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             p0 = fast_exp2(x0);
             p1 = fast_exp2(x1);
           }
-          ls[i & 3] += p0 + p1;
+          fadd2_acc(ls[2 * (i & 1)], ls[2 * (i & 1) + 1], p0, p1);  // packed row-sum accumulate
           pk[i] = pack_bf16x2(p0, p1);
         }
         if (qd == 0) wait_pv();

@@ -24,14 +24,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// try_wait with a suspend-time hint: a waiting thread sleeps in hardware until the phase
-// completes (or the hint expires) instead of spinning through issue slots
+// try_wait: a waiting thread may sleep in hardware until the phase completes (or a
+// system-dependent time limit passes) instead of spinning through issue slots.  No suspend-time
+// hint: with a long hint the waiters measured slower to resume.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -217,7 +218,9 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 // ---- whole-warp issue ----
 // The MMA warp runs its issue loop converged and one elected lane issues each tcgen05
 // instruction: the operands are then warp-uniform values the compiler keeps in uniform
-// registers, which makes an issue several times cheaper than from a lone diverged lane.
+// registers, and an issue costs about 22 cycles instead of about 63 from a lone diverged lane.
+// That pays where the issuing thread is the bottleneck; where it mostly waits on the softmax
+// warps, the lone lane (no warp-wide vote after each wait) measured faster.
 __device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
@@ -269,6 +272,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+// (a0, a1) += (b0, b1) with one packed f32x2 add
+__device__ __forceinline__ void fadd2_acc(float& a0, float& a1, float b0, float b1) {
+  uint64_t ra, rb, rd;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(ra) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(rb) : "f"(b0), "f"(b1));
+  asm("add.rn.ftz.f32x2 %0, %1, %2;\n" : "=l"(rd) : "l"(ra), "l"(rb));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(a0), "=f"(a1) : "l"(rd));
 }
 // (a0, a1) * (b, b) + (c, c) with one packed f32x2 FMA
 __device__ __forceinline__ void ffma2(float& r0, float& r1, float a0, float a1, float b, float c) {
