@@ -519,16 +519,18 @@ def run_backward(args):
     out = torch.empty(N, Hq, d, dtype=bf16, device=dev)
     idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
     lse = torch.empty(N, Hq, w.n_gates, dtype=torch.float32, device=dev)
+    # the forward keeps its per-branch outputs (bf16), so the backward streams each branch once
+    obr = torch.empty(N, Hq, w.n_gates, d, dtype=torch.bfloat16, device=dev)
     nsa.lsrm_nsa_forward(desc, x["off"], x["q"], x["k"], x["v"], x["gates"], x["coords"], nsa.ROUTE_GEOMETRIC,
-                         out, idx, lse, ws)
+                         out, idx, lse, ws, obr=obr)
     grads = {"dq": torch.empty(N, Hq, d, dtype=bf16, device=dev), "dk": torch.empty(N, Hkv, d, dtype=bf16, device=dev),
              "dv": torch.empty(N, Hkv, d, dtype=bf16, device=dev),
              "dgates": torch.empty(N, Hq, w.n_gates, dtype=bf16, device=dev)}
     stream = torch.cuda.current_stream(dev)
 
-    def step(t=x, g=grads, ix=idx, ls=lse):
+    def step(t=x, g=grads, ix=idx, ls=lse, ob=obr):
         nsa.lsrm_nsa_backward(desc, t["off"], t["q"], t["k"], t["v"], t["gates"], ix, 1, ls, t["dout"], g["dq"],
-                              g["dk"], g["dv"], g["dgates"], ws)
+                              g["dk"], g["dv"], g["dgates"], ws, obr=ob)
 
     # compress, then the inverse routing lists (count, scan, fill, sort), then the query, local-key,
     # compressed-key and finishing kernels
@@ -565,10 +567,12 @@ def run_backward(args):
         h_in = {n: t.pin_memory() for n, t in h_in.items() if n != "coords"}
         h_in["idx"] = idx.cpu().pin_memory()
         h_in["lse"] = lse.cpu().pin_memory()
+        h_in["obr"] = obr.cpu().pin_memory()
 
         def bwd(di, do, st):
             nsa.lsrm_nsa_backward(desc, di["off"], di["q"], di["k"], di["v"], di["gates"], di["idx"], 1, di["lse"],
-                                  di["dout"], do["dq"], do["dk"], do["dv"], do["dgates"], ws, stream=st)
+                                  di["dout"], do["dq"], do["dk"], do["dv"], do["dgates"], ws, stream=st,
+                                  obr=di["obr"])
 
         te, last = pipelined_e2e(dev, world, args.steps, args.warmup, h_in, grads, bwd)
         h2d = sum(t.numel() * t.element_size() for t in h_in.values())
@@ -588,7 +592,8 @@ def run_backward(args):
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": bwd_config(w, world, args.seed,
-                                     {"l2": "inputs larger than L2 (q, dO, dq 249 MB each per step)"}),
+                                     {"l2": "inputs larger than L2 (q, dO, dq 249 MB each per step)",
+                                      "saved_branch_outputs": "bf16 o_b from the forward (745 MB), one pass per branch"}),
                 "flops_per_step": flops,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                              "frac": achieved / peak, "traffic": profiled_traffic("bwd"),

@@ -116,6 +116,7 @@ struct TcParams {
   const int32_t* forced;
   uint16_t* out;
   float* obranch;
+  uint16_t* obr;  // optional saved branch outputs o_b, bf16 [N][Hq][n_gates][D] (fused forward only)
   float* lse;
   uint32_t* status;
   int N, B, Hq, Hkv, G, top_k, idx_heads, n_forced, window, n_gates, route_all, branches, lse_stride, lse_first;
@@ -487,6 +488,15 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (p.out != nullptr) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) acc[(32 * i + e) * 128] = fmaf(gi, __uint_as_float(o[e]), acc[(32 * i + e) * 128]);
+        }
+        if (p.obr != nullptr && valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.obr + (orow * p.n_gates + br) * D + 32 * i);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * e]) * inv, __uint_as_float(o[8 * e + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv));
         }
         if (p.obranch != nullptr && valid) {
           float4* dst = reinterpret_cast<float4*>(p.obranch + orow * D + 32 * i);
@@ -883,7 +893,7 @@ lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q
 lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                            const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                            int route_all, int branches, void* out, float* obranch, float* lse, int lse_stride,
-                           int lse_first, uint32_t* status, cudaStream_t stream) {
+                           int lse_first, uint32_t* status, cudaStream_t stream, void* obr) {
   const int G = d.n_q_heads / d.n_kv_heads;
   if (128 % G != 0) return LSRM_ERR_UNSUPPORTED;
   if ((!route_all && d.n_forced + d.top_k > kTcMaxSel) || d.n_blocks > 65535) return LSRM_ERR_UNSUPPORTED;
@@ -894,6 +904,7 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
   p.forced = d.forced_blocks;
   p.out = (uint16_t*)out;
   p.obranch = obranch;
+  p.obr = (uint16_t*)obr;
   p.lse = lse;
   p.status = status;
   p.N = (int)d.n_tokens;

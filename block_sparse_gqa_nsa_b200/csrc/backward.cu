@@ -39,6 +39,7 @@ struct BwdParams {
   const int32_t* idx;     // [B][idx_heads][top_k]
   const float* lse;       // [N][Hq][NG] natural log
   const uint16_t* dout;   // [N][Hq][D]
+  const uint16_t* obr;    // optional saved branch outputs o_b, bf16 [N][Hq][NG][D]: no pass A
   uint16_t* dq;
   uint16_t* dgates;
   float4* rowc;           // [NG][N][Hq]: lse (log2 units), gate, Delta, token position (int bits)
@@ -107,14 +108,18 @@ struct BqtSmem {
 };
 
 // chunk order: for each branch with keys, its chunks twice (pass A, then pass B)
+// chunk sequence of the query pass: per branch, pass A then pass B over the branch's chunks, or
+// pass B alone when the forward's branch outputs were saved (two_pass = 0)
 struct BqtSeq {
   int n[3];
   int total;
+  int two_pass;
   __device__ __forceinline__ void decode(int c, int& br, int& pass, int& local, bool& first, bool& last) const {
+    const int m = two_pass ? 2 : 1;
     br = 0;
-    while (c >= 2 * n[br]) { c -= 2 * n[br]; ++br; }
-    pass = c >= n[br];
-    local = c - pass * n[br];
+    while (c >= m * n[br]) { c -= m * n[br]; ++br; }
+    pass = two_pass ? (c >= n[br] ? 1 : 0) : 1;
+    local = c - (two_pass && pass ? n[br] : 0);
     first = local == 0;
     last = local == n[br] - 1;
   }
@@ -179,7 +184,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   seq.n[0] = (p.B + C::kKeys - 1) / C::kKeys;
   seq.n[1] = S.n_sel;
   seq.n[2] = (p.NG == 3 && p.window > 0) ? 1 : 0;
-  seq.total = 2 * (seq.n[0] + seq.n[1] + seq.n[2]);
+  seq.two_pass = p.obr == nullptr ? 1 : 0;
+  seq.total = (seq.two_pass ? 2 : 1) * (seq.n[0] + seq.n[1] + seq.n[2]);
   volatile int* abort = &S.abort;
   auto chunk_start = [&](int br, int local, int& start, int& nv) {
     if (br == 0) {
@@ -313,6 +319,33 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               make_float4(INFINITY, 0.f, 0.f, __int_as_float(tok_local));
         }
     }
+    // With the forward's branch outputs saved, dgates_b = <dO, o_b> and Delta_b = g_b dgates_b come
+    // straight from them (fp32 dot products over d) and pass A is skipped.
+    float delta_b[3] = {0.f, 0.f, 0.f};
+    if (p.obr != nullptr && valid) {
+      const uint4* go = reinterpret_cast<const uint4*>(p.dout + orow * D);
+      for (int b = 0; b < p.NG; ++b) {
+        if (seq.n[b] == 0) continue;
+        const uint4* ob = reinterpret_cast<const uint4*>(p.obr + (orow * p.NG + b) * D);
+        float dg = 0.f;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+          const uint4 x = go[i], y = ob[i];
+          const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            dg = fmaf(bf16_to_f32((uint16_t)(xs[e] & 0xffffu)), bf16_to_f32((uint16_t)(ys[e] & 0xffffu)), dg);
+            dg = fmaf(bf16_to_f32((uint16_t)(xs[e] >> 16)), bf16_to_f32((uint16_t)(ys[e] >> 16)), dg);
+          }
+        }
+        delta_b[b] = gate[b] * dg;
+        if (h == 0) {
+          p.dgates[orow * p.NG + b] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
+          p.rowc[((size_t)b * p.N + t0 + tok_local) * p.Hq + g * p.G + R % p.G] =
+              make_float4(lse2[b], gate[b], delta_b[b], __int_as_float(tok_local));
+        }
+      }
+    }
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       const bool w = mbar_wait(bar, parity, abort, p.status);
       return __all_sync(0xffffffffu, w);
@@ -338,33 +371,43 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     auto chunk_pass = [&](auto mask_tag, auto pass_tag, int nv, int br, float l2, float gb, float dlt) {
       constexpr bool kMask = decltype(mask_tag)::value;
       constexpr bool kPassB = decltype(pass_tag)::value;
+      const float nl2 = -l2, ndlt = -dlt;
       uint32_t sa[16], sb[16], da[16], db[16];
       auto quarter_pass = [&](const uint32_t* sr, const uint32_t* dr, int qd) {
         uint32_t pk[8];
-        float dgq = 0.f;
+        float dgq[2] = {0.f, 0.f};
+        // key pairs: the scale, the dS factor and the products are packed f32x2 operations
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          float v2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = 32 * h + 16 * qd + 2 * i + e;
-            bool kv = true;
-            if constexpr (kMask) {
-              kv = j < nv;
-              if (br == 2) kv = kv && j >= wlo && j <= whi;
+          const float s0 = __uint_as_float(sr[2 * i]), s1 = __uint_as_float(sr[2 * i + 1]);
+          const float d0 = __uint_as_float(dr[2 * i]), d1 = __uint_as_float(dr[2 * i + 1]);
+          float x0, x1;
+          ffma2(x0, x1, s0, s1, sc, nl2);
+          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          if constexpr (kMask) {
+            const int j = 32 * h + 16 * qd + 2 * i;
+            bool kv0 = j < nv, kv1 = j + 1 < nv;
+            if (br == 2) {
+              kv0 = kv0 && j >= wlo && j <= whi;
+              kv1 = kv1 && j + 1 >= wlo && j + 1 <= whi;
             }
-            float pr = fast_exp2(fmaf(__uint_as_float(sr[2 * i + e]), sc, -l2));
-            if constexpr (kMask) pr = kv ? pr : 0.f;
-            if constexpr (kPassB) v2[e] = pr * fmaf(gb, __uint_as_float(dr[2 * i + e]), -dlt);
-            else dgq = fmaf(pr, __uint_as_float(dr[2 * i + e]), dgq);
+            p0 = kv0 ? p0 : 0.f;
+            p1 = kv1 ? p1 : 0.f;
           }
-          if constexpr (kPassB) pk[i] = pack_bf16x2(v2[0], v2[1]);
+          if constexpr (kPassB) {
+            float t0, t1, v0, v1;
+            ffma2(t0, t1, d0, d1, gb, ndlt);  // g_b dP - Delta
+            fmul2(v0, v1, p0, p1, t0, t1);
+            pk[i] = pack_bf16x2(v0, v1);
+          } else {
+            ffma2_acc(dgq[0], dgq[1], p0, p1, d0, d1);
+          }
         }
         if constexpr (kPassB) {
           if (qd == 0) pv_ok = pv_wait_through(pv_before_store);
           if (pv_ok) tmem_st8(tbase + C::kColP + 16 * h + 8 * qd, pk);
         } else {
-          dg_part += dgq;
+          dg_part += dgq[0] + dgq[1];
         }
       };
       tmem_ld16(tbase + C::kColS + 32 * h, sa);
@@ -388,6 +431,7 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       tc_fence_after();
       pv_before_store = nb - 1;  // the dS columns are free once the previous dS K product is done
       if (!pass && first) dg_part = 0.f;
+      if (!seq.two_pass && first) delta = br == 0 ? delta_b[0] : (br == 1 ? delta_b[1] : delta_b[2]);
       const float l2 = br == 0 ? lse2[0] : (br == 1 ? lse2[1] : lse2[2]);
       const float gb = br == 0 ? gate[0] : (br == 1 ? gate[1] : gate[2]);
       const bool need_mask = br == 2 || nv < 32 * (h + 1);
@@ -936,7 +980,7 @@ static lsrm_status launch_backward_d(const lsrm_nsa_desc& d, const BwdParams& p,
 lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
-                            unsigned char* ws_bwd, uint32_t* status, cudaStream_t s) {
+                            unsigned char* ws_bwd, uint32_t* status, cudaStream_t s, const void* obr) {
   if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.n_blocks > 65535 || 64 % (d.n_q_heads / d.n_kv_heads) != 0)
     return LSRM_ERR_UNSUPPORTED;
   const BwdWs w = bwd_layout(d, idx_heads);
@@ -951,6 +995,7 @@ lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const vo
   p.idx = idx;
   p.lse = lse;
   p.dout = (const uint16_t*)dout;
+  p.obr = (const uint16_t*)obr;
   p.dq = (uint16_t*)dq;
   p.dgates = (uint16_t*)dgates;
   p.rowc = reinterpret_cast<float4*>(ws_bwd + w.rowc);

@@ -19,7 +19,7 @@ lsrm_status launch_gate_combine(const lsrm_nsa_desc& d, const float* oc, const f
 lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                         const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                         int route_all, int branches, void* out, float* obranch, float* lse, int lse_stride,
-                        int lse_first, uint32_t* status, cudaStream_t stream);
+                        int lse_first, uint32_t* status, cudaStream_t stream, void* obr = nullptr);
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
@@ -36,7 +36,7 @@ lsrm_status launch_speed3r_routed(const lsrm_nsa_desc& d, const int32_t* off, co
 lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
-                            unsigned char* ws_bwd, uint32_t* status, cudaStream_t stream);
+                            unsigned char* ws_bwd, uint32_t* status, cudaStream_t stream, const void* obr);
 }  // namespace lsrm
 
 using namespace lsrm;
@@ -235,12 +235,14 @@ lsrm_status lsrm_nsa_attend(const lsrm_nsa_desc* desc, const int32_t* off, const
 
 lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
                              const void* v, const void* gates, const int32_t* coords_or_null, int32_t route_mode,
-                             void* out, int32_t* idx_inout, float* lse_or_null, void* ws, void* stream) {
+                             void* out, int32_t* idx_inout, float* lse_or_null, void* obr_or_null, void* ws,
+                             void* stream) {
   LSRM_TRY(check_desc(desc));
   LSRM_TRY(check_ws(desc, ws));
   if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || gates == nullptr || out == nullptr)
     return LSRM_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return LSRM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(obr_or_null, 16)) return LSRM_ERR_INVALID_ARG;
+  if (obr_or_null != nullptr && desc->pooled_q) return LSRM_ERR_UNSUPPORTED;  // no pooled-query backward
   const lsrm_nsa_desc& d = *desc;
   const Workspace w = workspace_layout(d);
   cudaStream_t s = (cudaStream_t)stream;
@@ -304,13 +306,13 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
   }
   const int branches = BR_CMP | BR_SLC | ((d.n_gates == 3 && d.window > 0) ? BR_WIN : 0);
   return launch_attn(d, off, q, k, v, kc16, vc16, gates, idx, idx_heads, route_all, branches, out, nullptr,
-                     lse_or_null, d.n_gates, 0, status_of(ws), s);
+                     lse_or_null, d.n_gates, 0, status_of(ws), s, obr_or_null);
 }
 
 lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
                               const void* v, const void* gates, const int32_t* idx, int32_t idx_heads,
-                              const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates, void* ws,
-                              void* stream) {
+                              const float* lse, const void* obr_or_null, const void* dout, void* dq, void* dk, void* dv,
+                              void* dgates, void* ws, void* stream) {
   LSRM_TRY(check_desc(desc));
   LSRM_TRY(check_ws(desc, ws));
   if (desc->pooled_q) return LSRM_ERR_UNSUPPORTED;
@@ -318,13 +320,14 @@ lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t* off, con
       lse == nullptr || dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || dgates == nullptr)
     return LSRM_ERR_INVALID_ARG;
   if (idx_heads != 1 && idx_heads != desc->n_kv_heads) return LSRM_ERR_INVALID_ARG;
+  if (!aligned(obr_or_null, 16) || !aligned(dout, 16)) return LSRM_ERR_INVALID_ARG;
   const Workspace w = workspace_layout(*desc);
   cudaStream_t s = (cudaStream_t)stream;
   void* kc16 = wsp<void>(ws, w.kc16);
   void* vc16 = wsp<void>(ws, w.vc16);
   LSRM_TRY(launch_compress(*desc, off, nullptr, k, v, nullptr, kc16, nullptr, vc16, nullptr, nullptr, s));
   return launch_backward(*desc, off, q, k, v, kc16, vc16, gates, idx, idx_heads, lse, dout, dq, dk, dv, dgates,
-                         wsp<unsigned char>(ws, w.bwd), status_of(ws), s);
+                         wsp<unsigned char>(ws, w.bwd), status_of(ws), s, obr_or_null);
 }
 
 lsrm_status lsrm_nsa_last_device_status(void* ws, void* stream) {

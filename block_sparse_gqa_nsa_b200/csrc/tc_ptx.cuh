@@ -273,6 +273,23 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// (r0, r1) = (a0, a1) * (b0, b1) with one packed f32x2 multiply
+__device__ __forceinline__ void fmul2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+  uint64_t ra, rb, rd;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(ra) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(rb) : "f"(b0), "f"(b1));
+  asm("mul.rn.ftz.f32x2 %0, %1, %2;\n" : "=l"(rd) : "l"(ra), "l"(rb));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(r0), "=f"(r1) : "l"(rd));
+}
+// (c0, c1) += (a0, a1) * (b0, b1) with one packed f32x2 FMA
+__device__ __forceinline__ void ffma2_acc(float& c0, float& c1, float a0, float a1, float b0, float b1) {
+  uint64_t ra, rb, rc, rd;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(ra) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(rb) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(rc) : "f"(c0), "f"(c1));
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;\n" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(c0), "=f"(c1) : "l"(rd));
+}
 // (a0, a1) += (b0, b1) with one packed f32x2 add
 __device__ __forceinline__ void fadd2_acc(float& a0, float& a1, float b0, float b1) {
   uint64_t ra, rb, rd;

@@ -84,8 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsrm_nsa_window_attn": ([D, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_gate_combine": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp], ctypes.c_int),
-        "lsrm_nsa_forward": ([D, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp], ctypes.c_int),
-        "lsrm_nsa_backward": ([D, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "lsrm_nsa_forward": ([D, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "lsrm_nsa_backward": ([D, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_last_device_status": ([vp, vp], ctypes.c_int),
         "lsrm_status_string": ([ctypes.c_int], ctypes.c_char_p),
     }
@@ -225,23 +225,29 @@ def lsrm_nsa_attend(desc, off, q, k, v, kc, vc, gates, idx, idx_heads, route_all
           _ptr(gates), _ptr(idx), int(idx_heads), int(route_all), _ptr(out), _ptr(lse), _ptr(ws), _stream(stream))
 
 
-def lsrm_nsa_forward(desc, off, q, k, v, gates, coords, route_mode, out, idx=None, lse=None, ws=None, stream=None):
+def lsrm_nsa_forward(desc, off, q, k, v, gates, coords, route_mode, out, idx=None, lse=None, ws=None, stream=None,
+                     obr=None):
+    """obr: optional bf16 [N][Hq][n_gates][d] that receives the per-branch outputs for the backward."""
     for t, n, dt in ((off, "off", torch.int32), (q, "q", torch.bfloat16), (k, "k", torch.bfloat16),
                      (v, "v", torch.bfloat16), (gates, "gates", torch.bfloat16), (coords, "coords", torch.int32),
-                     (out, "out", torch.bfloat16), (idx, "idx", torch.int32), (lse, "lse", torch.float32)):
+                     (out, "out", torch.bfloat16), (idx, "idx", torch.int32), (lse, "lse", torch.float32),
+                     (obr, "obr", torch.bfloat16)):
         _check(t, dt, n)
     _call("lsrm_nsa_forward", ctypes.byref(desc), _ptr(off), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(coords),
-          int(route_mode), _ptr(out), _ptr(idx), _ptr(lse), _ptr(ws), _stream(stream))
+          int(route_mode), _ptr(out), _ptr(idx), _ptr(lse), _ptr(obr), _ptr(ws), _stream(stream))
 
 
-def lsrm_nsa_backward(desc, off, q, k, v, gates, idx, idx_heads, lse, dout, dq, dk, dv, dgates, ws, stream=None):
+def lsrm_nsa_backward(desc, off, q, k, v, gates, idx, idx_heads, lse, dout, dq, dk, dv, dgates, ws, stream=None,
+                      obr=None):
+    """obr: the forward's saved per-branch outputs (optional); with them each branch is streamed once."""
     for t, n, dt in ((off, "off", torch.int32), (q, "q", torch.bfloat16), (k, "k", torch.bfloat16),
                      (v, "v", torch.bfloat16), (gates, "gates", torch.bfloat16), (idx, "idx", torch.int32),
                      (lse, "lse", torch.float32), (dout, "dout", torch.bfloat16), (dq, "dq", torch.bfloat16),
-                     (dk, "dk", torch.bfloat16), (dv, "dv", torch.bfloat16), (dgates, "dgates", torch.bfloat16)):
+                     (dk, "dk", torch.bfloat16), (dv, "dv", torch.bfloat16), (dgates, "dgates", torch.bfloat16),
+                     (obr, "obr", torch.bfloat16)):
         _check(t, dt, n)
     _call("lsrm_nsa_backward", ctypes.byref(desc), _ptr(off), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(idx),
-          int(idx_heads), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgates), _ptr(ws),
+          int(idx_heads), _ptr(lse), _ptr(obr), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgates), _ptr(ws),
           _stream(stream))
 
 

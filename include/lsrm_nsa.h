@@ -193,19 +193,27 @@ LSRM_API lsrm_status lsrm_nsa_attend(const lsrm_nsa_desc* desc, const int32_t* o
  * workspace.  For pooled_q the routing is the Speed3R rule and idx_inout is
  * [B][Hq][top_k].
  * lse_or_null receives fp32 [N][Hq][n_gates] per-branch LSE (needed by the
- * backward). */
+ * backward).  obr_or_null (device, 16-byte aligned, caller-owned) receives the
+ * normalised per-branch outputs o_b as bf16 [N][Hq][n_gates][d], the
+ * activations that let the backward skip recomputing <dO, o_b>; it must be NULL
+ * for pooled_q (LSRM_ERR_UNSUPPORTED otherwise). */
 LSRM_API lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
                              const void* v, const void* gates, const int32_t* coords_or_null, int32_t route_mode,
-                             void* out, int32_t* idx_inout, float* lse_or_null, void* ws, void* stream);
+                             void* out, int32_t* idx_inout, float* lse_or_null, void* obr_or_null, void* ws,
+                             void* stream);
 
 /* S10 backward of the LSRM layer (pooled_q = 0) with routing indices fixed:
  * dq, dgates [N][Hq][.], dk, dv [N][Hkv][d] (bf16) of L = sum(out * dout),
  * through the gated sum, the three softmax branches and the block mean.
- * lse is the forward's per-branch LSE.  idx_heads as in lsrm_nsa_select_attn. */
+ * lse is the forward's per-branch LSE.  idx_heads as in lsrm_nsa_select_attn.
+ * obr_or_null: the forward's saved branch outputs (see lsrm_nsa_forward).  With
+ * them dgates_b = <dO, o_b> and Delta_b = g_b dgates_b are read off directly and
+ * every branch is streamed once; with NULL they are recomputed in an extra pass
+ * over each branch (P dP summed in fp32).  dout and obr must be 16-byte aligned. */
 LSRM_API lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
                               const void* v, const void* gates, const int32_t* idx, int32_t idx_heads,
-                              const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
-                              void* ws, void* stream);
+                              const float* lse, const void* obr_or_null, const void* dout, void* dq, void* dk,
+                              void* dv, void* dgates, void* ws, void* stream);
 
 /* Read (synchronising `stream`) and clear the device status word of the workspace. */
 LSRM_API lsrm_status lsrm_nsa_last_device_status(void* ws, void* stream);

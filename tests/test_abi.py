@@ -57,13 +57,17 @@ def test_workspace_size_and_validation_on_host(lib):
 def test_calls_reject_bad_arguments_before_any_launch(lib):
     d = _desc()
     # a dummy 256-byte-aligned workspace address: the null tensors are rejected before it is touched
-    rc = lib.lsrm_nsa_forward(ctypes.byref(d), None, None, None, None, None, None, 2, None, None, None, 256, None)
+    rc = lib.lsrm_nsa_forward(ctypes.byref(d), None, None, None, None, None, None, 2, None, None, None, None, 256,
+                              None)
     assert rc == 1  # invalid argument: null tensors
     d48 = _desc(head_dim=48)
     rc = lib.lsrm_nsa_compress(ctypes.byref(d48), None, None, None, None, None, None, None, None, None, None, None,
                                None)
     assert rc == 2  # unsupported head_dim
-    rc = lib.lsrm_nsa_forward(ctypes.byref(d), 16, 16, 16, 16, 16, 16, 2, 16, None, None, None, None)
+    rc = lib.lsrm_nsa_forward(ctypes.byref(d), 16, 16, 16, 16, 16, 16, 2, 16, None, None, None, None, None)
     assert rc == 6  # workspace missing
+    # a saved-branch-output pointer off the 16-byte grid is an invalid argument
+    rc = lib.lsrm_nsa_forward(ctypes.byref(d), 16, 16, 16, 16, 16, 16, 2, 16, None, None, 24, 256, None)
+    assert rc == 1
     assert lib.lsrm_nsa_last_device_status(None, None) == 6
     assert nsa.lsrm_status_string(5) == "device bounds check failed"

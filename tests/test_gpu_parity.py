@@ -202,16 +202,22 @@ def test_selected_branch_flags_out_of_range_indices():
 # S7 fused forward
 # ------------------------------------------------------------------------------------------------
 
-def _forward(c: DeviceCase, mode, idx=None):
+def _forward(c: DeviceCase, mode, idx=None, obr=None):
     w = c.w
     out = c.empty(w.n_tokens, w.n_q_heads, w.head_dim, dtype=torch.bfloat16)
     lse = c.empty(w.n_tokens, w.n_q_heads, w.n_gates)
     if idx is None and mode != nsa.ROUTE_ALL:
         heads = 1 if mode == nsa.ROUTE_GEOMETRIC else w.n_kv_heads
         idx = c.empty(w.n_blocks, heads, c.top_k, dtype=torch.int32)
-    nsa.lsrm_nsa_forward(c.desc, c.off, c.q, c.k, c.v, c.gates, c.coords, mode, out, idx, lse, c.ws)
+    nsa.lsrm_nsa_forward(c.desc, c.off, c.q, c.k, c.v, c.gates, c.coords, mode, out, idx, lse, c.ws, obr=obr)
     assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
     return out, idx, lse
+
+
+def _branch_outputs(c: DeviceCase):
+    """bf16 [N][Hq][n_gates][d] buffer for the forward's saved branch outputs."""
+    w = c.w
+    return c.empty(w.n_tokens, w.n_q_heads, w.n_gates, w.head_dim, dtype=torch.bfloat16)
 
 
 def test_fused_forward_tiny_score_routing():
@@ -387,14 +393,15 @@ def _dout(w, seed=7):
     return w.dout if w.dout is not None else normal_bf16(seed, 5, w.q.shape, 1.0)
 
 
-def _gpu_backward(c: DeviceCase, idx_t, idx_heads, lse, dout_t):
+def _gpu_backward(c: DeviceCase, idx_t, idx_heads, lse, dout_t, obr=None):
     w = c.w
     bf = torch.bfloat16
     dq = c.empty(w.n_tokens, w.n_q_heads, w.head_dim, dtype=bf)
     dk = c.empty(w.n_tokens, w.n_kv_heads, w.head_dim, dtype=bf)
     dv = c.empty(w.n_tokens, w.n_kv_heads, w.head_dim, dtype=bf)
     dg = c.empty(w.n_tokens, w.n_q_heads, w.n_gates, dtype=bf)
-    nsa.lsrm_nsa_backward(c.desc, c.off, c.q, c.k, c.v, c.gates, idx_t, idx_heads, lse, dout_t, dq, dk, dv, dg, c.ws)
+    nsa.lsrm_nsa_backward(c.desc, c.off, c.q, c.k, c.v, c.gates, idx_t, idx_heads, lse, dout_t, dq, dk, dv, dg, c.ws,
+                          obr=obr)
     assert nsa.lsrm_nsa_last_device_status(c.ws) == 0
     return dq, dk, dv, dg
 
@@ -407,6 +414,7 @@ def _check_grads(got, ref, rows=None):
         assert_grad_close(g, r, name)
 
 
+@pytest.mark.parametrize("saved", [False, True])
 @pytest.mark.parametrize("name,kw,mode", [
     ("backward_small", {}, "geom"),
     ("ragged_geo", {}, "geom"),
@@ -416,26 +424,46 @@ def _check_grads(got, ref, rows=None):
     ("tiny_geo", {"window": 2}, "geom"),
     ("ragged_geo", {"top_k": 1}, "geom"),
 ])
-def test_backward_matches_oracle(name, kw, mode):
+def test_backward_matches_oracle(name, kw, mode, saved):
+    # saved: the forward keeps its branch outputs and the backward reads dgates from them
     w = make_workload(name, **kw)
     c = DeviceCase(w)
-    out, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC if mode == "geom" else nsa.ROUTE_SCORE)
+    obr = _branch_outputs(c) if saved else None
+    out, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC if mode == "geom" else nsa.ROUTE_SCORE, obr=obr)
     heads = 1 if mode == "geom" else w.n_kv_heads
     gidx = to_np(idx).reshape(w.n_blocks, heads, w.top_k)
     dout = _dout(w)
-    got = _gpu_backward(c, idx, heads, lse, bf16_tensor(dout))
+    got = _gpu_backward(c, idx, heads, lse, bf16_tensor(dout), obr=obr)
     ref_idx = gidx[:, 0, :] if heads == 1 else gidx
     ref = O.backward(oracle_desc(w), w.off, w.q, w.k, w.v, w.gates, ref_idx, dout, nthreads=8)
     _check_grads(got, ref)
 
 
-def test_backward_is_deterministic():
+def test_saved_branch_outputs_match_single_branch_oracle():
+    # the forward's saved o_b equals the oracle layer with a one-hot gate on branch b
+    w = make_workload("ragged_geo")
+    c = DeviceCase(w)
+    obr = _branch_outputs(c)
+    _, idx, _ = _forward(c, nsa.ROUTE_GEOMETRIC, obr=obr)
+    D = oracle_desc(w)
+    ref_idx = to_np(idx).reshape(w.n_blocks, -1)
+    got = to_np(obr)
+    for b in range(w.n_gates):
+        one = np.zeros_like(w.gates)
+        one[..., b] = f32_to_bf16_bits(np.array([1.0], np.float32))[0]
+        ref = O.forward(D, w.off, w.q, w.k, w.v, one, ref_idx)
+        assert_close(got[:, :, b, :], ref, f"o_{b}")
+
+
+@pytest.mark.parametrize("saved", [False, True])
+def test_backward_is_deterministic(saved):
     w = make_workload("backward_small")
     c = DeviceCase(w)
-    _, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC)
+    obr = _branch_outputs(c) if saved else None
+    _, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC, obr=obr)
     dout = bf16_tensor(_dout(w))
-    a = _gpu_backward(c, idx, 1, lse, dout)
-    b = _gpu_backward(c, idx, 1, lse, dout)
+    a = _gpu_backward(c, idx, 1, lse, dout, obr=obr)
+    b = _gpu_backward(c, idx, 1, lse, dout, obr=obr)
     for x, y in zip(a, b):
         assert torch.equal(x.view(torch.int16), y.view(torch.int16))
 
@@ -457,17 +485,19 @@ def test_backward_compressed_only_gates_spread_block_gradient():
         assert np.array_equal(dv[blk], np.broadcast_to(dv[w.off[b]], dv[blk].shape))
 
 
-def test_backward_sparse_stage_full_size():
+@pytest.mark.parametrize("saved", [False, True])
+def test_backward_sparse_stage_full_size(saved):
     """The backward workload (sparse stage, 121 344 tokens, dO ~ N(0, 1)) at full size:
     sampled query blocks exactly against the oracle restricted to them, key-side sums against
     identities that hold at any size, and sampled key blocks with the compressed gate at zero
     against the oracle over the query blocks that reach them."""
     w = make_workload("backward")
     c = DeviceCase(w)
-    _, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC)
+    obr = _branch_outputs(c) if saved else None
+    _, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC, obr=obr)
     gidx = to_np(idx).reshape(w.n_blocks, w.top_k)
     dout_t = bf16_tensor(w.dout)
-    dq, dk, dv, dg = _gpu_backward(c, idx, 1, lse, dout_t)
+    dq, dk, dv, dg = _gpu_backward(c, idx, 1, lse, dout_t, obr=obr)
     D = oracle_desc(w)
     rng = np.random.default_rng(2)
     qb = np.sort(np.r_[rng.choice(w.n_blocks, 2, replace=False), [w.n_blocks - 1]]).astype(np.int32)
