@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r"],
                     help="sparse: the layer forward (the default line); backward: its gradients; dense: the "
                          "dense-stage shape with every block selected; speed3r: the pooled-query variant")
+    ap.add_argument("--frames", type=int, default=512,
+                    help="speed3r only: frames of the synthetic sequence (512 is the workload; fewer give the "
+                         "small cases that profiler captures use)")
     return ap.parse_args()
 
 
@@ -659,7 +662,11 @@ def run_extra(args):
     if world > 1:
         dist.barrier()
     nsa.load_library()
-    w = make_workload(args.workload, seed=args.seed)
+    if args.workload == "speed3r" and args.frames != 512:
+        w = make_workload("speed3r_small", seed=args.seed, n_frames=args.frames)
+        workload = workload.replace("512_frames", f"{args.frames}_frames")
+    else:
+        w = make_workload(args.workload, seed=args.seed)
     N, B, Hq, Hkv, d, k = w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k
 
     def bf(a):
