@@ -33,10 +33,12 @@ namespace lsrm {
 
 using namespace tc;
 
-// One pair in kPolyMod of the exponentials goes through poly_exp2 on the FMA pipe instead of
-// MUFU (whose 16 ex2 per clock per SM bound the kernel at d = 32); 0 keeps all on MUFU.
+// One pair in kPolyMod of the exponentials goes through poly_exp2_pair on the FMA pipe instead of
+// MUFU (whose 16 ex2 per clock per SM bound the kernel at d = 32); 0 keeps all on MUFU.  With the
+// packed f32x2 softmax arithmetic leaving issue slots free, 1 pair in 8 measured fastest
+// (4, 8 and 16 tried: sparse stage 3.96 / 3.89 / 3.93 ms against 4.06 ms with MUFU alone).
 #ifndef LSRM_POLY_MOD
-#define LSRM_POLY_MOD 0
+#define LSRM_POLY_MOD 8
 #endif
 constexpr int kPolyMod = LSRM_POLY_MOD;
 
@@ -627,8 +629,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           ffma2(x0, x1, s0, s1, sc, nm);  // one packed FMA for the pair
           float p0, p1;
           if (kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
-            p0 = poly_exp2(x0);
-            p1 = poly_exp2(x1);
+            poly_exp2_pair(p0, p1, x0, x1);
           } else {
             p0 = fast_exp2(x0);
             p1 = fast_exp2(x1);

@@ -267,6 +267,31 @@ __device__ __forceinline__ float poly_exp2(float x) {
   return __uint_as_float(__float_as_uint(t) * (1u << 23) + __float_as_uint(p));
 }
 
+// poly_exp2 of a pair with the float steps as packed f32x2 operations (the clamp and the exponent
+// add stay scalar): about 5 issue slots per element instead of 8
+__device__ __forceinline__ void poly_exp2_pair(float& r0, float& r1, float x0, float x1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  uint64_t rx, rt, rm, rn, rr, rf, rp, ra, rb, rc;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(rx) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};\n" : "=l"(rm) : "f"(12582912.0f));
+  asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(rt) : "l"(rx), "l"(rm));        // t = x + 1.5 * 2^23
+  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(rn) : "l"(rt), "l"(rm));        // round(x)
+  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(rf) : "l"(rx), "l"(rn));        // f = x - round(x)
+  asm("mov.b64 %0, {%1, %1};\n" : "=l"(ra) : "f"(0.0551716685f));
+  asm("mov.b64 %0, {%1, %1};\n" : "=l"(rb) : "f"(0.2426111251f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(rp) : "l"(rf), "l"(ra), "l"(rb));
+  asm("mov.b64 %0, {%1, %1};\n" : "=l"(rc) : "f"(0.6932609677f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(rr) : "l"(rp), "l"(rf), "l"(rc));
+  asm("mov.b64 %0, {%1, %1};\n" : "=l"(rc) : "f"(0.9999280572f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(rp) : "l"(rr), "l"(rf), "l"(rc));
+  float t0, t1, p0, p1;
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(t0), "=f"(t1) : "l"(rt));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(p0), "=f"(p1) : "l"(rp));
+  r0 = __uint_as_float(__float_as_uint(t0) * (1u << 23) + __float_as_uint(p0));
+  r1 = __uint_as_float(__float_as_uint(t1) * (1u << 23) + __float_as_uint(p1));
+}
+
 // max of three floats in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
