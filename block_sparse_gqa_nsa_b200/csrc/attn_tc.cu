@@ -35,10 +35,10 @@ using namespace tc;
 
 // One pair in kPolyMod of the exponentials goes through poly_exp2_pair on the FMA pipe instead of
 // MUFU (whose 16 ex2 per clock per SM bound the kernel at d = 32); 0 keeps all on MUFU.  With the
-// packed f32x2 softmax arithmetic leaving issue slots free, 1 pair in 8 measured fastest
-// (4, 8 and 16 tried: sparse stage 3.96 / 3.89 / 3.93 ms against 4.06 ms with MUFU alone).
+// packed f32x2 softmax arithmetic leaving issue slots free, 1 pair in 6 measured fastest on the
+// sparse stage (1 in 5 / 6 / 8 / 10: 3.775 / 3.773 / 3.80 / 3.83 ms; MUFU alone 3.95 ms).
 #ifndef LSRM_POLY_MOD
-#define LSRM_POLY_MOD 8
+#define LSRM_POLY_MOD 6
 #endif
 constexpr int kPolyMod = LSRM_POLY_MOD;
 
@@ -620,11 +620,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           const int j = 16 * qd + 2 * i;
           const float s0 = need_mask ? masked(r[2 * i], j) : __uint_as_float(r[2 * i]);
           const float s1 = need_mask ? masked(r[2 * i + 1], j + 1) : __uint_as_float(r[2 * i + 1]);
-          if constexpr (topk) {
-            qm[i & 1] = fmax3(qm[i & 1], s0, s1);
-          } else {
-            mx[i & 3] = fmax3(mx[i & 3], s0, s1);
-          }
+          // the running max is tracked only where it is the top-k gate; elsewhere the row sum
+          // tells when the reference has to move (see the caller)
+          if constexpr (topk) qm[i & 1] = fmax3(qm[i & 1], s0, s1);
           float x0, x1;
           ffma2(x0, x1, s0, s1, sc, nm);  // one packed FMA for the pair
           float p0, p1;
@@ -801,9 +799,24 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       } else {
         const float mraw = exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
         if (!pv_ok) { ok = false; break; }
-        // move the reference only when the row max would exceed it by more than 2^8
-        const float cand = mraw == -INFINITY ? -INFINITY : mraw * sc;
-        const bool grow = cand > m + 8.f;
+        // Move the reference only when it has fallen well behind the row max.  With the top-k on,
+        // the chunk max is at hand (the gate): move when it exceeds the reference by more than
+        // 2^8.  Otherwise the chunk's sum of P decides: every P is at most that sum, so a sum up
+        // to 2^16 keeps every P (and O) far inside range, and only a larger sum (or an infinite
+        // one) has the chunk max read back from S and the reference moved to it.
+        float cand;
+        bool grow;
+        if (topk_on && br == 0) {
+          cand = mraw == -INFINITY ? -INFINITY : mraw * sc;
+          grow = cand > m + 8.f;
+        } else {
+          grow = !(lsum <= 65536.f);
+          cand = -INFINITY;
+          if (__any_sync(0xffffffffu, grow)) {
+            const float mr = chunk_max(need_mask);
+            cand = mr == -INFINITY ? -INFINITY : mr * sc;
+          }
+        }
         if (__any_sync(0xffffffffu, grow)) {
           const float mn = grow ? cand : m;
           const float alpha = grow ? (m == -INFINITY ? 0.f : fast_exp2(m - mn)) : 1.f;
