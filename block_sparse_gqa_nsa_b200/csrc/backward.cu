@@ -98,6 +98,7 @@ struct BqtSmem {
   float acc[D][128];       // dQ of the tile, column-major
   float xdg[128];          // half 1's partial dgates sum, handed to half 0
   float dgs[128];          // the full sum, handed back
+  float dlt[3][2][128];    // with saved branch outputs: Delta_b of each thread's row (its own slot)
   uint64_t q_full, kv_full[C::kStages], kv_empty[C::kStages], s_full, p_full, pv_done, drain;
   uint64_t xfer[4], back[4];  // pass-A end hand-over between the two warps that own 32 rows
   uint32_t tmem_base;
@@ -107,7 +108,6 @@ struct BqtSmem {
   int sel_n[kBqtMaxSel];
 };
 
-// chunk order: for each branch with keys, its chunks twice (pass A, then pass B)
 // chunk sequence of the query pass: per branch, pass A then pass B over the branch's chunks, or
 // pass B alone when the forward's branch outputs were saved (two_pass = 0)
 struct BqtSeq {
@@ -321,9 +321,9 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     }
     // With the forward's branch outputs saved, dgates_b = <dO, o_b> and Delta_b = g_b dgates_b come
     // straight from them (fp32 dot products over d) and pass A is skipped.
-    float delta_b[3] = {0.f, 0.f, 0.f};
     if (p.obr != nullptr && valid) {
       const uint4* go = reinterpret_cast<const uint4*>(p.dout + orow * D);
+#pragma unroll 1
       for (int b = 0; b < p.NG; ++b) {
         if (seq.n[b] == 0) continue;
         const uint4* ob = reinterpret_cast<const uint4*>(p.obr + (orow * p.NG + b) * D);
@@ -338,11 +338,15 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
             dg = fmaf(bf16_to_f32((uint16_t)(xs[e] >> 16)), bf16_to_f32((uint16_t)(ys[e] >> 16)), dg);
           }
         }
-        delta_b[b] = gate[b] * dg;
+        // constant indices only (selects), so the per-branch arrays stay in registers
+        const float gb = b == 0 ? gate[0] : (b == 1 ? gate[1] : gate[2]);
+        const float lb = b == 0 ? lse2[0] : (b == 1 ? lse2[1] : lse2[2]);
+        const float db = gb * dg;
+        S.dlt[b][h][row] = db;  // read back when the branch's chunks start (kept out of registers)
         if (h == 0) {
           p.dgates[orow * p.NG + b] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
           p.rowc[((size_t)b * p.N + t0 + tok_local) * p.Hq + g * p.G + R % p.G] =
-              make_float4(lse2[b], gate[b], delta_b[b], __int_as_float(tok_local));
+              make_float4(lb, gb, db, __int_as_float(tok_local));
         }
       }
     }
@@ -431,7 +435,7 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       tc_fence_after();
       pv_before_store = nb - 1;  // the dS columns are free once the previous dS K product is done
       if (!pass && first) dg_part = 0.f;
-      if (!seq.two_pass && first) delta = br == 0 ? delta_b[0] : (br == 1 ? delta_b[1] : delta_b[2]);
+      if (!seq.two_pass && first) delta = valid ? S.dlt[br][h][row] : 0.f;
       const float l2 = br == 0 ? lse2[0] : (br == 1 ? lse2[1] : lse2[2]);
       const float gb = br == 0 ? gate[0] : (br == 1 ? gate[1] : gate[2]);
       const bool need_mask = br == 2 || nv < 32 * (h + 1);
@@ -752,7 +756,7 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       constexpr bool kWindow = decltype(window_tag)::value;
       constexpr bool kMask = decltype(mask_tag)::value;  // rows past the chunk's valid rows
       const int nrows = S.nrows[st];
-      uint32_t sa[16], sb[16], da[16], db[16];
+      uint32_t sa[16], da[16];
       auto quarter_pass = [&](const uint32_t* sr, const uint32_t* dr, int qd) {
         uint32_t pg[8], ds[8];
 #pragma unroll
@@ -780,14 +784,16 @@ bwd_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
           tmem_st8(tbase + C::kColDS + 16 * h + 8 * qd, ds);
         }
       };
+      // one quarter of S and dP in flight at a time: with two, the 64 registers of loads pushed the
+      // kernel past its 96-register budget into spills (sequential loads measured 5% faster)
       tmem_ld16(tbase + C::kColS + 32 * h, sa);
       tmem_ld16(tbase + C::kColDP + 32 * h, da);
       tmem_ld_wait();
-      tmem_ld16(tbase + C::kColS + 32 * h + 16, sb);
-      tmem_ld16(tbase + C::kColDP + 32 * h + 16, db);
       quarter_pass(sa, da, 0);
+      tmem_ld16(tbase + C::kColS + 32 * h + 16, sa);
+      tmem_ld16(tbase + C::kColDP + 32 * h + 16, da);
       tmem_ld_wait();
-      quarter_pass(sb, db, 1);
+      quarter_pass(sa, da, 1);
     };
     bool ok = active;
     for (int c = 0; ok && c < total; ++c) {
