@@ -142,6 +142,9 @@ struct TcParams {
   // pass (bound_pass = 1: scores only, no softmax, no P V) writes it; the top-k pass reads it
   float* topk_thr;
   int bound_pass;
+  // optional row -> block id map of the keys (the pooled keys may be stored in another order);
+  // the emitted top-k are block ids
+  const int32_t* topk_ids;
 };
 
 enum : int { TC_CMP = 1, TC_SLC = 2, TC_WIN = 4 };
@@ -246,11 +249,13 @@ __device__ __noinline__ KeepBest topk_keep_best(float* val, int* id, int n, int 
 
 // Emit the row's k best in order (logit desc, block asc); a row with fewer than k candidates pads
 // with -1.
-__device__ __noinline__ void topk_emit(const float* val, const int* id, int n, int k, int32_t* dst) {
-  if (!cand_ranks_fast(val, n, [&](int i, int r) { if (r < k) dst[r] = id[i * 128]; })) {
+__device__ __noinline__ void topk_emit(const float* val, const int* id, int n, int k, int32_t* dst,
+                                       const int32_t* ids) {
+  auto put = [&](int r, int i) { dst[r] = ids != nullptr ? ids[id[i * 128]] : id[i * 128]; };
+  if (!cand_ranks_fast(val, n, [&](int i, int r) { if (r < k) put(r, i); })) {
     for (int i = 0; i < n; ++i) {
       const int r = cand_rank_exact(val, n, i, val[i * 128]);
-      if (r < k) dst[r] = id[i * 128];
+      if (r < k) put(r, i);
     }
   }
   for (int r = n; r < k; ++r) dst[r] = -1;
@@ -853,7 +858,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       if (p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first] = -INFINITY;
     }
     if (ok && topk_on && valid)
-      topk_emit(cval, cid, ncand, p.topk_k, p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k);
+      topk_emit(cval, cid, ncand, p.topk_k, p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k, p.topk_ids);
     if (ok && cs.total > 0 && wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
       tc_fence_after();
       finalize(prev_br, m, l);
@@ -953,11 +958,13 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
 // branch (optionally with the streaming top-k that routes it) and the forced-block part of the
 // pooled-query selected branch.  Writes fp32 obranch [n_q][H][D] and the natural-log lse [n_q][H].
 // With topk_thr ([n_q][H] fp32 scratch) the top-k pass is preceded by the bound pass, whose
-// per-row lower bound on the k-th logit lets the top-k pass skip almost every candidate.
+// per-row lower bound on the k-th logit lets the top-k pass skip almost every candidate.  With
+// topk_ids the key rows are stored in another order (forced_bits then marks rows) and the
+// emitted indices are topk_ids[row].
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
-                              float* topk_thr, uint32_t* status, cudaStream_t stream) {
+                              float* topk_thr, uint32_t* status, cudaStream_t stream, const int32_t* topk_ids) {
   if (topk_idx != nullptr && (D != 64 || topk_k < 1 || topk_k > 32 || forced_bits == nullptr))
     return LSRM_ERR_UNSUPPORTED;
   if ((n_q + 255) / 256 > 65535 || n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
@@ -987,6 +994,7 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
   p.topk_idx = topk_idx;
   p.topk_k = topk_k;
   p.forced_bits = forced_bits;
+  p.topk_ids = topk_ids;
   if (D == 32) return launch_tc_d<32>(d, p, q, nullptr, nullptr, kc, vc, kc_rows, stream);
   if (D != 64) return LSRM_ERR_UNSUPPORTED;
   if (topk_idx != nullptr && topk_thr != nullptr) {

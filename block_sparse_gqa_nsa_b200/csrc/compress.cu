@@ -17,7 +17,8 @@ constexpr int kCompressThreads = 256;
 __global__ void __launch_bounds__(kCompressThreads)
 compress_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__ x0, const uint16_t* __restrict__ x1,
                 const uint16_t* __restrict__ x2, int32_t h0, int32_t h1, int32_t h2, int32_t d,
-                float* o32_0, uint16_t* o16_0, float* o32_1, uint16_t* o16_1, float* o32_2, uint16_t* o16_2) {
+                float* o32_0, uint16_t* o16_0, float* o32_1, uint16_t* o16_1, float* o32_2, uint16_t* o16_2,
+                const int32_t* __restrict__ kv_row) {
   extern __shared__ float red[];  // [groups][cols]
   const int b = blockIdx.x;
   const int which = blockIdx.y;
@@ -30,6 +31,8 @@ compress_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__ x0
   const int c8 = cols / 8;          // 16-byte column slices per token row
   const int t0 = off[b], t1 = off[b + 1];
   const int n = t1 - t0;
+  // the K and V means may go to a permuted row (kv_row[b]); Q means stay at row b
+  const int orow = (kv_row != nullptr && which < 2) ? kv_row[b] : b;
   const float inv_n = n > 0 ? 1.0f / (float)n : 0.0f;
   // process the columns in passes of at most kCompressThreads slices
   for (int cbase = 0; cbase < c8; cbase += kCompressThreads) {
@@ -59,7 +62,7 @@ compress_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__ x0
       float s = 0.0f;
       for (int g = 0; g < groups; ++g) s += red[(size_t)g * slices * 8 + e];
       const float m = s * inv_n;
-      const size_t oi = (size_t)b * cols + (size_t)cbase * 8 + e;
+      const size_t oi = (size_t)orow * cols + (size_t)cbase * 8 + e;
       if (o32) o32[oi] = m;
       if (o16) o16[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(m));
     }
@@ -69,13 +72,13 @@ compress_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__ x0
 
 lsrm_status launch_compress(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                             float* kc32, void* kc, float* vc32, void* vc, float* qc32, void* qc,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const int32_t* kv_row) {
   const int ny = (q != nullptr && (qc32 != nullptr || qc != nullptr)) ? 3 : 2;
   dim3 grid((unsigned)d.n_blocks, (unsigned)ny);
   const size_t smem = (size_t)kCompressThreads * 8 * sizeof(float);
   compress_kernel<<<grid, kCompressThreads, smem, stream>>>(
       off, (const uint16_t*)k, (const uint16_t*)v, (const uint16_t*)q, d.n_kv_heads, d.n_kv_heads, d.n_q_heads,
-      d.head_dim, kc32, (uint16_t*)kc, vc32, (uint16_t*)vc, qc32, (uint16_t*)qc);
+      d.head_dim, kc32, (uint16_t*)kc, vc32, (uint16_t*)vc, qc32, (uint16_t*)qc, kv_row);
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 

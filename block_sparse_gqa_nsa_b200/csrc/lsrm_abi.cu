@@ -9,7 +9,8 @@
 
 namespace lsrm {
 lsrm_status launch_compress(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
-                            float* kc32, void* kc, float* vc32, void* vc, float* qc32, void* qc, cudaStream_t s);
+                            float* kc32, void* kc, float* vc32, void* vc, float* qc32, void* qc, cudaStream_t s,
+                            const int32_t* kv_row = nullptr);
 lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, const int32_t* coords, int32_t* cen,
                                    int32_t* idx, uint32_t* status, cudaStream_t s);
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
@@ -23,12 +24,15 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
-                              float* topk_thr, uint32_t* status, cudaStream_t stream);
+                              float* topk_thr, uint32_t* status, cudaStream_t stream,
+                              const int32_t* topk_ids = nullptr);
 lsrm_status launch_pooled_broadcast(const lsrm_nsa_desc& d, const int32_t* off, const float* o_blk,
                                     const float* lse_blk, float* o_cmp, float* lse, cudaStream_t s);
 lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, const void* k, const void* v,
                                   uint32_t* bits, int* pre, int* total, void* kf, void* vf, uint32_t* status,
                                   cudaStream_t s);
+lsrm_status launch_key_order(const lsrm_nsa_desc& d, const uint32_t* bits, int32_t* row_of_block,
+                             int32_t* block_of_row, uint32_t* bits_part, cudaStream_t s);
 lsrm_status launch_speed3r_routed(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
                                   const void* v, const void* gates, const int32_t* idx, const float* o_forced,
                                   const float* lse_forced, const float* o_blk, const float* lse_blk, void* out,
@@ -259,18 +263,25 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
     if (route_mode == LSRM_ROUTE_GIVEN && idx_inout == nullptr) return LSRM_ERR_INVALID_ARG;
     if (d.head_dim != 64 || d.max_block_len > 16) return LSRM_ERR_UNSUPPORTED;
     void* qc16 = wsp<void>(ws, w.qc16);
-    LSRM_TRY(launch_compress(d, off, q, k, v, nullptr, kc16, nullptr, vc16, wsp<float>(ws, w.qc32), qc16, s));
     int* ftotal = wsp<int>(ws, w.ftotal);
     LSRM_TRY(launch_speed3r_forced(d, off, k, v, wsp<uint32_t>(ws, w.fbits), wsp<int>(ws, w.fpre), ftotal,
                                    wsp<void>(ws, w.kf), wsp<void>(ws, w.vf), status_of(ws), s));
+    // the pooled keys are stored non-forced first (in block order), then the forced blocks, so
+    // the routing passes meet forced keys only in their last chunks; rows map back to blocks
+    int32_t* row_of_block = wsp<int32_t>(ws, w.krow);
+    int32_t* block_of_row = wsp<int32_t>(ws, w.kblk);
+    uint32_t* bits_part = wsp<uint32_t>(ws, w.fbits_part);
+    LSRM_TRY(launch_key_order(d, wsp<uint32_t>(ws, w.fbits), row_of_block, block_of_row, bits_part, s));
+    LSRM_TRY(launch_compress(d, off, q, k, v, nullptr, kc16, nullptr, vc16, wsp<float>(ws, w.qc32), qc16, s,
+                             row_of_block));
     float* o_blk = wsp<float>(ws, w.obranch);
     float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
     const bool route = route_mode == LSRM_ROUTE_SCORE;
     if (route && d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
     LSRM_TRY(launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc16, kc16, vc16, d.n_blocks, d.n_blocks,
                                nullptr, tau_of(d), o_blk, l_blk, route ? idx : nullptr, route ? d.top_k : 0,
-                               route ? wsp<uint32_t>(ws, w.fbits) : nullptr, route ? wsp<float>(ws, w.rthr) : nullptr,
-                               status_of(ws), s));
+                               route ? bits_part : nullptr, route ? wsp<float>(ws, w.rthr) : nullptr,
+                               status_of(ws), s, route ? block_of_row : nullptr));
     float* ofrc = wsp<float>(ws, w.ofrc);
     float* lfrc = wsp<float>(ws, w.lfrc);
     const long long cap = (long long)(d.n_forced > 0 ? d.n_forced : 1) * d.max_block_len;

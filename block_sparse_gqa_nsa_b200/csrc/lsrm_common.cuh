@@ -24,6 +24,9 @@ struct Workspace {
   // and the forced part of the selected branch per token
   size_t fbits, fpre, ftotal, kf, vf, ofrc, lfrc;
   size_t rthr;  // per (block, head) lower bound on the k-th routing logit
+  // pooled keys stored non-forced first: row of each block, block of each row, and the forced
+  // bitmap over rows
+  size_t krow, kblk, fbits_part;
   size_t total;
 };
 
@@ -86,6 +89,9 @@ inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   w.ofrc = o;      o = align256(o + (d.pooled_q ? N * Hq * D * 4 : 0));
   w.lfrc = o;      o = align256(o + (d.pooled_q ? N * Hq * 4 : 0));
   w.rthr = o;      o = align256(o + (d.pooled_q ? B * Hq * 4 : 0));
+  w.krow = o;      o = align256(o + (d.pooled_q ? B * 4 : 0));
+  w.kblk = o;      o = align256(o + (d.pooled_q ? B * 4 : 0));
+  w.fbits_part = o; o = align256(o + (d.pooled_q ? (B / 32 + 2) * 4 : 0));
   w.total = o;
   return w;
 }

@@ -299,6 +299,48 @@ lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, co
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 
+// Row order of the pooled keys for the routing passes: non-forced blocks first, in block order,
+// then the forced blocks in block order (a stable partition, so among candidates row order is
+// block order and ties still go to the lower block id).  One CTA: per-word forced counts, their
+// exclusive prefix, then each block's row, the inverse map and the forced bitmap over rows.
+__global__ void key_order_kernel(const uint32_t* __restrict__ bits, int B, int32_t* row_of_block,
+                                 int32_t* block_of_row, uint32_t* bits_part) {
+  extern __shared__ int pre[];  // [n_words + 1]
+  const int n_words = (B + 31) / 32;
+  for (int w = threadIdx.x; w < n_words; w += blockDim.x) pre[w + 1] = __popc(bits[w]);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    pre[0] = 0;
+    for (int w = 0; w < n_words; ++w) pre[w + 1] += pre[w];
+  }
+  __syncthreads();
+  const int n_nf = B - pre[n_words];
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const uint32_t word = bits[b >> 5];
+    const int below = pre[b >> 5] + __popc(word & ((1u << (b & 31)) - 1u));  // forced blocks below b
+    const int r = ((word >> (b & 31)) & 1u) ? n_nf + below : b - below;
+    row_of_block[b] = r;
+    block_of_row[r] = b;
+  }
+  for (int w = threadIdx.x; w < B / 32 + 2; w += blockDim.x) {
+    const int lo = 32 * w, s0 = max(lo, n_nf) - lo, s1 = min(lo + 32, B) - lo;
+    uint32_t m = 0u;
+    if (s1 > s0) {
+      const uint32_t upto = s1 >= 32 ? 0xffffffffu : ((1u << s1) - 1u);
+      m = upto & ~((1u << s0) - 1u);
+    }
+    bits_part[w] = m;
+  }
+}
+
+lsrm_status launch_key_order(const lsrm_nsa_desc& d, const uint32_t* bits, int32_t* row_of_block,
+                             int32_t* block_of_row, uint32_t* bits_part, cudaStream_t s) {
+  const int n_words = (d.n_blocks + 31) / 32;
+  key_order_kernel<<<1, 1024, (size_t)(n_words + 1) * sizeof(int), s>>>(bits, d.n_blocks, row_of_block,
+                                                                        block_of_row, bits_part);
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
 lsrm_status launch_speed3r_routed(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
                                   const void* v, const void* gates, const int32_t* idx, const float* o_forced,
                                   const float* lse_forced, const float* o_blk, const float* lse_blk, void* out,

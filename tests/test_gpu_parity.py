@@ -620,18 +620,20 @@ def test_speed3r_routing_ties_break_by_block_id():
     assert checked > 0.9 * w.n_blocks * w.n_q_heads
 
 
-def test_two_gate_layer_forward_and_backward():
+@pytest.mark.parametrize("saved", [False, True])
+def test_two_gate_layer_forward_and_backward(saved):
     # n_gates = 2: compressed and selected branches only (no window), forward and backward
     w = make_workload("ragged_geo")
     w.gates = np.ascontiguousarray(w.gates[..., :2])
     w.n_gates = 2
     c = DeviceCase(w)
-    out, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC)
+    obr = _branch_outputs(c) if saved else None
+    out, idx, lse = _forward(c, nsa.ROUTE_GEOMETRIC, obr=obr)
     D = oracle_desc(w)
     ref_idx, _ = O.route_geometric(D, w.off, w.coords)
     assert np.array_equal(to_np(idx).reshape(w.n_blocks, -1), ref_idx)
     assert_close(to_np(out), O.forward(D, w.off, w.q, w.k, w.v, w.gates, ref_idx), "out")
     dout = _dout(w)
-    got = _gpu_backward(c, idx, 1, lse, bf16_tensor(dout))
+    got = _gpu_backward(c, idx, 1, lse, bf16_tensor(dout), obr=obr)
     ref = O.backward(D, w.off, w.q, w.k, w.v, w.gates, ref_idx, dout, nthreads=8)
     _check_grads(got, ref)
