@@ -699,8 +699,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     };
 
     if (D == 64 && p.bound_pass) {
-      // ---- bound pass (d = 64 only): per row, the max non-forced logit of each of 64 key groups (chunk c of
-      // kBoundKeys keys joins group c mod 64), then the topk_k-th largest group max.  Groups are disjoint, so
+      // ---- bound pass (d = 64 only): per row, the max non-forced logit of each of 64 key groups (the
+      // 32-key block b of the stream joins group b mod 64, so 1024 keys already fill 32 groups),
+      // then the topk_k-th largest group max.  Groups are disjoint, so
       // at least topk_k distinct keys score at or above that value: a lower bound on the
       // topk_k-th largest logit that needs no selection in the per-key loop.
       float* gmax = acc;  // gmax[i * 128], i < 64 (the output accumulator is unused here)
@@ -746,7 +747,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         // 32 columns at a time, each load issued before the previous block is reduced
         const uint32_t col = tbase + b * C::kBoundKeys;
         uint32_t ra[32], rb[32];
-        float mx = -INFINITY;
+        float mxs[kW];  // max of each 32-key block of the chunk
         tmem_ld32(col, ra);
         tmem_ld_wait();
 #pragma unroll
@@ -754,14 +755,17 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           uint32_t* cur = (h & 1) ? rb : ra;
           uint32_t* nxt = (h & 1) ? ra : rb;
           if (h + 1 < kW) tmem_ld32(col + 32 * (h + 1), nxt);
-          mx = fmaxf(mx, fmaxf(quarter_max(cur, 32 * h, fw[h] & 0xffffu, tail),
-                               quarter_max(cur + 16, 32 * h + 16, fw[h] >> 16, tail)));
+          mxs[h] = fmaxf(quarter_max(cur, 32 * h, fw[h] & 0xffffu, tail),
+                         quarter_max(cur + 16, 32 * h + 16, fw[h] >> 16, tail));
           if (h + 1 < kW) tmem_ld_wait();
         }
         tc_fence_before();
         mbar_arrive(&S.bs_free[t][b]);
-        float& gv = gmax[(c & 63) * 128];
-        gv = fmaxf(gv, mx);
+#pragma unroll
+        for (int h = 0; h < kW; ++h) {
+          float& gv = gmax[((c * kW + h) & 63) * 128];
+          gv = fmaxf(gv, mxs[h]);
+        }
       }
       if (okb && valid) {
         // the k-th largest of the 64 group maxima: the smallest value with fewer than k above it
