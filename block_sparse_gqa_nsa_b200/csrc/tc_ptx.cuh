@@ -36,26 +36,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// non-blocking probe of a phase (never suspends the thread)
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// try_wait with a short suspend-time hint (ns): sleeps at most that long when the phase is open
-__device__ __forceinline__ bool mbar_try_wait_short(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
@@ -251,24 +231,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
+
 // 2^x on the FMA pipe, for x <= 127 (anything below -125 returns about 2^-125).  Cody-Waite
 // style: x = j + f with j = round(x) taken from the low mantissa bits of x + 1.5 * 2^23 and
 // f in [-0.5, 0.5]; 2^f from a degree-3 polynomial (coefficients fitted here by a Remez
 // exchange on the relative error over [-0.5, 0.5]: max relative error 7.5e-5, far below
 // the bf16 rounding the result goes through); 2^j is added into the exponent field with one
 // integer multiply-add ((1.5 * 2^23 + j) * 2^23 == j * 2^23 mod 2^32).
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(f, 0.0551716685f, 0.2426111251f);
-  p = fmaf(p, f, 0.6932609677f);
-  p = fmaf(p, f, 0.9999280572f);
-  return __uint_as_float(__float_as_uint(t) * (1u << 23) + __float_as_uint(p));
-}
-
-// poly_exp2 of a pair with the float steps as packed f32x2 operations (the clamp and the exponent
-// add stay scalar): about 5 issue slots per element instead of 8
+// Two elements at once: the float steps run as packed f32x2 operations (the clamp and the
+// exponent add stay scalar), about 5 issue slots per element.
 __device__ __forceinline__ void poly_exp2_pair(float& r0, float& r1, float x0, float x1) {
   x0 = fmaxf(x0, -125.0f);
   x1 = fmaxf(x1, -125.0f);
