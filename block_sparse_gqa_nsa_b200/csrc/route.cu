@@ -104,49 +104,73 @@ geo_topk_kernel(const int32_t* __restrict__ cen, int32_t B, int32_t k, int32_t* 
 }
 
 // One CTA per query block for B <= kRouteThreads * kGeoPer: each thread computes its candidates'
-// distances once and keeps them in registers; every round takes the best candidate strictly after
-// the previous round's (key, index) with one block barrier (the per-warp winners alternate
-// between two shared buffers, and every thread reduces the eight winners itself).
+// distances once, keeps them in registers and sorts them by (distance, index) with a 19-comparator
+// network, so a thread's best remaining candidate is always its first.  Each round the block takes
+// the minimum of those heads (warp shuffle, then the eight warp winners through shared memory and
+// a 3-step shuffle, one block barrier per round with the winners alternating between two shared
+// buffers) and the thread that owned the winner drops it.  The selection is the same as taking, k
+// times, the best candidate strictly after the previous winner.
 constexpr int kGeoPer = 8;
+__device__ __forceinline__ void key_cswap(DistKey& a, DistKey& b) {
+  if (key_less(b, a)) {
+    const DistKey t = a;
+    a = b;
+    b = t;
+  }
+}
+__device__ __forceinline__ DistKey shfl_key(const DistKey& x, int src_or_mask, bool xor_mode) {
+  DistKey y;
+  y.d = xor_mode ? __shfl_xor_sync(0xffffffffu, x.d, src_or_mask) : __shfl_sync(0xffffffffu, x.d, src_or_mask);
+  y.j = xor_mode ? __shfl_xor_sync(0xffffffffu, x.j, src_or_mask) : __shfl_sync(0xffffffffu, x.j, src_or_mask);
+  return y;
+}
 __global__ void __launch_bounds__(kRouteThreads)
 geo_topk_reg_kernel(const int32_t* __restrict__ cen, int32_t B, int32_t k, int32_t* __restrict__ idx) {
+  static_assert(kGeoPer == 8 && kRouteThreads / 32 == 8, "the sorting network and the winner reduction are for 8");
   __shared__ DistKey s_warp[2][kRouteThreads / 32];
   const int a = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long ax = cen[a * 3 + 0], ay = cen[a * 3 + 1], az = cen[a * 3 + 2];
-  long long dist[kGeoPer];
+  DistKey key[kGeoPer];
 #pragma unroll
   for (int i = 0; i < kGeoPer; ++i) {
     const int j = tid + i * kRouteThreads;
     if (j < B) {
       const long long dx = cen[j * 3 + 0] - ax, dy = cen[j * 3 + 1] - ay, dz = cen[j * 3 + 2] - az;
-      dist[i] = dx * dx + dy * dy + dz * dz;
+      key[i] = DistKey{dx * dx + dy * dy + dz * dz, j};
     } else {
-      dist[i] = LLONG_MAX;
+      key[i] = DistKey{LLONG_MAX, INT_MAX};
     }
   }
-  DistKey last{-1, -1};
+  // Batcher's odd-even merge network for 8 inputs (19 comparators, depth 6)
+  key_cswap(key[0], key[2]); key_cswap(key[1], key[3]); key_cswap(key[4], key[6]); key_cswap(key[5], key[7]);
+  key_cswap(key[0], key[4]); key_cswap(key[1], key[5]); key_cswap(key[2], key[6]); key_cswap(key[3], key[7]);
+  key_cswap(key[0], key[1]); key_cswap(key[2], key[3]); key_cswap(key[4], key[5]); key_cswap(key[6], key[7]);
+  key_cswap(key[2], key[4]); key_cswap(key[3], key[5]);
+  key_cswap(key[1], key[4]); key_cswap(key[3], key[6]);
+  key_cswap(key[1], key[2]); key_cswap(key[3], key[4]); key_cswap(key[5], key[6]);
   for (int r = 0; r < k; ++r) {
-    DistKey best{LLONG_MAX, INT_MAX};
-#pragma unroll
-    for (int i = 0; i < kGeoPer; ++i) {
-      const int j = tid + i * kRouteThreads;
-      const DistKey cand{dist[i], j};
-      if (j < B && key_less(last, cand) && key_less(cand, best)) best = cand;
-    }
+    DistKey best = key[0];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      DistKey other{__shfl_xor_sync(0xffffffffu, best.d, o), __shfl_xor_sync(0xffffffffu, best.j, o)};
+      const DistKey other = shfl_key(best, o, true);
       if (key_less(other, best)) best = other;
     }
     if (lane == 0) s_warp[r & 1][warp] = best;
     __syncthreads();
-    DistKey b = s_warp[r & 1][0];
+    DistKey b = lane < kRouteThreads / 32 ? s_warp[r & 1][lane] : DistKey{LLONG_MAX, INT_MAX};
 #pragma unroll
-    for (int w = 1; w < kRouteThreads / 32; ++w)
-      if (key_less(s_warp[r & 1][w], b)) b = s_warp[r & 1][w];
+    for (int o = 4; o > 0; o >>= 1) {
+      const DistKey other = shfl_key(b, o, true);
+      if (key_less(other, b)) b = other;
+    }
+    b = shfl_key(b, 0, false);
     if (tid == 0) idx[(size_t)a * k + r] = b.j;
-    last = b;
+    if (key[0].j == b.j) {  // this thread owned the winner: drop it (indices are unique)
+#pragma unroll
+      for (int i = 0; i + 1 < kGeoPer; ++i) key[i] = key[i + 1];
+      key[kGeoPer - 1] = DistKey{LLONG_MAX, INT_MAX};
+    }
   }
 }
 
