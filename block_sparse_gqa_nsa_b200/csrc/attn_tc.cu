@@ -19,7 +19,13 @@
 // 2-5 and 6-9 are two softmax warpgroups, one per M tile, so one tile's exponentials
 // overlap the other tile's MMAs.  Every wait is bounded (see tc::mbar_wait).
 //
-// Tensor memory per M tile (256 columns): S [kKeys fp32] | P [kKeys/2, bf16 pairs] | O [D].
+// Tensor memory per M tile (kColsPerTile: 128 columns at d = 32, 256 at d = 64):
+// S [kKeys fp32] | P [kKeys/2, bf16 pairs] | O [D].
+//
+// The same kernel runs the dense passes of the pooled-query (Speed3R) variant at d = 64: the
+// compressed branch over all block means with a streaming top-k of its logits (candidates above a
+// per-row lower bound on the k-th logit, ranked at the end), the bound pass that computes that
+// bound (scores only), and the pass of every token against the gathered forced tokens.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -806,9 +812,25 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         wait_pv();
         if (!pv_ok) { ok = false; break; }
         if (c > 0) finalize(prev_br, m, l);
-        const float mraw = chunk_max(need_mask);
-        m = mraw == -INFINITY ? -INFINITY : mraw * sc;
-        exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
+        if (topk_on && br == 0) {
+          // the top-k pass moves its reference by the max (its gate), so it starts from the max
+          const float mraw = chunk_max(need_mask);
+          m = mraw == -INFINITY ? -INFINITY : mraw * sc;
+          exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
+        } else {
+          // Start the branch from reference 0 and keep it while the chunk's sum of P lies in
+          // [2^-64, 2^16]: every P then stays far inside the normal range (and the largest is at
+          // least 2^-70).  Otherwise (or with every key masked) the chunk max is read from S and
+          // the chunk redone from it.  Nothing has reached O yet: its first P V overwrites it.
+          m = 0.f;
+          exp_pass(need_mask, 0.f, &lsum);
+          const bool off_range = !(lsum <= 65536.f && lsum >= 5.421010862427522e-20f);
+          if (__any_sync(0xffffffffu, off_range)) {
+            const float mraw = chunk_max(need_mask);
+            if (off_range) m = mraw == -INFINITY ? -INFINITY : mraw * sc;
+            exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum, false);
+          }
+        }
         l = lsum;
       } else {
         const float mraw = exp_pass(need_mask, m == -INFINITY ? 0.f : m, &lsum);
