@@ -846,7 +846,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           cand = mraw == -INFINITY ? -INFINITY : mraw * sc;
           grow = cand > m + 8.f;
         } else {
-          grow = !(lsum <= 65536.f);
+          // (no reference yet, after a first chunk without valid keys: always take the max)
+          grow = !(lsum <= 65536.f) || m == -INFINITY;
           cand = -INFINITY;
           if (__any_sync(0xffffffffu, grow)) {
             const float mr = chunk_max(need_mask);
