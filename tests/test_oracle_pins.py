@@ -392,6 +392,36 @@ def test_speed3r_pooled_branch_and_routing():
             assert np.array_equal(order[:32], idx[i, h])
 
 
+def test_speed3r_routing_ties_go_to_the_lowest_non_forced_blocks():
+    # Speed3R page, section 2.1 (top-k of the pooled logits) and 2.2 (frame 0 and the camera
+    # blocks always selected, so never routed): with every pooled key equal, all logits of a row
+    # tie and the routing must be the k lowest non-forced block ids; a block whose pooled key is
+    # that key scaled up must come first whenever the row's logit on it is positive.
+    w = make_workload("speed3r_small", n_frames=3)
+    D = desc(w)
+    rng = np.random.default_rng(11)
+    qc = rng.standard_normal((w.n_blocks, 16, w.head_dim))
+    u = rng.standard_normal((16, w.head_dim))
+    kc = np.broadcast_to(u, (w.n_blocks, 16, w.head_dim)).copy()
+    forced = set(w.forced.tolist())
+    free = [b for b in range(w.n_blocks) if b not in forced]
+    qb = np.array([0, 7, 150, w.n_blocks - 1], dtype=np.int32)
+    idx, _ = O.route_pooled(D, qc, kc, w.forced, qblocks=qb)
+    for i in range(len(qb)):
+        for h in range(16):
+            assert idx[i, h].tolist() == free[:32], (i, h)
+    star = free[40]  # a late non-forced block
+    kc[star] = 3.0 * u
+    idx, _ = O.route_pooled(D, qc, kc, w.forced, qblocks=qb)
+    for i, a in enumerate(qb):
+        for h in range(16):
+            lu = float(qc[a, h] @ u[h])
+            if lu > 1e-9:
+                assert idx[i, h, 0] == star and idx[i, h, 1:].tolist() == [b for b in free if b != star][:31]
+            elif lu < -1e-9:
+                assert star not in idx[i, h].tolist() and idx[i, h].tolist() == free[:32]
+
+
 # ------------------------------------------------------------------------------------------------
 # S10 backward
 # ------------------------------------------------------------------------------------------------
