@@ -683,9 +683,10 @@ def run_extra(args):
 
         def step():
             nsa.lsrm_nsa_forward(desc, off, q, kk, v, gates, None, nsa.ROUTE_SCORE, out, idx, None, ws)
-        # compress (Q, K, V), forced bitmap / prefix / gather, pooled compressed pass with the
-        # streaming top-k, forced-token pass, routed part with the merge and gated combine
-        launches_per_step = 7
+        # forced bitmap / prefix / gather, key row order, compress (Q, K, V), the bound pass, the
+        # pooled compressed pass with the streaming top-k, the forced-token pass, the routed part
+        # with the merge and gated combine
+        launches_per_step = 9
     else:
         idx = None
 
