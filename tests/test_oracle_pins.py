@@ -457,6 +457,17 @@ def test_backward_matches_central_finite_differences():
             assert abs(fd - grad[i]) < 1e-7 * max(1.0, abs(fd)), (name, i, fd, grad[i])
 
 
+def test_gate_gradient_is_the_inner_product_with_the_branch_output():
+    # out = sum_b g_b o_b with o_b independent of the gates, so dL/dg_b = <dO, o_b> for every
+    # (token, head): the backward's gate gradient against the forward's own branch outputs, at
+    # every entry (the identity the saved-output backward reads dgates from)
+    D, off, qf, kf, vf, gf, idx, dout = _fd_case(5)
+    _, _, _, dg = O.backward_f64(D, off, qf, kf, vf, gf, idx, dout)
+    _, br, _ = O.forward_f64(D, off, qf, kf, vf, gf, idx, want_branches=True)
+    ref = np.einsum("thd,thbd->thb", dout, br)
+    assert np.abs(dg - ref).max() < 1e-12
+
+
 def test_backward_compressed_only_spreads_the_block_gradient_evenly():
     D, off, qf, kf, vf, gf, idx, dout = _fd_case(3)
     g_cmp = np.zeros_like(gf)
