@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r"],
                     help="sparse: the layer forward (the default line); backward: its gradients; dense: the "
                          "dense-stage shape with every block selected; speed3r: the pooled-query variant")
+    ap.add_argument("--record-traffic", nargs=4, metavar=("WHICH", "CSV", "KERNEL_REGEX", "LAUNCHES"),
+                    help="write profiles/traffic.json[WHICH] from an ncu raw CSV export and exit")
     ap.add_argument("--frames", type=int, default=512,
                     help="speed3r only: frames of the synthetic sequence (512 is the workload; fewer give the "
                          "small cases that profiler captures use)")
@@ -102,19 +104,66 @@ def kernel_source_hash(which: str) -> str:
     return h.hexdigest()[:16]
 
 
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+TRAFFIC_METRICS = ("dram__bytes_read.sum", "dram__bytes_write.sum")
+
+
 def profiled_traffic(which: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the kernel
-    sources as they are now (else None)."""
+    """DRAM bytes per launch from profiles/traffic.json (written by `bench.py --record-traffic`
+    from an ncu capture), used only while the kernel sources hash to the value recorded with
+    it (else None: the kernel has changed since the counters were taken)."""
+    if not os.path.exists(TRAFFIC_JSON):
+        return None
+    with open(TRAFFIC_JSON) as f:
+        rec = json.load(f).get(which)
+    if rec is None or rec.get("source_hash") != kernel_source_hash(which):
+        return None
+    return float(rec["bytes_per_launch"])
+
+
+def _ncu_bytes(value: str, unit: str) -> float:
+    scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12,
+             "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    return float(value.replace(",", "")) * scale[unit]
+
+
+def record_traffic(which: str, csv_path: str, kernel_regex: str, launches_per_unit: int, note: str) -> dict:
+    """Write profiles/traffic.json[which] from `ncu -i <rep> --page raw --csv` output: the DRAM
+    read + write bytes of the launches whose name matches kernel_regex, summed over each group of
+    launches_per_unit consecutive launches (one call) and averaged over the groups."""
+    import csv
     import re
-    path = os.path.join(ROOT, "profiles", "traffic.md")
-    if not os.path.exists(path):
-        return None
-    pat = re.compile(rf"^\|\s*{which}\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|", re.M)
-    with open(path) as f:
-        m = pat.search(f.read())
-    if m is None or m.group(2) != kernel_source_hash(which):
-        return None
-    return float(m.group(1))
+    with open(csv_path) as f:
+        rows = list(csv.reader(f))
+    head, units = rows[0], rows[1]
+    col = {n: i for i, n in enumerate(head)}
+    name_col = col["Kernel Name"]
+    per = []
+    for r in rows[2:]:
+        if len(r) != len(head) or not re.search(kernel_regex, r[name_col]):
+            continue
+        per.append(sum(_ncu_bytes(r[col[m]], units[col[m]]) for m in TRAFFIC_METRICS))
+    if not per or len(per) % launches_per_unit:
+        raise ValueError(f"{len(per)} matching launches, not a multiple of {launches_per_unit}")
+    groups = [sum(per[i:i + launches_per_unit]) for i in range(0, len(per), launches_per_unit)]
+    rec = {"bytes_per_launch": sum(groups) / len(groups), "source_hash": kernel_source_hash(which),
+           "kernel_regex": kernel_regex, "launches_per_unit": launches_per_unit, "captures": len(groups),
+           "note": note}
+    data = {}
+    if os.path.exists(TRAFFIC_JSON):
+        with open(TRAFFIC_JSON) as f:
+            data = json.load(f)
+    data[which] = rec
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return rec
+
+
+def cpu_baseline(value: float, sample: str) -> dict:
+    """The oracle's timing as a reported baseline: one thread of the host's cores."""
+    return {"value": value, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
+            "sample": sample}
 
 
 def max_over_ranks(ms: float, device, world: int) -> float:
@@ -241,6 +290,15 @@ class ClockSampler:
 # the oracle on the host: cpu_baseline of our arm, and the whole reference arm
 # ------------------------------------------------------------------------------------------------
 
+def sparse_config(w, world: int, seed: int) -> dict:
+    """The workload description both arms print (identical dicts, so the lines compare)."""
+    return {"workload": WORKLOAD, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
+            "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "top_k": w.top_k,
+            "window": w.window, "route": "geometric",
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (q 249 MB + out 249 MB per step)", "seed": seed}
+
+
 def oracle_sample(w, idx, n_blocks: int, seed: int):
     """Time the fp64 oracle on a seeded sample of query blocks of the workload (1 thread)."""
     import oracle as O
@@ -277,11 +335,9 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": 1000.0 * tsum / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": WORKLOAD, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
-                       "heads": "32q/2kv", "head_dim": 32, "top_k": 16, "window": 64,
-                       "sample": f"{per_step} seeded query blocks per step"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{per_step} query blocks ({per_step * 64} tokens) per step, fp64, 1 thread"},
+            "config": sparse_config(w, args.gpus, args.seed),
+            "cpu_baseline": cpu_baseline(value, f"{per_step} seeded query blocks ({per_step * 64} tokens) per "
+                                                f"step, fp64, 1 thread"),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -402,10 +458,7 @@ def run_ours(args):
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "n_tokens": N, "n_blocks": B, "heads": f"{Hq}q/{Hkv}kv",
-                           "head_dim": d, "top_k": k, "window": w.window, "route": "geometric",
-                           "parallelism": f"replicas{world}" if world > 1 else "single",
-                           "l2": "inputs larger than L2 (q 249 MB + out 249 MB per step)", "seed": args.seed},
+                "config": sparse_config(w, world, args.seed),
                 "effective_tflops": flops["total"] / (ms_per_step / 1000.0) / 1e12,
                 "flops_per_step": flops,
                 "kernel_ms": {"fused_attention": attn_avg, "compress_and_route": sum(pre_ms) / len(pre_ms)},
@@ -418,9 +471,8 @@ def run_ours(args):
         if not args.no_cpu_baseline and world == 1:
             n_blk = args.cpu_sample_blocks or 64
             tok, dt = oracle_sample(w, idx.cpu().numpy(), n_blk, 7)
-            line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"{n_blk} seeded query blocks ({tok} tokens) "
-                                              f"of the same workload, fp64, 1 thread, {dt:.1f} s"}
+            line["cpu_baseline"] = cpu_baseline(tok / dt, f"{n_blk} seeded query blocks ({tok} tokens) "
+                                                          f"of the same workload, fp64, 1 thread, {dt:.1f} s")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -448,13 +500,14 @@ def oracle_backward_sample(w, idx, n_blocks: int, seed: int):
     return int((w.off[qb + 1] - w.off[qb]).sum()), dt
 
 
-def bwd_config(w, world, seed, extra=None):
-    c = {"workload": BWD_WORKLOAD, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
-         "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "top_k": w.top_k,
-         "window": w.window, "route": "geometric (indices fixed from the forward)",
-         "parallelism": f"replicas{world}" if world > 1 else "single", "seed": seed}
-    c.update(extra or {})
-    return c
+def bwd_config(w, world, seed):
+    """The backward workload description both arms print (identical dicts)."""
+    return {"workload": BWD_WORKLOAD, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
+            "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "top_k": w.top_k,
+            "window": w.window, "route": "geometric (indices fixed from the forward)",
+            "parallelism": f"replicas{world}" if world > 1 else "single", "seed": seed,
+            "l2": "inputs larger than L2 (q, dO, dq 249 MB each per step)",
+            "saved_branch_outputs": "bf16 o_b from the forward (745 MB), one pass per branch"}
 
 
 def run_backward_reference(args):
@@ -476,9 +529,9 @@ def run_backward_reference(args):
     line = {"metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * tsum / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": bwd_config(w, 1, args.seed, {"sample": "1 seeded query block per step"}),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": "1 query block (64 tokens) per step, fp64, 1 thread"},
+            "config": bwd_config(w, args.gpus, args.seed),
+            "cpu_baseline": cpu_baseline(value, "1 seeded query block (64 tokens) per step, fp64 backward, "
+                                                "1 thread"),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -594,9 +647,7 @@ def run_backward(args):
         line = {"metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": bwd_config(w, world, args.seed,
-                                     {"l2": "inputs larger than L2 (q, dO, dq 249 MB each per step)",
-                                      "saved_branch_outputs": "bf16 o_b from the forward (745 MB), one pass per branch"}),
+                "config": bwd_config(w, world, args.seed),
                 "flops_per_step": flops,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                              "frac": achieved / peak, "traffic": profiled_traffic("bwd"),
@@ -606,9 +657,8 @@ def run_backward(args):
         if not args.no_cpu_baseline and world == 1:
             n_blk = args.cpu_sample_blocks or 24
             tok, dt = oracle_backward_sample(w, idx.view(B, k).cpu().numpy(), n_blk, 7)
-            line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"{n_blk} seeded query blocks ({tok} tokens) of the same workload, "
-                                              f"fp64 backward, 1 thread, {dt:.1f} s"}
+            line["cpu_baseline"] = cpu_baseline(tok / dt, f"{n_blk} seeded query blocks ({tok} tokens) of the "
+                                                          f"same workload, fp64 backward, 1 thread, {dt:.1f} s")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -623,6 +673,14 @@ EXTRA = {
     "dense": ("sparse-attn fwd tokens/s, dense-stage shape (k = B)", "lsrm_dense_stage_all_blocks"),
     "speed3r": ("sparse-attn fwd tokens/s, Speed3R pooled-query variant", "speed3r_512_frames_top32_forced"),
 }
+
+
+def extra_config(w, workload: str, world: int, seed: int) -> dict:
+    return {"workload": workload, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
+            "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "top_k": w.top_k,
+            "window": w.window, "n_forced": int(len(w.forced)),
+            "parallelism": f"replicas{world}" if world > 1 else "single", "seed": seed,
+            "l2": "inputs larger than L2"}
 
 
 def speed3r_flops(w, idx: np.ndarray) -> dict:
@@ -726,10 +784,7 @@ def run_extra(args):
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic",
-                "config": {"workload": workload, "n_tokens": N, "n_blocks": B, "heads": f"{Hq}q/{Hkv}kv",
-                           "head_dim": d, "top_k": k, "window": w.window, "n_forced": int(len(w.forced)),
-                           "parallelism": f"replicas{world}" if world > 1 else "single", "seed": args.seed,
-                           "l2": "inputs larger than L2"},
+                "config": extra_config(w, workload, world, args.seed),
                 "flops_per_step": flops,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                              "frac": achieved / peak, "traffic": None,
@@ -739,9 +794,8 @@ def run_extra(args):
         if not args.no_cpu_baseline and world == 1:
             n_blk = args.cpu_sample_blocks or 4
             tok, dt = extra_oracle_sample(w, idx.cpu().numpy() if idx is not None else None, n_blk, 7)
-            line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"{n_blk} seeded query blocks ({tok} tokens) of the same workload, "
-                                              f"fp64, 1 thread, {dt:.1f} s"}
+            line["cpu_baseline"] = cpu_baseline(tok / dt, f"{n_blk} seeded query blocks ({tok} tokens) of the "
+                                                          f"same workload, fp64, 1 thread, {dt:.1f} s")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -804,10 +858,8 @@ def run_extra_reference(args, metric, workload):
     line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * tsum / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": workload, "n_tokens": w.n_tokens, "n_blocks": w.n_blocks,
-                       "sample": "1 seeded query block per step"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": "1 query block per step, fp64, 1 thread"},
+            "config": extra_config(w, workload, args.gpus, args.seed),
+            "cpu_baseline": cpu_baseline(value, "1 seeded query block per step, fp64, 1 thread"),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -815,6 +867,10 @@ def run_extra_reference(args, metric, workload):
 
 def main():
     args = parse()
+    if args.record_traffic:
+        which, csv_path, regex, launches = args.record_traffic
+        print(json.dumps(record_traffic(which, csv_path, regex, int(launches), f"from {os.path.basename(csv_path)}")))
+        return 0
     if args.workload == "backward":
         return run_backward_reference(args) if args.impl == "reference" else run_backward(args)
     if args.workload in EXTRA:

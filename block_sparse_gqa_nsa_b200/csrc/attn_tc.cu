@@ -642,7 +642,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           float x0, x1;
           ffma2(x0, x1, s0, s1, sc, nm);  // one packed FMA for the pair
           float p0, p1;
-          if (kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
+          // the polynomial only where every key of the chunk is valid (see poly_exp2_pair)
+          if (!need_mask && kPolyMod > 0 && (8 * qd + i) % (kPolyMod > 0 ? kPolyMod : 1) == kPolyMod - 1) {
             poly_exp2_pair(p0, p1, x0, x1);
           } else {
             p0 = fast_exp2(x0);

@@ -3,6 +3,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include "lsrm_nsa.h"
@@ -10,6 +11,25 @@
 namespace lsrm {
 
 constexpr int kMaxBlockLen = 64;
+
+// Descriptor checks shared by every entry point (host side).
+inline lsrm_status check_desc(const lsrm_nsa_desc* d) {
+  if (d == nullptr) return LSRM_ERR_INVALID_ARG;
+  if (d->n_tokens < 1 || d->n_blocks < 1 || d->n_blocks > d->n_tokens) return LSRM_ERR_INVALID_ARG;
+  if (d->n_tokens > (int64_t)INT32_MAX) return LSRM_ERR_UNSUPPORTED;
+  if (d->max_block_len < 1 || d->max_block_len > kMaxBlockLen) return LSRM_ERR_INVALID_ARG;
+  if (d->n_kv_heads < 1 || d->n_q_heads < d->n_kv_heads || d->n_q_heads % d->n_kv_heads) return LSRM_ERR_INVALID_ARG;
+  if (d->head_dim != 32 && d->head_dim != 64) return LSRM_ERR_UNSUPPORTED;
+  if (d->top_k < 1 || d->top_k > d->n_blocks) return LSRM_ERR_INVALID_ARG;
+  if (d->window < 0 || (d->window & 1)) return LSRM_ERR_INVALID_ARG;
+  if (!(d->scale >= 0.0f) || isinf(d->scale)) return LSRM_ERR_INVALID_ARG;
+  if (d->pooled_q != 0 && d->pooled_q != 1) return LSRM_ERR_INVALID_ARG;
+  if (d->n_gates != 2 && d->n_gates != 3) return LSRM_ERR_INVALID_ARG;
+  if (d->n_forced < 0 || (d->n_forced > 0 && d->forced_blocks == nullptr)) return LSRM_ERR_INVALID_ARG;
+  if (d->pooled_q && (d->n_q_heads != d->n_kv_heads || d->n_gates != 2)) return LSRM_ERR_INVALID_ARG;
+  if (d->pooled_q && d->top_k + d->n_forced > d->n_blocks) return LSRM_ERR_INVALID_ARG;
+  return LSRM_OK;
+}
 
 // ---- device status word (first 4 bytes of the workspace) ---------------------------------------
 // Kernels OR a status bit in; the host reads and clears it.  Bit i set <=> status (i+1) was raised.

@@ -7,8 +7,6 @@
 // lsrm_route_geometric, but keeps the per-block centroids in a fixed array that lives in
 // the library's own device memory (a file-scope __device__ array, held by every GPU that
 // loads the library until the process exits).
-#include <mutex>
-
 #include "lsrm_common.cuh"
 
 namespace lsrm {
@@ -22,22 +20,14 @@ static __device__ __align__(256) int32_t g_noalloc_centroids[kNoAllocMaxBlocks *
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-int32_t* g_cen_ptr[kMaxDevices] = {};
-
-// The host-side name of the array is not a device address: look the address up once per
-// device, with that device current, and hand the result to the kernels.
+// The host-side name of the array is not a device address.  Its address on the current device
+// is looked up on every call (a host-side query that allocates nothing), so that no address
+// outlives the context it belongs to: a pointer cached across a device reset or a recreated
+// primary context would point into a dead module.
 lsrm_status scratch_for_current_device(int32_t** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LSRM_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_cen_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_centroids) != cudaSuccess || p == nullptr) return LSRM_ERR_CUDA;
-    g_cen_ptr[dev] = static_cast<int32_t*>(p);
-  }
-  *out = g_cen_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_centroids) != cudaSuccess || p == nullptr) return LSRM_ERR_CUDA;
+  *out = static_cast<int32_t*>(p);
   return LSRM_OK;
 }
 
@@ -48,9 +38,10 @@ extern "C" lsrm_status lsrm_route_geometric_noalloc(const lsrm_nsa_desc* desc, c
                                                     const int32_t* coords, int32_t* idx, uint32_t* status_or_null,
                                                     void* stream) {
   using namespace lsrm;
-  if (desc == nullptr || off == nullptr || coords == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
-  if (desc->n_blocks < 1 || desc->n_tokens < desc->n_blocks || desc->top_k < 1 || desc->top_k > desc->n_blocks)
-    return LSRM_ERR_INVALID_ARG;
+  // the same descriptor checks as lsrm_route_geometric, then the size limit of the fixed scratch
+  const lsrm_status ds = check_desc(desc);
+  if (ds != LSRM_OK) return ds;
+  if (off == nullptr || coords == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
   if (desc->n_blocks > kNoAllocMaxBlocks) return LSRM_ERR_WORKSPACE;  // the fixed scratch is too small
   int32_t* cen = nullptr;
   const lsrm_status st = scratch_for_current_device(&cen);

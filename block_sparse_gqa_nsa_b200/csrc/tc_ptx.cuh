@@ -232,12 +232,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 
-// 2^x on the FMA pipe, for x <= 127 (anything below -125 returns about 2^-125).  Cody-Waite
-// style: x = j + f with j = round(x) taken from the low mantissa bits of x + 1.5 * 2^23 and
-// f in [-0.5, 0.5]; 2^f from a degree-3 polynomial (coefficients fitted here by a Remez
-// exchange on the relative error over [-0.5, 0.5]: max relative error 7.5e-5, far below
-// the bf16 rounding the result goes through); 2^j is added into the exponent field with one
-// integer multiply-add ((1.5 * 2^23 + j) * 2^23 == j * 2^23 mod 2^32).
+// 2^x on the FMA pipe, for x <= 127.  Cody-Waite style: x = j + f with j = round(x) taken from
+// the low mantissa bits of x + 1.5 * 2^23 and f in [-0.5, 0.5]; 2^f from a degree-3 polynomial
+// whose coefficients are the minimax fit of the relative error on [-0.5, 0.5] (Remez exchange,
+// block_sparse_gqa_nsa_b200/exp2_fit.py: max relative error 7.5e-5, far below the bf16 rounding
+// the result goes through); 2^j is added into the exponent field with one integer multiply-add
+// ((1.5 * 2^23 + j) * 2^23 == j * 2^23 mod 2^32).  Inputs below -125 (masked keys at -inf among
+// them) are clamped there and return about 2^-125, not 0: callers use it only where every key is
+// valid (a key that far below the reference then weighs under 2^-125 against a row sum of at
+// least 2^-64), and keep masked keys on the hardware ex2, whose ex2(-inf) is exactly 0.
 // Two elements at once: the float steps run as packed f32x2 operations (the clamp and the
 // exponent add stay scalar), about 5 issue slots per element.
 __device__ __forceinline__ void poly_exp2_pair(float& r0, float& r1, float x0, float x1) {

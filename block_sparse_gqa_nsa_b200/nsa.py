@@ -29,7 +29,7 @@ ROUTE_GIVEN, ROUTE_SCORE, ROUTE_GEOMETRIC, ROUTE_ALL = 0, 1, 2, 3
 EXPORTS = ("lsrm_nsa_workspace_size", "lsrm_nsa_workspace_init", "lsrm_nsa_compress", "lsrm_route_score_topk",
            "lsrm_route_geometric", "lsrm_route_geometric_noalloc", "lsrm_route_pooled_topk", "lsrm_nsa_cmp_attn", "lsrm_nsa_select_attn",
            "lsrm_nsa_window_attn", "lsrm_nsa_gate_combine", "lsrm_nsa_attend", "lsrm_nsa_forward", "lsrm_nsa_backward",
-           "lsrm_nsa_last_device_status", "lsrm_status_string")
+           "lsrm_nsa_last_device_status", "lsrm_status_string", "lsrm_diag_exp2_poly")
 
 
 class NsaError(RuntimeError):
@@ -88,6 +88,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsrm_nsa_backward": ([D, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_last_device_status": ([vp, vp], ctypes.c_int),
         "lsrm_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "lsrm_diag_exp2_poly": ([vp, vp, ctypes.c_int64, vp], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -169,8 +170,10 @@ def lsrm_route_geometric(desc, off, coords, idx, ws, stream=None):
 def lsrm_route_geometric_noalloc(desc, off, coords, idx, status=None, stream=None):
     """Geometric routing without a workspace, for callers that cannot allocate device memory
     (its scratch is a fixed array inside the library; at most 16384 blocks; calls that
-    overlap on the GPU race).  `status` is an optional device uint32 tensor that receives
-    the bounds bit."""
+    overlap on the GPU race).  `status` is an optional one-element device tensor that receives
+    the bounds bit.  The C entry point declares it uint32_t*; torch has no unsigned 32-bit
+    tensor type, so it is passed as torch.int32, which has the same size and layout (the bit
+    LSRM_ERR_BOUNDS sets, 1 << 4, reads the same in either type)."""
     _check(off, torch.int32, "off"); _check(coords, torch.int32, "coords"); _check(idx, torch.int32, "idx")
     _check(status, torch.int32, "status")
     _call("lsrm_route_geometric_noalloc", ctypes.byref(desc), _ptr(off), _ptr(coords), _ptr(idx), _ptr(status),
@@ -261,3 +264,11 @@ def lsrm_status_string(status: int) -> str:
 
 def default_scale(head_dim: int) -> float:
     return 1.0 / math.sqrt(head_dim)
+
+
+def lsrm_diag_exp2_poly(x, y, stream=None):
+    """y = 2^x through the attention kernels' FMA-pipe polynomial (a diagnostic)."""
+    _check(x, torch.float32, "x"); _check(y, torch.float32, "y")
+    if x.numel() != y.numel():
+        raise ValueError("x and y differ in size")
+    _call("lsrm_diag_exp2_poly", _ptr(x), _ptr(y), ctypes.c_int64(x.numel()), _stream(stream))

@@ -123,14 +123,17 @@ LSRM_API lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32
 /* Geometric routing that allocates nothing and takes no workspace, for callers that may
  * not allocate device memory at call time and have none to lend (for example a plugin in
  * a host framework whose memory pool owns the whole GPU, or a loop whose policy forbids
- * allocation after start-up).  The pages have no counterpart of this call; it computes
- * exactly what lsrm_route_geometric computes.  Its centroid scratch is a fixed array in
- * the library's own device memory (192 KiB, held on every GPU that loads the library until
+ * allocation after start-up).  The pages have no counterpart of this call; it accepts the
+ * same descriptors as lsrm_route_geometric (the same checks, same status codes) and
+ * computes exactly what it computes.  Its centroid scratch is a fixed array in the
+ * library's own device memory (192 KiB, held on every GPU that loads the library until
  * the process exits), so n_blocks may be at most 16384; larger descriptors are rejected
- * with LSRM_ERR_WORKSPACE.  The first call on each device looks up that array's device
- * address (with the device current); make that first call before any stream capture.
- * Every call shares the one array: calls that may overlap on the GPU (different streams,
- * or different host threads on one device) race and must be serialised by the caller.
+ * with LSRM_ERR_WORKSPACE.  Every call looks up that array's address on the current
+ * device (a host-side query that allocates nothing; no address is cached across calls, so
+ * a device reset cannot leave a stale one).  The first call on a device may load the
+ * library's device code there, so make it before any stream capture.  Every call shares
+ * the one array: calls that may overlap on the GPU (different streams, or different host
+ * threads on one device) race and must be serialised by the caller.
  * status_or_null (device uint32, may be NULL) receives LSRM_ERR_BOUNDS as bit
  * (1 << (LSRM_ERR_BOUNDS - 1)) OR-ed in when a coordinate lies outside [-2^29, 2^29];
  * the caller clears it. */
@@ -214,6 +217,13 @@ LSRM_API lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t*
                               const void* v, const void* gates, const int32_t* idx, int32_t idx_heads,
                               const float* lse, const void* obr_or_null, const void* dout, void* dq, void* dk,
                               void* dv, void* dgates, void* ws, void* stream);
+
+/* Diagnostic (no counterpart in the pages): y[i] = 2^x[i] as the attention kernels' FMA-pipe
+ * polynomial computes it (the exponentials of the softmax that do not go to the hardware ex2).
+ * x and y are device float arrays of n elements (caller-owned); valid for x <= 127, and inputs
+ * below -125 return about 2^-125.  Lets a test compare the polynomial with CUDA's exp2f over
+ * its whole range; not part of the layer. */
+LSRM_API lsrm_status lsrm_diag_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
 /* Read (synchronising `stream`) and clear the device status word of the workspace. */
 LSRM_API lsrm_status lsrm_nsa_last_device_status(void* ws, void* stream);

@@ -49,6 +49,17 @@ def test_noalloc_routing_rejects_too_many_blocks_and_reports_bad_coordinates():
     with pytest.raises(nsa.NsaError) as e:
         nsa.lsrm_route_geometric_noalloc(big, off, coords, torch.empty(1, dtype=torch.int32, device="cuda"))
     assert e.value.status == 6  # LSRM_ERR_WORKSPACE: beyond the fixed scratch
+    # descriptors that lsrm_route_geometric rejects are rejected here too, with the same status
+    ws = nsa.workspace(desc)
+    idx0 = torch.empty(w.n_blocks, w.top_k, dtype=torch.int32, device="cuda")
+    for bad_desc in (nsa.make_desc(w.n_tokens, w.n_blocks, 65, 32, 2, 32, w.top_k, 64),      # block > 64
+                     nsa.make_desc(w.n_tokens, w.n_blocks, w.max_block_len, 32, 2, 48, w.top_k, 64),  # d = 48
+                     nsa.make_desc(w.n_tokens, w.n_blocks, w.max_block_len, 32, 2, 32, w.top_k, 63)):  # odd w
+        with pytest.raises(nsa.NsaError) as e_ref:
+            nsa.lsrm_route_geometric(bad_desc, off, coords, idx0, ws)
+        with pytest.raises(nsa.NsaError) as e_na:
+            nsa.lsrm_route_geometric_noalloc(bad_desc, off, coords, idx0)
+        assert e_na.value.status == e_ref.value.status
     bad = coords.clone()
     bad[3, 0] = (1 << 29) + 5
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
