@@ -151,6 +151,14 @@ struct TcParams {
   // optional row -> block id map of the keys (the pooled keys may be stored in another order);
   // the emitted top-k are block ids
   const int32_t* topk_ids;
+  // optional exact ranking: fp32 pooled queries [rows][topk_heads][64] and keys [key rows][heads][64]
+  // (key rows in the stored order) and the largest |key mean| of all keys (float bits); with them
+  // the candidates are ranked by fp32 logits recomputed from the means, and the gate is widened by
+  // a bound on the error of the bf16-operand logits, so the result is the ranking of the exact
+  // means rather than of their bf16 roundings
+  const float* rescore_q;
+  const float* rescore_k;
+  const uint32_t* rescore_kmax;
 };
 
 enum : int { TC_CMP = 1, TC_SLC = 2, TC_WIN = 4 };
@@ -231,6 +239,29 @@ struct KeepBest {
   int n;
   float thr;
 };
+
+// fp32 logit (unscaled dot product) of a pooled query row and a pooled key row, 64 dims each
+__device__ __noinline__ float rescore_dot64(const float* __restrict__ q, const float* __restrict__ k) {
+  const float4* a = reinterpret_cast<const float4*>(q);
+  const float4* b = reinterpret_cast<const float4*>(k);
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const float4 x = __ldg(a + i), y = __ldg(b + i);
+    s0 = fmaf(x.x, y.x, s0);
+    s1 = fmaf(x.y, y.y, s1);
+    s2 = fmaf(x.z, y.z, s2);
+    s3 = fmaf(x.w, y.w, s3);
+  }
+  return (s0 + s1) + (s2 + s3);
+}
+
+// Replace the row's n buffered logits by fp32 logits recomputed from the pooled means (the
+// key row of candidate i is id[i * 128]).
+__device__ __noinline__ void topk_rescore(float* val, const int* id, int n, const float* qrow, const float* kbase,
+                                          size_t krow_stride) {
+  for (int i = 0; i < n; ++i) val[i * 128] = rescore_dot64(qrow, kbase + (size_t)id[i * 128] * krow_stride);
+}
 
 // Keep the k best of a row's n > k buffered candidates, in buffer order; the new gate is the k-th
 // best logit (a later key, from a larger block, has to beat it strictly).
@@ -569,16 +600,35 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         ++ncand;
       }
     };
+    // exact ranking (see TcParams::rescore_q): every bf16-operand logit lies within err of the
+    // fp32 logit of the means, err = 2^-7 * |q|_1 * max|k| (each operand rounded to bf16 moves a
+    // product by at most 2^-9 of it; the factor leaves room for the fp32 sums).  A key among the
+    // exact k best then has a bf16 logit at least (bound - 2 err), which is where the gate starts,
+    // and after a compaction a key can enter only with a bf16 logit above (k-th exact - err).
+    const bool exact = topk_on && p.rescore_q != nullptr;
+    const float* qrow = nullptr;
+    const float* kbase = nullptr;
+    size_t kstride = 0;
+    float err = 0.f;
+    if (exact && valid) {
+      qrow = p.rescore_q + ((size_t)(t0 + R) * p.Hkv + g) * 64;
+      kbase = p.rescore_k + (size_t)g * 64;
+      kstride = (size_t)p.Hkv * 64;
+      float n1 = 0.f;
+      for (int i = 0; i < 64; ++i) n1 += fabsf(__ldg(qrow + i));
+      err = 0.0078125f * n1 * __uint_as_float(*p.rescore_kmax) + 1e-30f;
+    }
     auto topk_compact = [&]() {
       if (ncand > p.topk_k) {
+        if (exact && valid) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
         const KeepBest kb = topk_keep_best(cval, cid, ncand, p.topk_k);
         ncand = kb.n;
-        thr = kb.thr;
+        thr = exact ? kb.thr - err : kb.thr;
       }
     };
     if (topk_on && p.topk_thr != nullptr && valid) {
       const float b = p.topk_thr[(size_t)(t0 + R) * p.Hkv + g];
-      if (b > -INFINITY) thr = nextafterf(b, -INFINITY);
+      if (b > -INFINITY) thr = nextafterf(exact ? b - 2.f * err : b, -INFINITY);
     }
     // forced blocks among compressed-key chunk c (bit j: block 64 c + j); the next chunk's mask
     // is loaded one chunk ahead
@@ -885,8 +935,10 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         for (int i = 0; i < D; ++i) p.obranch[orow * D + i] = 0.f;
       if (p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first] = -INFINITY;
     }
-    if (ok && topk_on && valid)
+    if (ok && topk_on && valid) {
+      if (exact) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
       topk_emit(cval, cid, ncand, p.topk_k, p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k, p.topk_ids);
+    }
     if (ok && cs.total > 0 && wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
       tc_fence_after();
       finalize(prev_br, m, l);
@@ -988,11 +1040,14 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
 // With topk_thr ([n_q][H] fp32 scratch) the top-k pass is preceded by the bound pass, whose
 // per-row lower bound on the k-th logit lets the top-k pass skip almost every candidate.  With
 // topk_ids the key rows are stored in another order (forced_bits then marks rows) and the
-// emitted indices are topk_ids[row].
+// emitted indices are topk_ids[row].  With rescore_q / rescore_k (fp32 pooled queries [n_q][H][64]
+// and keys in the stored row order) and rescore_kmax (the largest |key| as float bits) the top-k
+// is the ranking of the fp32 logits of the means (see TcParams).
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
-                              float* topk_thr, uint32_t* status, cudaStream_t stream, const int32_t* topk_ids) {
+                              float* topk_thr, uint32_t* status, cudaStream_t stream, const int32_t* topk_ids,
+                              const float* rescore_q, const float* rescore_k, const uint32_t* rescore_kmax) {
   if (topk_idx != nullptr && (D != 64 || topk_k < 1 || topk_k > 32 || forced_bits == nullptr))
     return LSRM_ERR_UNSUPPORTED;
   if ((n_q + 255) / 256 > 65535 || n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
@@ -1023,6 +1078,11 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
   p.topk_k = topk_k;
   p.forced_bits = forced_bits;
   p.topk_ids = topk_ids;
+  if (topk_idx != nullptr && rescore_q != nullptr && rescore_k != nullptr && rescore_kmax != nullptr) {
+    p.rescore_q = rescore_q;
+    p.rescore_k = rescore_k;
+    p.rescore_kmax = rescore_kmax;
+  }
   if (D == 32) return launch_tc_d<32>(d, p, q, nullptr, nullptr, kc, vc, kc_rows, stream);
   if (D != 64) return LSRM_ERR_UNSUPPORTED;
   if (topk_idx != nullptr && topk_thr != nullptr) {

@@ -25,7 +25,9 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
                               float* topk_thr, uint32_t* status, cudaStream_t stream,
-                              const int32_t* topk_ids = nullptr);
+                              const int32_t* topk_ids = nullptr, const float* rescore_q = nullptr,
+                              const float* rescore_k = nullptr, const uint32_t* rescore_kmax = nullptr);
+lsrm_status launch_absmax(const float* x, long long n, uint32_t* out, cudaStream_t s);
 lsrm_status launch_pooled_broadcast(const lsrm_nsa_desc& d, const int32_t* off, const float* o_blk,
                                     const float* lse_blk, float* o_cmp, float* lse, cudaStream_t s);
 lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, const void* k, const void* v,
@@ -66,10 +68,16 @@ uint32_t* status_of(void* ws) { return wsp<uint32_t>(ws, 0); }
 
 float tau_of(const lsrm_nsa_desc& d) { return d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim); }
 
+#define LSRM_TRY(x)                         \
+  do {                                      \
+    lsrm_status _s = (x);                   \
+    if (_s != LSRM_OK) return _s;           \
+  } while (0)
+
 // pooled compressed branch over all B block means, per head (and, with idx, the Speed3R routing:
 // top_k blocks by pooled logit outside the forced set); o_blk / lse_blk go to the workspace
 lsrm_status pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, const void* vc, int32_t* idx,
-                       void* ws, cudaStream_t s) {
+                       void* ws, cudaStream_t s, const float* qc32 = nullptr, const float* kc32 = nullptr) {
   const Workspace w = workspace_layout(d);
   uint32_t* bits = wsp<uint32_t>(ws, w.fbits);
   float* o_blk = wsp<float>(ws, w.obranch);
@@ -84,16 +92,15 @@ lsrm_status pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, c
       if (st != LSRM_OK) return st;
     }
   }
+  const bool exact = idx != nullptr && qc32 != nullptr && kc32 != nullptr;
+  if (exact)
+    LSRM_TRY(launch_absmax(kc32, (long long)d.n_blocks * d.n_kv_heads * d.head_dim, wsp<uint32_t>(ws, w.kmax), s));
   return launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc, kc, vc, d.n_blocks, d.n_blocks, nullptr,
                            tau_of(d), o_blk, l_blk, idx, idx ? d.top_k : 0, idx ? bits : nullptr,
-                           idx ? wsp<float>(ws, w.rthr) : nullptr, status_of(ws), s);
+                           idx ? wsp<float>(ws, w.rthr) : nullptr, status_of(ws), s, nullptr,
+                           exact ? qc32 : nullptr, exact ? kc32 : nullptr, exact ? wsp<uint32_t>(ws, w.kmax) : nullptr);
 }
 
-#define LSRM_TRY(x)                         \
-  do {                                      \
-    lsrm_status _s = (x);                   \
-    if (_s != LSRM_OK) return _s;           \
-  } while (0)
 
 }  // namespace
 
@@ -141,14 +148,17 @@ lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, 
                                 (cudaStream_t)stream);
 }
 
-lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc, int32_t* idx,
-                                   void* ws, void* stream) {
+lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc,
+                                   const float* qc32_or_null, const float* kc32_or_null, int32_t* idx, void* ws,
+                                   void* stream) {
   LSRM_TRY(check_desc(desc));
   LSRM_TRY(check_ws(desc, ws));
   if (!desc->pooled_q || qc == nullptr || kc == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
+  if ((qc32_or_null == nullptr) != (kc32_or_null == nullptr)) return LSRM_ERR_INVALID_ARG;
+  if (!aligned(qc32_or_null, 16) || !aligned(kc32_or_null, 16)) return LSRM_ERR_INVALID_ARG;
   // the routing pass is the pooled compressed branch with its top-k; values are not needed, so the
   // keys stand in for them and the branch output stays in the workspace
-  return pooled_cmp(*desc, qc, kc, kc, idx, ws, (cudaStream_t)stream);
+  return pooled_cmp(*desc, qc, kc, kc, idx, ws, (cudaStream_t)stream, qc32_or_null, kc32_or_null);
 }
 
 lsrm_status lsrm_nsa_cmp_attn(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* kc,
@@ -253,16 +263,22 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
     int32_t* block_of_row = wsp<int32_t>(ws, w.kblk);
     uint32_t* bits_part = wsp<uint32_t>(ws, w.fbits_part);
     LSRM_TRY(launch_key_order(d, wsp<uint32_t>(ws, w.fbits), row_of_block, block_of_row, bits_part, s));
-    LSRM_TRY(launch_compress(d, off, q, k, v, nullptr, kc16, nullptr, vc16, wsp<float>(ws, w.qc32), qc16, s,
-                             row_of_block));
-    float* o_blk = wsp<float>(ws, w.obranch);
-    float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
     const bool route = route_mode == LSRM_ROUTE_SCORE;
     if (route && d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
+    // the routing ranks the fp32 logits of the means: their fp32 copies (keys in row order) and
+    // the largest |pooled key| feed the exact ranking of the candidates
+    float* qc32 = wsp<float>(ws, w.qc32);
+    LSRM_TRY(launch_compress(d, off, q, k, v, route ? kc32 : nullptr, kc16, nullptr, vc16, qc32, qc16, s,
+                             row_of_block));
+    uint32_t* kmax = wsp<uint32_t>(ws, w.kmax);
+    if (route) LSRM_TRY(launch_absmax(kc32, (long long)d.n_blocks * d.n_kv_heads * d.head_dim, kmax, s));
+    float* o_blk = wsp<float>(ws, w.obranch);
+    float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
     LSRM_TRY(launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc16, kc16, vc16, d.n_blocks, d.n_blocks,
                                nullptr, tau_of(d), o_blk, l_blk, route ? idx : nullptr, route ? d.top_k : 0,
                                route ? bits_part : nullptr, route ? wsp<float>(ws, w.rthr) : nullptr,
-                               status_of(ws), s, route ? block_of_row : nullptr));
+                               status_of(ws), s, route ? block_of_row : nullptr, route ? qc32 : nullptr,
+                               route ? kc32 : nullptr, route ? kmax : nullptr));
     float* ofrc = wsp<float>(ws, w.ofrc);
     float* lfrc = wsp<float>(ws, w.lfrc);
     const long long cap = (long long)(d.n_forced > 0 ? d.n_forced : 1) * d.max_block_len;

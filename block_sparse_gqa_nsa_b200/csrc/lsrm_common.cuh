@@ -47,6 +47,7 @@ struct Workspace {
   // pooled keys stored non-forced first: row of each block, block of each row, and the forced
   // bitmap over rows
   size_t krow, kblk, fbits_part;
+  size_t kmax;  // largest |pooled key| (float bits), the width of the exact-ranking gate
   size_t total;
 };
 
@@ -112,6 +113,7 @@ inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   w.krow = o;      o = align256(o + (d.pooled_q ? B * 4 : 0));
   w.kblk = o;      o = align256(o + (d.pooled_q ? B * 4 : 0));
   w.fbits_part = o; o = align256(o + (d.pooled_q ? (B / 32 + 2) * 4 : 0));
+  w.kmax = o;      o = align256(o + (d.pooled_q ? 16 : 0));
   w.total = o;
   return w;
 }

@@ -299,6 +299,40 @@ lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, co
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 
+// Largest |x| over n floats, OR-ed in as float bits (non-negative floats order like their bits):
+// the bound on the pooled keys that sets the width of the exact-ranking gate.  *out must be zero
+// (or a smaller bound) before the launch.
+__global__ void absmax_kernel(const float* __restrict__ x, long long n, uint32_t* out) {
+  float m = 0.f;
+  const float4* x4 = reinterpret_cast<const float4*>(x);
+  const long long n4 = n / 4;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 v = __ldg(x4 + i);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  for (long long i = 4 * n4 + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wm[32];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wm[w]);
+    if (!(m <= 3.0e38f)) m = 3.0e38f;  // a NaN or infinite mean: a huge (finite) bound
+    atomicMax(out, __float_as_uint(m));
+  }
+}
+
+lsrm_status launch_absmax(const float* x, long long n, uint32_t* out, cudaStream_t s) {
+  if (cudaMemsetAsync(out, 0, sizeof(uint32_t), s) != cudaSuccess) return LSRM_ERR_CUDA;
+  if (n <= 0) return LSRM_OK;
+  const long long want = (n / 4 + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 8 ? (want > 0 ? want : 1) : 148 * 8);
+  absmax_kernel<<<blocks, 256, 0, s>>>(x, n, out);
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
 // Row order of the pooled keys for the routing passes: non-forced blocks first, in block order,
 // then the forced blocks in block order (a stable partition, so among candidates row order is
 // block order and ties still go to the lower block id).  One CTA: per-word forced counts, their

@@ -78,7 +78,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsrm_route_score_topk": ([D, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_route_geometric": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_route_geometric_noalloc": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
-        "lsrm_route_pooled_topk": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
+        "lsrm_route_pooled_topk": ([D, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_cmp_attn": ([D, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_select_attn": ([D, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_window_attn": ([D, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
@@ -180,9 +180,13 @@ def lsrm_route_geometric_noalloc(desc, off, coords, idx, status=None, stream=Non
           _stream(stream))
 
 
-def lsrm_route_pooled_topk(desc, qc, kc, idx, ws, stream=None):
+def lsrm_route_pooled_topk(desc, qc, kc, idx, ws, stream=None, qc32=None, kc32=None):
+    """Speed3R routing from the bf16 pooled tensors; with the fp32 means qc32 / kc32 the ranking is
+    that of the fp32 means (the exact mode)."""
     _check(qc, torch.bfloat16, "qc"); _check(kc, torch.bfloat16, "kc"); _check(idx, torch.int32, "idx")
-    _call("lsrm_route_pooled_topk", ctypes.byref(desc), _ptr(qc), _ptr(kc), _ptr(idx), _ptr(ws), _stream(stream))
+    _check(qc32, torch.float32, "qc32"); _check(kc32, torch.float32, "kc32")
+    _call("lsrm_route_pooled_topk", ctypes.byref(desc), _ptr(qc), _ptr(kc), _ptr(qc32), _ptr(kc32), _ptr(idx),
+          _ptr(ws), _stream(stream))
 
 
 def lsrm_nsa_cmp_attn(desc, off, q, kc, vc, o_cmp, lse=None, ws=None, stream=None):

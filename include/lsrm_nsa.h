@@ -143,9 +143,15 @@ LSRM_API lsrm_status lsrm_route_geometric_noalloc(const lsrm_nsa_desc* desc, con
 
 /* Speed3R routing (Speed3R page 2.1 selection branch, 2.2 forced frame-0 and
  * camera blocks): per block a and head h, the top_k blocks j outside the forced
- * set by (tau * qc[a,h] . kc[j,h] desc, j asc), computed from the bf16 pooled
- * tensors with fp32 accumulation.  idx is int32 [B][Hq][top_k]. */
-LSRM_API lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc, int32_t* idx,
+ * set by (tau * qc[a,h] . kc[j,h] desc, j asc).  qc / kc are the bf16 pooled
+ * tensors [B][H][d] the tensor cores score with.  With qc32_or_null and
+ * kc32_or_null (both or neither; fp32 [B][H][64], 16-byte aligned) the ranking is
+ * that of the fp32 pooled means themselves: candidates are gathered from the bf16
+ * logits with a gate widened by a bound on their error (2^-7 |qc32|_1 max|kc32|)
+ * and ranked by fp32 dot products of the means; without them it is the ranking of
+ * the bf16 operands, products accumulated in fp32.  idx is int32 [B][Hq][top_k]. */
+LSRM_API lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc,
+                                   const float* qc32_or_null, const float* kc32_or_null, int32_t* idx,
                                    void* ws, void* stream);
 
 /* S3 compressed branch (LSRM page, k^cmp/v^cmp give the global coarse context;
@@ -194,7 +200,8 @@ LSRM_API lsrm_status lsrm_nsa_attend(const lsrm_nsa_desc* desc, const int32_t* o
  * required) writes [B][top_k]; LSRM_ROUTE_ALL needs top_k == B and selects every
  * block (idx_inout may be NULL).  With a NULL idx_inout the indices live in the
  * workspace.  For pooled_q the routing is the Speed3R rule and idx_inout is
- * [B][Hq][top_k].
+ * [B][Hq][top_k], ranked by the fp32 logits of the pooled means (as
+ * lsrm_route_pooled_topk with fp32 inputs).
  * lse_or_null receives fp32 [N][Hq][n_gates] per-branch LSE (needed by the
  * backward).  obr_or_null (device, 16-byte aligned, caller-owned) receives the
  * normalised per-branch outputs o_b as bf16 [N][Hq][n_gates][d], the

@@ -299,18 +299,16 @@ def test_fused_forward_dense_equals_dense_gqa_sampled():
 # S9 Speed3R pooled-query variant
 # ------------------------------------------------------------------------------------------------
 
-def check_pooled_routing(gpu_idx, w, qblocks, k, operands_bf16=False):
-    """Validity of Speed3R routing: k distinct, non-forced blocks, each with an oracle pooled logit
-    within 1e-3 of the k-th best; where the oracle gap exceeds 1e-3 the sets must agree.
-    With operands_bf16 the oracle ranks with the pooled Q and K rounded to bf16, the precision the
-    kernel's MMA operands have (the top-k is an integer decision taken from those products)."""
+def check_pooled_routing(gpu_idx, w, qblocks, k, qc=None, kc=None):
+    """Validity of Speed3R routing against the oracle's fp64 pooled logits: k distinct, non-forced
+    blocks, each with an oracle logit within 1e-3 of the k-th best; where the oracle gap exceeds
+    1e-3 the sets must agree.  qc / kc default to the oracle's fp64 block means; a test of the
+    bf16-operand mode passes the bf16 operands it gave the kernel."""
     D = oracle_desc(w, top_k=k)
-    qc = O.compress(D, w.off, w.q, w.n_q_heads)
-    kc = O.compress(D, w.off, w.k, w.n_kv_heads)
-    if operands_bf16:
-        from workloads.nsa_workloads import bf16_bits_to_f32
-        qc = bf16_bits_to_f32(f32_to_bf16_bits(qc.astype(np.float32))).astype(np.float64)
-        kc = bf16_bits_to_f32(f32_to_bf16_bits(kc.astype(np.float32))).astype(np.float64)
+    if qc is None:
+        qc = O.compress(D, w.off, w.q, w.n_q_heads)
+    if kc is None:
+        kc = O.compress(D, w.off, w.k, w.n_kv_heads)
     _, logits = O.route_pooled(D, qc, kc, w.forced, qblocks=qblocks, want_logits=True)
     forced = set(w.forced.tolist())
     for i, a in enumerate(qblocks):
@@ -356,8 +354,15 @@ def test_speed3r_pooled_routing_and_compressed_branch_calls():
     B, H, d = w.n_blocks, w.n_q_heads, w.head_dim
     qc, kc, vc = (c.empty(B, H, d, dtype=torch.bfloat16) for _ in range(3))
     nsa.lsrm_nsa_compress(c.desc, c.off, c.q, c.k, c.v, None, kc, None, vc, None, qc, ws=c.ws)
+    qc32, kc32 = c.empty(B, H, d), c.empty(B, H, d)
+    nsa.lsrm_nsa_compress(c.desc, c.off, c.q, c.k, c.v, kc32, kc, None, vc, qc32, qc, ws=c.ws)
     idx = c.empty(B, H, w.top_k, dtype=torch.int32)
+    # bf16-operand mode: the ranking of the operands given
     nsa.lsrm_route_pooled_topk(c.desc, qc, kc, idx, c.ws)
+    check_pooled_routing(to_np(idx), w, np.arange(B, dtype=np.int32), w.top_k, qc=to_np(qc).astype(np.float64),
+                         kc=to_np(kc).astype(np.float64))
+    # exact mode: the ranking of the means
+    nsa.lsrm_route_pooled_topk(c.desc, qc, kc, idx, c.ws, qc32=qc32, kc32=kc32)
     check_pooled_routing(to_np(idx), w, np.arange(B, dtype=np.int32), w.top_k)
     o, lse = c.empty(w.n_tokens, H, d), c.empty(w.n_tokens, H)
     nsa.lsrm_nsa_cmp_attn(c.desc, c.off, qc, kc, vc, o, lse, c.ws)
@@ -572,9 +577,10 @@ def test_speed3r_routing_with_a_late_dominant_block():
     for row in gidx.reshape(-1, w.top_k):
         assert len(set(row.tolist())) == w.top_k  # distinct: no candidate offered twice
     qb = np.arange(w.n_blocks, dtype=np.int32)
-    # the dominant block's logits are ~400x the others': bf16 rounding of the pooled queries moves
-    # them by more than the 1e-3 gap rule, so the ranking is checked at the operands' precision
-    check_pooled_routing(gidx, w, qb, w.top_k, operands_bf16=True)
+    # the dominant block's logits are ~400x the others' (bf16 rounding of the pooled queries alone
+    # would move them by more than the 1e-3 gap): the forward ranks the fp32 means, so the plain
+    # gap rule against the fp64 oracle holds
+    check_pooled_routing(gidx, w, qb, w.top_k)
     ref = O.forward(oracle_desc(w), w.off, w.q, w.k, w.v, w.gates, gidx, forced=w.forced)
     assert_close(to_np(out), ref, "out")
 
@@ -603,7 +609,7 @@ def test_speed3r_routing_ties_break_by_block_id():
     gidx = to_np(idx)
     D = oracle_desc(w)
     from workloads.nsa_workloads import bf16_bits_to_f32
-    qc = bf16_bits_to_f32(f32_to_bf16_bits(O.compress(D, w.off, w.q, w.n_q_heads).astype(np.float32)))
+    qc = O.compress(D, w.off, w.q, w.n_q_heads)  # the forward ranks the means themselves
     uf = bf16_bits_to_f32(u).astype(np.float64)
     even = [b for b in range(0, w.n_blocks, 2) if b not in forced]
     odd = [b for b in range(1, w.n_blocks, 2) if b not in forced]
