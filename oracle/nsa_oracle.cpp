@@ -554,15 +554,181 @@ int impl_backward(const Desc* D, const int32_t* off, const T* q, const T* k, con
   return 0;
 }
 
+// ---- S9 backward: the Speed3R pooled-query layer (pooled_q = 1, MHA, gates (cmp, slc)) with the
+// routing indices fixed (Speed3R page, 2.1: compression, selection and gated aggregation; the
+// model trains end to end, so the gradient flows through all of them).  Chain rule:
+//   compressed: every token t of block a receives o_blk(a), the softmax attention of the
+//     block-mean query Qbar_a = (1/n_a) sum_{t in a} q_t over all block means, so its upstream
+//     gradient is Gbar_a = sum_{t in a} g_cmp[t] dO[t];
+//     dS_j = P_j (Gbar_a . Vbar_j - Gbar_a . o_blk(a)),
+//     dQbar_a = tau sum_j dS_j Kbar_j,  dKbar_j += tau dS_j Qbar_a,  dVbar_j += P_j Gbar_a,
+//     and each token t of a receives dQbar_a / n_a;
+//   selected: per token as in the LSRM layer, over the tokens of (forced U routed) blocks;
+//   dgates[t,h,0] = <dO[t], o_blk(a)>, dgates[t,h,1] = <dO[t], o_slc(t)>;
+//   mean-pool of K and V: every token u of block j receives dKbar_j / n_j and dVbar_j / n_j.
+// idx [B][H][k].  nthreads > 1 splits the query blocks across threads (own accumulators, summed
+// in thread order).
+template <typename T>
+int impl_backward_pooled(const Desc* D, const int32_t* off, const T* q, const T* k, const T* v, const T* gates,
+                         const int32_t* idx, int32_t n_forced, const int32_t* forced, const T* dout, double* dq,
+                         double* dk, double* dv, double* dgates, int32_t nthreads) {
+  const int32_t B = D->n_blocks, H = D->n_q_heads, d = D->head_dim, NG = D->n_gates, K = D->top_k;
+  if (H != D->n_kv_heads || NG != 2) return 1;
+  const int64_t N = D->n_tokens;
+  const double tau = tau_of(*D);
+  std::vector<double> qc((size_t)B * H * d), kc((size_t)B * H * d), vc((size_t)B * H * d);
+  mean_pool(*D, off, q, H, qc.data());
+  mean_pool(*D, off, k, H, kc.data());
+  mean_pool(*D, off, v, H, vc.data());
+  const std::vector<double> Kw = widen(k, (size_t)(N * H * d)), Vw = widen(v, (size_t)(N * H * d));
+  if (nthreads < 1) nthreads = 1;
+  const size_t kv_sz = (size_t)(N * H * d), kvc_sz = (size_t)B * H * d;
+  std::vector<std::vector<double>> dK(nthreads, std::vector<double>(kv_sz, 0.0)),
+      dV(nthreads, std::vector<double>(kv_sz, 0.0)), dKc(nthreads, std::vector<double>(kvc_sz, 0.0)),
+      dVc(nthreads, std::vector<double>(kvc_sz, 0.0));
+  auto work = [&](int tid) {
+    std::vector<double> qv((size_t)d), go((size_t)d), ob((size_t)d), dqv((size_t)d), gbar((size_t)d);
+    std::vector<double> s, p;
+    for (int32_t a = tid; a < B; a += nthreads) {
+      const int64_t n_a = (int64_t)off[a + 1] - off[a];
+      for (int32_t h = 0; h < H; ++h) {
+        // ---- compressed branch of block a, head h (pooled query)
+        const double* qbar = &qc[((size_t)a * H + h) * d];
+        s.assign((size_t)B, 0.0);
+        double m = -INFINITY;
+        for (int32_t j = 0; j < B; ++j) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += qbar[c] * kc[((size_t)j * H + h) * d + c];
+          s[(size_t)j] = tau * acc;
+          m = std::max(m, s[(size_t)j]);
+        }
+        double l = 0.0;
+        for (int32_t j = 0; j < B; ++j) { s[(size_t)j] = std::exp(s[(size_t)j] - m); l += s[(size_t)j]; }
+        for (int c = 0; c < d; ++c) { ob[(size_t)c] = 0.0; gbar[(size_t)c] = 0.0; }
+        for (int32_t j = 0; j < B; ++j)
+          for (int c = 0; c < d; ++c) ob[(size_t)c] += s[(size_t)j] / l * vc[((size_t)j * H + h) * d + c];
+        for (int64_t t = off[a]; t < off[a + 1]; ++t) {
+          const double gc = bf(gates[(t * H + h) * NG + 0]);
+          double dg = 0.0;
+          for (int c = 0; c < d; ++c) {
+            const double g_out = bf(dout[(t * H + h) * d + c]);
+            dg += g_out * ob[(size_t)c];
+            gbar[(size_t)c] += gc * g_out;
+          }
+          dgates[(t * H + h) * NG + 0] = dg;
+        }
+        double Dt = 0.0;
+        for (int c = 0; c < d; ++c) Dt += gbar[(size_t)c] * ob[(size_t)c];
+        std::vector<double> dqbar((size_t)d, 0.0);
+        for (int32_t j = 0; j < B; ++j) {
+          const double pj = s[(size_t)j] / l;
+          double dp = 0.0;
+          for (int c = 0; c < d; ++c) dp += gbar[(size_t)c] * vc[((size_t)j * H + h) * d + c];
+          const double ds = pj * (dp - Dt);
+          double* dkr = &dKc[(size_t)tid][((size_t)j * H + h) * d];
+          double* dvr = &dVc[(size_t)tid][((size_t)j * H + h) * d];
+          for (int c = 0; c < d; ++c) {
+            dqbar[(size_t)c] += tau * ds * kc[((size_t)j * H + h) * d + c];
+            dkr[c] += tau * ds * qbar[c];
+            dvr[c] += pj * gbar[(size_t)c];
+          }
+        }
+        // ---- selected branch of every token of a, head h: forced U routed blocks
+        std::vector<int64_t> sel;
+        for (int32_t j : selected_blocks(*D, idx + ((int64_t)a * H + h) * K, n_forced, forced))
+          for (int64_t u = off[j]; u < off[j + 1]; ++u) sel.push_back(u);
+        const size_t n = sel.size();
+        for (int64_t t = off[a]; t < off[a + 1]; ++t) {
+          for (int c = 0; c < d; ++c) {
+            qv[(size_t)c] = bf(q[(t * H + h) * d + c]);
+            dqv[(size_t)c] = dqbar[(size_t)c] / (double)n_a;
+          }
+          if (n == 0) {
+            dgates[(t * H + h) * NG + 1] = 0.0;
+          } else {
+            s.assign(n, 0.0);
+            double ms = -INFINITY;
+            for (size_t u = 0; u < n; ++u) {
+              double acc = 0.0;
+              for (int c = 0; c < d; ++c) acc += qv[(size_t)c] * Kw[(size_t)((sel[u] * H + h) * d + c)];
+              s[u] = tau * acc;
+              ms = std::max(ms, s[u]);
+            }
+            double ls = 0.0;
+            for (size_t u = 0; u < n; ++u) { s[u] = std::exp(s[u] - ms); ls += s[u]; }
+            p.assign(n, 0.0);
+            for (int c = 0; c < d; ++c) ob[(size_t)c] = 0.0;
+            for (size_t u = 0; u < n; ++u) {
+              p[u] = s[u] / ls;
+              for (int c = 0; c < d; ++c) ob[(size_t)c] += p[u] * Vw[(size_t)((sel[u] * H + h) * d + c)];
+            }
+            const double gb = bf(gates[(t * H + h) * NG + 1]);
+            double dg = 0.0, Ds = 0.0;
+            for (int c = 0; c < d; ++c) {
+              const double g_out = bf(dout[(t * H + h) * d + c]);
+              dg += g_out * ob[(size_t)c];
+              go[(size_t)c] = gb * g_out;
+              Ds += go[(size_t)c] * ob[(size_t)c];
+            }
+            dgates[(t * H + h) * NG + 1] = dg;
+            for (size_t u = 0; u < n; ++u) {
+              const double* ku = &Kw[(size_t)((sel[u] * H + h) * d)];
+              const double* vu = &Vw[(size_t)((sel[u] * H + h) * d)];
+              double dp = 0.0;
+              for (int c = 0; c < d; ++c) dp += go[(size_t)c] * vu[c];
+              const double ds = p[u] * (dp - Ds);
+              double* dkr = &dK[(size_t)tid][(size_t)((sel[u] * H + h) * d)];
+              double* dvr = &dV[(size_t)tid][(size_t)((sel[u] * H + h) * d)];
+              for (int c = 0; c < d; ++c) {
+                dqv[(size_t)c] += tau * ds * ku[c];
+                dkr[c] += tau * ds * qv[(size_t)c];
+                dvr[c] += p[u] * go[(size_t)c];
+              }
+            }
+          }
+          for (int c = 0; c < d; ++c) dq[(t * H + h) * d + c] = dqv[(size_t)c];
+        }
+      }
+    }
+  };
+  if (nthreads == 1) work(0);
+  else {
+    std::vector<std::thread> th;
+    for (int i = 0; i < nthreads; ++i) th.emplace_back(work, i);
+    for (auto& x : th) x.join();
+  }
+  for (size_t i = 0; i < kv_sz; ++i) { dk[i] = 0.0; dv[i] = 0.0; }
+  for (int tid = 0; tid < nthreads; ++tid)
+    for (size_t i = 0; i < kv_sz; ++i) { dk[i] += dK[(size_t)tid][i]; dv[i] += dV[(size_t)tid][i]; }
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t n = (int64_t)off[b + 1] - off[b];
+    for (int32_t h = 0; h < H; ++h)
+      for (int c = 0; c < d; ++c) {
+        double gk = 0.0, gv = 0.0;
+        for (int tid = 0; tid < nthreads; ++tid) {
+          gk += dKc[(size_t)tid][((size_t)b * H + h) * d + c];
+          gv += dVc[(size_t)tid][((size_t)b * H + h) * d + c];
+        }
+        for (int64_t u = off[b]; u < off[b + 1]; ++u) {
+          dk[(u * H + h) * d + c] += gk / (double)n;
+          dv[(u * H + h) * d + c] += gv / (double)n;
+        }
+      }
+  }
+  return 0;
+}
+
 // ---- a scalar loss L = sum O * dO for the listed blocks (finite-difference checks of the backward)
 template <typename T>
 double impl_loss(const Desc* D, const int32_t* off, const T* q, const T* k, const T* v,
-                   const T* gates, const int32_t* idx, int32_t idx_heads, const T* dout) {
+                   const T* gates, const int32_t* idx, int32_t idx_heads, const T* dout, int32_t n_forced = 0,
+                   const int32_t* forced = nullptr) {
   const int32_t B = D->n_blocks, Hq = D->n_q_heads, d = D->head_dim;
   std::vector<int32_t> all((size_t)B);
   for (int32_t b = 0; b < B; ++b) all[(size_t)b] = b;
   std::vector<double> out((size_t)(D->n_tokens * Hq * d));
-  impl_forward<T>(D, off, q, k, v, gates, idx, idx_heads, 0, nullptr, B, all.data(), out.data(), nullptr, nullptr);
+  impl_forward<T>(D, off, q, k, v, gates, idx, idx_heads, n_forced, forced, B, all.data(), out.data(), nullptr,
+                  nullptr);
   double L = 0.0;
   for (size_t i = 0; i < out.size(); ++i) L += out[i] * bf(dout[i]);
   return L;
@@ -639,6 +805,25 @@ int oracle_backward_f64(const Desc* D, const int32_t* off, const double* q, cons
 double oracle_loss_f64(const Desc* D, const int32_t* off, const double* q, const double* k, const double* v,
                        const double* gates, const int32_t* idx, int32_t idx_heads, const double* dout) {
   return impl_loss<double>(D, off, q, k, v, gates, idx, idx_heads, dout);
+}
+double oracle_loss_forced_f64(const Desc* D, const int32_t* off, const double* q, const double* k, const double* v,
+                              const double* gates, const int32_t* idx, int32_t idx_heads, const double* dout,
+                              int32_t n_forced, const int32_t* forced) {
+  return impl_loss<double>(D, off, q, k, v, gates, idx, idx_heads, dout, n_forced, forced);
+}
+int oracle_backward_pooled(const Desc* D, const int32_t* off, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const uint16_t* gates, const int32_t* idx, int32_t n_forced,
+                           const int32_t* forced, const uint16_t* dout, double* dq, double* dk, double* dv,
+                           double* dgates, int32_t nthreads) {
+  return impl_backward_pooled<uint16_t>(D, off, q, k, v, gates, idx, n_forced, forced, dout, dq, dk, dv, dgates,
+                                        nthreads);
+}
+int oracle_backward_pooled_f64(const Desc* D, const int32_t* off, const double* q, const double* k,
+                               const double* v, const double* gates, const int32_t* idx, int32_t n_forced,
+                               const int32_t* forced, const double* dout, double* dq, double* dk, double* dv,
+                               double* dgates, int32_t nthreads) {
+  return impl_backward_pooled<double>(D, off, q, k, v, gates, idx, n_forced, forced, dout, dq, dk, dv, dgates,
+                                      nthreads);
 }
 
 }  // extern "C"

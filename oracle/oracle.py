@@ -22,7 +22,7 @@ _LIB = os.path.join(_HERE, "liboracle_nsa.so")
 
 __all__ = ["build_oracle", "OracleDesc", "desc_for", "compress", "route_geometric", "route_score",
            "route_pooled", "cmp_attn", "select_attn", "window_attn", "forward", "backward", "loss_f64",
-           "forward_f64", "backward_f64", "rows_of"]
+           "forward_f64", "backward_f64", "backward_pooled", "backward_pooled_f64", "loss_forced_f64", "rows_of"]
 
 
 class OracleDesc(ctypes.Structure):
@@ -65,11 +65,14 @@ def _L():
             "oracle_backward": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, vp, i32],
             "oracle_backward_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, vp, i32],
             "oracle_loss_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp],
+            "oracle_loss_forced_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp, i32, vp],
+            "oracle_backward_pooled": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, i32],
+            "oracle_backward_pooled_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, i32],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
             f.argtypes = args
-            f.restype = ctypes.c_double if name == "oracle_loss_f64" else ctypes.c_int
+            f.restype = ctypes.c_double if name.startswith("oracle_loss") else ctypes.c_int
         _lib = lib
     return _lib
 
@@ -249,3 +252,43 @@ def loss_f64(D, off, q, k, v, gates, idx, dout) -> float:
 
 def default_scale(head_dim: int) -> float:
     return 1.0 / math.sqrt(head_dim)
+
+
+def _backward_pooled(fn, dtype, D, off, q, k, v, gates, idx, forced, dout, nthreads):
+    off = _c(off, np.int32)
+    q, k, v, gates, dout = _inputs(dtype, q, k, v, gates, dout)
+    idx = _c(idx, np.int32)
+    forced = np.zeros(0, np.int32) if forced is None else _c(forced, np.int32)
+    N = D.n_tokens
+    dq = np.zeros((N, D.n_q_heads, D.head_dim))
+    dk = np.zeros((N, D.n_kv_heads, D.head_dim))
+    dv = np.zeros((N, D.n_kv_heads, D.head_dim))
+    dg = np.zeros((N, D.n_q_heads, D.n_gates))
+    rc = fn(ctypes.byref(D), _p(off), _p(q), _p(k), _p(v), _p(gates), _p(idx), len(forced), _p(forced), _p(dout),
+            _p(dq), _p(dk), _p(dv), _p(dg), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle pooled backward: unsupported configuration")
+    return dq, dk, dv, dg
+
+
+def backward_pooled(D, off, q, k, v, gates, idx, forced, dout, nthreads=1):
+    """(dq, dk, dv, dgates) of L = sum(O * dO) for the Speed3R pooled-query layer (MHA, gates
+    (cmp, slc)); idx [B][H][k] routing indices fixed, forced blocks joined to every selected set."""
+    return _backward_pooled(_L().oracle_backward_pooled, np.uint16, D, off, q, k, v, gates, idx, forced, dout,
+                            nthreads)
+
+
+def backward_pooled_f64(D, off, q, k, v, gates, idx, forced, dout, nthreads=1):
+    return _backward_pooled(_L().oracle_backward_pooled_f64, np.float64, D, off, q, k, v, gates, idx, forced, dout,
+                            nthreads)
+
+
+def loss_forced_f64(D, off, q, k, v, gates, idx, dout, forced) -> float:
+    """L = sum(O * dO) with forced blocks joined to every selected set (pooled-query layer)."""
+    off = _c(off, np.int32)
+    q, k, v, gates, dout = _inputs(np.float64, q, k, v, gates, dout)
+    idx = _c(idx, np.int32)
+    idx_heads = 1 if idx.ndim == 2 else idx.shape[1]
+    forced = _c(forced, np.int32)
+    return float(_L().oracle_loss_forced_f64(ctypes.byref(D), _p(off), _p(q), _p(k), _p(v), _p(gates), _p(idx),
+                                             idx_heads, _p(dout), len(forced), _p(forced)))
