@@ -52,9 +52,10 @@ def parse():
                          "10-20 s of one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r"],
+    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r", "bandwidth"],
                     help="sparse: the layer forward (the default line); backward: its gradients; dense: the "
-                         "dense-stage shape with every block selected; speed3r: the pooled-query variant")
+                         "dense-stage shape with every block selected; speed3r: the pooled-query variant; "
+                         "bandwidth: achieved HBM GB/s of the memory-bound kernels (pooling, routing, combine)")
     ap.add_argument("--record-traffic", nargs=4, metavar=("WHICH", "CSV", "KERNEL_REGEX", "LAUNCHES"),
                     help="write profiles/traffic.json[WHICH] from an ncu raw CSV export and exit")
     ap.add_argument("--frames", type=int, default=512,
@@ -865,8 +866,95 @@ def run_extra_reference(args, metric, workload):
     return 0
 
 
+# ------------------------------------------------------------------------------------------------
+# the memory-bound kernels on their own: achieved HBM bandwidth against the measured copy peak
+# ------------------------------------------------------------------------------------------------
+
+def run_bandwidth(args):
+    """Block mean-pool of Q, K and V (Speed3R shape, --frames frames), the standalone gated combine
+    of two fp32 branch outputs (same shape) and the geometric routing of the sparse stage, each
+    timed alone with CUDA events (mean of --steps launches after --warmup); algorithmic bytes =
+    every input byte read once plus every output byte written once."""
+    import torch
+    from block_sparse_gqa_nsa_b200 import nsa
+    from block_sparse_gqa_nsa_b200.build import build
+    from workloads import make_workload
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    if args.impl == "reference":
+        print(json.dumps({"impl": "reference", "unavailable": "the bandwidth workload times single kernels; "
+                          "the oracle has no counterpart of a kernel's memory traffic"}))
+        return 0
+    build()
+    nsa.load_library()
+    dev = torch.device("cuda", 0)
+    peaks, src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    res = {}
+    w = make_workload("speed3r_small", seed=args.seed, n_frames=args.frames)
+    N, B, H, d = w.n_tokens, w.n_blocks, w.n_q_heads, w.head_dim
+    q, k, v, g = bf(w.q), bf(w.k), bf(w.v), bf(w.gates)
+    off = torch.from_numpy(w.off.astype(np.int32)).to(dev)
+    desc = nsa.make_desc(N, B, w.max_block_len, H, H, d, w.top_k, 0, 0.0, True, 2)
+    ws = nsa.workspace(desc, dev)
+    outs = {n: torch.empty(B, H, d, dtype=dt, device=dev) for n, dt in
+            (("kc32", torch.float32), ("kc", torch.bfloat16), ("vc32", torch.float32), ("vc", torch.bfloat16),
+             ("qc32", torch.float32), ("qc", torch.bfloat16))}
+    ms = timed(lambda: nsa.lsrm_nsa_compress(desc, off, q, k, v, outs["kc32"], outs["kc"], outs["vc32"], outs["vc"],
+                                             outs["qc32"], outs["qc"], ws))
+    byt = 3 * N * H * d * 2 + 3 * B * H * d * 6 + (B + 1) * 4
+    res["compress_kernel"] = {"what": f"mean-pool of q, k, v over {B} blocks ({N} tokens, {H}x{d})",
+                              "ms": ms, "bytes": byt}
+    oc = torch.randn(N, H, d, device=dev)
+    osl = torch.randn(N, H, d, device=dev)
+    out = torch.empty(N, H, d, dtype=torch.bfloat16, device=dev)
+    ms = timed(lambda: nsa.lsrm_nsa_gate_combine(desc, oc, osl, None, g, out))
+    byt = 2 * N * H * d * 4 + N * H * 2 * 2 + N * H * d * 2
+    res["gate_combine_kernel"] = {"what": f"out = g_cmp o_cmp + g_slc o_slc, {N} tokens x {H}x{d} fp32 in, bf16 out",
+                                  "ms": ms, "bytes": byt}
+    del q, k, v, oc, osl, out, outs, ws
+    ws_ = make_workload("sparse", seed=args.seed)
+    offs = torch.from_numpy(ws_.off.astype(np.int32)).to(dev)
+    coords = torch.from_numpy(ws_.coords.astype(np.int32)).to(dev)
+    dsc = nsa.make_desc(ws_.n_tokens, ws_.n_blocks, ws_.max_block_len, ws_.n_q_heads, ws_.n_kv_heads, ws_.head_dim,
+                        ws_.top_k, ws_.window, 0.0, False, ws_.n_gates)
+    wsp = nsa.workspace(dsc, dev)
+    idx = torch.empty(ws_.n_blocks, ws_.top_k, dtype=torch.int32, device=dev)
+    ms = timed(lambda: nsa.lsrm_route_geometric(dsc, offs, coords, idx, wsp))
+    byt = ws_.n_tokens * 12 + (ws_.n_blocks + 1) * 4 + ws_.n_blocks * ws_.top_k * 4
+    res["centroid_kernel+geo_topk_reg_kernel"] = {
+        "what": f"geometric routing of the sparse stage ({ws_.n_blocks} blocks, top-{ws_.top_k}); the centroids "
+                f"({ws_.n_blocks * 12} B) stay in L2 for the top-k's {ws_.n_blocks}^2 distances", "ms": ms,
+        "bytes": byt}
+    for r in res.values():
+        r["gbs"] = r["bytes"] / (r["ms"] / 1000.0) / 1e9
+        r["frac"] = r["gbs"] / hbm
+    print(json.dumps({"metric": "achieved HBM GB/s of the memory-bound kernels", "unit": "GB/s",
+                      "peak": hbm, "peak_source": f"{src} hbm_gbs", "steps": args.steps, "warmup": args.warmup,
+                      "frames": args.frames, "kernels": res}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload == "bandwidth":
+        return run_bandwidth(args)
     if args.record_traffic:
         which, csv_path, regex, launches = args.record_traffic
         print(json.dumps(record_traffic(which, csv_path, regex, int(launches), f"from {os.path.basename(csv_path)}")))
