@@ -148,6 +148,7 @@ struct TcParams {
   // pass (bound_pass = 1: scores only, no softmax, no P V) writes it; the top-k pass reads it
   float* topk_thr;
   int bound_pass;
+  int n_pairs;  // 128-row tile pairs per query block (set by the launcher; part of grid x)
   // optional row -> block id map of the keys (the pooled keys may be stored in another order);
   // the emitted top-k are block ids
   const int32_t* topk_ids;
@@ -308,7 +309,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   const uint32_t raw = smem_u32(smem_raw);
   TcSmem<D>& S = *reinterpret_cast<TcSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x, g = blockIdx.y, a = blockIdx.z;
+  // grid: x = query block * pairs + pair (block-major, so a block's tile pairs run side by side
+  // and the query-block count is not bounded by the 65535 limit of grid y / z), y = KV group
+  const int pair = (int)(blockIdx.x % (unsigned)p.n_pairs), g = blockIdx.y, a = (int)(blockIdx.x / (unsigned)p.n_pairs);
   const int t0 = p.uniform_block ? a * p.uniform_block : p.off[a];
   const int n_a = p.uniform_block ? min(p.uniform_block, p.N - t0) : p.off[a + 1] - t0;
   const int rows_total = n_a * p.G;
@@ -987,8 +990,12 @@ lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q
       cudaSuccess)
     return LSRM_ERR_CUDA;
   const int tiles = (d.max_block_len * p.G + 127) / 128;
-  dim3 grid((unsigned)((tiles + 1) / 2), (unsigned)d.n_kv_heads, (unsigned)d.n_blocks);
-  nsa_attn_tc_kernel<D><<<grid, kTcThreads, smem, stream>>>(qm, km, vm, kcm, vcm, p);
+  TcParams pp = p;
+  pp.n_pairs = (tiles + 1) / 2;
+  const long long nx = (long long)d.n_blocks * pp.n_pairs;
+  if (nx > INT32_MAX || d.n_kv_heads > 65535) return LSRM_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)nx, (unsigned)d.n_kv_heads);
+  nsa_attn_tc_kernel<D><<<grid, kTcThreads, smem, stream>>>(qm, km, vm, kcm, vcm, pp);
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 
@@ -1000,7 +1007,7 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
                            int lse_first, uint32_t* status, cudaStream_t stream, void* obr) {
   const int G = d.n_q_heads / d.n_kv_heads;
   if (128 % G != 0) return LSRM_ERR_UNSUPPORTED;
-  if ((!route_all && d.n_forced + d.top_k > kTcMaxSel) || d.n_blocks > 65535) return LSRM_ERR_UNSUPPORTED;
+  if (!route_all && d.n_forced + d.top_k > kTcMaxSel) return LSRM_ERR_UNSUPPORTED;
   TcParams p{};
   p.off = off;
   p.gates = (const uint16_t*)gates;
@@ -1050,7 +1057,7 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
                               const float* rescore_q, const float* rescore_k, const uint32_t* rescore_kmax) {
   if (topk_idx != nullptr && (D != 64 || topk_k < 1 || topk_k > 32 || forced_bits == nullptr))
     return LSRM_ERR_UNSUPPORTED;
-  if ((n_q + 255) / 256 > 65535 || n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
+  if (n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
   lsrm_nsa_desc d{};
   d.n_tokens = n_q;
   d.n_blocks = (int32_t)((n_q + 255) / 256);  // query groups (grid z)

@@ -54,6 +54,7 @@ struct BwdParams {
   uint32_t* status;
   long long N;
   int B, Hq, Hkv, G, NG, top_k, idx_heads, window, n_lists;
+  int q_tiles;  // 128-row tiles per query block in the query pass (part of its grid x)
   float tau, scale_log2;
 };
 
@@ -137,7 +138,8 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   const uint32_t raw = smem_u32(smem_raw);
   BqtSmem<D>& S = *reinterpret_cast<BqtSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, g = blockIdx.y, a = blockIdx.z;
+  // grid: x = query block * tiles + tile (the query-block count is not bounded by grid y / z)
+  const int tile = (int)(blockIdx.x % (unsigned)p.q_tiles), g = blockIdx.y, a = (int)(blockIdx.x / (unsigned)p.q_tiles);
   const int t0 = p.off[a], n_a = p.off[a + 1] - t0;
   const int rows_total = n_a * p.G;
   if (tile * 128 >= rows_total) return;
@@ -959,7 +961,11 @@ static lsrm_status launch_backward_d(const lsrm_nsa_desc& d, const BwdParams& p,
   if (cudaFuncSetAttribute(bwd_query_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
       cudaSuccess)
     return LSRM_ERR_CUDA;
-  bwd_query_tc_kernel<D><<<dim3(tiles, d.n_kv_heads, d.n_blocks), kBqtThreads, sm, s>>>(qm, om, km, vm, kcm, vcm, p);
+  if ((long long)tiles * d.n_blocks > INT32_MAX || d.n_kv_heads > 65535) return LSRM_ERR_UNSUPPORTED;
+  BwdParams pq = p;
+  pq.q_tiles = tiles;
+  bwd_query_tc_kernel<D><<<dim3((unsigned)(tiles * d.n_blocks), d.n_kv_heads, 1), kBqtThreads, sm, s>>>(qm, om, km, vm,
+                                                                                                     kcm, vcm, pq);
   CUtensorMap k64, v64, kc128, vc128, q64, o64;
   if (!make_map(&k64, p.k, D, d.n_kv_heads, d.n_tokens, 1, 64) || !make_map(&v64, p.v, D, d.n_kv_heads, d.n_tokens, 1, 64) ||
       !make_map(&kc128, p.kc, D, d.n_kv_heads, d.n_blocks, 1, 128) ||
@@ -987,7 +993,7 @@ lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const vo
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
                             unsigned char* ws_bwd, uint32_t* status, cudaStream_t s, const void* obr) {
-  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.n_blocks > 65535 || 64 % (d.n_q_heads / d.n_kv_heads) != 0)
+  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || 64 % (d.n_q_heads / d.n_kv_heads) != 0)
     return LSRM_ERR_UNSUPPORTED;
   const BwdWs w = bwd_layout(d, idx_heads);
   BwdParams p{};
