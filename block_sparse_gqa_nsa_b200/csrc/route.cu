@@ -190,11 +190,13 @@ lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, c
 }
 
 // ---- score routing -------------------------------------------------------------------------------
-// One CTA per (query block a, KV group g), fp32 throughout.  Pass 1 gets each row's
-// softmax max and normaliser over all B compressed keys; pass 2 accumulates the
-// probabilities per key (per-warp partials summed in a fixed order).  Scores stay in
-// shared memory; then k rounds of arg-max by (score desc, j asc).
-constexpr int kScoreChunk = 128;  // compressed keys staged per step
+// One CTA per (query block a, KV group g), fp32 throughout, one thread per query row (the row's q
+// in registers; the compressed keys staged in shared memory in chunks of kScoreChunk and read
+// as broadcasts).  Pass 1 forms each row's softmax max and normaliser over all B compressed keys
+// (log2 units); pass 2 forms the probabilities chunk by chunk, each thread summing them over its
+// rows, and the per-thread partial sums are added in a fixed order (threads in index order), so
+// the scores are reproducible bit for bit.  Then k rounds of arg-max by (score desc, j asc).
+constexpr int kScoreChunk = 32;  // compressed keys per chunk (one register per key per thread)
 constexpr int kMaxScoreRows = 64 * 64;
 
 template <int D>
@@ -203,10 +205,9 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
                    int32_t B, int32_t Hq, int32_t Hkv, int32_t k, float scale, int32_t* __restrict__ idx,
                    float* __restrict__ score_out, uint32_t* status) {
   extern __shared__ float smem[];
-  float* s_k = smem;                                   // [kScoreChunk][D + 1]
-  float* s_part = s_k + kScoreChunk * (D + 1);         // [8 warps][kScoreChunk]
-  float* s_score = s_part + 8 * kScoreChunk;           // [B]
-  float2* s_ml = reinterpret_cast<float2*>(s_score + ((B + 1) & ~1));  // [rows] (max, 1/sum)
+  float* s_k = smem;                                   // [kScoreChunk][D] compressed keys of the chunk
+  float* s_part = s_k + kScoreChunk * D;               // [kRouteThreads][kScoreChunk + 1] partial sums
+  float* s_score = s_part + kRouteThreads * (kScoreChunk + 1);  // [B]
   __shared__ float s_bv[kRouteThreads / 32];
   __shared__ int s_bj[kRouteThreads / 32];
   __shared__ float s_lv;
@@ -215,7 +216,7 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
   const int G = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = off[a];
-  // a block longer than the descriptor allows would overrun the row table: flag it and clip
+  // a block longer than the descriptor allows: flag it and clip
   int rows = (off[a + 1] - t0) * G;
   if (rows > kMaxScoreRows) {
     if (tid == 0) raise_status(status, LSRM_ERR_BOUNDS);
@@ -223,98 +224,99 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
   }
   const float sl2 = scale * 1.4426950408889634f;  // logits in log2 units
   const int nchunks = (B + kScoreChunk - 1) / kScoreChunk;
-  constexpr int KPL = kScoreChunk / 32;  // keys per lane per chunk
+  constexpr int kRowsPerThread = kMaxScoreRows / kRouteThreads;
 
   auto load_chunk = [&](int c) {
     __syncthreads();
     for (int e = tid; e < kScoreChunk * D; e += kRouteThreads) {
       const int kk = e / D, col = e % D;
       const int j = c * kScoreChunk + kk;
-      s_k[kk * (D + 1) + col] = j < B ? kc32[((size_t)j * Hkv + g) * D + col] : 0.0f;
+      s_k[e] = j < B ? kc32[((size_t)j * Hkv + g) * D + col] : 0.0f;
     }
     __syncthreads();
   };
   auto load_q = [&](int r, float* qv) {
     const int t = t0 + r / G, h = g * G + r % G;
-    const uint16_t* src = q + ((size_t)t * Hq + h) * D;
+    const uint4* src = reinterpret_cast<const uint4*>(q + ((size_t)t * Hq + h) * D);
 #pragma unroll
-    for (int c = 0; c < D; ++c) qv[c] = bf16_to_f32(__ldg(src + c));
-  };
-
-  // pass 1: per-row running max / sum (lane-local over its keys, merged at the end)
-  for (int r0 = 0; r0 < rows; r0 += 8 * 8) {
-    float m[8], l[8];
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 u = __ldg(src + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { m[i] = -INFINITY; l[i] = 0.0f; }
-    for (int c = 0; c < nchunks; ++c) {
-      load_chunk(c);
-#pragma unroll 1
-      for (int i = 0; i < 8; ++i) {
-        const int r = r0 + warp * 8 + i;
-        if (r >= rows) break;
-        float qv[D];
-        load_q(r, qv);
-#pragma unroll
-        for (int e = 0; e < KPL; ++e) {
-          const int kk = lane + 32 * e;
-          const int j = c * kScoreChunk + kk;
-          if (j >= B) continue;
-          float s = 0.0f;
-#pragma unroll
-          for (int cc = 0; cc < D; ++cc) s = fmaf(qv[cc], s_k[kk * (D + 1) + cc], s);
-          s *= sl2;
-          if (s > m[i]) { l[i] = l[i] * exp2f(m[i] - s) + 1.0f; m[i] = s; }
-          else l[i] += exp2f(s - m[i]);
-        }
+      for (int e = 0; e < 4; ++e) {
+        qv[8 * c + 2 * e] = __uint_as_float(w[e] << 16);
+        qv[8 * c + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
       }
     }
+  };
+  // raw logits of one row against the chunk's keys (keys past B give -inf)
+  auto chunk_logits = [&](const float* qv, int c, float* sv) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + warp * 8 + i;
-      float mi = m[i], li = l[i];
+    for (int kk = 0; kk < kScoreChunk; ++kk) {
+      float s = 0.0f;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float mo = __shfl_xor_sync(0xffffffffu, mi, o), lo = __shfl_xor_sync(0xffffffffu, li, o);
-        const float mn = fmaxf(mi, mo);
-        li = (mi == -INFINITY ? 0.0f : li * exp2f(mi - mn)) + (mo == -INFINITY ? 0.0f : lo * exp2f(mo - mn));
-        mi = mn;
+      for (int cc = 0; cc < D; ++cc) s = fmaf(qv[cc], s_k[kk * D + cc], s);
+      sv[kk] = c * kScoreChunk + kk < B ? s * sl2 : -INFINITY;
+    }
+  };
+
+  // pass 1: every row's max and normaliser (each thread its rows r = tid, tid + 256, ...)
+  float m[kRowsPerThread], linv[kRowsPerThread];
+#pragma unroll
+  for (int i = 0; i < kRowsPerThread; ++i) { m[i] = -INFINITY; linv[i] = 0.0f; }
+  for (int c = 0; c < nchunks; ++c) {
+    load_chunk(c);
+#pragma unroll 1
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const int r = tid + i * kRouteThreads;
+      if (r >= rows) break;
+      float qv[D], sv[kScoreChunk];
+      load_q(r, qv);
+      chunk_logits(qv, c, sv);
+      float cm = -INFINITY;
+#pragma unroll
+      for (int kk = 0; kk < kScoreChunk; ++kk) cm = fmaxf(cm, sv[kk]);
+      const float mn = fmaxf(m[i], cm);
+      float l = m[i] == -INFINITY ? 0.0f : linv[i] * exp2f(m[i] - mn);  // linv holds the running sum here
+#pragma unroll
+      for (int kk = 0; kk < kScoreChunk; ++kk) l += exp2f(sv[kk] - mn);
+      m[i] = mn;
+      linv[i] = l;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kRowsPerThread; ++i) linv[i] = linv[i] > 0.0f ? 1.0f / linv[i] : 0.0f;
+  // pass 2: probabilities summed per key
+  for (int c = 0; c < nchunks; ++c) {
+    load_chunk(c);
+    float acc[kScoreChunk];
+#pragma unroll
+    for (int kk = 0; kk < kScoreChunk; ++kk) acc[kk] = 0.0f;
+#pragma unroll 1
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const int r = tid + i * kRouteThreads;
+      if (r >= rows) break;
+      float qv[D], sv[kScoreChunk];
+      load_q(r, qv);
+      chunk_logits(qv, c, sv);
+#pragma unroll
+      for (int kk = 0; kk < kScoreChunk; ++kk) acc[kk] += exp2f(sv[kk] - m[i]) * linv[i];
+    }
+#pragma unroll
+    for (int kk = 0; kk < kScoreChunk; ++kk) s_part[tid * (kScoreChunk + 1) + kk] = acc[kk];
+    __syncthreads();
+    // fixed-order sum over threads: warp w adds threads 32 u + lane ... for key kk = tid % 32
+    for (int kk = tid; kk < kScoreChunk; kk += kRouteThreads) {
+      const int j = c * kScoreChunk + kk;
+      float sum = 0.0f;
+      for (int th = 0; th < kRouteThreads; ++th) sum += s_part[th * (kScoreChunk + 1) + kk];
+      if (j < B) {
+        s_score[j] = sum;
+        if (score_out) score_out[((size_t)a * Hkv + g) * B + j] = sum;
       }
-      if (lane == 0 && r < rows) s_ml[r] = make_float2(mi, 1.0f / li);
     }
   }
   __syncthreads();
-  // pass 2: probabilities summed per key, chunk by chunk
-  for (int c = 0; c < nchunks; ++c) {
-    load_chunk(c);
-    float acc[KPL];
-#pragma unroll
-    for (int e = 0; e < KPL; ++e) acc[e] = 0.0f;
-    for (int r = warp; r < rows; r += 8) {
-      float qv[D];
-      load_q(r, qv);
-      const float2 ml = s_ml[r];
-#pragma unroll
-      for (int e = 0; e < KPL; ++e) {
-        const int kk = lane + 32 * e;
-        float s = 0.0f;
-#pragma unroll
-        for (int cc = 0; cc < D; ++cc) s = fmaf(qv[cc], s_k[kk * (D + 1) + cc], s);
-        acc[e] += exp2f(s * sl2 - ml.x) * ml.y;
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < KPL; ++e) s_part[warp * kScoreChunk + lane + 32 * e] = acc[e];
-    __syncthreads();
-    for (int kk = tid; kk < kScoreChunk; kk += kRouteThreads) {
-      const int j = c * kScoreChunk + kk;
-      if (j < B) {
-        float s = 0.0f;
-        for (int w = 0; w < 8; ++w) s += s_part[w * kScoreChunk + kk];
-        s_score[j] = s;
-        if (score_out) score_out[((size_t)a * Hkv + g) * B + j] = s;
-      }
-    }
-  }
   // top-k by (score desc, j asc)
   if (tid == 0) { s_lv = INFINITY; s_lj = -1; }
   __syncthreads();
@@ -351,8 +353,7 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
 }
 
 size_t score_route_smem(int B, int D) {
-  return (size_t)kScoreChunk * (D + 1) * 4 + 8 * kScoreChunk * 4 + (size_t)((B + 1) & ~1) * 4 +
-         (size_t)kMaxScoreRows * 8;
+  return (size_t)kScoreChunk * D * 4 + (size_t)kRouteThreads * (kScoreChunk + 1) * 4 + (size_t)B * 4;
 }
 
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
