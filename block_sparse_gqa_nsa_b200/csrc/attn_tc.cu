@@ -104,6 +104,7 @@ struct TcSmem {
   uint32_t tmem_base;
   int abort;
   int n_sel;
+  int win_lo, win_hi;  // window band of the CTA's tokens, relative to the block start
   int sel_start[kTcMaxSel];
   int sel_n[kTcMaxSel];
 };
@@ -170,7 +171,7 @@ struct Chunks {
   __device__ __forceinline__ int branch(int c, int& local) const {
     if (c < n_cmp) { local = c; return 0; }
     if (c < n_cmp + n_slc) { local = c - n_cmp; return 1; }
-    local = 0;
+    local = c - n_cmp - n_slc;  // window chunks (several when the band spans more than 64 keys)
     return 2;
   }
   __device__ __forceinline__ bool first_of_branch(int c) const {
@@ -178,10 +179,13 @@ struct Chunks {
   }
 };
 
-// first key row (block-mean index or token index) and number of valid keys of chunk (br, local)
+// first key row (block-mean index or token index) and number of valid keys of chunk (br, local).
+// Selected blocks longer than 64 tokens are listed as several 64-key chunks; the window branch
+// covers the band of the CTA's tokens, [win_lo, win_hi] relative to the block start, in 64-key
+// chunks (one for blocks of at most 64 tokens).
 template <int D>
 __device__ __forceinline__ void chunk_keys(const TcSmem<D>& S, const TcParams& p, int br, int local, int t0,
-                                           int n_a, int n_ckeys, int& start, int& nvalid) {
+                                           int n_ckeys, int& start, int& nvalid) {
   if (br == 0) {
     start = local * 64;
     nvalid = min(64, n_ckeys - start);
@@ -194,8 +198,8 @@ __device__ __forceinline__ void chunk_keys(const TcSmem<D>& S, const TcParams& p
       nvalid = S.sel_n[local];
     }
   } else {
-    start = t0;
-    nvalid = n_a;
+    start = t0 + S.win_lo + 64 * local;
+    nvalid = min(64, S.win_hi + 1 - (S.win_lo + 64 * local));
   }
 }
 
@@ -327,12 +331,17 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       for (int i = 0; i < p.n_forced + p.top_k && n < kTcMaxSel; ++i) {
         const int j = i < p.n_forced ? p.forced[i] : r[i - p.n_forced];
         if (j < 0 || j >= p.B) { raise_status(p.status, LSRM_ERR_BOUNDS); continue; }
-        S.sel_start[n] = p.off[j];
-        S.sel_n[n] = p.off[j + 1] - p.off[j];
-        ++n;
+        // one 64-key chunk per 64 tokens of the block
+        for (int s0 = p.off[j]; s0 < p.off[j + 1] && n < kTcMaxSel; s0 += 64) {
+          S.sel_start[n] = s0;
+          S.sel_n[n] = min(64, p.off[j + 1] - s0);
+          ++n;
+        }
       }
     }
     S.n_sel = n;
+    S.win_lo = max(0, tile0 * tokens_per_tile - p.window / 2);
+    S.win_hi = min(n_a - 1, min(n_a, (tile0 + 2) * tokens_per_tile) - 1 + p.window / 2 - 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&S.q_full[t], 1);
       mbar_init(&S.s_full[t], 1);
@@ -367,7 +376,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   const int n_ckeys = p.n_ckeys_dev != nullptr ? *p.n_ckeys_dev : p.n_ckeys;
   cs.n_cmp = (p.branches & TC_CMP) ? (n_ckeys + C::kKeys - 1) / C::kKeys : 0;
   cs.n_slc = (p.branches & TC_SLC) ? (p.route_all ? p.B : S.n_sel) : 0;
-  cs.n_win = ((p.branches & TC_WIN) && p.window > 0) ? 1 : 0;
+  // the window band of this CTA's tokens in 64-key chunks (one for blocks of at most 64 tokens)
+  cs.n_win = ((p.branches & TC_WIN) && p.window > 0) ? (S.win_hi - S.win_lo + 64) / 64 : 0;
   cs.total = cs.n_cmp + cs.n_slc + cs.n_win;
   volatile int* abort = &S.abort;
 
@@ -396,7 +406,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (c >= C::kStages && !mbar_wait(&S.kv_empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
         int local, start, nvalid;
         const int br = cs.branch(c, local);
-        chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nvalid);
+        chunk_keys<D>(S, p, br, local, t0, n_ckeys, start, nvalid);
         mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
         tma_load_3d(S.k[st], br == 0 ? &kcmap : &kmap, &S.kv_full[st], 0, g, start);
         tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
@@ -573,11 +583,11 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     };
     const int wlo = tok_local - p.window / 2, whi = tok_local + p.window / 2 - 1;
     const float sc = p.scale_log2;
-    int br = 0, nv = 0;
+    int br = 0, nv = 0, kofs = 0;  // kofs: position in the block of a window chunk's first key
     // raw score of key j of the chunk, or -inf where masked (short block or outside the window band)
     auto masked = [&](uint32_t raw, int j) -> float {
       bool kv = j < nv;
-      if (br == 2) kv = kv && j >= wlo && j <= whi;
+      if (br == 2) kv = kv && kofs + j >= wlo && kofs + j <= whi;
       return kv ? __uint_as_float(raw) : -INFINITY;
     };
     // ---- streaming top-k of the compressed-branch logits (pooled-query routing) ----
@@ -854,7 +864,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       int local, start;
       br = cs.branch(c, local);
       const bool first = cs.first_of_branch(c);
-      chunk_keys<D>(S, p, br, local, t0, n_a, n_ckeys, start, nv);
+      chunk_keys<D>(S, p, br, local, t0, n_ckeys, start, nv);
+      if (br == 2) kofs = S.win_lo + 64 * local;
       const bool need_mask = br == 2 || nv < 64;
       if (topk_on && br == 0) {
         key_base = local * 64;
@@ -1007,7 +1018,10 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
                            int lse_first, uint32_t* status, cudaStream_t stream, void* obr) {
   const int G = d.n_q_heads / d.n_kv_heads;
   if (128 % G != 0) return LSRM_ERR_UNSUPPORTED;
-  if (!route_all && d.n_forced + d.top_k > kTcMaxSel) return LSRM_ERR_UNSUPPORTED;
+  // selected blocks longer than 64 tokens take several 64-key chunks each
+  const int chunks_per_block = (d.max_block_len + 63) / 64;
+  if (!route_all && (long long)(d.n_forced + d.top_k) * chunks_per_block > kTcMaxSel) return LSRM_ERR_UNSUPPORTED;
+  if (route_all && d.max_block_len > 64) return LSRM_ERR_UNSUPPORTED;
   TcParams p{};
   p.off = off;
   p.gates = (const uint16_t*)gates;

@@ -993,7 +993,7 @@ lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const vo
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
                             unsigned char* ws_bwd, uint32_t* status, cudaStream_t s, const void* obr) {
-  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || 64 % (d.n_q_heads / d.n_kv_heads) != 0)
+  if (d.top_k > 256 || d.n_gates < 2 || d.n_gates > 3 || d.max_block_len > 64 || 64 % (d.n_q_heads / d.n_kv_heads) != 0)
     return LSRM_ERR_UNSUPPORTED;
   const BwdWs w = bwd_layout(d, idx_heads);
   BwdParams p{};

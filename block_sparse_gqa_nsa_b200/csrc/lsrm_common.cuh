@@ -10,7 +10,9 @@
 
 namespace lsrm {
 
-constexpr int kMaxBlockLen = 64;
+// Blocks of up to 512 tokens (the 8x8x8 volume bricks) in the forward; the backward, score routing
+// and the pooled-query variant keep their own (smaller) limits.
+constexpr int kMaxBlockLen = 512;
 
 // Descriptor checks shared by every entry point (host side).
 inline lsrm_status check_desc(const lsrm_nsa_desc* d) {

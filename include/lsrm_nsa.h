@@ -19,7 +19,10 @@
  *   a gate mixes the compressed and selected outputs.
  *
  * Notation: N tokens in block-major order; block b owns tokens off[b] .. off[b+1]-1
- * (n_b = off[b+1] - off[b], 1 <= n_b <= max_block_len <= 64).  Hq query heads,
+ * (n_b = off[b+1] - off[b], 1 <= n_b <= max_block_len <= 512: the pages' 8x8x8 volume
+ * blocks next to 8x8 image tiles.  The backward, score routing beyond 4096 rows per block and
+ * the pooled-query variant take blocks of at most 64 / 64 / 16 tokens and answer
+ * LSRM_ERR_UNSUPPORTED otherwise).  Hq query heads,
  * Hkv KV heads, G = Hq / Hkv, query head h reads KV head h / G.  d = head_dim.
  * tau = scale (0 means 1/sqrt(d)).
  *
@@ -77,7 +80,7 @@ enum { LSRM_ROUTE_GIVEN = 0, LSRM_ROUTE_SCORE = 1, LSRM_ROUTE_GEOMETRIC = 2, LSR
 typedef struct {
   int64_t n_tokens;       /* N >= 1 */
   int32_t n_blocks;       /* B >= 1 */
-  int32_t max_block_len;  /* upper bound of every n_b, 1..64 */
+  int32_t max_block_len;  /* upper bound of every n_b, 1..512 */
   int32_t n_q_heads;      /* Hq, multiple of n_kv_heads */
   int32_t n_kv_heads;     /* Hkv >= 1 */
   int32_t head_dim;       /* d in {32, 64} */

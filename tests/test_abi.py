@@ -49,7 +49,7 @@ def test_workspace_size_and_validation_on_host(lib):
     n = nsa.lsrm_nsa_workspace_size(_desc())
     assert n > 0 and n % 256 == 0
     for bad in (dict(head_dim=48), dict(top_k=17), dict(top_k=0), dict(n_q_heads=3), dict(window=3),
-                dict(max_block_len=65), dict(n_gates=4), dict(scale=-1.0), dict(n_blocks=0),
+                dict(max_block_len=513), dict(n_gates=4), dict(scale=-1.0), dict(n_blocks=0),
                 dict(pooled_q=True, n_gates=3)):
         assert nsa.lsrm_nsa_workspace_size(_desc(**bad)) == 0, bad
 

@@ -346,6 +346,8 @@ def make_workload(name: str, seed: int = 0, **kw) -> Workload:
     speed3r   512 frames x (1 camera + 37x37 patches); MHA 16 heads, d 64; pooled-Q
               compression; top-32 plus forced blocks (frame 0, camera tokens); 2 gates.
     backward  the sparse workload plus an upstream gradient dO ~ N(0, 1).
+    sparse_vol512 / small_vol512 / ragged_vol512: the pages' 8x8x8 volume blocks (512 tokens) with
+              8x8 image tiles (the sparse stage, a small case, and a voxel-exact case of ragged blocks).
     small variants (test sizes): tiny_geo, ragged_geo (voxel-exact shell: partial blocks),
               speed3r_small, backward_small.
     """
@@ -382,6 +384,17 @@ def make_workload(name: str, seed: int = 0, **kw) -> Workload:
         hq, hkv, d, k, w, route = 16, 16, 64, 32, 0, "score"
         fixed, ng, sc, pooled = None, 2, 1.0 / 8.0, True
         desc = f"{nf} frames x (1 camera + 37x37 patches), MHA 16 x 64, pooled-Q, top-32 + forced"
+    elif name in ("sparse_vol512", "small_vol512", "ragged_vol512"):
+        # the pages' 8x8x8 volume blocks (512 tokens) with 8x8 image tiles
+        if name == "sparse_vol512":
+            lay = lsrm_layout(64, 16, 64, 32, (0.35, 0.45), True, seed=seed, brick=8)
+        elif name == "small_vol512":
+            lay = lsrm_layout(16, 4, 32, 8, (0.3, 0.45), True, seed=seed, brick=8)
+        else:
+            lay = lsrm_layout(16, 2, 16, 3, (0.3, 0.45), False, seed=seed, brick=8)
+        hq, hkv, d, k, w, route = 32, 2, 32, 16 if name == "sparse_vol512" else 4, 64, "geom"
+        fixed, ng, sc, pooled = None, 3, d32, False
+        desc = f"{name}: 8x8x8 volume blocks (512 tokens) + 8x8 image tiles, geometric top-{k}, window 64"
     elif name == "backward_small":
         lay = lsrm_layout(16, 4, 32, 8, (0.3, 0.45), True, seed=seed)
         hq, hkv, d, k, w, route = 32, 2, 32, 8, 64, "geom"
