@@ -149,7 +149,7 @@ struct TcParams {
   // pass (bound_pass = 1: scores only, no softmax, no P V) writes it; the top-k pass reads it
   float* topk_thr;
   int bound_pass;
-  int n_pairs;  // 128-row tile pairs per query block (set by the launcher; part of grid x)
+  int n_pairs, n_groups;  // 128-row tile pairs per query block, KV groups (grid x = (a * groups + g) * pairs + pair)
   // optional row -> block id map of the keys (the pooled keys may be stored in another order);
   // the emitted top-k are block ids
   const int32_t* topk_ids;
@@ -303,7 +303,9 @@ __device__ __noinline__ void topk_emit(const float* val, const int* id, int n, i
   for (int r = n; r < k; ++r) dst[r] = -1;
 }
 
-template <int D>
+// kLong: blocks may exceed 64 tokens (the window band of a CTA may then start inside the block and
+// span several chunks); without it a CTA's band is its whole block, one chunk from the block start.
+template <int D, bool kLong>
 __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kCtasPerSm)
 nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
@@ -313,9 +315,12 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   const uint32_t raw = smem_u32(smem_raw);
   TcSmem<D>& S = *reinterpret_cast<TcSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid: x = query block * pairs + pair (block-major, so a block's tile pairs run side by side
-  // and the query-block count is not bounded by the 65535 limit of grid y / z), y = KV group
-  const int pair = (int)(blockIdx.x % (unsigned)p.n_pairs), g = blockIdx.y, a = (int)(blockIdx.x / (unsigned)p.n_pairs);
+  // grid x = (query block * KV groups + group) * pairs + pair of 128-row tiles: the tile pairs and
+  // groups of one query block run side by side (they read the same selected blocks, whose K and V
+  // rows hold both groups' heads), and the query-block count is not bounded by grid y / z
+  const unsigned bg = blockIdx.x / (unsigned)p.n_pairs;
+  const int pair = (int)(blockIdx.x - bg * (unsigned)p.n_pairs);
+  const int a = (int)(bg / (unsigned)p.n_groups), g = (int)(bg - (unsigned)a * (unsigned)p.n_groups);
   const int t0 = p.uniform_block ? a * p.uniform_block : p.off[a];
   const int n_a = p.uniform_block ? min(p.uniform_block, p.N - t0) : p.off[a + 1] - t0;
   const int rows_total = n_a * p.G;
@@ -340,8 +345,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       }
     }
     S.n_sel = n;
-    S.win_lo = max(0, tile0 * tokens_per_tile - p.window / 2);
-    S.win_hi = min(n_a - 1, min(n_a, (tile0 + 2) * tokens_per_tile) - 1 + p.window / 2 - 1);
+    S.win_lo = kLong ? max(0, tile0 * tokens_per_tile - p.window / 2) : 0;
+    S.win_hi = kLong ? min(n_a - 1, min(n_a, (tile0 + 2) * tokens_per_tile) - 1 + p.window / 2 - 1) : n_a - 1;
     for (int t = 0; t < 2; ++t) {
       mbar_init(&S.q_full[t], 1);
       mbar_init(&S.s_full[t], 1);
@@ -581,13 +586,15 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       const bool w = mbar_wait(bar, parity, abort, p.status);
       return __all_sync(0xffffffffu, w);
     };
-    const int wlo = tok_local - p.window / 2, whi = tok_local + p.window / 2 - 1;
+    // this row's window band relative to the first key of the current window chunk (with long
+    // blocks, moved along as the window chunks come, which are the last of the stream)
+    int wlo = tok_local - p.window / 2, whi = tok_local + p.window / 2 - 1;
     const float sc = p.scale_log2;
-    int br = 0, nv = 0, kofs = 0;  // kofs: position in the block of a window chunk's first key
+    int br = 0, nv = 0;
     // raw score of key j of the chunk, or -inf where masked (short block or outside the window band)
     auto masked = [&](uint32_t raw, int j) -> float {
       bool kv = j < nv;
-      if (br == 2) kv = kv && kofs + j >= wlo && kofs + j <= whi;
+      if (br == 2) kv = kv && j >= wlo && j <= whi;
       return kv ? __uint_as_float(raw) : -INFINITY;
     };
     // ---- streaming top-k of the compressed-branch logits (pooled-query routing) ----
@@ -865,7 +872,11 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       br = cs.branch(c, local);
       const bool first = cs.first_of_branch(c);
       chunk_keys<D>(S, p, br, local, t0, n_ckeys, start, nv);
-      if (br == 2) kofs = S.win_lo + 64 * local;
+      if (kLong && br == 2) {
+        const int shift = local == 0 ? S.win_lo : 64;  // the chunk starts this many keys further on
+        wlo -= shift;
+        whi -= shift;
+      }
       const bool need_mask = br == 2 || nv < 64;
       if (topk_on && br == 0) {
         key_base = local * 64;
@@ -982,8 +993,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 // ---- host side ------------------------------------------------------------------------------------
 namespace {
 
-template <int D>
-lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q, const void* k, const void* v,
+template <int D, bool kLong>
+lsrm_status launch_tc_dl(const lsrm_nsa_desc& d, const TcParams& p, const void* q, const void* k, const void* v,
                         const void* kc, const void* vc, long long kc_rows, cudaStream_t stream) {
   CUtensorMap qm, km, vm, kcm, vcm;
   const void* kk = k ? k : kc;
@@ -997,17 +1008,26 @@ lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q
     return LSRM_ERR_CUDA;
   if (!make_map(&vcm, vvc, D, d.n_kv_heads, vc ? kc_rows : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
   const size_t smem = sizeof(TcSmem<D>) + 1024;
-  if (cudaFuncSetAttribute(nsa_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (cudaFuncSetAttribute(nsa_attn_tc_kernel<D, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LSRM_ERR_CUDA;
   const int tiles = (d.max_block_len * p.G + 127) / 128;
   TcParams pp = p;
   pp.n_pairs = (tiles + 1) / 2;
-  const long long nx = (long long)d.n_blocks * pp.n_pairs;
-  if (nx > INT32_MAX || d.n_kv_heads > 65535) return LSRM_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)nx, (unsigned)d.n_kv_heads);
-  nsa_attn_tc_kernel<D><<<grid, kTcThreads, smem, stream>>>(qm, km, vm, kcm, vcm, pp);
+  pp.n_groups = d.n_kv_heads;
+  const long long nx = (long long)d.n_blocks * d.n_kv_heads * pp.n_pairs;
+  if (nx > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
+  nsa_attn_tc_kernel<D, kLong><<<(unsigned)nx, kTcThreads, smem, stream>>>(qm, km, vm, kcm, vcm, pp);
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
+template <int D>
+lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q, const void* k, const void* v,
+                        const void* kc, const void* vc, long long kc_rows, cudaStream_t stream) {
+  // the window band of long blocks only exists in the layer passes (the dense passes use no window)
+  if (d.max_block_len > 64 && p.uniform_block == 0)
+    return launch_tc_dl<D, true>(d, p, q, k, v, kc, vc, kc_rows, stream);
+  return launch_tc_dl<D, false>(d, p, q, k, v, kc, vc, kc_rows, stream);
 }
 
 }  // namespace
@@ -1074,7 +1094,7 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
   if (n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
   lsrm_nsa_desc d{};
   d.n_tokens = n_q;
-  d.n_blocks = (int32_t)((n_q + 255) / 256);  // query groups (grid z)
+  d.n_blocks = (int32_t)((n_q + 255) / 256);  // groups of 256 query rows (the query blocks of the grid)
   d.max_block_len = 256;
   d.n_q_heads = H;
   d.n_kv_heads = H;

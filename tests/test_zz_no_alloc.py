@@ -52,7 +52,7 @@ def test_noalloc_routing_rejects_too_many_blocks_and_reports_bad_coordinates():
     # descriptors that lsrm_route_geometric rejects are rejected here too, with the same status
     ws = nsa.workspace(desc)
     idx0 = torch.empty(w.n_blocks, w.top_k, dtype=torch.int32, device="cuda")
-    for bad_desc in (nsa.make_desc(w.n_tokens, w.n_blocks, 65, 32, 2, 32, w.top_k, 64),      # block > 64
+    for bad_desc in (nsa.make_desc(w.n_tokens, w.n_blocks, 513, 32, 2, 32, w.top_k, 64),     # block > 512
                      nsa.make_desc(w.n_tokens, w.n_blocks, w.max_block_len, 32, 2, 48, w.top_k, 64),  # d = 48
                      nsa.make_desc(w.n_tokens, w.n_blocks, w.max_block_len, 32, 2, 32, w.top_k, 63)):  # odd w
         with pytest.raises(nsa.NsaError) as e_ref:
