@@ -20,6 +20,11 @@
 //                paragraph; Speed3R page, 2.1 (compression / selection branches).
 //   gates: Sigmoid(Linear(x)) gate values weight the branch outputs — LSRM page,
 //                方法, gate equations; Speed3R page, 2.1 gated aggregation.
+//   camera routing: the query point is projected into every view, the view's
+//                nearby image blocks are candidates, ranked by their smallest
+//                token-to-query distance — LSRM page, 方法, 3D-aware routing paragraph.
+//   self/cross mixture: o^x = w CrossAttn(x,x) + w CrossAttn(x,y) and likewise for
+//                y — LSRM page, 方法, the dense blocks' gated cross-attention equations.
 //
 // Readings where the pages are silent (each also listed in the design notes):
 //   * softmax scale tau = 1/sqrt(d); query head h uses KV group floor(h / (Hq/Hkv)).
@@ -734,6 +739,139 @@ double impl_loss(const Desc* D, const int32_t* off, const T* q, const T* k, cons
   return L;
 }
 
+// ---- f4: decoupled self/cross gated mixture over two token streams (LSRM page, 方法, the
+// gated cross-attention equations of the dense transformer blocks):
+//   o^x = w^{x-self} CrossAttn(x, x) + w^{x-cross} CrossAttn(x, y),
+//   o^y = w^{y-self} CrossAttn(y, y) + w^{y-cross} CrossAttn(y, x).
+// Stream x is blocks [0, bx) (tokens [0, off[bx])), stream y blocks [bx, B).  CrossAttn(a, b) is
+// softmax attention of a's queries over every token of b (grouped-query heads as elsewhere).
+// gates [N][Hq][2] = (w_self, w_cross), inputs like the NSA gates (the Sigmoid(Linear) that makes
+// them is trained and out of scope).  An empty stream contributes a zero output (LSE -inf).
+// branches (optional): [rows][Hq][2][d] = (self, cross); lse (optional): [rows][Hq][2].
+template <typename T>
+int impl_mixture(const Desc* D, const int32_t* off, const T* q, const T* k, const T* v, const T* gates, int32_t bx,
+                 int32_t n_qb, const int32_t* qblocks, double* out, double* branches, double* lse) {
+  const int32_t B = D->n_blocks, Hq = D->n_q_heads, Hkv = D->n_kv_heads, d = D->head_dim;
+  if (bx < 0 || bx > B) return 1;
+  const int32_t G = Hq / Hkv;
+  const double tau = tau_of(*D);
+  const int64_t nx = off[bx], N = off[B];
+  // the key/value rows of both streams, widened once
+  const std::vector<double> kw = widen(k, (size_t)(N * Hkv * d)), vw = widen(v, (size_t)(N * Hkv * d));
+  std::vector<double> qv((size_t)d), o2((size_t)(2 * d));
+  int64_t row = 0;
+  for (int32_t qi = 0; qi < n_qb; ++qi) {
+    const int32_t a = qblocks[qi];
+    const bool in_x = a < bx;
+    // token ranges of the query's own stream and of the other one
+    const int64_t self_lo = in_x ? 0 : nx, self_hi = in_x ? nx : N;
+    const int64_t cross_lo = in_x ? nx : 0, cross_hi = in_x ? N : nx;
+    for (int64_t t = off[a]; t < off[a + 1]; ++t, ++row)
+      for (int32_t h = 0; h < Hq; ++h) {
+        const int32_t g = h / G;
+        for (int c = 0; c < d; ++c) qv[(size_t)c] = bf(q[(t * Hq + h) * d + c]);
+        double L[2];
+        for (int s = 0; s < 2; ++s) {
+          const int64_t lo = s == 0 ? self_lo : cross_lo, hi = s == 0 ? self_hi : cross_hi;
+          std::vector<const double*> keys, vals;
+          for (int64_t u = lo; u < hi; ++u) {
+            keys.push_back(&kw[(size_t)((u * Hkv + g) * d)]);
+            vals.push_back(&vw[(size_t)((u * Hkv + g) * d)]);
+          }
+          L[s] = attend(qv, keys, vals, d, tau, &o2[(size_t)(s * d)]);
+        }
+        const T* w = gates + (t * Hq + h) * 2;
+        for (int c = 0; c < d; ++c)
+          out[(row * Hq + h) * d + c] = bf(w[0]) * o2[(size_t)c] + bf(w[1]) * o2[(size_t)(d + c)];
+        if (branches)
+          for (int s = 0; s < 2; ++s)
+            for (int c = 0; c < d; ++c) branches[((row * Hq + h) * 2 + s) * d + c] = o2[(size_t)(s * d + c)];
+        if (lse)
+          for (int s = 0; s < 2; ++s) lse[(row * Hq + h) * 2 + s] = L[s];
+      }
+  }
+  return 0;
+}
+
+// ---- f2: camera-projection routing (LSRM page, 方法, 3D-aware routing paragraph).  Each token
+// has a 3D point; the query point of block a is its centroid (as in S2b).
+//   volume part: the k_vol volume blocks (ids [0, n_vol)) nearest by centroid distance, as S2b;
+//   image part: the query point is projected into every view by that view's camera,
+//     h = P_v [c; 1] (int64), pixel = (floor(h0 / h2), floor(h1 / h2)) when h2 > 0 (in front of
+//     the camera; views behind it give nothing), tile = floor(pixel / tile_px); the image blocks
+//     of the tiles within Chebyshev distance `radius` of that tile in the view's tile grid
+//     (tile_block[v][ty][tx], -1 = no block) are the candidates, ranked by the smallest squared
+//     distance from any of their tokens to the query point, ties to the lower block id; the
+//     k_img best are kept.  Should fewer than k_img candidates exist, the other image blocks
+//     fill the list by centroid distance (ties to the lower id).
+// idx [B][k_vol + k_img]: the volume part in rank order, then the image part.
+int impl_route_camera(const Desc* D, const int32_t* off, const int32_t* coords, int32_t n_vol, int32_t n_views,
+                      const int32_t* proj, int32_t tiles_x, int32_t tiles_y, int32_t tile_px,
+                      const int32_t* tile_block, int32_t radius, int32_t k_vol, int32_t k_img, int32_t* idx) {
+  const int32_t B = D->n_blocks;
+  if (n_vol < k_vol || B - n_vol < k_img || tile_px < 1 || radius < 0) return 1;
+  std::vector<int64_t> c((size_t)B * 3);
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t n = (int64_t)off[b + 1] - off[b];
+    for (int a = 0; a < 3; ++a) {
+      int64_t S = 0;
+      for (int64_t t = off[b]; t < off[b + 1]; ++t) S += coords[t * 3 + a];
+      c[(size_t)b * 3 + a] = floor_div(2 * S + n, 2 * n);
+    }
+  }
+  auto dist2 = [](const int64_t* p, const int64_t* q) {
+    int64_t s = 0;
+    for (int a = 0; a < 3; ++a) s += (p[a] - q[a]) * (p[a] - q[a]);
+    return s;
+  };
+  const int32_t K = k_vol + k_img;
+  for (int32_t a = 0; a < B; ++a) {
+    const int64_t* qa = &c[(size_t)a * 3];
+    std::vector<std::pair<int64_t, int32_t>> vol;
+    for (int32_t j = 0; j < n_vol; ++j) vol.push_back({dist2(qa, &c[(size_t)j * 3]), j});
+    std::sort(vol.begin(), vol.end());
+    for (int32_t i = 0; i < k_vol; ++i) idx[(int64_t)a * K + i] = vol[(size_t)i].second;
+    // candidates from every view's tile neighbourhood
+    std::vector<int32_t> cand;
+    for (int32_t v = 0; v < n_views; ++v) {
+      int64_t h[3];
+      for (int r = 0; r < 3; ++r) {
+        const int32_t* P = proj + ((int64_t)v * 3 + r) * 4;
+        h[r] = (int64_t)P[0] * qa[0] + (int64_t)P[1] * qa[1] + (int64_t)P[2] * qa[2] + (int64_t)P[3];
+      }
+      if (h[2] <= 0) continue;
+      const int64_t tx = floor_div(floor_div(h[0], h[2]), tile_px), ty = floor_div(floor_div(h[1], h[2]), tile_px);
+      for (int64_t y = ty - radius; y <= ty + radius; ++y)
+        for (int64_t x = tx - radius; x <= tx + radius; ++x) {
+          if (x < 0 || y < 0 || x >= tiles_x || y >= tiles_y) continue;
+          const int32_t b = tile_block[((int64_t)v * tiles_y + y) * tiles_x + x];
+          if (b >= 0) cand.push_back(b);
+        }
+    }
+    std::sort(cand.begin(), cand.end());
+    cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
+    std::vector<std::pair<int64_t, int32_t>> img;
+    for (int32_t b : cand) {
+      int64_t best = INT64_MAX;
+      for (int64_t t = off[b]; t < off[b + 1]; ++t) {
+        const int64_t p[3] = {coords[t * 3], coords[t * 3 + 1], coords[t * 3 + 2]};
+        best = std::min(best, dist2(qa, p));
+      }
+      img.push_back({best, b});
+    }
+    std::sort(img.begin(), img.end());
+    int32_t n = 0;
+    for (; n < k_img && n < (int32_t)img.size(); ++n) idx[(int64_t)a * K + k_vol + n] = img[(size_t)n].second;
+    if (n < k_img) {
+      std::vector<std::pair<int64_t, int32_t>> fill;
+      for (int32_t j = n_vol; j < B; ++j)
+        if (!std::binary_search(cand.begin(), cand.end(), j)) fill.push_back({dist2(qa, &c[(size_t)j * 3]), j});
+      std::sort(fill.begin(), fill.end());
+      for (size_t i = 0; n < k_img; ++n, ++i) idx[(int64_t)a * K + k_vol + n] = fill[i].second;
+    }
+  }
+  return 0;
+}
 
 }  // namespace
 
@@ -824,6 +962,17 @@ int oracle_backward_pooled_f64(const Desc* D, const int32_t* off, const double* 
                                double* dgates, int32_t nthreads) {
   return impl_backward_pooled<double>(D, off, q, k, v, gates, idx, n_forced, forced, dout, dq, dk, dv, dgates,
                                       nthreads);
+}
+int oracle_route_camera(const Desc* D, const int32_t* off, const int32_t* coords, int32_t n_vol, int32_t n_views,
+                        const int32_t* proj, int32_t tiles_x, int32_t tiles_y, int32_t tile_px,
+                        const int32_t* tile_block, int32_t radius, int32_t k_vol, int32_t k_img, int32_t* idx) {
+  return impl_route_camera(D, off, coords, n_vol, n_views, proj, tiles_x, tiles_y, tile_px, tile_block, radius, k_vol,
+                           k_img, idx);
+}
+int oracle_mixture(const Desc* D, const int32_t* off, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const uint16_t* gates, int32_t bx, int32_t n_qb, const int32_t* qblocks, double* out,
+                   double* branches, double* lse) {
+  return impl_mixture<uint16_t>(D, off, q, k, v, gates, bx, n_qb, qblocks, out, branches, lse);
 }
 
 }  // extern "C"

@@ -22,7 +22,7 @@ _LIB = os.path.join(_HERE, "liboracle_nsa.so")
 
 __all__ = ["build_oracle", "OracleDesc", "desc_for", "compress", "route_geometric", "route_score",
            "route_pooled", "cmp_attn", "select_attn", "window_attn", "forward", "backward", "loss_f64",
-           "forward_f64", "backward_f64", "backward_pooled", "backward_pooled_f64", "loss_forced_f64", "rows_of"]
+           "forward_f64", "backward_f64", "backward_pooled", "backward_pooled_f64", "loss_forced_f64", "mixture", "route_camera", "rows_of"]
 
 
 class OracleDesc(ctypes.Structure):
@@ -68,6 +68,8 @@ def _L():
             "oracle_loss_forced_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp, i32, vp],
             "oracle_backward_pooled": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, i32],
             "oracle_backward_pooled_f64": [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, i32],
+            "oracle_mixture": [P, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp],
+            "oracle_route_camera": [P, vp, vp, i32, i32, vp, i32, i32, i32, vp, i32, i32, i32, vp],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -292,3 +294,42 @@ def loss_forced_f64(D, off, q, k, v, gates, idx, dout, forced) -> float:
     forced = _c(forced, np.int32)
     return float(_L().oracle_loss_forced_f64(ctypes.byref(D), _p(off), _p(q), _p(k), _p(v), _p(gates), _p(idx),
                                              idx_heads, _p(dout), len(forced), _p(forced)))
+
+
+def mixture(D: OracleDesc, off, q, k, v, gates, bx: int, qblocks=None, want_branches=False):
+    """Decoupled self/cross gated mixture (LSRM page, 方法, gated cross-attention equations):
+    stream x = blocks [0, bx), stream y = blocks [bx, B); gates [N][Hq][2] = (w_self, w_cross).
+    With want_branches: (out, branches [rows][Hq][2][d] = (self, cross), lse [rows][Hq][2])."""
+    qblocks = np.arange(D.n_blocks, dtype=np.int32) if qblocks is None else _c(qblocks, np.int32)
+    off = _c(off, np.int32)
+    q, k, v, gates = _inputs(np.uint16, q, k, v, gates)
+    rows = rows_of(off, qblocks)
+    out = np.zeros((rows, D.n_q_heads, D.head_dim))
+    br = np.zeros((rows, D.n_q_heads, 2, D.head_dim)) if want_branches else None
+    lse = np.zeros((rows, D.n_q_heads, 2)) if want_branches else None
+    rc = _L().oracle_mixture(ctypes.byref(D), _p(off), _p(q), _p(k), _p(v), _p(gates), int(bx), len(qblocks),
+                             _p(qblocks), _p(out), _p(br), _p(lse))
+    if rc != 0:
+        raise ValueError("oracle_mixture: stream split outside [0, n_blocks]")
+    return (out, br, lse) if want_branches else out
+
+
+def route_camera(D: OracleDesc, off, coords, n_vol: int, proj, tile_block, tile_px: int, radius: int, k_vol: int,
+                 k_img: int) -> np.ndarray:
+    """Camera-projection routing (LSRM page, 方法, 3D-aware routing paragraph): idx [B][k_vol + k_img],
+    the k_vol nearest volume blocks by centroid distance, then the k_img image blocks of the
+    projected tile neighbourhoods nearest by their closest token.  proj int32 [V][3][4],
+    tile_block int32 [V][tiles_y][tiles_x] (-1 = no block)."""
+    off = _c(off, np.int32)
+    coords = _c(coords, np.int32)
+    proj = _c(proj, np.int32)
+    tile_block = _c(tile_block, np.int32)
+    V, ty, tx = tile_block.shape
+    assert proj.shape == (V, 3, 4)
+    idx = np.zeros((D.n_blocks, k_vol + k_img), dtype=np.int32)
+    rc = _L().oracle_route_camera(ctypes.byref(D), _p(off), _p(coords), int(n_vol), int(V), _p(proj), int(tx),
+                                  int(ty), int(tile_px), _p(tile_block), int(radius), int(k_vol), int(k_img),
+                                  _p(idx))
+    if rc != 0:
+        raise ValueError("oracle_route_camera: k_vol / k_img above the block counts, or bad tile size / radius")
+    return idx

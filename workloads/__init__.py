@@ -9,6 +9,7 @@ from .nsa_workloads import (  # noqa: F401
     Workload,
     make_workload,
     lsrm_layout,
+    camera_inputs,
     speed3r_layout,
     WORKLOAD_NAMES,
     gen_lib,

@@ -235,7 +235,37 @@ def lsrm_layout(grid: int, n_views: int, view_res: int, keep_tiles: Optional[int
     assert coords_all.shape[0] == off[-1]
     return Layout(off=off, coords=coords_all, n_vol_blocks=n_vol_blocks, n_img_blocks=n_img_blocks,
                   meta=dict(grid=grid, n_views=n_views, view_res=view_res, keep_tiles=keep_tiles,
-                            shell=shell, brick_granular=brick_granular, tan_half_fov=tan_half))
+                            shell=shell, brick_granular=brick_granular, tan_half_fov=tan_half, tile=tile,
+                            cam_pos=pos, cam_fwd=fwd, cam_right=right, cam_up=up, kept_tiles=kept))
+
+
+def camera_inputs(layout: Layout, max_entry: int = 1 << 23):
+    """The cameras of an LSRM layout as inputs of camera-projection routing.
+
+    proj int32 [V][3][4]: per view a homogeneous projection of a lattice point c (the coords'
+    units) to pixel coordinates, u = h0 / h2, v = h1 / h2 with h = P [c; 1] (h2 = depth along
+    the view direction), the same pinhole model the image tokens were generated with (pixel
+    (u, v) covers [u, u+1) x [v, v+1), rows from the top), scaled so that the largest entry is
+    about max_entry and rounded to integers.  tile_block int32 [V][tiles][tiles]: the block id
+    of each kept tile, -1 elsewhere.  tile_px: pixels per tile side.  Returns
+    (proj, tile_block, tile_px)."""
+    m = layout.meta
+    G, R, tile, th = m["grid"], m["view_res"], m["tile"], m["tan_half_fov"]
+    s = 1.0 / (16.0 * G)                     # lattice unit in world units; world = s c - 0.5
+    V = m["n_views"]
+    tpr = R // tile
+    proj = np.zeros((V, 3, 4), dtype=np.int32)
+    tile_block = np.full((V, tpr, tpr), -1, dtype=np.int32)
+    kept = m["kept_tiles"]
+    for v in range(V):
+        pos, fwd, right, up = m["cam_pos"][v], m["cam_fwd"][v], m["cam_right"][v], m["cam_up"][v]
+        rows = np.stack([0.5 * R * (right / th + fwd), 0.5 * R * (fwd - up / th), fwd])  # [3][3]
+        o = -0.5 - pos                         # world offset of lattice point 0, relative to the camera
+        P = np.concatenate([rows * s, (rows @ o)[:, None]], axis=1)
+        proj[v] = np.rint(P * (max_entry / np.abs(P).max())).astype(np.int32)
+        for r, t in enumerate(kept):
+            tile_block[v, t // tpr, t % tpr] = layout.n_vol_blocks + v * len(kept) + r
+    return proj, tile_block, tile
 
 
 def speed3r_layout(n_frames: int, patch: int = 37, pool: int = 4) -> Layout:
@@ -314,6 +344,11 @@ class Workload:
     def scale(self):
         return 1.0 / math.sqrt(self.head_dim)
 
+    @property
+    def n_blocks_x(self):
+        """Blocks of the first stream (the volume tokens) in the self/cross mixture."""
+        return int(self.layout.n_vol_blocks)
+
 
 def _tensors(layout: Layout, hq: int, hkv: int, d: int, n_gates: int, seed: int, scale: float,
              fixed_gates=None, with_dout=False):
@@ -331,7 +366,8 @@ def _tensors(layout: Layout, hq: int, hkv: int, d: int, n_gates: int, seed: int,
 
 
 WORKLOAD_NAMES = ("tiny", "dense", "sparse", "speed3r", "backward",
-                  "tiny_geo", "ragged_geo", "speed3r_small", "backward_small")
+                  "tiny_geo", "ragged_geo", "speed3r_small", "backward_small",
+                  "mixture", "mixture_small", "mixture_ragged")
 
 
 def make_workload(name: str, seed: int = 0, **kw) -> Workload:
@@ -350,6 +386,10 @@ def make_workload(name: str, seed: int = 0, **kw) -> Workload:
               8x8 image tiles (the sparse stage, a small case, and a voxel-exact case of ragged blocks).
     small variants (test sizes): tiny_geo, ragged_geo (voxel-exact shell: partial blocks),
               speed3r_small, backward_small.
+    mixture   the decoupled self/cross gated mixture at the dense-stage shape (16^3 volume tokens
+              + 16 views of 32x32 image tokens, 20480 tokens); 2 gates (self, cross) ~ sigmoid(N(0,1)).
+    mixture_small / mixture_ragged: the same on the tiny layout, and on the voxel-exact shell
+              (ragged volume blocks).
     """
     d32 = 1.0 / math.sqrt(32.0)
     if name == "tiny":
@@ -395,6 +435,16 @@ def make_workload(name: str, seed: int = 0, **kw) -> Workload:
         hq, hkv, d, k, w, route = 32, 2, 32, 16 if name == "sparse_vol512" else 4, 64, "geom"
         fixed, ng, sc, pooled = None, 3, d32, False
         desc = f"{name}: 8x8x8 volume blocks (512 tokens) + 8x8 image tiles, geometric top-{k}, window 64"
+    elif name in ("mixture", "mixture_small", "mixture_ragged"):
+        if name == "mixture":
+            lay = lsrm_layout(16, 16, 32, None, None, seed=seed)
+        elif name == "mixture_small":
+            lay = lsrm_layout(8, 2, 16, None, None, seed=seed)
+        else:
+            lay = lsrm_layout(16, 2, 16, 3, (0.3, 0.45), False, seed=seed)
+        hq, hkv, d, k, w, route = 32, 2, 32, 1, 0, "mixture"
+        fixed, ng, sc, pooled = None, 2, d32, False
+        desc = f"{name}: self/cross gated mixture of the volume and image streams ({lay.n_tokens} tokens)"
     elif name == "backward_small":
         lay = lsrm_layout(16, 4, 32, 8, (0.3, 0.45), True, seed=seed)
         hq, hkv, d, k, w, route = 32, 2, 32, 8, 64, "geom"
