@@ -52,7 +52,7 @@ def parse():
                          "10-20 s of one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r", "bandwidth"],
+    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r", "mixture", "bandwidth"],
                     help="sparse: the layer forward (the default line); backward: its gradients; dense: the "
                          "dense-stage shape with every block selected; speed3r: the pooled-query variant; "
                          "bandwidth: achieved HBM GB/s of the memory-bound kernels (pooling, routing, combine)")
@@ -673,6 +673,7 @@ def run_backward(args):
 EXTRA = {
     "dense": ("sparse-attn fwd tokens/s, dense-stage shape (k = B)", "lsrm_dense_stage_all_blocks"),
     "speed3r": ("sparse-attn fwd tokens/s, Speed3R pooled-query variant", "speed3r_512_frames_top32_forced"),
+    "mixture": ("self/cross gated mixture fwd tokens/s, dense-stage shape", "lsrm_dense_stage_self_cross_mixture"),
 }
 
 
@@ -695,6 +696,16 @@ def speed3r_flops(w, idx: np.ndarray) -> dict:
     slc = float((n[:, None] * (forced_tok + routed_tok)).sum())
     f = 4 * d
     return {"cmp": f * cmp, "slc": f * slc, "total": f * (cmp + slc)}
+
+
+def mixture_flops(w) -> dict:
+    """4 d per (query, key) pair: every query attends every key of its own stream (self) and of
+    the other stream (cross), for each query head."""
+    nx = int(w.off[w.n_blocks_x])
+    ny = w.n_tokens - nx
+    f = 4 * w.head_dim * w.n_q_heads
+    return {"self": float(f * (nx * nx + ny * ny)), "cross": float(f * 2 * nx * ny),
+            "total": float(f * w.n_tokens * w.n_tokens)}
 
 
 def run_extra(args):
@@ -737,7 +748,14 @@ def run_extra(args):
     desc = nsa.make_desc(N, B, w.max_block_len, Hq, Hkv, d, k, w.window, 0.0, w.pooled_q, w.n_gates, forced)
     ws = nsa.workspace(desc, dev)
     out = torch.empty(N, Hq, d, dtype=torch.bfloat16, device=dev)
-    if args.workload == "speed3r":
+    if args.workload == "mixture":
+        idx = None
+        bx = w.n_blocks_x
+
+        def step():
+            nsa.lsrm_nsa_mixture(desc, off, bx, q, kk, v, gates, out, None, ws)
+        launches_per_step = 1  # both attentions and the gated sum in one kernel
+    elif args.workload == "speed3r":
         idx = torch.empty(B, Hq, k, dtype=torch.int32, device=dev)
 
         def step():
@@ -759,6 +777,8 @@ def run_extra(args):
         raise RuntimeError(f"device status {st} after warm-up")
     if args.workload == "speed3r":
         flops = speed3r_flops(w, idx.cpu().numpy())
+    elif args.workload == "mixture":
+        flops = mixture_flops(w)
     else:
         flops = algorithmic_flops(w, np.tile(np.arange(B, dtype=np.int32), (B, 1)))
     sampler = ClockSampler(local) if rank == 0 else None
@@ -789,7 +809,8 @@ def run_extra(args):
                 "flops_per_step": flops,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                              "frac": achieved / peak, "traffic": None,
-                             "kernel": "lsrm_nsa_forward (all launches of one call)",
+                             "kernel": ("nsa_attn_tc_kernel (mixture mode, one launch)" if args.workload == "mixture"
+                                        else "lsrm_nsa_forward (all launches of one call)"),
                              "peak_source": f"{src} bf16_tflops (burst)"},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
         if not args.no_cpu_baseline and world == 1:
@@ -815,7 +836,9 @@ def extra_oracle_sample(w, idx, n_blocks: int, seed: int):
     if idx is None:
         idx = np.tile(np.arange(w.n_blocks, dtype=np.int32), (w.n_blocks, 1))
     t0 = time.perf_counter()
-    if w.pooled_q:
+    if w.route == "mixture":
+        O.mixture(D, w.off, w.q, w.k, w.v, w.gates, w.n_blocks_x, qblocks=qb)
+    elif w.pooled_q:
         O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, forced=w.forced, qblocks=qb)
     else:
         O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, qblocks=qb)
@@ -839,7 +862,9 @@ def run_extra_reference(args, metric, workload):
         # one seeded query block: (Speed3R: its routing by the oracle, then) the layer forward
         qb = np.array([np.random.default_rng(seed).integers(w.n_blocks)], dtype=np.int32)
         t0 = time.perf_counter()
-        if w.pooled_q:
+        if w.route == "mixture":
+            O.mixture(D, w.off, w.q, w.k, w.v, w.gates, w.n_blocks_x, qblocks=qb)
+        elif w.pooled_q:
             rows, _ = O.route_pooled(D, qc, kc, w.forced, qblocks=qb)
             idx = np.zeros((w.n_blocks, w.n_q_heads, w.top_k), dtype=np.int32)
             idx[qb] = rows

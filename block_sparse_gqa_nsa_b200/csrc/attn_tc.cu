@@ -105,6 +105,9 @@ struct TcSmem {
   int abort;
   int n_sel;
   int win_lo, win_hi;  // window band of the CTA's tokens, relative to the block start
+  // key rows of the compressed slot start at c_lo; with the self/cross mixture the compressed slot
+  // is the token range [c_lo, c_hi) and the selected slot the token range [s_lo, s_hi)
+  int c_lo, c_hi, s_lo, s_hi;
   int sel_start[kTcMaxSel];
   int sel_n[kTcMaxSel];
 };
@@ -140,6 +143,10 @@ struct TcParams {
   const int* n_ckeys_dev;
   // query blocks of a fixed size instead of `off` (dense passes over pooled queries or all tokens)
   int uniform_block;
+  // self/cross mixture (kModeMix): blocks [0, mix_bx) are stream x, the rest stream y; the
+  // compressed slot (gate 0) attends every token of the query's own stream and the selected slot
+  // (gate 1) every token of the other one, both read from the token K / V
+  int mix_bx;
   // streaming top-k of the compressed-branch logits (pooled-query routing, d = 64 only):
   // topk_idx [rows][topk_heads][topk_k]; blocks whose bit is set in forced_bits are skipped
   int32_t* topk_idx;
@@ -179,42 +186,52 @@ struct Chunks {
   }
 };
 
-// first key row (block-mean index or token index) and number of valid keys of chunk (br, local).
-// Selected blocks longer than 64 tokens are listed as several 64-key chunks; the window branch
-// covers the band of the CTA's tokens, [win_lo, win_hi] relative to the block start, in 64-key
-// chunks (one for blocks of at most 64 tokens).
-template <int D>
+// Kernel modes.  kModeShort: blocks of at most 64 tokens (a CTA's window band is its whole block,
+// one chunk from the block start).  kModeLong: blocks of up to 512 tokens (selected blocks take
+// several 64-key chunks, and the window band of a CTA may start inside the block and span several
+// chunks).  kModeMix: the self/cross mixture (the compressed slot is the query's own stream and the
+// selected slot the other stream, both token ranges in 64-key chunks; no window).
+enum : int { kModeShort = 0, kModeLong = 1, kModeMix = 2 };
+
+// first key row (block-mean index or token index) and number of valid keys of chunk (br, local)
+template <int D, int kMode>
 __device__ __forceinline__ void chunk_keys(const TcSmem<D>& S, const TcParams& p, int br, int local, int t0,
-                                           int n_ckeys, int& start, int& nvalid) {
+                                           int n_a, int n_ckeys, int& start, int& nvalid) {
   if (br == 0) {
-    start = local * 64;
-    nvalid = min(64, n_ckeys - start);
+    start = (kMode == kModeMix ? S.c_lo : 0) + local * 64;
+    nvalid = min(64, n_ckeys - local * 64);
   } else if (br == 1) {
-    if (p.route_all) {
+    if (kMode == kModeMix) {
+      start = S.s_lo + 64 * local;
+      nvalid = min(64, S.s_hi - start);
+    } else if (p.route_all) {
       start = p.off[local];
       nvalid = p.off[local + 1] - start;
     } else {
       start = S.sel_start[local];
       nvalid = S.sel_n[local];
     }
-  } else {
+  } else if (kMode == kModeLong) {
     start = t0 + S.win_lo + 64 * local;
     nvalid = min(64, S.win_hi + 1 - (S.win_lo + 64 * local));
+  } else {
+    start = t0;
+    nvalid = n_a;
   }
 }
 
-// Top-k over a row's buffered candidates (logits at val[i * 128], block ids at id[i * 128], in
-// arrival order, which is increasing block order).  The rank of entry i in the order (logit desc,
-// block asc) is the number of entries with a larger logit plus the earlier entries with an equal
-// one; ranks form a permutation of 0..n-1.
+// Top-k over a row's buffered candidates (logits at val[i * 128], key rows at id[i * 128]).  The
+// rank of entry i in the order (logit desc, row asc) is the number of entries with a larger logit
+// plus those with an equal logit and a lower row; ranks form a permutation of 0..n-1.
 constexpr int kMaxCand = 64;
 
 // exact rank from shared memory, ties included (the fallback when two logits are equal)
-__device__ __forceinline__ int cand_rank_exact(const float* val, int n, int i, float vi) {
+__device__ __forceinline__ int cand_rank_exact(const float* val, const int* id, int n, int i, float vi) {
   int r = 0;
+  const int ji = id[i * 128];
   for (int j = 0; j < n; ++j) {
     const float vj = val[j * 128];
-    r += (vj > vi || (vj == vi && j < i)) ? 1 : 0;
+    r += (vj > vi || (vj == vi && id[j * 128] < ji)) ? 1 : 0;
   }
   return r;
 }
@@ -274,7 +291,7 @@ __device__ __noinline__ KeepBest topk_keep_best(float* val, int* id, int n, int 
   uint64_t keep = 0;
   if (!cand_ranks_fast(val, n, [&](int i, int r) { keep |= (uint64_t)(r < k) << i; })) {
     keep = 0;
-    for (int i = 0; i < n; ++i) keep |= (uint64_t)(cand_rank_exact(val, n, i, val[i * 128]) < k) << i;
+    for (int i = 0; i < n; ++i) keep |= (uint64_t)(cand_rank_exact(val, id, n, i, val[i * 128]) < k) << i;
   }
   int m = 0;
   float lo = INFINITY;
@@ -289,23 +306,40 @@ __device__ __noinline__ KeepBest topk_keep_best(float* val, int* id, int n, int 
   return KeepBest{m, lo};
 }
 
-// Emit the row's k best in order (logit desc, block asc); a row with fewer than k candidates pads
+// A full buffer (k above kCand - 16, where keeping the k best would leave less room than one quarter
+// of a chunk can append): the new candidate (logit v, key row j) replaces the worst entry when it
+// ranks above it; returns the buffer's new worst logit, the gate for the next candidates.
+__device__ __noinline__ float topk_insert_full(float* val, int* id, int n, float v, int j) {
+  int w = 0;
+  for (int i = 1; i < n; ++i) {
+    const float vi = val[i * 128], vw = val[w * 128];
+    if (vi < vw || (vi == vw && id[i * 128] > id[w * 128])) w = i;
+  }
+  const float vw = val[w * 128];
+  if (v > vw || (v == vw && j < id[w * 128])) {
+    val[w * 128] = v;
+    id[w * 128] = j;
+  }
+  float lo = INFINITY;
+  for (int i = 0; i < n; ++i) lo = fminf(lo, val[i * 128]);
+  return lo;
+}
+
+// Emit the row's k best in order (logit desc, row asc); a row with fewer than k candidates pads
 // with -1.
 __device__ __noinline__ void topk_emit(const float* val, const int* id, int n, int k, int32_t* dst,
                                        const int32_t* ids) {
   auto put = [&](int r, int i) { dst[r] = ids != nullptr ? ids[id[i * 128]] : id[i * 128]; };
   if (!cand_ranks_fast(val, n, [&](int i, int r) { if (r < k) put(r, i); })) {
     for (int i = 0; i < n; ++i) {
-      const int r = cand_rank_exact(val, n, i, val[i * 128]);
+      const int r = cand_rank_exact(val, id, n, i, val[i * 128]);
       if (r < k) put(r, i);
     }
   }
   for (int r = n; r < k; ++r) dst[r] = -1;
 }
 
-// kLong: blocks may exceed 64 tokens (the window band of a CTA may then start inside the block and
-// span several chunks); without it a CTA's band is its whole block, one chunk from the block start.
-template <int D, bool kLong>
+template <int D, int kMode>
 __global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kCtasPerSm)
 nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
@@ -315,12 +349,21 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   const uint32_t raw = smem_u32(smem_raw);
   TcSmem<D>& S = *reinterpret_cast<TcSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid x = (query block * KV groups + group) * pairs + pair of 128-row tiles: the tile pairs and
-  // groups of one query block run side by side (they read the same selected blocks, whose K and V
-  // rows hold both groups' heads), and the query-block count is not bounded by grid y / z
-  const unsigned bg = blockIdx.x / (unsigned)p.n_pairs;
-  const int pair = (int)(blockIdx.x - bg * (unsigned)p.n_pairs);
-  const int a = (int)(bg / (unsigned)p.n_groups), g = (int)(bg - (unsigned)a * (unsigned)p.n_groups);
+  // grid (pair of 128-row tiles, KV group, query block): the tile pairs and groups of one query
+  // block run side by side (they read the same selected blocks, whose K and V rows hold both
+  // groups' heads).  Past 65535 query blocks the grid is one-dimensional in the same order,
+  // x = (query block * KV groups + group) * pairs + pair.
+  int pair, g, a;
+  if (gridDim.y * gridDim.z > 1) {
+    pair = blockIdx.x;
+    g = blockIdx.y;
+    a = blockIdx.z;
+  } else {
+    const unsigned bg = blockIdx.x / (unsigned)p.n_pairs;
+    pair = (int)(blockIdx.x - bg * (unsigned)p.n_pairs);
+    a = (int)(bg / (unsigned)p.n_groups);
+    g = (int)(bg - (unsigned)a * (unsigned)p.n_groups);
+  }
   const int t0 = p.uniform_block ? a * p.uniform_block : p.off[a];
   const int n_a = p.uniform_block ? min(p.uniform_block, p.N - t0) : p.off[a + 1] - t0;
   const int rows_total = n_a * p.G;
@@ -336,17 +379,33 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       for (int i = 0; i < p.n_forced + p.top_k && n < kTcMaxSel; ++i) {
         const int j = i < p.n_forced ? p.forced[i] : r[i - p.n_forced];
         if (j < 0 || j >= p.B) { raise_status(p.status, LSRM_ERR_BOUNDS); continue; }
-        // one 64-key chunk per 64 tokens of the block
-        for (int s0 = p.off[j]; s0 < p.off[j + 1] && n < kTcMaxSel; s0 += 64) {
-          S.sel_start[n] = s0;
-          S.sel_n[n] = min(64, p.off[j + 1] - s0);
+        if (kMode == kModeLong) {
+          // one 64-key chunk per 64 tokens of the block
+          for (int s0 = p.off[j]; s0 < p.off[j + 1] && n < kTcMaxSel; s0 += 64) {
+            S.sel_start[n] = s0;
+            S.sel_n[n] = min(64, p.off[j + 1] - s0);
+            ++n;
+          }
+        } else {
+          S.sel_start[n] = p.off[j];
+          S.sel_n[n] = p.off[j + 1] - p.off[j];
           ++n;
         }
       }
     }
     S.n_sel = n;
-    S.win_lo = kLong ? max(0, tile0 * tokens_per_tile - p.window / 2) : 0;
-    S.win_hi = kLong ? min(n_a - 1, min(n_a, (tile0 + 2) * tokens_per_tile) - 1 + p.window / 2 - 1) : n_a - 1;
+    if (kMode == kModeLong) {
+      S.win_lo = max(0, tile0 * tokens_per_tile - p.window / 2);
+      S.win_hi = min(n_a - 1, min(n_a, (tile0 + 2) * tokens_per_tile) - 1 + p.window / 2 - 1);
+    }
+    if (kMode == kModeMix) {
+      const int nx = p.off[p.mix_bx], nall = p.off[p.B];
+      const bool in_x = a < p.mix_bx;
+      S.c_lo = in_x ? 0 : nx;  // own stream
+      S.c_hi = in_x ? nx : nall;
+      S.s_lo = in_x ? nx : 0;  // the other stream (may be empty)
+      S.s_hi = in_x ? nall : nx;
+    }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&S.q_full[t], 1);
       mbar_init(&S.s_full[t], 1);
@@ -378,11 +437,16 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   const uint32_t tmem = S.tmem_base;
 
   Chunks cs;
-  const int n_ckeys = p.n_ckeys_dev != nullptr ? *p.n_ckeys_dev : p.n_ckeys;
+  const int n_ckeys = kMode == kModeMix              ? S.c_hi - S.c_lo
+                      : p.n_ckeys_dev != nullptr ? *p.n_ckeys_dev
+                                                 : p.n_ckeys;
   cs.n_cmp = (p.branches & TC_CMP) ? (n_ckeys + C::kKeys - 1) / C::kKeys : 0;
-  cs.n_slc = (p.branches & TC_SLC) ? (p.route_all ? p.B : S.n_sel) : 0;
+  cs.n_slc = (p.branches & TC_SLC) ? (kMode == kModeMix ? (S.s_hi - S.s_lo + 63) / 64 : p.route_all ? p.B : S.n_sel)
+                                   : 0;
   // the window band of this CTA's tokens in 64-key chunks (one for blocks of at most 64 tokens)
-  cs.n_win = ((p.branches & TC_WIN) && p.window > 0) ? (S.win_hi - S.win_lo + 64) / 64 : 0;
+  cs.n_win = ((p.branches & TC_WIN) && p.window > 0 && kMode != kModeMix)
+                 ? (kMode == kModeLong ? (S.win_hi - S.win_lo + 64) / 64 : 1)
+                 : 0;
   cs.total = cs.n_cmp + cs.n_slc + cs.n_win;
   volatile int* abort = &S.abort;
 
@@ -411,7 +475,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         if (c >= C::kStages && !mbar_wait(&S.kv_empty[st], ((c / C::kStages) + 1) & 1, abort, p.status)) break;
         int local, start, nvalid;
         const int br = cs.branch(c, local);
-        chunk_keys<D>(S, p, br, local, t0, n_ckeys, start, nvalid);
+        chunk_keys<D, kMode>(S, p, br, local, t0, n_a, n_ckeys, start, nvalid);
         mbar_arrive_expect_tx(&S.kv_full[st], 2 * C::kKVBytes);
         tma_load_3d(S.k[st], br == 0 ? &kcmap : &kmap, &S.kv_full[st], 0, g, start);
         tma_load_3d(S.v[st], br == 0 ? &vcmap : &vmap, &S.kv_full[st], 0, g, start);
@@ -604,8 +668,10 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     // non-forced logit (from the bound pass), so every key at or above the bound is a candidate and
     // no key below it can be among the k best (k keys at or above it exist).  With that bound a
     // row collects a few dozen candidates over the whole stream; should the buffer run short, the
-    // warp's rows keep their k best and the gate rises to the k-th of them.  The k best of the
-    // buffer are ranked at the end.
+    // warp's rows keep their k best and the gate rises to the k-th of them (for k above kCand - 16,
+    // where that would leave less room than a quarter chunk appends, a full buffer instead takes
+    // each new candidate in place of its worst entry).  The k best of the buffer are ranked at the
+    // end.
     const bool topk_on = (D == 64) && p.topk_idx != nullptr;
     float thr = -INFINITY;
     int key_base = 0;    // block id of key 0 of the current chunk
@@ -613,13 +679,6 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     int ncand = 0;       // this row's buffered candidates
     float* cval = acc;
     int* cid = &S.cand_id[t][0][row];
-    auto topk_append = [&](float sv, int j) {
-      if (sv > thr) {
-        cval[ncand * 128] = sv;
-        cid[ncand * 128] = key_base + j;
-        ++ncand;
-      }
-    };
     // exact ranking (see TcParams::rescore_q): every bf16-operand logit lies within err of the
     // fp32 logit of the means, err = 2^-7 * |q|_1 * max|k| (each operand rounded to bf16 moves a
     // product by at most 2^-9 of it; the factor leaves room for the fp32 sums).  A key among the
@@ -644,6 +703,25 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         const KeepBest kb = topk_keep_best(cval, cid, ncand, p.topk_k);
         ncand = kb.n;
         thr = exact ? kb.thr - err : kb.thr;
+      }
+    };
+    const bool big_k = topk_on && p.topk_k > C::kCand - 16;
+    bool rescored = false;  // a full buffer holds the fp32 logits of the means (exact ranking)
+    auto topk_append = [&](float sv, int j) {
+      if (sv > thr) {
+        if (ncand < C::kCand) {
+          cval[ncand * 128] = sv;
+          cid[ncand * 128] = key_base + j;
+          ++ncand;
+        } else {
+          if (exact && valid) {
+            if (!rescored) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
+            rescored = true;
+            sv = rescore_dot64(qrow, kbase + (size_t)(key_base + j) * kstride);
+          }
+          const float lo = topk_insert_full(cval, cid, ncand, sv, key_base + j);
+          thr = exact ? lo - err : lo;
+        }
       }
     };
     if (topk_on && p.topk_thr != nullptr && valid) {
@@ -746,7 +824,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 #pragma unroll
             for (int i = 0; i < 16; ++i) topk_append(sv[i], 16 * qd + i);
             // a quarter appends at most 16 candidates per row
-            if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_compact();
+            if (!big_k && __any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_compact();
           }
         }
       };
@@ -871,8 +949,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       int local, start;
       br = cs.branch(c, local);
       const bool first = cs.first_of_branch(c);
-      chunk_keys<D>(S, p, br, local, t0, n_ckeys, start, nv);
-      if (kLong && br == 2) {
+      chunk_keys<D, kMode>(S, p, br, local, t0, n_a, n_ckeys, start, nv);
+      if (kMode == kModeLong && br == 2) {
         const int shift = local == 0 ? S.win_lo : 64;  // the chunk starts this many keys further on
         wlo -= shift;
         whi -= shift;
@@ -960,6 +1038,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         for (int i = 0; i < D; ++i) p.obranch[orow * D + i] = 0.f;
       if (p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first] = -INFINITY;
     }
+    // the mixture's cross slot over an empty stream: no keys, a zero output and LSE -inf
+    if (kMode == kModeMix && cs.n_slc == 0 && valid && p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first + 1] = -INFINITY;
     if (ok && topk_on && valid) {
       if (exact) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
       topk_emit(cval, cid, ncand, p.topk_k, p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k, p.topk_ids);
@@ -993,7 +1073,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 // ---- host side ------------------------------------------------------------------------------------
 namespace {
 
-template <int D, bool kLong>
+template <int D, int kMode>
 lsrm_status launch_tc_dl(const lsrm_nsa_desc& d, const TcParams& p, const void* q, const void* k, const void* v,
                         const void* kc, const void* vc, long long kc_rows, cudaStream_t stream) {
   CUtensorMap qm, km, vm, kcm, vcm;
@@ -1008,7 +1088,7 @@ lsrm_status launch_tc_dl(const lsrm_nsa_desc& d, const TcParams& p, const void* 
     return LSRM_ERR_CUDA;
   if (!make_map(&vcm, vvc, D, d.n_kv_heads, vc ? kc_rows : d.n_tokens, 1, 64)) return LSRM_ERR_CUDA;
   const size_t smem = sizeof(TcSmem<D>) + 1024;
-  if (cudaFuncSetAttribute(nsa_attn_tc_kernel<D, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (cudaFuncSetAttribute(nsa_attn_tc_kernel<D, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LSRM_ERR_CUDA;
   const int tiles = (d.max_block_len * p.G + 127) / 128;
@@ -1016,18 +1096,21 @@ lsrm_status launch_tc_dl(const lsrm_nsa_desc& d, const TcParams& p, const void* 
   pp.n_pairs = (tiles + 1) / 2;
   pp.n_groups = d.n_kv_heads;
   const long long nx = (long long)d.n_blocks * d.n_kv_heads * pp.n_pairs;
-  if (nx > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
-  nsa_attn_tc_kernel<D, kLong><<<(unsigned)nx, kTcThreads, smem, stream>>>(qm, km, vm, kcm, vcm, pp);
+  if (nx > INT32_MAX || d.n_kv_heads > 65535) return LSRM_ERR_UNSUPPORTED;
+  const dim3 grid = d.n_blocks <= 65535 ? dim3((unsigned)pp.n_pairs, (unsigned)d.n_kv_heads, (unsigned)d.n_blocks)
+                                        : dim3((unsigned)nx, 1, 1);
+  nsa_attn_tc_kernel<D, kMode><<<grid, kTcThreads, smem, stream>>>(qm, km, vm, kcm, vcm, pp);
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 
 template <int D>
 lsrm_status launch_tc_d(const lsrm_nsa_desc& d, const TcParams& p, const void* q, const void* k, const void* v,
-                        const void* kc, const void* vc, long long kc_rows, cudaStream_t stream) {
-  // the window band of long blocks only exists in the layer passes (the dense passes use no window)
+                        const void* kc, const void* vc, long long kc_rows, cudaStream_t stream, bool mix = false) {
+  if (mix) return launch_tc_dl<D, kModeMix>(d, p, q, k, v, kc, vc, kc_rows, stream);
+  // long blocks only exist in the layer passes (the dense passes have fixed 256-row query groups)
   if (d.max_block_len > 64 && p.uniform_block == 0)
-    return launch_tc_dl<D, true>(d, p, q, k, v, kc, vc, kc_rows, stream);
-  return launch_tc_dl<D, false>(d, p, q, k, v, kc, vc, kc_rows, stream);
+    return launch_tc_dl<D, kModeLong>(d, p, q, k, v, kc, vc, kc_rows, stream);
+  return launch_tc_dl<D, kModeShort>(d, p, q, k, v, kc, vc, kc_rows, stream);
 }
 
 }  // namespace
@@ -1074,6 +1157,38 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
   return LSRM_ERR_UNSUPPORTED;
 }
 
+// Decoupled self/cross gated mixture over two token streams (blocks [0, bx) and [bx, B)): one
+// launch, the compressed slot over the query's own stream and the selected slot over the other,
+// gated by gates [N][Hq][2] = (self, cross) and summed in the epilogue.
+lsrm_status launch_mixture(const lsrm_nsa_desc& d, const int32_t* off, int32_t bx, const void* q, const void* k,
+                           const void* v, const void* gates, void* out, float* lse, uint32_t* status,
+                           cudaStream_t stream) {
+  const int G = d.n_q_heads / d.n_kv_heads;
+  if (128 % G != 0) return LSRM_ERR_UNSUPPORTED;
+  TcParams p{};
+  p.off = off;
+  p.gates = (const uint16_t*)gates;
+  p.out = (uint16_t*)out;
+  p.lse = lse;
+  p.status = status;
+  p.N = (int)d.n_tokens;
+  p.B = d.n_blocks;
+  p.Hq = d.n_q_heads;
+  p.Hkv = d.n_kv_heads;
+  p.G = G;
+  p.n_gates = 2;
+  p.branches = TC_CMP | TC_SLC;
+  p.lse_stride = 2;
+  p.lse_first = 0;
+  p.mix_bx = bx;
+  const float tau = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim);
+  p.scale_log2 = tau * 1.4426950408889634f;
+  // both slots read token rows: the compressed slot's tensor maps cover K and V
+  if (d.head_dim == 32) return launch_tc_d<32>(d, p, q, k, v, k, v, d.n_tokens, stream, true);
+  if (d.head_dim == 64) return launch_tc_d<64>(d, p, q, k, v, k, v, d.n_tokens, stream, true);
+  return LSRM_ERR_UNSUPPORTED;
+}
+
 // Dense multi-head attention of n_q query rows (q [n_q][H][D]) against n_ckeys rows of
 // (kc, vc) ([kc_rows][H][D]), in fixed groups of 256 query rows: the pooled-query compressed
 // branch (optionally with the streaming top-k that routes it) and the forced-block part of the
@@ -1089,7 +1204,7 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
                               float* topk_thr, uint32_t* status, cudaStream_t stream, const int32_t* topk_ids,
                               const float* rescore_q, const float* rescore_k, const uint32_t* rescore_kmax) {
-  if (topk_idx != nullptr && (D != 64 || topk_k < 1 || topk_k > 32 || forced_bits == nullptr))
+  if (topk_idx != nullptr && (D != 64 || topk_k < 1 || topk_k > TcCfg<64>::kCand || forced_bits == nullptr))
     return LSRM_ERR_UNSUPPORTED;
   if (n_q > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
   lsrm_nsa_desc d{};

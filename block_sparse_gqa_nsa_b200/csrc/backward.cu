@@ -138,11 +138,19 @@ bwd_query_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   const uint32_t raw = smem_u32(smem_raw);
   BqtSmem<D>& S = *reinterpret_cast<BqtSmem<D>*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid x = (query block * KV groups + group) * tiles + tile (the query-block count is not
-  // bounded by grid y / z; a block's groups and tiles run side by side)
-  const unsigned bg = blockIdx.x / (unsigned)p.q_tiles;
-  const int tile = (int)(blockIdx.x - bg * (unsigned)p.q_tiles);
-  const int a = (int)(bg / (unsigned)p.Hkv), g = (int)(bg - (unsigned)a * (unsigned)p.Hkv);
+  // grid (tile, KV group, query block), a block's groups and tiles side by side; past 65535
+  // query blocks one-dimensional in the same order, x = (query block * KV groups + group) * tiles + tile
+  int tile, g, a;
+  if (gridDim.y * gridDim.z > 1) {
+    tile = blockIdx.x;
+    g = blockIdx.y;
+    a = blockIdx.z;
+  } else {
+    const unsigned bg = blockIdx.x / (unsigned)p.q_tiles;
+    tile = (int)(blockIdx.x - bg * (unsigned)p.q_tiles);
+    a = (int)(bg / (unsigned)p.Hkv);
+    g = (int)(bg - (unsigned)a * (unsigned)p.Hkv);
+  }
   const int t0 = p.off[a], n_a = p.off[a + 1] - t0;
   const int rows_total = n_a * p.G;
   if (tile * 128 >= rows_total) return;
@@ -964,11 +972,13 @@ static lsrm_status launch_backward_d(const lsrm_nsa_desc& d, const BwdParams& p,
   if (cudaFuncSetAttribute(bwd_query_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
       cudaSuccess)
     return LSRM_ERR_CUDA;
-  if ((long long)tiles * d.n_kv_heads * d.n_blocks > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
+  const long long nx = (long long)tiles * d.n_kv_heads * d.n_blocks;
+  if (nx > INT32_MAX || d.n_kv_heads > 65535) return LSRM_ERR_UNSUPPORTED;
   BwdParams pq = p;
   pq.q_tiles = tiles;
-  bwd_query_tc_kernel<D><<<(unsigned)((long long)tiles * d.n_kv_heads * d.n_blocks), kBqtThreads, sm, s>>>(
-      qm, om, km, vm, kcm, vcm, pq);
+  const dim3 grid = d.n_blocks <= 65535 ? dim3((unsigned)tiles, (unsigned)d.n_kv_heads, (unsigned)d.n_blocks)
+                                        : dim3((unsigned)nx, 1, 1);
+  bwd_query_tc_kernel<D><<<grid, kBqtThreads, sm, s>>>(qm, om, km, vm, kcm, vcm, pq);
   CUtensorMap k64, v64, kc128, vc128, q64, o64;
   if (!make_map(&k64, p.k, D, d.n_kv_heads, d.n_tokens, 1, 64) || !make_map(&v64, p.v, D, d.n_kv_heads, d.n_tokens, 1, 64) ||
       !make_map(&kc128, p.kc, D, d.n_kv_heads, d.n_blocks, 1, 128) ||

@@ -13,6 +13,10 @@ lsrm_status launch_compress(const lsrm_nsa_desc& d, const int32_t* off, const vo
                             const int32_t* kv_row = nullptr);
 lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, const int32_t* coords, int32_t* cen,
                                    int32_t* idx, uint32_t* status, cudaStream_t s);
+lsrm_status launch_route_camera(const lsrm_nsa_desc& d, const int32_t* off, const int32_t* coords, int32_t n_vol,
+                                int32_t n_views, const int32_t* proj, int32_t tiles_x, int32_t tiles_y,
+                                int32_t tile_px, const int32_t* tile_block, int32_t radius, int32_t k_vol,
+                                int32_t* cen, int32_t* idx, uint32_t* status, cudaStream_t stream);
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
                                int32_t* idx, float* score, uint32_t* status, cudaStream_t s);
 lsrm_status launch_gate_combine(const lsrm_nsa_desc& d, const float* oc, const float* os, const float* ow,
@@ -21,6 +25,9 @@ lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* 
                         const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                         int route_all, int branches, void* out, float* obranch, float* lse, int lse_stride,
                         int lse_first, uint32_t* status, cudaStream_t stream, void* obr = nullptr);
+lsrm_status launch_mixture(const lsrm_nsa_desc& d, const int32_t* off, int32_t bx, const void* q, const void* k,
+                           const void* v, const void* gates, void* out, float* lse, uint32_t* status,
+                           cudaStream_t stream);
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,
                               float* lse, int32_t* topk_idx, int topk_k, const uint32_t* forced_bits,
@@ -38,7 +45,11 @@ lsrm_status launch_key_order(const lsrm_nsa_desc& d, const uint32_t* bits, int32
 lsrm_status launch_speed3r_routed(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
                                   const void* v, const void* gates, const int32_t* idx, const float* o_forced,
                                   const float* lse_forced, const float* o_blk, const float* lse_blk, void* out,
-                                  float* lse_out, uint32_t* status, cudaStream_t s);
+                                  float* lse_out, uint32_t* status, cudaStream_t s, void* obr);
+lsrm_status launch_speed3r_backward(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
+                                    const void* v, const void* gates, const int32_t* idx, const float* lse,
+                                    const void* obr, const void* dout, void* dq, void* dk, void* dv, void* dgates,
+                                    void* ws, uint32_t* status, cudaStream_t s);
 lsrm_status launch_backward(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
                             const void* kc, const void* vc, const void* gates, const int32_t* idx, int idx_heads,
                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* dgates,
@@ -83,7 +94,7 @@ lsrm_status pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, c
   float* o_blk = wsp<float>(ws, w.obranch);
   float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
   if (idx != nullptr) {
-    if (d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
+    if (d.top_k > 64) return LSRM_ERR_UNSUPPORTED;
     if (cudaMemsetAsync(bits, 0, ((size_t)d.n_blocks / 32 + 2) * 4, s) != cudaSuccess) return LSRM_ERR_CUDA;
     if (d.n_forced > 0) {
       // bits only (the prefix/gather outputs of this call are not needed here)
@@ -146,6 +157,24 @@ lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, 
   const Workspace w = workspace_layout(*desc);
   return launch_route_geometric(*desc, off, coords, wsp<int32_t>(ws, w.centroids), idx, status_of(ws),
                                 (cudaStream_t)stream);
+}
+
+lsrm_status lsrm_route_camera(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords,
+                              int32_t n_vol_blocks, int32_t n_views, const int32_t* proj, int32_t tiles_x,
+                              int32_t tiles_y, int32_t tile_px, const int32_t* tile_block, int32_t radius,
+                              int32_t k_vol, int32_t* idx, void* ws, void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (off == nullptr || coords == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
+  const int32_t B = desc->n_blocks, k_img = desc->top_k - k_vol;
+  if (n_vol_blocks < 0 || n_vol_blocks > B || k_vol < 0 || k_vol > n_vol_blocks || k_img < 0 ||
+      k_img > B - n_vol_blocks)
+    return LSRM_ERR_INVALID_ARG;
+  if (n_views < 0 || tiles_x < 1 || tiles_y < 1 || tile_px < 1 || radius < 0) return LSRM_ERR_INVALID_ARG;
+  if (n_views > 0 && (proj == nullptr || tile_block == nullptr)) return LSRM_ERR_INVALID_ARG;
+  const Workspace w = workspace_layout(*desc);
+  return launch_route_camera(*desc, off, coords, n_vol_blocks, n_views, proj, tiles_x, tiles_y, tile_px, tile_block,
+                             radius, k_vol, wsp<int32_t>(ws, w.centroids), idx, status_of(ws), (cudaStream_t)stream);
 }
 
 lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc,
@@ -228,6 +257,19 @@ lsrm_status lsrm_nsa_attend(const lsrm_nsa_desc* desc, const int32_t* off, const
                      lse_or_null, desc->n_gates, 0, status_of(ws), (cudaStream_t)stream);
 }
 
+lsrm_status lsrm_nsa_mixture(const lsrm_nsa_desc* desc, const int32_t* off, int32_t n_blocks_x, const void* q,
+                             const void* k, const void* v, const void* gates, void* out, float* lse_or_null, void* ws,
+                             void* stream) {
+  LSRM_TRY(check_desc(desc));
+  LSRM_TRY(check_ws(desc, ws));
+  if (desc->pooled_q || desc->n_gates != 2 || desc->n_forced != 0) return LSRM_ERR_INVALID_ARG;
+  if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || gates == nullptr || out == nullptr)
+    return LSRM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return LSRM_ERR_INVALID_ARG;
+  if (n_blocks_x < 0 || n_blocks_x > desc->n_blocks) return LSRM_ERR_INVALID_ARG;
+  return launch_mixture(*desc, off, n_blocks_x, q, k, v, gates, out, lse_or_null, status_of(ws), (cudaStream_t)stream);
+}
+
 lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
                              const void* v, const void* gates, const int32_t* coords_or_null, int32_t route_mode,
                              void* out, int32_t* idx_inout, float* lse_or_null, void* obr_or_null, void* ws,
@@ -237,7 +279,6 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
   if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || gates == nullptr || out == nullptr)
     return LSRM_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(obr_or_null, 16)) return LSRM_ERR_INVALID_ARG;
-  if (obr_or_null != nullptr && desc->pooled_q) return LSRM_ERR_UNSUPPORTED;  // no pooled-query backward
   const lsrm_nsa_desc& d = *desc;
   const Workspace w = workspace_layout(d);
   cudaStream_t s = (cudaStream_t)stream;
@@ -264,7 +305,7 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
     uint32_t* bits_part = wsp<uint32_t>(ws, w.fbits_part);
     LSRM_TRY(launch_key_order(d, wsp<uint32_t>(ws, w.fbits), row_of_block, block_of_row, bits_part, s));
     const bool route = route_mode == LSRM_ROUTE_SCORE;
-    if (route && d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
+    if (route && d.top_k > 64) return LSRM_ERR_UNSUPPORTED;
     // the routing ranks the fp32 logits of the means: their fp32 copies (keys in row order) and
     // the largest |pooled key| feed the exact ranking of the candidates
     float* qc32 = wsp<float>(ws, w.qc32);
@@ -285,7 +326,7 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
     LSRM_TRY(launch_attn_dense(d.head_dim, d.n_tokens, d.n_q_heads, q, wsp<void>(ws, w.kf), wsp<void>(ws, w.vf),
                                cap, 0, ftotal, tau_of(d), ofrc, lfrc, nullptr, 0, nullptr, nullptr, status_of(ws), s));
     return launch_speed3r_routed(d, off, q, k, v, gates, idx, ofrc, lfrc, o_blk, l_blk, out, lse_or_null,
-                                 status_of(ws), s);
+                                 status_of(ws), s, obr_or_null);
   }
 
   LSRM_TRY(launch_compress(d, off, nullptr, k, v, route_mode == LSRM_ROUTE_SCORE ? kc32 : nullptr, kc16, nullptr,
@@ -323,10 +364,18 @@ lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t* off, con
                               void* dgates, void* ws, void* stream) {
   LSRM_TRY(check_desc(desc));
   LSRM_TRY(check_ws(desc, ws));
-  if (desc->pooled_q) return LSRM_ERR_UNSUPPORTED;
   if (off == nullptr || q == nullptr || k == nullptr || v == nullptr || gates == nullptr || idx == nullptr ||
       lse == nullptr || dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || dgates == nullptr)
     return LSRM_ERR_INVALID_ARG;
+  if (desc->pooled_q) {
+    // Speed3R: per-head routing lists and the forward's saved branch outputs are required
+    if (idx_heads != desc->n_q_heads || obr_or_null == nullptr) return LSRM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(obr_or_null, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+      return LSRM_ERR_INVALID_ARG;
+    return launch_speed3r_backward(*desc, off, q, k, v, gates, idx, lse, obr_or_null, dout, dq, dk, dv, dgates, ws,
+                                   status_of(ws), (cudaStream_t)stream);
+  }
   if (idx_heads != 1 && idx_heads != desc->n_kv_heads) return LSRM_ERR_INVALID_ARG;
   if (!aligned(obr_or_null, 16) || !aligned(dout, 16)) return LSRM_ERR_INVALID_ARG;
   const Workspace w = workspace_layout(*desc);

@@ -81,6 +81,41 @@ inline BwdWs bwd_layout(const lsrm_nsa_desc& d, int idx_heads) {
   return w;
 }
 
+// backward scratch of the pooled-query (Speed3R) layer: the pooled branch's upstream gradient
+// (bf16, for the tensor cores), its LSE (log2 units) and Delta per (block, head) as float2; the pooled
+// gradients dQbar, dKbar, dVbar (fp32); per (token, head) the selected branch's LSE (log2 units) and
+// Delta as float2 and its upstream gradient g_slc dO (bf16); the forced part of dq (fp32); dK, dV of
+// the packed forced tokens (fp32) and each packed token's (token, block); the inverse routing lists
+// per (block, head)
+struct PooledBwdWs {
+  size_t gbar16, rowcb, dqbar, dkbar, dvbar, rowc, dos16, dqf, dkf, dvf, fmap;
+  size_t inv_count, inv_cursor, inv_start, inv_list, total;
+};
+inline PooledBwdWs pooled_bwd_layout(const lsrm_nsa_desc& d) {
+  PooledBwdWs w{};
+  size_t o = 0;
+  const size_t N = (size_t)d.n_tokens, B = (size_t)d.n_blocks, H = (size_t)d.n_q_heads, D = (size_t)d.head_dim;
+  const size_t nf_tok = (size_t)(d.n_forced > 0 ? d.n_forced : 0) * (size_t)d.max_block_len;
+  const size_t nl = B * H, K = (size_t)(d.top_k > 0 ? d.top_k : 0);
+  w.gbar16 = o;     o = align256(o + B * H * D * 2);
+  w.rowcb = o;      o = align256(o + B * H * 8);
+  w.dqbar = o;      o = align256(o + B * H * D * 4);
+  w.dkbar = o;      o = align256(o + B * H * D * 4);
+  w.dvbar = o;      o = align256(o + B * H * D * 4);
+  w.rowc = o;       o = align256(o + N * H * 8);
+  w.dos16 = o;      o = align256(o + N * H * D * 2);
+  w.dqf = o;        o = align256(o + N * H * D * 4);
+  w.dkf = o;        o = align256(o + nf_tok * H * D * 4);
+  w.dvf = o;        o = align256(o + nf_tok * H * D * 4);
+  w.fmap = o;       o = align256(o + nf_tok * 8);
+  w.inv_count = o;  o = align256(o + nl * 4);
+  w.inv_cursor = o; o = align256(o + nl * 4);
+  w.inv_start = o;  o = align256(o + (nl + 1) * 4);
+  w.inv_list = o;   o = align256(o + nl * K * 4);
+  w.total = o;
+  return w;
+}
+
 inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   Workspace w{};
   size_t o = 0;
@@ -101,7 +136,8 @@ inline Workspace workspace_layout(const lsrm_nsa_desc& d) {
   // pooled compressed-branch output [B][Hq][d] fp32 (Speed3R) + its LSE [B][Hq]
   w.obranch = o;   o = align256(o + (d.pooled_q ? B * Hq * (D + 1) * 4 : 0));
   // backward scratch, sized for per-group routing lists (the larger case)
-  w.bwd = o;       o = align256(o + (d.pooled_q ? 0 : bwd_layout(d, d.n_kv_heads > 0 ? d.n_kv_heads : 1).total));
+  w.bwd = o;       o = align256(o + (d.pooled_q ? pooled_bwd_layout(d).total
+                                                : bwd_layout(d, d.n_kv_heads > 0 ? d.n_kv_heads : 1).total));
   const size_t nf = d.pooled_q ? (size_t)(d.n_forced > 0 ? d.n_forced : 0) : 0;
   const size_t nf_tok = nf * (size_t)d.max_block_len;
   w.fbits = o;     o = align256(o + (d.pooled_q ? (B / 32 + 2) * 4 : 0));

@@ -189,6 +189,182 @@ lsrm_status launch_route_geometric(const lsrm_nsa_desc& d, const int32_t* off, c
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 
+// ---- camera-projection routing ------------------------------------------------------------------
+// LSRM page, 方法, 3D-aware routing paragraph: the query point (the query block's centroid) is
+// projected into every view; the image blocks of the tiles near the projected tile are the
+// candidates, ranked by the smallest squared distance from any of their tokens to the query point;
+// volume blocks are ranked by centroid distance.  One CTA per query block:
+//   1. k_vol rounds of "best volume block strictly after the previous winner" by (centroid
+//      distance, id);
+//   2. one slot per (view, neighbour tile): the projection h = P [c; 1] in int64, pixel =
+//      floor(h0 / h2), floor(h1 / h2) for h2 > 0, tile = floor(pixel / tile_px); the slot holds the
+//      tile's block (or -1); a bitmap over image blocks marks the candidates (a block reached twice
+//      keeps one slot);
+//   3. one warp per slot: the smallest token distance;
+//   4. k_img rounds over the slots by (token distance, id), and, once they run out, over the
+//      image blocks outside the bitmap by (centroid distance, id).
+// Every distance is exact int64, so the result is bit-exact.
+constexpr int kCamMaxSlots = 4096;
+
+__device__ __forceinline__ DistKey block_min_key(DistKey best, DistKey* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const DistKey other = shfl_key(best, o, true);
+    if (key_less(other, best)) best = other;
+  }
+  if (lane == 0) s_warp[warp] = best;
+  __syncthreads();
+  DistKey b = s_warp[0];
+  for (int w = 1; w < kRouteThreads / 32; ++w)
+    if (key_less(s_warp[w], b)) b = s_warp[w];
+  __syncthreads();  // s_warp is reused by the next call
+  return b;
+}
+
+__device__ __forceinline__ long long floor_div_ll(long long a, long long b) {  // b > 0
+  long long q = a / b;
+  if ((a % b != 0) && (a < 0)) --q;
+  return q;
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+camera_route_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ coords,
+                    const int32_t* __restrict__ cen, int32_t B, int32_t n_vol, int32_t n_views,
+                    const int32_t* __restrict__ proj, int32_t tiles_x, int32_t tiles_y, int32_t tile_px,
+                    const int32_t* __restrict__ tile_block, int32_t radius, int32_t k_vol, int32_t k_img,
+                    int32_t* __restrict__ idx, uint32_t* status) {
+  extern __shared__ __align__(16) unsigned char cam_smem[];
+  __shared__ DistKey s_warp[kRouteThreads / 32];
+  const int side = 2 * radius + 1, per_view = side * side;
+  const int n_slots = n_views * per_view;
+  const int n_img = B - n_vol;
+  long long* s_d = reinterpret_cast<long long*>(cam_smem);
+  int32_t* s_blk = reinterpret_cast<int32_t*>(s_d + n_slots);
+  uint32_t* s_bits = reinterpret_cast<uint32_t*>(s_blk + n_slots);
+  const int n_words = (n_img + 31) / 32;
+  const int a = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K = k_vol + k_img;
+  const long long ax = cen[a * 3 + 0], ay = cen[a * 3 + 1], az = cen[a * 3 + 2];
+  auto cdist = [&](int j) {
+    const long long dx = cen[j * 3 + 0] - ax, dy = cen[j * 3 + 1] - ay, dz = cen[j * 3 + 2] - az;
+    return dx * dx + dy * dy + dz * dz;
+  };
+  const DistKey none{LLONG_MAX, INT_MAX};
+
+  // 1. volume blocks by centroid distance
+  DistKey last{-1, -1};
+  for (int r = 0; r < k_vol; ++r) {
+    DistKey best = none;
+    for (int j = tid; j < n_vol; j += kRouteThreads) {
+      const DistKey c{cdist(j), j};
+      if (key_less(last, c) && key_less(c, best)) best = c;
+    }
+    last = block_min_key(best, s_warp);
+    if (tid == 0) idx[(size_t)a * K + r] = last.j;
+  }
+  if (k_img == 0) return;
+
+  // 2. candidate slots
+  for (int i = tid; i < n_words; i += kRouteThreads) s_bits[i] = 0u;
+  __syncthreads();
+  for (int i = tid; i < n_slots; i += kRouteThreads) {
+    const int v = i / per_view, e = i - v * per_view;
+    const int32_t* P = proj + (size_t)v * 12;
+    long long h[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+      h[r] = (long long)P[4 * r] * ax + (long long)P[4 * r + 1] * ay + (long long)P[4 * r + 2] * az + P[4 * r + 3];
+    int b = -1;
+    if (h[2] > 0) {
+      const long long tx = floor_div_ll(floor_div_ll(h[0], h[2]), tile_px) + (e % side) - radius;
+      const long long ty = floor_div_ll(floor_div_ll(h[1], h[2]), tile_px) + (e / side) - radius;
+      if (tx >= 0 && ty >= 0 && tx < tiles_x && ty < tiles_y) {
+        b = tile_block[((size_t)v * tiles_y + ty) * tiles_x + tx];
+        if (b >= B || (b >= 0 && b < n_vol)) {
+          raise_status(status, LSRM_ERR_BOUNDS);
+          b = -1;
+        } else if (b >= 0) {
+          const uint32_t bit = 1u << ((b - n_vol) & 31);
+          if (atomicOr(&s_bits[(b - n_vol) >> 5], bit) & bit) b = -1;  // reached before: one slot
+        }
+      }
+    }
+    s_blk[i] = b;
+  }
+  __syncthreads();
+
+  // 3. smallest token distance of each candidate (one warp per slot)
+  for (int i = warp; i < n_slots; i += kRouteThreads / 32) {
+    const int b = s_blk[i];
+    if (b < 0) continue;
+    long long m = LLONG_MAX;
+    for (int t = off[b] + lane; t < off[b + 1]; t += 32) {
+      const long long dx = coords[(size_t)t * 3] - ax, dy = coords[(size_t)t * 3 + 1] - ay,
+                      dz = coords[(size_t)t * 3 + 2] - az;
+      m = min(m, dx * dx + dy * dy + dz * dz);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = min(m, (long long)__shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_d[i] = m;
+  }
+  __syncthreads();
+
+  // 4. image blocks: the candidates, then the fill
+  last = DistKey{-1, -1};
+  bool fill = false;
+  for (int r = 0; r < k_img; ++r) {
+    DistKey best = none;
+    if (!fill) {
+      for (int i = tid; i < n_slots; i += kRouteThreads) {
+        const int b = s_blk[i];
+        if (b < 0) continue;
+        const DistKey c{s_d[i], b};
+        if (key_less(last, c) && key_less(c, best)) best = c;
+      }
+      best = block_min_key(best, s_warp);
+      if (best.j == INT_MAX) {  // no candidate left: the fill starts from the beginning
+        fill = true;
+        last = DistKey{-1, -1};
+      }
+    }
+    if (fill) {
+      best = none;
+      for (int j = n_vol + tid; j < B; j += kRouteThreads) {
+        if ((s_bits[(j - n_vol) >> 5] >> ((j - n_vol) & 31)) & 1u) continue;
+        const DistKey c{cdist(j), j};
+        if (key_less(last, c) && key_less(c, best)) best = c;
+      }
+      best = block_min_key(best, s_warp);
+    }
+    last = best;
+    if (tid == 0) idx[(size_t)a * K + k_vol + r] = best.j;
+  }
+}
+
+size_t camera_route_smem(int B, int n_vol, int n_slots) {
+  return (size_t)n_slots * (sizeof(long long) + sizeof(int32_t)) + (size_t)((B - n_vol + 31) / 32) * 4;
+}
+
+lsrm_status launch_route_camera(const lsrm_nsa_desc& d, const int32_t* off, const int32_t* coords, int32_t n_vol,
+                                int32_t n_views, const int32_t* proj, int32_t tiles_x, int32_t tiles_y,
+                                int32_t tile_px, const int32_t* tile_block, int32_t radius, int32_t k_vol,
+                                int32_t* cen, int32_t* idx, uint32_t* status, cudaStream_t stream) {
+  const int B = d.n_blocks;
+  const long long side = 2LL * radius + 1;
+  const long long n_slots = (long long)n_views * side * side;
+  if (n_slots > kCamMaxSlots) return LSRM_ERR_UNSUPPORTED;
+  const size_t smem = camera_route_smem(B, n_vol, (int)n_slots);
+  if (smem > 200 * 1024) return LSRM_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(camera_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return LSRM_ERR_CUDA;
+  centroid_kernel<<<(B * 32 + 255) / 256, 256, 0, stream>>>(off, coords, B, cen, status);
+  camera_route_kernel<<<B, kRouteThreads, smem, stream>>>(off, coords, cen, B, n_vol, n_views, proj, tiles_x, tiles_y,
+                                                          tile_px, tile_block, radius, k_vol, d.top_k - k_vol, idx,
+                                                          status);
+  return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
+}
+
 // ---- score routing -------------------------------------------------------------------------------
 // One CTA per (query block a, KV group g), fp32 throughout, one thread per query row (the row's q
 // in registers; the compressed keys staged in shared memory in chunks of kScoreChunk and read

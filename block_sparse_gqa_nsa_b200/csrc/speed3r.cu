@@ -6,7 +6,7 @@
 // computed in two parts whose softmaxes are merged exactly through their log-sum-exps:
 //   forced part: dense attention of every token against the forced tokens, gathered once
 //     into a contiguous [n_f][H][d] copy (tcgen05 kernel, launch_attn_dense);
-//   routed part: here, one warp per (a, h), 16 query rows x (routed tokens) with mma.sync
+//   routed part: here, one warp per (a, h) and up to 64 routed blocks, 16 query rows x (routed tokens) with mma.sync
 //     m16n8k16 (the routed key set of (a, h) is shared by at most 16 rows, which is exactly
 //     one MMA row tile).  Its epilogue merges in the forced part, adds the compressed branch
 //     (pooled query, one output per block) and applies the two gates.
@@ -80,6 +80,7 @@ struct RoutedParams {
   const float* lse_blk;     // [B][H]
   uint16_t* out;            // [N][H][64]
   float* lse_out;           // [N][H][2] (cmp, slc), optional
+  uint16_t* obr;            // [N][H][2][64] bf16 branch outputs (cmp, slc) for the backward, optional
   uint32_t* status;
   int B, H, top_k;
   float scale_log2;
@@ -104,25 +105,36 @@ __global__ void __launch_bounds__(kRtWarps * 32) speed3r_routed_kernel(const Rou
   const int t0 = p.off[a], n_a = min(16, p.off[a + 1] - t0);
   const int H = p.H;
 
-  // routed blocks of (a, h): lane i holds block i; warp prefix of their token counts
-  int my_start = 0, my_n = 0;
-  if (lane < p.top_k) {
-    const int j = p.idx[((size_t)a * H + h) * p.top_k + lane];
-    if (j >= 0 && j < p.B) {
-      my_start = p.off[j];
-      my_n = p.off[j + 1] - my_start;
-    } else if (j >= p.B) {
-      raise_status(p.status, LSRM_ERR_BOUNDS);
+  // routed blocks of (a, h): lane i holds blocks i and 32 + i (list entries in order); exclusive
+  // prefix of their token counts over the whole list
+  int my_start[2] = {0, 0}, my_n[2] = {0, 0}, excl[2];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int e = 32 * half + lane;
+    if (e < p.top_k) {
+      const int j = p.idx[((size_t)a * H + h) * p.top_k + e];
+      if (j >= 0 && j < p.B) {
+        my_start[half] = p.off[j];
+        my_n[half] = p.off[j + 1] - my_start[half];
+      } else if (j >= p.B) {
+        raise_status(p.status, LSRM_ERR_BOUNDS);
+      }
     }
   }
-  int incl = my_n;
+  int base = 0;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+  for (int half = 0; half < 2; ++half) {
+    int incl = my_n[half];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    excl[half] = base + incl - my_n[half];
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  const int excl = incl - my_n;
-  const int nk = __shfl_sync(0xffffffffu, incl, 31);
+  const int nk = base;
+  const int second0 = __shfl_sync(0xffffffffu, excl[1], 0);  // first key position of entry 32
 
   // Q rows of the block (zero beyond n_a)
   unsigned char* qs = reinterpret_cast<unsigned char*>(S.q[warp]);
@@ -160,14 +172,20 @@ __global__ void __launch_bounds__(kRtWarps * 32) speed3r_routed_kernel(const Rou
       const int kr = e >> 3, ch = e & 7;
       const int pos = c * kRtKeys + kr;
       const bool ok = pos < nk;
-      // largest lane whose exclusive prefix <= pos (fixed five steps: every lane joins each shuffle)
+      // the list entry holding position pos: the half first (entries 32.. start at second0), then
+      // the largest lane of that half whose exclusive prefix <= pos (five fixed steps; every lane
+      // joins each shuffle, reading both halves and keeping its own)
+      const bool hi = p.top_k > 32 && pos >= second0;
       int lo = 0;
 #pragma unroll
       for (int step = 16; step > 0; step >>= 1) {
-        const int pm = __shfl_sync(0xffffffffu, excl, lo + step);
-        if (pm <= pos) lo += step;
+        const int pm0 = __shfl_sync(0xffffffffu, excl[0], lo + step);
+        const int pm1 = __shfl_sync(0xffffffffu, excl[1], lo + step);
+        if ((hi ? pm1 : pm0) <= pos) lo += step;
       }
-      const int st = __shfl_sync(0xffffffffu, my_start, lo), pre = __shfl_sync(0xffffffffu, excl, lo);
+      const int st0 = __shfl_sync(0xffffffffu, my_start[0], lo), pre0 = __shfl_sync(0xffffffffu, excl[0], lo);
+      const int st1 = __shfl_sync(0xffffffffu, my_start[1], lo), pre1 = __shfl_sync(0xffffffffu, excl[1], lo);
+      const int st = hi ? st1 : st0, pre = hi ? pre1 : pre0;
       const long long u = ok ? (long long)st + (pos - pre) : t0;
       const size_t base = ((size_t)u * H + h) * kRtD + ch * 8;
       cp_async16(ks + rt_swz(kr, ch), p.k + base, ok);
@@ -273,6 +291,10 @@ __global__ void __launch_bounds__(kRtWarps * 32) speed3r_routed_kernel(const Rou
       const float s0 = cf * of.x + cr * o[n][2 * i], s1 = cf * of.y + cr * o[n][2 * i + 1];
       *reinterpret_cast<uint32_t*>(p.out + row * kRtD + col) =
           pack_bf16x2(g_cmp * oc.x + g_slc * s0, g_cmp * oc.y + g_slc * s1);
+      if (p.obr != nullptr) {
+        *reinterpret_cast<uint32_t*>(p.obr + (row * 2 + 0) * kRtD + col) = pack_bf16x2(oc.x, oc.y);
+        *reinterpret_cast<uint32_t*>(p.obr + (row * 2 + 1) * kRtD + col) = pack_bf16x2(s0, s1);
+      }
     }
     if (p.lse_out != nullptr && cq == 0) {
       p.lse_out[row * 2 + 0] = lse_c;
@@ -378,8 +400,8 @@ lsrm_status launch_key_order(const lsrm_nsa_desc& d, const uint32_t* bits, int32
 lsrm_status launch_speed3r_routed(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k,
                                   const void* v, const void* gates, const int32_t* idx, const float* o_forced,
                                   const float* lse_forced, const float* o_blk, const float* lse_blk, void* out,
-                                  float* lse_out, uint32_t* status, cudaStream_t s) {
-  if (d.head_dim != kRtD || d.max_block_len > 16 || d.top_k > 32) return LSRM_ERR_UNSUPPORTED;
+                                  float* lse_out, uint32_t* status, cudaStream_t s, void* obr) {
+  if (d.head_dim != kRtD || d.max_block_len > 16 || d.top_k > 64) return LSRM_ERR_UNSUPPORTED;
   RoutedParams p{};
   p.off = off;
   p.q = (const uint16_t*)q;
@@ -393,6 +415,7 @@ lsrm_status launch_speed3r_routed(const lsrm_nsa_desc& d, const int32_t* off, co
   p.lse_blk = lse_blk;
   p.out = (uint16_t*)out;
   p.lse_out = lse_out;
+  p.obr = (uint16_t*)obr;
   p.status = status;
   p.B = d.n_blocks;
   p.H = d.n_q_heads;

@@ -27,8 +27,8 @@ ROUTE_GIVEN, ROUTE_SCORE, ROUTE_GEOMETRIC, ROUTE_ALL = 0, 1, 2, 3
 
 # every symbol include/lsrm_nsa.h declares
 EXPORTS = ("lsrm_nsa_workspace_size", "lsrm_nsa_workspace_init", "lsrm_nsa_compress", "lsrm_route_score_topk",
-           "lsrm_route_geometric", "lsrm_route_geometric_noalloc", "lsrm_route_pooled_topk", "lsrm_nsa_cmp_attn", "lsrm_nsa_select_attn",
-           "lsrm_nsa_window_attn", "lsrm_nsa_gate_combine", "lsrm_nsa_attend", "lsrm_nsa_forward", "lsrm_nsa_backward",
+           "lsrm_route_geometric", "lsrm_route_geometric_noalloc", "lsrm_route_camera", "lsrm_route_pooled_topk", "lsrm_nsa_cmp_attn", "lsrm_nsa_select_attn",
+           "lsrm_nsa_window_attn", "lsrm_nsa_gate_combine", "lsrm_nsa_attend", "lsrm_nsa_mixture", "lsrm_nsa_forward", "lsrm_nsa_backward",
            "lsrm_nsa_last_device_status", "lsrm_status_string", "lsrm_diag_exp2_poly")
 
 
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsrm_nsa_window_attn": ([D, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_gate_combine": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_attend": ([D, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp], ctypes.c_int),
+        "lsrm_nsa_mixture": ([D, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "lsrm_route_camera": ([D, vp, vp, i32, i32, vp, i32, i32, i32, vp, i32, i32, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_forward": ([D, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_backward": ([D, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsrm_nsa_last_device_status": ([vp, vp], ctypes.c_int),
@@ -230,6 +232,32 @@ def lsrm_nsa_attend(desc, off, q, k, v, kc, vc, gates, idx, idx_heads, route_all
         _check(t, dt, n)
     _call("lsrm_nsa_attend", ctypes.byref(desc), _ptr(off), _ptr(q), _ptr(k), _ptr(v), _ptr(kc), _ptr(vc),
           _ptr(gates), _ptr(idx), int(idx_heads), int(route_all), _ptr(out), _ptr(lse), _ptr(ws), _stream(stream))
+
+
+def lsrm_route_camera(desc, off, coords, n_vol_blocks, proj, tile_block, tile_px, radius, k_vol, idx, ws,
+                      stream=None):
+    """Camera-projection routing: proj int32 [V][3][4], tile_block int32 [V][tiles_y][tiles_x]
+    (device); idx int32 [B][top_k] = k_vol volume blocks, then top_k - k_vol image blocks."""
+    for t, n, dt in ((off, "off", torch.int32), (coords, "coords", torch.int32), (proj, "proj", torch.int32),
+                     (tile_block, "tile_block", torch.int32), (idx, "idx", torch.int32)):
+        _check(t, dt, n)
+    V, ty, tx = tile_block.shape
+    if tuple(proj.shape) != (V, 3, 4):
+        raise ValueError("proj: expected [views][3][4]")
+    _call("lsrm_route_camera", ctypes.byref(desc), _ptr(off), _ptr(coords), int(n_vol_blocks), int(V), _ptr(proj),
+          int(tx), int(ty), int(tile_px), _ptr(tile_block), int(radius), int(k_vol), _ptr(idx), _ptr(ws),
+          _stream(stream))
+
+
+def lsrm_nsa_mixture(desc, off, n_blocks_x, q, k, v, gates, out, lse=None, ws=None, stream=None):
+    """Self/cross gated mixture: blocks [0, n_blocks_x) are one stream, the rest the other;
+    gates [N][Hq][2] = (self, cross); lse (optional) fp32 [N][Hq][2]."""
+    for t, n, dt in ((off, "off", torch.int32), (q, "q", torch.bfloat16), (k, "k", torch.bfloat16),
+                     (v, "v", torch.bfloat16), (gates, "gates", torch.bfloat16), (out, "out", torch.bfloat16),
+                     (lse, "lse", torch.float32)):
+        _check(t, dt, n)
+    _call("lsrm_nsa_mixture", ctypes.byref(desc), _ptr(off), int(n_blocks_x), _ptr(q), _ptr(k), _ptr(v),
+          _ptr(gates), _ptr(out), _ptr(lse), _ptr(ws), _stream(stream))
 
 
 def lsrm_nsa_forward(desc, off, q, k, v, gates, coords, route_mode, out, idx=None, lse=None, ws=None, stream=None,

@@ -123,6 +123,39 @@ LSRM_API lsrm_status lsrm_route_score_topk(const lsrm_nsa_desc* desc, const int3
 LSRM_API lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords,
                                  int32_t* idx, void* ws, void* stream);
 
+/* Camera-projection routing (LSRM page, 方法, 3D-aware routing paragraph: for
+ * image blocks the query point is projected into every input view, the view's
+ * nearby image blocks are retrieved and ranked by their smallest 3D distance to
+ * the query point; volume blocks are ranked by the distance between centres).
+ * The query point of block a is its centroid c_a (as lsrm_route_geometric).
+ * Blocks [0, n_vol_blocks) are volume blocks, the rest image blocks.
+ *   volume part: the k_vol volume blocks nearest to c_a by centroid distance,
+ *     ties to the lower id;
+ *   image part (k_img = top_k - k_vol): for each view v, h = proj[v] [c_a; 1]
+ *     (int64); if h2 > 0 the projected tile is (floor(floor(h0/h2) / tile_px),
+ *     floor(floor(h1/h2) / tile_px)) (x = column, y = row) and the blocks
+ *     tile_block[v][y'][x'] of the tiles within Chebyshev distance `radius` of
+ *     it inside the tiles_x x tiles_y grid are candidates (-1 entries hold no
+ *     block); candidates are ranked by min over their tokens of the squared
+ *     distance to c_a, ties to the lower id.  When fewer than k_img candidates
+ *     exist, the remaining image blocks fill the list by centroid distance.
+ * idx (device, int32 [B][top_k]) gets the volume part then the image part, each
+ * in rank order; it serves as the shared index list (idx_heads = 1) of the
+ * selected branch.  proj (device, int32 [n_views][3][4], any common scale per
+ * view: only ratios matter) and tile_block (device, int32
+ * [n_views][tiles_y][tiles_x]) are caller-owned; tile_block entries must be
+ * image block ids or -1 (others raise LSRM_ERR_BOUNDS in the device status and
+ * are skipped).  Errors: LSRM_ERR_INVALID_ARG for counts outside their ranges
+ * (k_vol > n_vol_blocks, k_img > B - n_vol_blocks, tile_px < 1, radius < 0);
+ * LSRM_ERR_UNSUPPORTED for more than 4096 (view, tile) neighbourhood slots
+ * or more image blocks than the per-CTA bitmap holds (over a million).
+ * Coordinates beyond +-2^29 raise LSRM_ERR_BOUNDS. */
+LSRM_API lsrm_status lsrm_route_camera(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords,
+                                       int32_t n_vol_blocks, int32_t n_views, const int32_t* proj,
+                                       int32_t tiles_x, int32_t tiles_y, int32_t tile_px,
+                                       const int32_t* tile_block, int32_t radius, int32_t k_vol, int32_t* idx,
+                                       void* ws, void* stream);
+
 /* Geometric routing that allocates nothing and takes no workspace, for callers that may
  * not allocate device memory at call time and have none to lend (for example a plugin in
  * a host framework whose memory pool owns the whole GPU, or a loop whose policy forbids
@@ -152,7 +185,9 @@ LSRM_API lsrm_status lsrm_route_geometric_noalloc(const lsrm_nsa_desc* desc, con
  * that of the fp32 pooled means themselves: candidates are gathered from the bf16
  * logits with a gate widened by a bound on their error (2^-7 |qc32|_1 max|kc32|)
  * and ranked by fp32 dot products of the means; without them it is the ranking of
- * the bf16 operands, products accumulated in fp32.  idx is int32 [B][Hq][top_k]. */
+ * the bf16 operands, products accumulated in fp32.  idx is int32 [B][Hq][top_k]
+ * (top_k at most 64, else LSRM_ERR_UNSUPPORTED; a row with fewer eligible blocks
+ * pads with -1). */
 LSRM_API lsrm_status lsrm_route_pooled_topk(const lsrm_nsa_desc* desc, const void* qc, const void* kc,
                                    const float* qc32_or_null, const float* kc32_or_null, int32_t* idx,
                                    void* ws, void* stream);
@@ -196,13 +231,36 @@ LSRM_API lsrm_status lsrm_nsa_attend(const lsrm_nsa_desc* desc, const int32_t* o
                                      const int32_t* idx, int32_t idx_heads, int32_t route_all, void* out,
                                      float* lse_or_null, void* ws, void* stream);
 
+/* Decoupled self/cross gated mixture (LSRM page, 方法: the dense transformer
+ * blocks' gated cross-attention equations, o^x = w^{x-self} CrossAttn(x, x) +
+ * w^{x-cross} CrossAttn(x, y) and o^y likewise with x and y swapped).  The
+ * concatenated tokens hold two streams: blocks [0, n_blocks_x) are x (volume
+ * tokens) and blocks [n_blocks_x, B) are y (image tokens).  For a token t of one
+ * stream and head h (KV group g = h / (Hq/Hkv)):
+ *   out[t,h] = gates[t,h,0] * softmax-attention of q[t,h] over every token of
+ *              its own stream + gates[t,h,1] * the same over every token of the
+ *              other stream,
+ * one kernel launch (both attentions and the gated sum; an empty other stream
+ * contributes 0).  q [N][Hq][d], k/v [N][Hkv][d], gates [N][Hq][2] (self,
+ * cross), out [N][Hq][d], all bf16, 16-byte aligned; lse_or_null receives fp32
+ * [N][Hq][2] (natural log; -inf for an empty stream).  desc: n_gates = 2,
+ * pooled_q = 0, n_forced = 0; top_k and window are not used (top_k must still be
+ * valid).  Blocks of any length up to 512 tokens.  Errors: LSRM_ERR_INVALID_ARG
+ * for a bad descriptor, pointer, alignment or n_blocks_x outside [0, B];
+ * LSRM_ERR_UNSUPPORTED when 128 is not a multiple of Hq/Hkv.  The gates are
+ * inputs: the Sigmoid(Linear) that makes them is a trained layer. */
+LSRM_API lsrm_status lsrm_nsa_mixture(const lsrm_nsa_desc* desc, const int32_t* off, int32_t n_blocks_x,
+                                      const void* q, const void* k, const void* v, const void* gates, void* out,
+                                      float* lse_or_null, void* ws, void* stream);
+
 /* S7 the fused layer forward: compression, routing (route_mode), then the three
  * branches and the gated combine in one attention kernel whose epilogue writes
  * out.  route_mode: LSRM_ROUTE_GIVEN reads idx_inout as [B][Hkv][top_k];
  * LSRM_ROUTE_SCORE writes it as [B][Hkv][top_k]; LSRM_ROUTE_GEOMETRIC (coords
  * required) writes [B][top_k]; LSRM_ROUTE_ALL needs top_k == B and selects every
  * block (idx_inout may be NULL).  With a NULL idx_inout the indices live in the
- * workspace.  For pooled_q the routing is the Speed3R rule and idx_inout is
+ * workspace.  For pooled_q (top_k at most 64, blocks of at most 16 tokens,
+ * head_dim 64) the routing is the Speed3R rule and idx_inout is
  * [B][Hq][top_k], ranked by the fp32 logits of the pooled means (as
  * lsrm_route_pooled_topk with fp32 inputs).
  * lse_or_null receives fp32 [N][Hq][n_gates] per-branch LSE (needed by the

@@ -9,6 +9,9 @@ from block_sparse_gqa_nsa_b200 import nsa
 # acceptance bounds for attention outputs from bf16 inputs
 MAX_ABS = 1e-2
 REL_L2 = 5e-3
+# score-routing gap rule: where the oracle's k-th and (k+1)-th scores differ by more than GAP the
+# chosen sets must agree; otherwise every chosen block lies within GAP of the k-th score
+GAP = 1e-3
 
 
 def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
@@ -78,3 +81,28 @@ def assert_grad_close(got, ref, what=""):
     """Gradient bounds: max-abs 1e-2 scaled by max(1, max|ref|), relative L2 5e-3."""
     ref = np.asarray(ref, dtype=np.float64)
     return assert_close(got, ref, what, max_abs=MAX_ABS * max(1.0, float(np.abs(ref).max())), rel=REL_L2)
+
+
+def check_pooled_routing(gpu_idx, w, qblocks, k, qc=None, kc=None):
+    """Validity of Speed3R routing against the oracle's fp64 pooled logits: k distinct, non-forced
+    blocks, each with an oracle logit within 1e-3 of the k-th best; where the oracle gap exceeds
+    1e-3 the sets must agree.  qc / kc default to the oracle's fp64 block means; a test of the
+    bf16-operand mode passes the bf16 operands it gave the kernel."""
+    D = oracle_desc(w, top_k=k)
+    if qc is None:
+        qc = O.compress(D, w.off, w.q, w.n_q_heads)
+    if kc is None:
+        kc = O.compress(D, w.off, w.k, w.n_kv_heads)
+    _, logits = O.route_pooled(D, qc, kc, w.forced, qblocks=qblocks, want_logits=True)
+    forced = set(w.forced.tolist())
+    for i, a in enumerate(qblocks):
+        for h in range(w.n_q_heads):
+            chosen = gpu_idx[a, h].tolist()
+            assert len(set(chosen)) == k and not (set(chosen) & forced), (a, h)
+            lg = logits[i, h].copy()
+            lg[list(forced)] = -np.inf
+            order = np.lexsort((np.arange(w.n_blocks), -lg))
+            sk = lg[order[k - 1]]
+            assert np.all(lg[chosen] >= sk - GAP), (a, h)
+            if k < len(order) and sk - lg[order[k]] > GAP:
+                assert set(chosen) == set(order[:k].tolist()), (a, h)

@@ -12,7 +12,8 @@ import torch
 import oracle as O
 from block_sparse_gqa_nsa_b200 import nsa
 from block_sparse_gqa_nsa_b200.build import build
-from nsa_case import DeviceCase, oracle_desc, assert_close, assert_grad_close, rows_for, to_np, i32, bf16_tensor
+from nsa_case import (DeviceCase, oracle_desc, assert_close, assert_grad_close, rows_for, to_np, i32, bf16_tensor,
+                      check_pooled_routing)
 from workloads import make_workload
 from workloads.nsa_workloads import f32_to_bf16_bits
 
@@ -298,31 +299,6 @@ def test_fused_forward_dense_equals_dense_gqa_sampled():
 # ------------------------------------------------------------------------------------------------
 # S9 Speed3R pooled-query variant
 # ------------------------------------------------------------------------------------------------
-
-def check_pooled_routing(gpu_idx, w, qblocks, k, qc=None, kc=None):
-    """Validity of Speed3R routing against the oracle's fp64 pooled logits: k distinct, non-forced
-    blocks, each with an oracle logit within 1e-3 of the k-th best; where the oracle gap exceeds
-    1e-3 the sets must agree.  qc / kc default to the oracle's fp64 block means; a test of the
-    bf16-operand mode passes the bf16 operands it gave the kernel."""
-    D = oracle_desc(w, top_k=k)
-    if qc is None:
-        qc = O.compress(D, w.off, w.q, w.n_q_heads)
-    if kc is None:
-        kc = O.compress(D, w.off, w.k, w.n_kv_heads)
-    _, logits = O.route_pooled(D, qc, kc, w.forced, qblocks=qblocks, want_logits=True)
-    forced = set(w.forced.tolist())
-    for i, a in enumerate(qblocks):
-        for h in range(w.n_q_heads):
-            chosen = gpu_idx[a, h].tolist()
-            assert len(set(chosen)) == k and not (set(chosen) & forced), (a, h)
-            lg = logits[i, h].copy()
-            lg[list(forced)] = -np.inf
-            order = np.lexsort((np.arange(w.n_blocks), -lg))
-            sk = lg[order[k - 1]]
-            assert np.all(lg[chosen] >= sk - GAP), (a, h)
-            if k < len(order) and sk - lg[order[k]] > GAP:
-                assert set(chosen) == set(order[:k].tolist()), (a, h)
-
 
 @pytest.mark.parametrize("n_frames", [3, 6])
 def test_speed3r_forward_small(n_frames):
