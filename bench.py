@@ -52,7 +52,7 @@ def parse():
                          "10-20 s of one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r", "mixture", "bandwidth"],
+    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r", "speed3r_backward", "mixture", "bandwidth"],
                     help="sparse: the layer forward (the default line); backward: its gradients; dense: the "
                          "dense-stage shape with every block selected; speed3r: the pooled-query variant; "
                          "bandwidth: achieved HBM GB/s of the memory-bound kernels (pooling, routing, combine)")
@@ -674,6 +674,8 @@ EXTRA = {
     "dense": ("sparse-attn fwd tokens/s, dense-stage shape (k = B)", "lsrm_dense_stage_all_blocks"),
     "speed3r": ("sparse-attn fwd tokens/s, Speed3R pooled-query variant", "speed3r_512_frames_top32_forced"),
     "mixture": ("self/cross gated mixture fwd tokens/s, dense-stage shape", "lsrm_dense_stage_self_cross_mixture"),
+    "speed3r_backward": ("sparse-attn bwd tokens/s, Speed3R pooled-query variant",
+                         "speed3r_512_frames_top32_forced_backward"),
 }
 
 
@@ -717,6 +719,11 @@ def run_extra(args):
     if args.impl == "reference":
         if rank != 0:
             return 0
+        if args.workload == "speed3r_backward":
+            print(json.dumps({"impl": "reference", "metric": metric,
+                              "unavailable": "the oracle's pooled-query backward has no per-block sampling: "
+                                             "it runs at the test sizes only"}), flush=True)
+            return 0
         return run_extra_reference(args, metric, workload)
     if world > 1:
         import torch.distributed as dist
@@ -732,11 +739,12 @@ def run_extra(args):
     if world > 1:
         dist.barrier()
     nsa.load_library()
-    if args.workload == "speed3r" and args.frames != 512:
+    base = "speed3r" if args.workload == "speed3r_backward" else args.workload
+    if base == "speed3r" and args.frames != 512:
         w = make_workload("speed3r_small", seed=args.seed, n_frames=args.frames)
         workload = workload.replace("512_frames", f"{args.frames}_frames")
     else:
-        w = make_workload(args.workload, seed=args.seed)
+        w = make_workload(base, seed=args.seed)
     N, B, Hq, Hkv, d, k = w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k
 
     def bf(a):
@@ -748,7 +756,23 @@ def run_extra(args):
     desc = nsa.make_desc(N, B, w.max_block_len, Hq, Hkv, d, k, w.window, 0.0, w.pooled_q, w.n_gates, forced)
     ws = nsa.workspace(desc, dev)
     out = torch.empty(N, Hq, d, dtype=torch.bfloat16, device=dev)
-    if args.workload == "mixture":
+    if args.workload == "speed3r_backward":
+        from workloads.nsa_workloads import STREAM_DOUT, normal_bf16
+        idx = torch.empty(B, Hq, k, dtype=torch.int32, device=dev)
+        lse = torch.empty(N, Hq, 2, dtype=torch.float32, device=dev)
+        obr = torch.empty(N, Hq, 2, d, dtype=torch.bfloat16, device=dev)
+        nsa.lsrm_nsa_forward(desc, off, q, kk, v, gates, None, nsa.ROUTE_SCORE, out, idx, lse, ws, obr=obr)
+        dout = bf(normal_bf16(args.seed, STREAM_DOUT, (N, Hq, d), 1.0))
+        dq, dk, dv = (torch.empty(N, Hq, d, dtype=torch.bfloat16, device=dev) for _ in range(3))
+        dg = torch.empty(N, Hq, 2, dtype=torch.bfloat16, device=dev)
+
+        def step():
+            nsa.lsrm_nsa_backward(desc, off, q, kk, v, gates, idx, Hq, lse, dout, dq, dk, dv, dg, ws, obr=obr)
+        # forced bitmap / prefix / gather, compress, two preparation passes, the pooled branch's dq and
+        # dK/dV, the forced part's dq and dK/dV, four inverse-list passes, the routed dq and dK/dV, the
+        # forced-token map and scatter
+        launches_per_step = 18
+    elif args.workload == "mixture":
         idx = None
         bx = w.n_blocks_x
 
@@ -777,6 +801,10 @@ def run_extra(args):
         raise RuntimeError(f"device status {st} after warm-up")
     if args.workload == "speed3r":
         flops = speed3r_flops(w, idx.cpu().numpy())
+    elif args.workload == "speed3r_backward":
+        # 10 d per attended (query, key) pair against the forward's 4 d: the score recompute, dV, dP,
+        # dq and dK
+        flops = {kk_: 2.5 * v_ for kk_, v_ in speed3r_flops(w, idx.cpu().numpy()).items()}
     elif args.workload == "mixture":
         flops = mixture_flops(w)
     else:
@@ -810,10 +838,17 @@ def run_extra(args):
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                              "frac": achieved / peak, "traffic": None,
                              "kernel": ("nsa_attn_tc_kernel (mixture mode, one launch)" if args.workload == "mixture"
+                                        else "lsrm_nsa_backward (all launches of one call)"
+                                        if args.workload == "speed3r_backward"
                                         else "lsrm_nsa_forward (all launches of one call)"),
                              "peak_source": f"{src} bf16_tflops (burst)"},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and world == 1 and args.workload == "speed3r_backward":
+            tok, dt = speed3r_backward_oracle_sample(args.seed)
+            line["cpu_baseline"] = cpu_baseline(tok / dt, f"the whole backward of the 3-frame case ({tok} tokens, "
+                                                          f"the oracle has no per-block sampling), fp64, "
+                                                          f"1 thread, {dt:.1f} s")
+        elif not args.no_cpu_baseline and world == 1:
             n_blk = args.cpu_sample_blocks or 4
             tok, dt = extra_oracle_sample(w, idx.cpu().numpy() if idx is not None else None, n_blk, 7)
             line["cpu_baseline"] = cpu_baseline(tok / dt, f"{n_blk} seeded query blocks ({tok} tokens) of the "
@@ -823,6 +858,24 @@ def run_extra(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def speed3r_backward_oracle_sample(seed: int):
+    """The fp64 oracle's pooled-query backward on the 3-frame case (1 thread), with routing
+    indices from the oracle's own pooled routing."""
+    import oracle as O
+    from workloads import make_workload
+    from workloads.nsa_workloads import STREAM_DOUT, normal_bf16
+    w = make_workload("speed3r_small", seed=seed, n_frames=3)
+    D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window,
+                   n_gates=w.n_gates, pooled_q=w.pooled_q)
+    qc = O.compress(D, w.off, w.q, w.n_q_heads)
+    kc = O.compress(D, w.off, w.k, w.n_kv_heads)
+    idx, _ = O.route_pooled(D, qc, kc, w.forced)
+    dout = normal_bf16(seed, STREAM_DOUT, (w.n_tokens, w.n_q_heads, w.head_dim), 1.0)
+    t0 = time.perf_counter()
+    O.backward_pooled(D, w.off, w.q, w.k, w.v, w.gates, idx, w.forced, dout, nthreads=1)
+    return w.n_tokens, time.perf_counter() - t0
 
 
 def extra_oracle_sample(w, idx, n_blocks: int, seed: int):

@@ -273,14 +273,21 @@ LSRM_API lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* 
                              void* out, int32_t* idx_inout, float* lse_or_null, void* obr_or_null, void* ws,
                              void* stream);
 
-/* S10 backward of the LSRM layer (pooled_q = 0) with routing indices fixed:
+/* S10 backward of the layer with routing indices fixed:
  * dq, dgates [N][Hq][.], dk, dv [N][Hkv][d] (bf16) of L = sum(out * dout),
  * through the gated sum, the three softmax branches and the block mean.
  * lse is the forward's per-branch LSE.  idx_heads as in lsrm_nsa_select_attn.
  * obr_or_null: the forward's saved branch outputs (see lsrm_nsa_forward).  With
  * them dgates_b = <dO, o_b> and Delta_b = g_b dgates_b are read off directly and
  * every branch is streamed once; with NULL they are recomputed in an extra pass
- * over each branch (P dP summed in fp32).  dout and obr must be 16-byte aligned. */
+ * over each branch (P dP summed in fp32).  dout and obr must be 16-byte aligned.
+ * With pooled_q (the Speed3R layer, Speed3R page section 2: trained end to end)
+ * idx is the forward's [B][Hq][top_k] routing (idx_heads = Hq), lse its
+ * [N][Hq][2] output and obr_or_null is required (LSRM_ERR_INVALID_ARG without
+ * it): the chain rule runs through the pooled query (dQbar / n_b to every token
+ * of the block), the copy of the pooled output to the block's tokens, the joint
+ * softmax of the forced and routed keys and the two gates; all sums have a fixed
+ * order, so results are reproducible bit for bit. */
 LSRM_API lsrm_status lsrm_nsa_backward(const lsrm_nsa_desc* desc, const int32_t* off, const void* q, const void* k,
                               const void* v, const void* gates, const int32_t* idx, int32_t idx_heads,
                               const float* lse, const void* obr_or_null, const void* dout, void* dq, void* dk,
