@@ -85,11 +85,16 @@ inline BwdWs bwd_layout(const lsrm_nsa_desc& d, int idx_heads) {
 // (bf16, for the tensor cores), its LSE (log2 units) and Delta per (block, head) as float2; the pooled
 // gradients dQbar, dKbar, dVbar (fp32); per (token, head) the selected branch's LSE (log2 units) and
 // Delta as float2 and its upstream gradient g_slc dO (bf16); the forced part of dq (fp32); dK, dV of
-// the packed forced tokens (fp32) and each packed token's (token, block); the inverse routing lists
-// per (block, head)
+// the packed forced tokens (fp32, one partial per split of the query rows) and each packed token's
+// (token, block); the inverse routing lists per (block, head), the lists longer than one segment
+// (their ids; per list its first segment and per segment its list) and each such segment's partial
+// dK, dV (fp32, 16 rows each)
+constexpr int kForcedSplits = 8;
+constexpr int kListSeg = 256;  // inverse-list entries per segment of the routed dK / dV pass
 struct PooledBwdWs {
   size_t gbar16, rowcb, dqbar, dkbar, dvbar, rowc, dos16, dqf, dkf, dvf, fmap;
-  size_t inv_count, inv_cursor, inv_start, inv_list, total;
+  size_t inv_count, inv_cursor, inv_start, inv_list, n_long, long_ids, seg_count, seg_start, seg_list, seg_part;
+  size_t max_segs, total;
 };
 inline PooledBwdWs pooled_bwd_layout(const lsrm_nsa_desc& d) {
   PooledBwdWs w{};
@@ -105,13 +110,21 @@ inline PooledBwdWs pooled_bwd_layout(const lsrm_nsa_desc& d) {
   w.rowc = o;       o = align256(o + N * H * 8);
   w.dos16 = o;      o = align256(o + N * H * D * 2);
   w.dqf = o;        o = align256(o + N * H * D * 4);
-  w.dkf = o;        o = align256(o + nf_tok * H * D * 4);
-  w.dvf = o;        o = align256(o + nf_tok * H * D * 4);
+  w.dkf = o;        o = align256(o + (size_t)kForcedSplits * nf_tok * H * D * 4);
+  w.dvf = o;        o = align256(o + (size_t)kForcedSplits * nf_tok * H * D * 4);
   w.fmap = o;       o = align256(o + nf_tok * 8);
   w.inv_count = o;  o = align256(o + nl * 4);
   w.inv_cursor = o; o = align256(o + nl * 4);
   w.inv_start = o;  o = align256(o + (nl + 1) * 4);
   w.inv_list = o;   o = align256(o + nl * K * 4);
+  w.n_long = o;     o = align256(o + 16);
+  w.long_ids = o;   o = align256(o + nl * 4);
+  w.seg_count = o;  o = align256(o + nl * 4);
+  w.seg_start = o;  o = align256(o + (nl + 1) * 4);
+  // a list longer than kListSeg has ceil(n / kListSeg) < 2 n / kListSeg segments
+  w.max_segs = 2 * nl * K / (size_t)kListSeg + 1;
+  w.seg_list = o;   o = align256(o + w.max_segs * 4);
+  w.seg_part = o;   o = align256(o + w.max_segs * 2 * 16 * D * 4);
   w.total = o;
   return w;
 }

@@ -197,8 +197,9 @@ struct DenseBwd {
   int H;
   float scale_log2, tau;
   float* dq;  // [n_rows][H][64] = tau sum dS k          (dq kernel)
-  float* dk;  // [n_keys][H][64] = tau sum dS^T q        (dkdv kernel)
-  float* dv;  // [n_keys][H][64] = sum P^T dout
+  float* dk;  // [n_keys][H][64] = tau sum dS^T q        (dkdv kernel; one partial per grid z of
+  float* dv;  // [n_keys][H][64] = sum P^T dout            the query rows, split_stride apart)
+  long long split_stride;
 };
 
 constexpr int kDbThreads = 128;  // 4 warps, 16 rows (or keys) each
@@ -289,8 +290,13 @@ __global__ void __launch_bounds__(kDbThreads) sb_dense_dkdv_kernel(const DenseBw
   if (k0 >= nk) return;
   sb_load_tile(S.a[0], p.k, k0, nk, p.H, h, 64, tid, kDbThreads);
   sb_load_tile(S.a[1], p.v, k0, nk, p.H, h, 64, tid, kDbThreads);
-  const long long n_chunks = (p.n_rows + 63) / 64;
-  auto load_rows = [&](int st, long long c) {
+  // this CTA's share of the query-row chunks (grid z splits them; partial sums per split)
+  const long long all_chunks = (p.n_rows + 63) / 64;
+  const long long per = (all_chunks + gridDim.z - 1) / gridDim.z;
+  const long long c_lo = blockIdx.z * per, c_hi = c_lo + per < all_chunks ? c_lo + per : all_chunks;
+  const long long n_chunks = c_hi > c_lo ? c_hi - c_lo : 0;
+  auto load_rows = [&](int st, long long cc) {
+    const long long c = c_lo + cc;
     sb_load_tile(S.s[st][0], p.q, c * 64, p.n_rows, p.H, h, 64, tid, kDbThreads);
     sb_load_tile(S.s[st][1], p.dout, c * 64, p.n_rows, p.H, h, 64, tid, kDbThreads);
     if (tid < 64) {
@@ -298,7 +304,7 @@ __global__ void __launch_bounds__(kDbThreads) sb_dense_dkdv_kernel(const DenseBw
       S.rc[st][tid] = r < p.n_rows ? p.rowc[(size_t)r * p.H + h] : make_float2(INFINITY, 0.f);
     }
   };
-  load_rows(0, 0);
+  if (n_chunks > 0) load_rows(0, 0);
   cp_async_commit();
   const int cq = lane & 3;
   float dk[8][4], dv[8][4];
@@ -343,8 +349,8 @@ __global__ void __launch_bounds__(kDbThreads) sb_dense_dkdv_kernel(const DenseBw
   for (int i = 0; i < 2; ++i) {
     const int kr = k0 + warp * 16 + gq + 8 * i;
     if (kr >= nk) continue;
-    float* dkr = p.dk + ((size_t)kr * p.H + h) * kSbD;
-    float* dvr = p.dv + ((size_t)kr * p.H + h) * kSbD;
+    float* dkr = p.dk + blockIdx.z * p.split_stride + ((size_t)kr * p.H + h) * kSbD;
+    float* dvr = p.dv + blockIdx.z * p.split_stride + ((size_t)kr * p.H + h) * kSbD;
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       *reinterpret_cast<float2*>(dkr + n * 8 + 2 * cq) = make_float2(p.tau * dk[n][2 * i], p.tau * dk[n][2 * i + 1]);
@@ -512,40 +518,46 @@ __global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dq_kernel(const Route
   }
 }
 
-// One warp per (key block j, head h), j not forced: dK, dV of j's tokens from the query blocks that
-// routed to j (the inverse list, ascending), plus the pooled branch's share dKbar / n_j, dVbar / n_j.
-__global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dkdv_kernel(const RoutedBwd p) {
-  extern __shared__ __align__(128) unsigned char sb_smem[];
-  RbSmem& S = *reinterpret_cast<RbSmem*>(sb_smem);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long pair = (long long)blockIdx.x * kRbWarps + warp;
-  if (pair >= (long long)p.B * p.H) return;
-  const int h = (int)(pair / p.B), j = (int)(pair % p.B);
-  if ((p.fbits[j >> 5] >> (j & 31)) & 1u) return;  // forced: written with the forced part
+// ---- routed dK, dV: per (key block j, head h), j not forced, over the query blocks that routed to j
+// (the inverse list, ascending).  Lists of at most kListSeg entries are done by one warp, which
+// writes the final rows; longer lists are cut into segments of kListSeg entries, one warp each,
+// whose partial sums are added in segment order afterwards (routing concentrates on a few blocks,
+// so some lists are thousands long).
+struct RkSmem {
+  unsigned char k[kRbWarps][16 * 128];
+  unsigned char v[kRbWarps][16 * 128];
+  unsigned char q[kRbWarps][2][16 * 128];
+  unsigned char d[kRbWarps][2][16 * 128];
+};
+
+// dK, dV (without tau / the pooled share) of block j's 16 key rows from list entries [e_begin, e_end);
+// the next entry's query rows are copied while the current one is computed
+__device__ __forceinline__ void rk_range(const RoutedBwd& p, RkSmem& S, int warp, int lane, int j, int h,
+                                         int e_begin, int e_end, float (&dk)[8][4], float (&dv)[8][4]) {
   const int H = p.H;
   const int u0 = p.off[j], n_j = min(16, p.off[j + 1] - u0);
-  // K_j, V_j (16 rows) as A fragments; the per-warp K / V areas hold them, the Q / dO areas the
-  // query block of the current list entry
   sb_load_tile(S.k[warp], p.k, u0, u0 + n_j, H, h, 16, lane, 32);
   sb_load_tile(S.v[warp], p.v, u0, u0 + n_j, H, h, 16, lane, 32);
+  auto issue = [&](int e, int st) {
+    const int a = p.inv_list[e];
+    const int t0 = p.off[a], n_a = min(16, p.off[a + 1] - t0);
+    sb_load_tile(S.q[warp][st], p.q, t0, t0 + n_a, H, h, 16, lane, 32);
+    sb_load_tile(S.d[warp][st], p.dos, t0, t0 + n_a, H, h, 16, lane, 32);
+  };
+  if (e_begin < e_end) issue(e_begin, 0);
   cp_async_commit();
   cp_async_wait<0>();
   __syncwarp();
   uint32_t ka[4][4], va[4][4];
   sb_frag_a(ka, S.k[warp], 0, lane);
   sb_frag_a(va, S.v[warp], 0, lane);
-  const int cq = lane & 3, gq = lane >> 2;
-  float dk[8][4], dv[8][4];
-  sb_zero(dk);
-  sb_zero(dv);
-  const int e0 = p.inv_start[(size_t)j * H + h], e1 = p.inv_start[(size_t)j * H + h + 1];
-  for (int e = e0; e < e1; ++e) {
+  const int cq = lane & 3;
+  for (int e = e_begin; e < e_end; ++e) {
+    const int st = (e - e_begin) & 1;
+    if (e + 1 < e_end) issue(e + 1, st ^ 1);
+    cp_async_commit();
     const int a = p.inv_list[e];
     const int t0 = p.off[a], n_a = min(16, p.off[a + 1] - t0);
-    __syncwarp();
-    sb_load_tile(S.q[warp], p.q, t0, t0 + n_a, H, h, 16, lane, 32);
-    sb_load_tile(S.d[warp], p.dos, t0, t0 + n_a, H, h, 16, lane, 32);
-    cp_async_commit();
     // this lane's query columns: rows 2 cq + (0, 1) of each 8-row n-tile
     float2 rc[2][2];
 #pragma unroll
@@ -555,13 +567,13 @@ __global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dkdv_kernel(const Rou
         const int r = nt * 8 + 2 * cq + b;
         rc[nt][b] = r < n_a ? p.rowc[(size_t)(t0 + r) * H + h] : make_float2(INFINITY, 0.f);
       }
-    cp_async_wait<0>();
+    cp_async_wait<1>();
     __syncwarp();
     float s[2][4], dp[2][4];
     sb_zero(s);
     sb_zero(dp);
-    sb_mma_abt<2>(s, ka, S.q[warp], lane);   // S^T: 16 keys x 16 query rows
-    sb_mma_abt<2>(dp, va, S.d[warp], lane);  // dP^T = V dO_s^T
+    sb_mma_abt<2>(s, ka, S.q[warp][st], lane);   // S^T: 16 keys x 16 query rows
+    sb_mma_abt<2>(dp, va, S.d[warp][st], lane);  // dP^T = V dO_s^T
     float pt[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -574,13 +586,23 @@ __global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dkdv_kernel(const Rou
       }
     uint32_t pa[1][4];
     sb_to_a<2>(pa, pt);
-    sb_mma_pb<1>(dv, pa, S.d[warp], lane);
+    sb_mma_pb<1>(dv, pa, S.d[warp][st], lane);
     sb_to_a<2>(pa, s);
-    sb_mma_pb<1>(dk, pa, S.q[warp], lane);
+    sb_mma_pb<1>(dk, pa, S.q[warp][st], lane);
+    __syncwarp();  // stage st is refilled by the next iteration's copy
   }
+  cp_async_wait<0>();
+}
+
+// final bf16 rows of block j: tau dK + dKbar / n_j, dV + dVbar / n_j
+__device__ __forceinline__ void rk_write(const RoutedBwd& p, int lane, int j, int h, const float (&dk)[8][4],
+                                         const float (&dv)[8][4]) {
+  const int H = p.H;
+  const int u0 = p.off[j], n_j = min(16, p.off[j + 1] - u0);
   const float inv_n = 1.f / (float)(p.off[j + 1] - u0);
   const float* kb = p.dkbar + ((size_t)j * H + h) * kSbD;
   const float* vb = p.dvbar + ((size_t)j * H + h) * kSbD;
+  const int cq = lane & 3, gq = lane >> 2;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int r = gq + 8 * i;
@@ -597,6 +619,104 @@ __global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dkdv_kernel(const Rou
   }
 }
 
+// one warp per (key block, head) whose list has at most kListSeg entries
+__global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dkdv_kernel(const RoutedBwd p) {
+  extern __shared__ __align__(128) unsigned char sb_smem[];
+  RkSmem& S = *reinterpret_cast<RkSmem*>(sb_smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long pair = (long long)blockIdx.x * kRbWarps + warp;
+  if (pair >= (long long)p.B * p.H) return;
+  const int h = (int)(pair / p.B), j = (int)(pair % p.B);
+  if ((p.fbits[j >> 5] >> (j & 31)) & 1u) return;  // forced: written with the forced part
+  const size_t li = (size_t)j * p.H + h;
+  const int e0 = p.inv_start[li], e1 = p.inv_start[li + 1];
+  if (e1 - e0 > kListSeg) return;  // segmented
+  float dk[8][4], dv[8][4];
+  sb_zero(dk);
+  sb_zero(dv);
+  rk_range(p, S, warp, lane, j, h, e0, e1, dk, dv);
+  rk_write(p, lane, j, h, dk, dv);
+}
+
+// segments of the long lists: per list the number of segments (0 for short or forced lists), then
+// per segment its list
+__global__ void sb_seg_count_kernel(const int* __restrict__ inv_start, const uint32_t* __restrict__ fbits, int B,
+                                    int H, int* seg_count, int* long_ids, int* n_long) {
+  const long long li = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (li >= (long long)B * H) return;
+  const int j = (int)(li / H);
+  const int n = inv_start[li + 1] - inv_start[li];
+  const bool forced = (fbits[j >> 5] >> (j & 31)) & 1u;
+  seg_count[li] = (!forced && n > kListSeg) ? (n + kListSeg - 1) / kListSeg : 0;
+  if (n > 64) long_ids[atomicAdd(n_long, 1)] = (int)li;  // sorted by the bitmap pass
+}
+__global__ void sb_seg_fill_kernel(const int* __restrict__ seg_count, const int* __restrict__ seg_start,
+                                   long long n_lists, int* seg_list) {
+  const long long li = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (li >= n_lists) return;
+  for (int sgm = 0; sgm < seg_count[li]; ++sgm) seg_list[seg_start[li] + sgm] = (int)li;
+}
+
+// one warp per segment: the partial dK, dV of its entries, [segment][dK | dV][16 rows][64]
+__global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dkdv_seg_kernel(const RoutedBwd p, const int* seg_start,
+                                                                           const int* seg_list, long long n_lists,
+                                                                           float* seg_part) {
+  extern __shared__ __align__(128) unsigned char sb_smem[];
+  RkSmem& S = *reinterpret_cast<RkSmem*>(sb_smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long i = (long long)blockIdx.x * kRbWarps + warp;
+  if (i >= seg_start[n_lists]) return;
+  const int li = seg_list[i];
+  const int j = li / p.H, h = li % p.H;
+  const int sgm = (int)(i - seg_start[li]);
+  const int e0 = p.inv_start[li] + sgm * kListSeg, e1 = min(p.inv_start[li + 1], e0 + kListSeg);
+  float dk[8][4], dv[8][4];
+  sb_zero(dk);
+  sb_zero(dv);
+  rk_range(p, S, warp, lane, j, h, e0, e1, dk, dv);
+  float* out = seg_part + (size_t)i * 2 * 16 * kSbD;
+  const int cq = lane & 3, gq = lane >> 2;
+#pragma unroll
+  for (int r2 = 0; r2 < 2; ++r2)
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int r = gq + 8 * r2, col = n * 8 + 2 * cq;
+      *reinterpret_cast<float2*>(out + r * kSbD + col) = make_float2(dk[n][2 * r2], dk[n][2 * r2 + 1]);
+      *reinterpret_cast<float2*>(out + (16 + r) * kSbD + col) = make_float2(dv[n][2 * r2], dv[n][2 * r2 + 1]);
+    }
+}
+
+// one warp per long list: its segments' partials added in segment order, then the final rows
+__global__ void __launch_bounds__(kRbWarps * 32) sb_routed_dkdv_reduce_kernel(const RoutedBwd p, const int* seg_start,
+                                                                              const float* seg_part) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long li = (long long)blockIdx.x * kRbWarps + warp;
+  if (li >= (long long)p.B * p.H) return;
+  const int s0 = seg_start[li], s1 = seg_start[li + 1];
+  if (s1 == s0) return;
+  const int j = (int)(li / p.H), h = (int)(li % p.H);
+  const int cq = lane & 3, gq = lane >> 2;
+  float dk[8][4], dv[8][4];
+  sb_zero(dk);
+  sb_zero(dv);
+  for (int sg = s0; sg < s1; ++sg) {
+    const float* in = seg_part + (size_t)sg * 2 * 16 * kSbD;
+#pragma unroll
+    for (int r2 = 0; r2 < 2; ++r2)
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const int r = gq + 8 * r2, col = n * 8 + 2 * cq;
+        const float2 a = *reinterpret_cast<const float2*>(in + r * kSbD + col);
+        const float2 b = *reinterpret_cast<const float2*>(in + (16 + r) * kSbD + col);
+        dk[n][2 * r2] += a.x;
+        dk[n][2 * r2 + 1] += a.y;
+        dv[n][2 * r2] += b.x;
+        dv[n][2 * r2 + 1] += b.y;
+      }
+  }
+  rk_write(p, lane, j, h, dk, dv);
+}
+
 // ---- forced tokens: map of the packed copy, and the final dK, dV ----------------------------------
 __global__ void sb_forced_map_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ forced,
                                      const int* __restrict__ pre, int B, int max_len, int2* __restrict__ fmap) {
@@ -607,11 +727,13 @@ __global__ void sb_forced_map_kernel(const int32_t* __restrict__ off, const int3
   for (int r = threadIdx.x; r < n; r += blockDim.x) fmap[pre[i] + r] = make_int2(t0 + r, j);
 }
 
-// one thread per (packed forced token, head, 8 dims): dk = dK_forced + dKbar / n_j (bf16)
+// one thread per (packed forced token, head, 8 dims): dk = the forced part's split partials summed
+// in split order + dKbar / n_j (bf16)
 __global__ void sb_forced_scatter_kernel(const int2* __restrict__ fmap, const int* __restrict__ ftotal,
                                          const int32_t* __restrict__ off, const float* __restrict__ dkf,
                                          const float* __restrict__ dvf, const float* __restrict__ dkbar,
-                                         const float* __restrict__ dvbar, int H, long long cap, uint4* dk, uint4* dv) {
+                                         const float* __restrict__ dvbar, int H, long long cap, int n_split,
+                                         long long split_stride, uint4* dk, uint4* dv) {
   const long long n = (long long)*ftotal * H * 8;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
     const long long uh = e >> 3;
@@ -625,11 +747,23 @@ __global__ void sb_forced_scatter_kernel(const int2* __restrict__ fmap, const in
     const float* b = dvf + (size_t)uh * kSbD + c * 8;
     const float* ab = dkbar + ((size_t)m.y * H + h) * kSbD + c * 8;
     const float* bb = dvbar + ((size_t)m.y * H + h) * kSbD + c * 8;
+    float sk[8], sv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sk[i] = a[i];
+      sv[i] = b[i];
+    }
+    for (int z = 1; z < n_split; ++z)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        sk[i] += a[z * split_stride + i];
+        sv[i] += b[z * split_stride + i];
+      }
     uint32_t wk[4], wv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      wk[i] = pack_bf16x2(a[2 * i] + ab[2 * i] * inv_n, a[2 * i + 1] + ab[2 * i + 1] * inv_n);
-      wv[i] = pack_bf16x2(b[2 * i] + bb[2 * i] * inv_n, b[2 * i + 1] + bb[2 * i + 1] * inv_n);
+      wk[i] = pack_bf16x2(sk[2 * i] + ab[2 * i] * inv_n, sk[2 * i + 1] + ab[2 * i + 1] * inv_n);
+      wv[i] = pack_bf16x2(sv[2 * i] + bb[2 * i] * inv_n, sv[2 * i + 1] + bb[2 * i + 1] * inv_n);
     }
     const size_t dst = ((size_t)m.x * H + h) * 8 + c;
     dk[dst] = make_uint4(wk[0], wk[1], wk[2], wk[3]);
@@ -680,17 +814,68 @@ __global__ void sb_inv_fill_kernel(const int32_t* __restrict__ idx, int B, int H
     list[start[li] + slot] = a;
   }
 }
-// insertion sort of each list (a query block appears once per list: lists are short)
+// ascending order of each list (a query block appears at most once per list): insertion sort of the
+// lists of at most 64 entries here, one CTA per longer list below
 __global__ void sb_inv_sort_kernel(const int* start, int n_lists, int* list) {
   const int li = blockIdx.x * blockDim.x + threadIdx.x;
   if (li >= n_lists) return;
   int* x = list + start[li];
   const int n = start[li + 1] - start[li];
+  if (n > 64) return;
   for (int i = 1; i < n; ++i) {
     const int v = x[i];
     int j = i - 1;
     while (j >= 0 && x[j] > v) { x[j + 1] = x[j]; --j; }
     x[j + 1] = v;
+  }
+}
+
+// a long list through a bitmap over the query blocks: set the entries' bits, then write the set bits
+// in order (each thread owns a run of words; a scan of the per-thread counts places them)
+constexpr int kSortThreads = 256;
+__global__ void __launch_bounds__(kSortThreads) sb_inv_sort_long_kernel(const int* __restrict__ start,
+                                                                        const int* __restrict__ long_ids,
+                                                                        const int* __restrict__ n_long, int B,
+                                                                        int* list) {
+  extern __shared__ uint32_t bits[];
+  __shared__ int part[kSortThreads];
+  const int W = (B + 31) / 32;
+  const int per = (W + kSortThreads - 1) / kSortThreads;
+  const int w0 = min(W, (int)threadIdx.x * per), w1 = min(W, w0 + per);
+  const int count = *n_long;
+  for (int i = blockIdx.x; i < count; i += gridDim.x) {
+    const int li = long_ids[i];
+    int* x = list + start[li];
+    const int n = start[li + 1] - start[li];
+    for (int w = threadIdx.x; w < W; w += kSortThreads) bits[w] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += kSortThreads) {
+      const int a = x[e];
+      atomicOr(&bits[a >> 5], 1u << (a & 31));
+    }
+    __syncthreads();
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(bits[w]);
+    part[threadIdx.x] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int acc = 0;
+      for (int t = 0; t < kSortThreads; ++t) {
+        const int v = part[t];
+        part[t] = acc;
+        acc += v;
+      }
+    }
+    __syncthreads();
+    int pos = part[threadIdx.x];
+    for (int w = w0; w < w1; ++w) {
+      uint32_t m = bits[w];
+      while (m != 0u) {
+        x[pos++] = w * 32 + (__ffs(m) - 1);
+        m &= m - 1u;
+      }
+    }
+    __syncthreads();  // the bitmap is cleared for the next list
   }
 }
 
@@ -764,6 +949,7 @@ lsrm_status launch_speed3r_backward(const lsrm_nsa_desc& d, const int32_t* off, 
   pb.dq = dqbar;
   pb.dk = dkbar;
   pb.dv = dvbar;
+  pb.split_stride = 0;
   const dim3 gblk((unsigned)((B + 63) / 64), (unsigned)H);
   sb_dense_dq_kernel<<<gblk, kDbThreads, db_smem, s>>>(pb);
   sb_dense_dkdv_kernel<<<gblk, kDbThreads, db_smem, s>>>(pb);
@@ -787,9 +973,11 @@ lsrm_status launch_speed3r_backward(const lsrm_nsa_desc& d, const int32_t* off, 
     pf.dq = dqf;
     pf.dk = reinterpret_cast<float*>(wb + b.dkf);
     pf.dv = reinterpret_cast<float*>(wb + b.dvf);
+    pf.split_stride = cap * H * kSbD;
     if ((N + 63) / 64 > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
     sb_dense_dq_kernel<<<dim3((unsigned)((N + 63) / 64), (unsigned)H), kDbThreads, db_smem, s>>>(pf);
-    sb_dense_dkdv_kernel<<<dim3((unsigned)((cap + 63) / 64), (unsigned)H), kDbThreads, db_smem, s>>>(pf);
+    sb_dense_dkdv_kernel<<<dim3((unsigned)((cap + 63) / 64), (unsigned)H, kForcedSplits), kDbThreads, db_smem, s>>>(
+        pf);
   }
   // inverse routing lists
   const int n_lists = B * H;
@@ -807,6 +995,23 @@ lsrm_status launch_speed3r_backward(const lsrm_nsa_desc& d, const int32_t* off, 
   sb_inv_scan_kernel<<<1, kSbScan, 0, s>>>(count, n_lists, start);
   sb_inv_fill_kernel<<<gi, 256, 0, s>>>(idx, B, H, d.top_k, start, cursor, list);
   sb_inv_sort_kernel<<<(n_lists + 127) / 128, 128, 0, s>>>(start, n_lists, list);
+  int* n_long = reinterpret_cast<int*>(wb + b.n_long);
+  int* seg_count = reinterpret_cast<int*>(wb + b.seg_count);
+  int* seg_start = reinterpret_cast<int*>(wb + b.seg_start);
+  int* seg_list = reinterpret_cast<int*>(wb + b.seg_list);
+  float* seg_part = reinterpret_cast<float*>(wb + b.seg_part);
+  if (cudaMemsetAsync(n_long, 0, 4, s) != cudaSuccess) return LSRM_ERR_CUDA;
+  sb_seg_count_kernel<<<(n_lists + 255) / 256, 256, 0, s>>>(start, fbits, B, H, seg_count,
+                                                            reinterpret_cast<int*>(wb + b.long_ids), n_long);
+  const size_t sort_smem = (size_t)((B + 31) / 32) * 4;
+  if (sort_smem > 200 * 1024) return LSRM_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(sb_inv_sort_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sort_smem) !=
+      cudaSuccess)
+    return LSRM_ERR_CUDA;
+  sb_inv_sort_long_kernel<<<148 * 2, kSortThreads, sort_smem, s>>>(start, reinterpret_cast<int*>(wb + b.long_ids),
+                                                                   n_long, B, list);
+  sb_inv_scan_kernel<<<1, kSbScan, 0, s>>>(seg_count, n_lists, seg_start);
+  sb_seg_fill_kernel<<<(n_lists + 255) / 256, 256, 0, s>>>(seg_count, seg_start, n_lists, seg_list);
   // routed part: dq per (block, head); dK, dV per (non-forced key block, head)
   RoutedBwd pr{};
   pr.off = off;
@@ -832,23 +1037,30 @@ lsrm_status launch_speed3r_backward(const lsrm_nsa_desc& d, const int32_t* off, 
   pr.top_k = d.top_k;
   pr.scale_log2 = sl;
   pr.tau = tau;
-  const size_t rb_smem = sizeof(RbSmem);
+  const size_t rb_smem = sizeof(RbSmem), rk_smem = sizeof(RkSmem);
   if (cudaFuncSetAttribute(sb_routed_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rb_smem) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(sb_routed_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rb_smem) !=
+      cudaFuncSetAttribute(sb_routed_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rk_smem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(sb_routed_dkdv_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rk_smem) !=
           cudaSuccess)
     return LSRM_ERR_CUDA;
   const long long pairs = (long long)B * H;
   const unsigned grb = (unsigned)((pairs + kRbWarps - 1) / kRbWarps);
   sb_routed_dq_kernel<<<grb, kRbWarps * 32, rb_smem, s>>>(pr);
-  sb_routed_dkdv_kernel<<<grb, kRbWarps * 32, rb_smem, s>>>(pr);
+  sb_routed_dkdv_kernel<<<grb, kRbWarps * 32, rk_smem, s>>>(pr);
+  const long long seg_grid = ((long long)b.max_segs + kRbWarps - 1) / kRbWarps;
+  if (seg_grid > INT32_MAX) return LSRM_ERR_UNSUPPORTED;
+  sb_routed_dkdv_seg_kernel<<<(unsigned)seg_grid, kRbWarps * 32, rk_smem, s>>>(pr, seg_start, seg_list, pairs,
+                                                                               seg_part);
+  sb_routed_dkdv_reduce_kernel<<<grb, kRbWarps * 32, 0, s>>>(pr, seg_start, seg_part);
   // forced tokens: dK, dV of the forced part plus the pooled share
   if (cap > 0) {
     int2* fmap = reinterpret_cast<int2*>(wb + b.fmap);
     sb_forced_map_kernel<<<d.n_forced, 64, 0, s>>>(off, d.forced_blocks, fpre, B, d.max_block_len, fmap);
     sb_forced_scatter_kernel<<<148 * 8, 256, 0, s>>>(fmap, ftotal, off, reinterpret_cast<const float*>(wb + b.dkf),
                                                      reinterpret_cast<const float*>(wb + b.dvf), dkbar, dvbar, H, cap,
-                                                     (uint4*)dk, (uint4*)dv);
+                                                     kForcedSplits, cap * H * kSbD, (uint4*)dk, (uint4*)dv);
   }
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
