@@ -52,7 +52,7 @@ def parse():
                          "10-20 s of one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "speed3r", "speed3r_backward", "mixture", "bandwidth"],
+    ap.add_argument("--workload", default="sparse", choices=["sparse", "backward", "dense", "tiny", "speed3r", "speed3r_backward", "mixture", "bandwidth"],
                     help="sparse: the layer forward (the default line); backward: its gradients; dense: the "
                          "dense-stage shape with every block selected; speed3r: the pooled-query variant; "
                          "bandwidth: achieved HBM GB/s of the memory-bound kernels (pooling, routing, combine)")
@@ -672,6 +672,7 @@ def run_backward(args):
 # ------------------------------------------------------------------------------------------------
 EXTRA = {
     "dense": ("sparse-attn fwd tokens/s, dense-stage shape (k = B)", "lsrm_dense_stage_all_blocks"),
+    "tiny": ("sparse-attn fwd tokens/s, score-routed small case", "lsrm_tiny_score_top4"),
     "speed3r": ("sparse-attn fwd tokens/s, Speed3R pooled-query variant", "speed3r_512_frames_top32_forced"),
     "mixture": ("self/cross gated mixture fwd tokens/s, dense-stage shape", "lsrm_dense_stage_self_cross_mixture"),
     "speed3r_backward": ("sparse-attn bwd tokens/s, Speed3R pooled-query variant",
@@ -794,6 +795,12 @@ def run_extra(args):
         def step():
             nsa.lsrm_nsa_forward(desc, off, q, kk, v, gates, None, nsa.ROUTE_ALL, out, None, None, ws)
         launches_per_step = 2  # compress, fused attention over every block
+    if args.workload == "tiny":
+        idx = torch.empty(B, Hkv, k, dtype=torch.int32, device=dev)
+
+        def step():
+            nsa.lsrm_nsa_forward(desc, off, q, kk, v, gates, None, nsa.ROUTE_SCORE, out, idx, None, ws)
+        launches_per_step = 4  # compress, score routing (row splits, then the top-k), fused attention
     for _ in range(max(3, args.warmup)):
         step()
     st = nsa.lsrm_nsa_last_device_status(ws)
@@ -807,8 +814,30 @@ def run_extra(args):
         flops = {kk_: 2.5 * v_ for kk_, v_ in speed3r_flops(w, idx.cpu().numpy()).items()}
     elif args.workload == "mixture":
         flops = mixture_flops(w)
+    elif args.workload == "tiny":
+        flops = algorithmic_flops(w, idx.cpu().numpy())
     else:
         flops = algorithmic_flops(w, np.tile(np.arange(B, dtype=np.int32), (B, 1)))
+    kernel_ms = None
+    if args.workload == "tiny":
+        # the score routing against the fused attention it feeds, each timed alone (CUDA events)
+        kc32 = torch.empty(B, Hkv, d, dtype=torch.float32, device=dev)
+        kc16, vc16 = (torch.empty(B, Hkv, d, dtype=torch.bfloat16, device=dev) for _ in range(2))
+        nsa.lsrm_nsa_compress(desc, off, None, kk, v, kc32, kc16, None, vc16, ws=ws)
+
+        def timed_ms(fn, n=100):
+            for _ in range(5):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            return e0.elapsed_time(e1) / n
+        kernel_ms = {"score_route": timed_ms(lambda: nsa.lsrm_route_score_topk(desc, off, q, kc32, idx, None, ws)),
+                     "fused_attention": timed_ms(lambda: nsa.lsrm_nsa_attend(desc, off, q, kk, v, kc16, vc16, gates,
+                                                                             idx, Hkv, 0, out, None, ws))}
     sampler = ClockSampler(local) if rank == 0 else None
     if world > 1:
         dist.barrier()
@@ -843,6 +872,8 @@ def run_extra(args):
                                         else "lsrm_nsa_forward (all launches of one call)"),
                              "peak_source": f"{src} bf16_tflops (burst)"},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+        if kernel_ms is not None:
+            line["kernel_ms"] = kernel_ms
         if not args.no_cpu_baseline and world == 1 and args.workload == "speed3r_backward":
             tok, dt = speed3r_backward_oracle_sample(args.seed)
             line["cpu_baseline"] = cpu_baseline(tok / dt, f"the whole backward of the 3-frame case ({tok} tokens, "
@@ -905,7 +936,9 @@ def run_extra_reference(args, metric, workload):
     w = make_workload(args.workload, seed=args.seed)
     D = O.desc_for(w.n_tokens, w.n_blocks, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k, w.window,
                    n_gates=w.n_gates, pooled_q=w.pooled_q)
-    qc = kc = None
+    qc = kc = kc_score = None
+    if w.route == "score" and not w.pooled_q:
+        kc_score = O.compress(D, w.off, w.k, w.n_kv_heads)
     if w.pooled_q:
         qc = O.compress(D, w.off, w.q, w.n_q_heads)
         kc = O.compress(D, w.off, w.k, w.n_kv_heads)
@@ -917,6 +950,11 @@ def run_extra_reference(args, metric, workload):
         t0 = time.perf_counter()
         if w.route == "mixture":
             O.mixture(D, w.off, w.q, w.k, w.v, w.gates, w.n_blocks_x, qblocks=qb)
+        elif w.route == "score":
+            rows, _ = O.route_score(D, w.off, w.q, kc_score, qblocks=qb)
+            idx = np.zeros((w.n_blocks, w.n_kv_heads, w.top_k), dtype=np.int32)
+            idx[qb] = rows
+            O.forward(D, w.off, w.q, w.k, w.v, w.gates, idx, qblocks=qb)
         elif w.pooled_q:
             rows, _ = O.route_pooled(D, qc, kc, w.forced, qblocks=qb)
             idx = np.zeros((w.n_blocks, w.n_q_heads, w.top_k), dtype=np.int32)

@@ -161,7 +161,7 @@ struct TcParams {
   // the emitted top-k are block ids
   const int32_t* topk_ids;
   // optional exact ranking: fp32 pooled queries [rows][topk_heads][64] and keys [key rows][heads][64]
-  // (key rows in the stored order) and the largest |key mean| of all keys (float bits); with them
+  // (key rows in the stored order) and the largest L2 norm of a key mean (float bits); with them
   // the candidates are ranked by fp32 logits recomputed from the means, and the gate is widened by
   // a bound on the error of the bf16-operand logits, so the result is the ranking of the exact
   // means rather than of their bf16 roundings
@@ -680,10 +680,12 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     float* cval = acc;
     int* cid = &S.cand_id[t][0][row];
     // exact ranking (see TcParams::rescore_q): every bf16-operand logit lies within err of the
-    // fp32 logit of the means, err = 2^-7 * |q|_1 * max|k| (each operand rounded to bf16 moves a
-    // product by at most 2^-9 of it; the factor leaves room for the fp32 sums).  A key among the
-    // exact k best then has a bf16 logit at least (bound - 2 err), which is where the gate starts,
-    // and after a compaction a key can enter only with a bf16 logit above (k-th exact - err).
+    // fp32 logit of the means, err = (2^-7 + 2^-14) |q|_2 max_j |k_j|_2: rounding each operand to
+    // bf16 moves it by at most 2^-8 of itself, so a product q_i k_i moves by at most
+    // (2^-7 + 2^-16) |q_i k_i|; the fp32 sums of 64 products add at most about 2^-18 of
+    // sum_i |q_i k_i|; and sum_i |q_i k_i| <= |q|_2 |k|_2.  A key among the exact k best then has a bf16
+    // logit at least (bound - 2 err), which is where the gate starts, and after a compaction a key
+    // can enter only with a bf16 logit above (k-th exact - err).
     const bool exact = topk_on && p.rescore_q != nullptr;
     const float* qrow = nullptr;
     const float* kbase = nullptr;
@@ -693,12 +695,15 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       qrow = p.rescore_q + ((size_t)(t0 + R) * p.Hkv + g) * 64;
       kbase = p.rescore_k + (size_t)g * 64;
       kstride = (size_t)p.Hkv * 64;
-      float n1 = 0.f;
-      for (int i = 0; i < 64; ++i) n1 += fabsf(__ldg(qrow + i));
-      err = 0.0078125f * n1 * __uint_as_float(*p.rescore_kmax) + 1e-30f;
+      float n2 = 0.f;
+      for (int i = 0; i < 64; ++i) n2 = fmaf(__ldg(qrow + i), __ldg(qrow + i), n2);
+      // (the extra 2^-7 of the bound also covers the rounding of the fp32 norms themselves)
+      err = 0.0078125f * 1.0078125f * sqrtf(n2) * __uint_as_float(*p.rescore_kmax) + 1e-30f;
     }
     auto topk_compact = [&]() {
       if (ncand > p.topk_k) {
+        // with the exact ranking the buffer is re-scored in fp32 first (keeping the entries within
+        // the error slack of the k-th bf16 value instead was measured slower: too many of them stay)
         if (exact && valid) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
         const KeepBest kb = topk_keep_best(cval, cid, ncand, p.topk_k);
         ncand = kb.n;
@@ -1197,7 +1202,7 @@ lsrm_status launch_mixture(const lsrm_nsa_desc& d, const int32_t* off, int32_t b
 // per-row lower bound on the k-th logit lets the top-k pass skip almost every candidate.  With
 // topk_ids the key rows are stored in another order (forced_bits then marks rows) and the
 // emitted indices are topk_ids[row].  With rescore_q / rescore_k (fp32 pooled queries [n_q][H][64]
-// and keys in the stored row order) and rescore_kmax (the largest |key| as float bits) the top-k
+// and keys in the stored row order) and rescore_kmax (the largest key L2 norm as float bits) the top-k
 // is the ranking of the fp32 logits of the means (see TcParams).
 lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const void* kc, const void* vc,
                               long long kc_rows, int n_ckeys, const int* n_ckeys_dev, float tau, float* obranch,

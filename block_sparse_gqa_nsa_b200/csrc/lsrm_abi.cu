@@ -18,7 +18,8 @@ lsrm_status launch_route_camera(const lsrm_nsa_desc& d, const int32_t* off, cons
                                 int32_t tile_px, const int32_t* tile_block, int32_t radius, int32_t k_vol,
                                 int32_t* cen, int32_t* idx, uint32_t* status, cudaStream_t stream);
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
-                               int32_t* idx, float* score, uint32_t* status, cudaStream_t s);
+                               int32_t* idx, float* score, uint32_t* status, cudaStream_t s, float* scratch,
+                               size_t scratch_bytes);
 lsrm_status launch_gate_combine(const lsrm_nsa_desc& d, const float* oc, const float* os, const float* ow,
                                 const void* gates, void* out, cudaStream_t s);
 lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
@@ -34,7 +35,7 @@ lsrm_status launch_attn_dense(int D, long long n_q, int H, const void* q, const 
                               float* topk_thr, uint32_t* status, cudaStream_t stream,
                               const int32_t* topk_ids = nullptr, const float* rescore_q = nullptr,
                               const float* rescore_k = nullptr, const uint32_t* rescore_kmax = nullptr);
-lsrm_status launch_absmax(const float* x, long long n, uint32_t* out, cudaStream_t s);
+lsrm_status launch_rownorm_max(const float* x, long long rows, uint32_t* out, cudaStream_t s);
 lsrm_status launch_pooled_broadcast(const lsrm_nsa_desc& d, const int32_t* off, const float* o_blk,
                                     const float* lse_blk, float* o_cmp, float* lse, cudaStream_t s);
 lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, const void* k, const void* v,
@@ -77,6 +78,11 @@ T* wsp(void* ws, size_t off) {
 
 uint32_t* status_of(void* ws) { return wsp<uint32_t>(ws, 0); }
 
+// bytes of the workspace's backward scratch region (as workspace_layout sizes it)
+size_t bwd_region_bytes(const lsrm_nsa_desc& d) {
+  return d.pooled_q ? pooled_bwd_layout(d).total : bwd_layout(d, d.n_kv_heads > 0 ? d.n_kv_heads : 1).total;
+}
+
 float tau_of(const lsrm_nsa_desc& d) { return d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim); }
 
 #define LSRM_TRY(x)                         \
@@ -105,7 +111,7 @@ lsrm_status pooled_cmp(const lsrm_nsa_desc& d, const void* qc, const void* kc, c
   }
   const bool exact = idx != nullptr && qc32 != nullptr && kc32 != nullptr;
   if (exact)
-    LSRM_TRY(launch_absmax(kc32, (long long)d.n_blocks * d.n_kv_heads * d.head_dim, wsp<uint32_t>(ws, w.kmax), s));
+    LSRM_TRY(launch_rownorm_max(kc32, (long long)d.n_blocks * d.n_kv_heads, wsp<uint32_t>(ws, w.kmax), s));
   return launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc, kc, vc, d.n_blocks, d.n_blocks, nullptr,
                            tau_of(d), o_blk, l_blk, idx, idx ? d.top_k : 0, idx ? bits : nullptr,
                            idx ? wsp<float>(ws, w.rthr) : nullptr, status_of(ws), s, nullptr,
@@ -146,7 +152,10 @@ lsrm_status lsrm_route_score_topk(const lsrm_nsa_desc* desc, const int32_t* off,
   LSRM_TRY(check_desc(desc));
   LSRM_TRY(check_ws(desc, ws));
   if (off == nullptr || q == nullptr || kc32 == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
-  return launch_route_score(*desc, off, q, kc32, idx, score_or_null, status_of(ws), (cudaStream_t)stream);
+  const Workspace w = workspace_layout(*desc);
+  // the backward scratch is idle during routing: it holds the per-split partial scores
+  return launch_route_score(*desc, off, q, kc32, idx, score_or_null, status_of(ws), (cudaStream_t)stream,
+                            wsp<float>(ws, w.bwd), bwd_region_bytes(*desc));
 }
 
 lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords, int32_t* idx,
@@ -312,7 +321,7 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
     LSRM_TRY(launch_compress(d, off, q, k, v, route ? kc32 : nullptr, kc16, nullptr, vc16, qc32, qc16, s,
                              row_of_block));
     uint32_t* kmax = wsp<uint32_t>(ws, w.kmax);
-    if (route) LSRM_TRY(launch_absmax(kc32, (long long)d.n_blocks * d.n_kv_heads * d.head_dim, kmax, s));
+    if (route) LSRM_TRY(launch_rownorm_max(kc32, (long long)d.n_blocks * d.n_kv_heads, kmax, s));
     float* o_blk = wsp<float>(ws, w.obranch);
     float* l_blk = o_blk + (size_t)d.n_blocks * d.n_q_heads * d.head_dim;
     LSRM_TRY(launch_attn_dense(d.head_dim, d.n_blocks, d.n_q_heads, qc16, kc16, vc16, d.n_blocks, d.n_blocks,
@@ -339,7 +348,8 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
       break;
     case LSRM_ROUTE_SCORE:
       idx_heads = d.n_kv_heads;
-      LSRM_TRY(launch_route_score(d, off, q, kc32, idx, nullptr, status_of(ws), s));
+      LSRM_TRY(launch_route_score(d, off, q, kc32, idx, nullptr, status_of(ws), s, wsp<float>(ws, w.bwd),
+                                  bwd_region_bytes(d)));
       break;
     case LSRM_ROUTE_GEOMETRIC:
       if (coords_or_null == nullptr) return LSRM_ERR_INVALID_ARG;

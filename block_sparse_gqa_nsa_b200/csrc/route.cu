@@ -374,30 +374,92 @@ lsrm_status launch_route_camera(const lsrm_nsa_desc& d, const int32_t* off, cons
 // the scores are reproducible bit for bit.  Then k rounds of arg-max by (score desc, j asc).
 constexpr int kScoreChunk = 32;  // compressed keys per chunk (one register per key per thread)
 constexpr int kMaxScoreRows = 64 * 64;
+constexpr int kMaxScoreSplits = 8;
 
+// k rounds of "best key strictly after the previous winner" by (score desc, j asc) over s_score[B]
+__device__ void score_topk_rounds(const float* s_score, int B, int k, int32_t* dst, float* s_bv, int* s_bj,
+                                  float* s_lv, int* s_lj) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) { *s_lv = INFINITY; *s_lj = -1; }
+  __syncthreads();
+  for (int r = 0; r < k; ++r) {
+    const float lv = *s_lv;
+    const int lj = *s_lj;
+    float bv = -INFINITY;
+    int bj = INT_MAX;
+    for (int j = tid; j < B; j += kRouteThreads) {
+      const float v = s_score[j];
+      const bool after_last = (v < lv) || (v == lv && j > lj);
+      const bool better = (v > bv) || (v == bv && j < bj);
+      if (after_last && better) { bv = v; bj = j; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
+    }
+    if (lane == 0) { s_bv[warp] = bv; s_bj[warp] = bj; }
+    __syncthreads();
+    if (tid == 0) {
+      float v = s_bv[0];
+      int j = s_bj[0];
+      for (int w = 1; w < kRouteThreads / 32; ++w)
+        if (s_bv[w] > v || (s_bv[w] == v && s_bj[w] < j)) { v = s_bv[w]; j = s_bj[w]; }
+      dst[r] = j;
+      *s_lv = v;
+      *s_lj = j;
+    }
+    __syncthreads();
+  }
+}
+
+// Sum of acc[kk] over the warp's lanes for every key kk, by a fixed butterfly: at each stage a lane
+// keeps the half of its keys its lane bit selects and adds the partner's copy of that half, so lane l
+// ends with key l; out[l] receives it.
+__device__ __forceinline__ void warp_key_sums(float (&acc)[kScoreChunk], int lane, float* out) {
+#pragma unroll
+  for (int o = kScoreChunk / 2; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = upper ? acc[i] : acc[i + o];
+      const float keep = upper ? acc[i + o] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  out[lane] = acc[0];
+}
+
+// One CTA per (query block a, KV group g, split of the block's rows).  With one split the CTA also
+// ranks the scores; with several it writes its partial sums part[((a Hkv + g) splits + split)][B]
+// and score_topk_kernel adds the splits in order and ranks.  Per key, the threads' partial sums are
+// added by a fixed shuffle tree within each warp (lane l ends with key l) and then warp by warp.
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
 score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__ q, const float* __restrict__ kc32,
                    int32_t B, int32_t Hq, int32_t Hkv, int32_t k, float scale, int32_t* __restrict__ idx,
-                   float* __restrict__ score_out, uint32_t* status) {
+                   float* __restrict__ score_out, float* __restrict__ part, uint32_t* status) {
   extern __shared__ float smem[];
-  float* s_k = smem;                                   // [kScoreChunk][D] compressed keys of the chunk
-  float* s_part = s_k + kScoreChunk * D;               // [kRouteThreads][kScoreChunk + 1] partial sums
-  float* s_score = s_part + kRouteThreads * (kScoreChunk + 1);  // [B]
+  float* s_k = smem;                                            // [kScoreChunk][D] compressed keys of the chunk
+  float* s_wsum = s_k + kScoreChunk * D;                        // [warps][kScoreChunk] per-warp sums
+  float* s_score = s_wsum + (kRouteThreads / 32) * kScoreChunk;  // [B]
   __shared__ float s_bv[kRouteThreads / 32];
   __shared__ int s_bj[kRouteThreads / 32];
   __shared__ float s_lv;
   __shared__ int s_lj;
-  const int a = blockIdx.x, g = blockIdx.y;
+  const int a = blockIdx.x, g = blockIdx.y, split = blockIdx.z, n_split = gridDim.z;
   const int G = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = off[a];
   // a block longer than the descriptor allows: flag it and clip
   int rows = (off[a + 1] - t0) * G;
   if (rows > kMaxScoreRows) {
-    if (tid == 0) raise_status(status, LSRM_ERR_BOUNDS);
+    if (tid == 0 && split == 0) raise_status(status, LSRM_ERR_BOUNDS);
     rows = kMaxScoreRows;
   }
+  const int rows_per = (rows + n_split - 1) / n_split;
+  const int r_lo = split * rows_per, r_hi = min(rows, r_lo + rows_per);
   const float sl2 = scale * 1.4426950408889634f;  // logits in log2 units
   const int nchunks = (B + kScoreChunk - 1) / kScoreChunk;
   constexpr int kRowsPerThread = kMaxScoreRows / kRouteThreads;
@@ -425,18 +487,63 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
       }
     }
   };
-  // raw logits of one row against the chunk's keys (keys past B give -inf)
+  // raw logits of one row against the chunk's keys (keys past B give -inf and are not computed)
   auto chunk_logits = [&](const float* qv, int c, float* sv) {
+    const int nk = B - c * kScoreChunk;
 #pragma unroll
     for (int kk = 0; kk < kScoreChunk; ++kk) {
       float s = 0.0f;
+      if (kk < nk) {
 #pragma unroll
-      for (int cc = 0; cc < D; ++cc) s = fmaf(qv[cc], s_k[kk * D + cc], s);
-      sv[kk] = c * kScoreChunk + kk < B ? s * sl2 : -INFINITY;
+        for (int cc = 0; cc < D; ++cc) s = fmaf(qv[cc], s_k[kk * D + cc], s);
+      }
+      sv[kk] = kk < nk ? s * sl2 : -INFINITY;
     }
   };
 
-  // pass 1: every row's max and normaliser (each thread its rows r = tid, tid + 256, ...)
+  // one chunk of keys and at most one row per thread: the logits are formed once and kept
+  if (nchunks == 1 && r_hi - r_lo <= kRouteThreads) {
+    float acc[kScoreChunk];
+    const int r = r_lo + tid;
+    float qv[D];
+    if (r < r_hi) load_q(r, qv);  // issued before the keys' copy so the two loads overlap
+    load_chunk(0);
+    if (r < r_hi) {
+      chunk_logits(qv, 0, acc);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int kk = 0; kk < kScoreChunk; ++kk) mx = fmaxf(mx, acc[kk]);
+      float l = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < kScoreChunk; ++kk) {
+        acc[kk] = exp2f(acc[kk] - mx);
+        l += acc[kk];
+      }
+      const float li = 1.0f / l;
+#pragma unroll
+      for (int kk = 0; kk < kScoreChunk; ++kk) acc[kk] *= li;
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < kScoreChunk; ++kk) acc[kk] = 0.0f;
+    }
+    warp_key_sums(acc, lane, s_wsum + warp * kScoreChunk);
+    __syncthreads();
+    if (tid < kScoreChunk && tid < B) {
+      float sum = 0.0f;
+      for (int w = 0; w < kRouteThreads / 32; ++w) sum += s_wsum[w * kScoreChunk + tid];
+      if (n_split > 1) {
+        part[(((size_t)a * Hkv + g) * n_split + split) * B + tid] = sum;
+      } else {
+        s_score[tid] = sum;
+        if (score_out) score_out[((size_t)a * Hkv + g) * B + tid] = sum;
+      }
+    }
+    if (n_split > 1) return;
+    __syncthreads();
+    score_topk_rounds(s_score, B, k, idx + ((size_t)a * Hkv + g) * k, s_bv, s_bj, &s_lv, &s_lj);
+    return;
+  }
+  // pass 1: every row's max and normaliser (each thread its rows r = r_lo + tid, + 256, ...)
   float m[kRowsPerThread], linv[kRowsPerThread];
 #pragma unroll
   for (int i = 0; i < kRowsPerThread; ++i) { m[i] = -INFINITY; linv[i] = 0.0f; }
@@ -444,8 +551,8 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
     load_chunk(c);
 #pragma unroll 1
     for (int i = 0; i < kRowsPerThread; ++i) {
-      const int r = tid + i * kRouteThreads;
-      if (r >= rows) break;
+      const int r = r_lo + tid + i * kRouteThreads;
+      if (r >= r_hi) break;
       float qv[D], sv[kScoreChunk];
       load_q(r, qv);
       chunk_logits(qv, c, sv);
@@ -470,87 +577,112 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
     for (int kk = 0; kk < kScoreChunk; ++kk) acc[kk] = 0.0f;
 #pragma unroll 1
     for (int i = 0; i < kRowsPerThread; ++i) {
-      const int r = tid + i * kRouteThreads;
-      if (r >= rows) break;
+      const int r = r_lo + tid + i * kRouteThreads;
+      if (r >= r_hi) break;
       float qv[D], sv[kScoreChunk];
       load_q(r, qv);
       chunk_logits(qv, c, sv);
 #pragma unroll
       for (int kk = 0; kk < kScoreChunk; ++kk) acc[kk] += exp2f(sv[kk] - m[i]) * linv[i];
     }
-#pragma unroll
-    for (int kk = 0; kk < kScoreChunk; ++kk) s_part[tid * (kScoreChunk + 1) + kk] = acc[kk];
+    warp_key_sums(acc, lane, s_wsum + warp * kScoreChunk);
     __syncthreads();
-    // fixed-order sum over threads: warp w adds threads 32 u + lane ... for key kk = tid % 32
-    for (int kk = tid; kk < kScoreChunk; kk += kRouteThreads) {
-      const int j = c * kScoreChunk + kk;
+    if (tid < kScoreChunk) {
+      const int j = c * kScoreChunk + tid;
       float sum = 0.0f;
-      for (int th = 0; th < kRouteThreads; ++th) sum += s_part[th * (kScoreChunk + 1) + kk];
+      for (int w = 0; w < kRouteThreads / 32; ++w) sum += s_wsum[w * kScoreChunk + tid];
       if (j < B) {
-        s_score[j] = sum;
-        if (score_out) score_out[((size_t)a * Hkv + g) * B + j] = sum;
+        if (n_split > 1) {
+          part[(((size_t)a * Hkv + g) * n_split + split) * B + j] = sum;
+        } else {
+          s_score[j] = sum;
+          if (score_out) score_out[((size_t)a * Hkv + g) * B + j] = sum;
+        }
       }
     }
   }
+  if (n_split > 1) return;
   __syncthreads();
-  // top-k by (score desc, j asc)
-  if (tid == 0) { s_lv = INFINITY; s_lj = -1; }
-  __syncthreads();
-  for (int r = 0; r < k; ++r) {
-    const float lv = s_lv;
-    const int lj = s_lj;
-    float bv = -INFINITY;
-    int bj = INT_MAX;
-    for (int j = tid; j < B; j += kRouteThreads) {
-      const float v = s_score[j];
-      const bool after_last = (v < lv) || (v == lv && j > lj);
-      const bool better = (v > bv) || (v == bv && j < bj);
-      if (after_last && better) { bv = v; bj = j; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-      if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
-    }
-    if (lane == 0) { s_bv[warp] = bv; s_bj[warp] = bj; }
-    __syncthreads();
-    if (tid == 0) {
-      float v = s_bv[0];
-      int j = s_bj[0];
-      for (int w = 1; w < kRouteThreads / 32; ++w)
-        if (s_bv[w] > v || (s_bv[w] == v && s_bj[w] < j)) { v = s_bv[w]; j = s_bj[w]; }
-      idx[((size_t)a * Hkv + g) * k + r] = j;
-      s_lv = v;
-      s_lj = j;
-    }
-    __syncthreads();
+  score_topk_rounds(s_score, B, k, idx + ((size_t)a * Hkv + g) * k, s_bv, s_bj, &s_lv, &s_lj);
+}
+
+// One CTA per (query block, group): the splits' partial scores added in split order, then the top-k.
+__global__ void __launch_bounds__(kRouteThreads)
+score_topk_kernel(const float* __restrict__ part, int n_split, int32_t B, int32_t Hkv, int32_t k,
+                  int32_t* __restrict__ idx, float* __restrict__ score_out) {
+  extern __shared__ float s_score[];
+  __shared__ float s_bv[kRouteThreads / 32];
+  __shared__ int s_bj[kRouteThreads / 32];
+  __shared__ float s_lv;
+  __shared__ int s_lj;
+  const size_t ag = (size_t)blockIdx.x * Hkv + blockIdx.y;
+  // launched as a programmatic dependent of the partial-score kernel: wait for its results here
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  for (int j = threadIdx.x; j < B; j += kRouteThreads) {
+    float sum = 0.0f;
+    for (int sp = 0; sp < n_split; ++sp) sum += part[(ag * n_split + sp) * B + j];
+    s_score[j] = sum;
+    if (score_out) score_out[ag * B + j] = sum;
   }
+  __syncthreads();
+  score_topk_rounds(s_score, B, k, idx + ag * k, s_bv, s_bj, &s_lv, &s_lj);
 }
 
 size_t score_route_smem(int B, int D) {
-  return (size_t)kScoreChunk * D * 4 + (size_t)kRouteThreads * (kScoreChunk + 1) * 4 + (size_t)B * 4;
+  return (size_t)kScoreChunk * D * 4 + (size_t)(kRouteThreads / 32) * kScoreChunk * 4 + (size_t)B * 4;
 }
 
+// scratch / scratch_bytes: room for the per-split partial scores; small problems (few query blocks)
+// split each block's rows over several CTAs so that the GPU is filled
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
-                               int32_t* idx, float* score, uint32_t* status, cudaStream_t stream) {
+                               int32_t* idx, float* score, uint32_t* status, cudaStream_t stream, float* scratch,
+                               size_t scratch_bytes) {
   const int B = d.n_blocks, D = d.head_dim;
   if ((size_t)d.max_block_len * (d.n_q_heads / d.n_kv_heads) > (size_t)kMaxScoreRows) return LSRM_ERR_UNSUPPORTED;
   const size_t smem = score_route_smem(B, D);
   if (smem > 200 * 1024) return LSRM_ERR_UNSUPPORTED;
   const float scale = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)D);
-  dim3 grid((unsigned)B, (unsigned)d.n_kv_heads);
+  const long long ctas = (long long)B * d.n_kv_heads;
+  const int max_rows = d.max_block_len * (d.n_q_heads / d.n_kv_heads);
+  int n_split = (int)((148LL * 4 + ctas - 1) / ctas);
+  n_split = min(n_split, min(kMaxScoreSplits, (max_rows + kRouteThreads - 1) / kRouteThreads));
+  if (n_split < 1) n_split = 1;
+  if (n_split > 1 && (scratch == nullptr || (size_t)ctas * n_split * B * 4 > scratch_bytes)) n_split = 1;
+  dim3 grid((unsigned)B, (unsigned)d.n_kv_heads, (unsigned)n_split);
+  float* part = n_split > 1 ? scratch : nullptr;
   cudaError_t e;
   if (D == 32) {
     e = cudaFuncSetAttribute(score_route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return LSRM_ERR_CUDA;
     score_route_kernel<32><<<grid, kRouteThreads, smem, stream>>>(off, (const uint16_t*)q, kc32, B, d.n_q_heads,
-                                                                  d.n_kv_heads, d.top_k, scale, idx, score, status);
+                                                                  d.n_kv_heads, d.top_k, scale, idx, score, part,
+                                                                  status);
   } else {
     e = cudaFuncSetAttribute(score_route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return LSRM_ERR_CUDA;
     score_route_kernel<64><<<grid, kRouteThreads, smem, stream>>>(off, (const uint16_t*)q, kc32, B, d.n_q_heads,
-                                                                  d.n_kv_heads, d.top_k, scale, idx, score, status);
+                                                                  d.n_kv_heads, d.top_k, scale, idx, score, part,
+                                                                  status);
+  }
+  if (n_split > 1) {
+    const size_t tsmem = (size_t)B * 4;
+    if (cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
+        cudaSuccess)
+      return LSRM_ERR_CUDA;
+    // a programmatic dependent launch: its launch overlaps the tail of the partial-score kernel
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)B, (unsigned)d.n_kv_heads);
+    cfg.blockDim = dim3(kRouteThreads);
+    cfg.dynamicSmemBytes = tsmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, score_topk_kernel, (const float*)part, n_split, (int32_t)B, (int32_t)d.n_kv_heads,
+                           (int32_t)d.top_k, idx, score) != cudaSuccess)
+      return LSRM_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }

@@ -321,19 +321,20 @@ lsrm_status launch_speed3r_forced(const lsrm_nsa_desc& d, const int32_t* off, co
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 
-// Largest |x| over n floats, OR-ed in as float bits (non-negative floats order like their bits):
-// the bound on the pooled keys that sets the width of the exact-ranking gate.  *out must be zero
-// (or a smaller bound) before the launch.
-__global__ void absmax_kernel(const float* __restrict__ x, long long n, uint32_t* out) {
+// Largest L2 norm over the rows of x (rows of 64 floats, the fp32 pooled keys) as float bits (a
+// positive float orders like its bits), the key side of the exact-ranking gate's error bound.
+__global__ void rownorm_max_kernel(const float* __restrict__ x, long long rows, uint32_t* out) {
   float m = 0.f;
-  const float4* x4 = reinterpret_cast<const float4*>(x);
-  const long long n4 = n / 4;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
-    const float4 v = __ldg(x4 + i);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  for (long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += (long long)gridDim.x * blockDim.x) {
+    const float4* x4 = reinterpret_cast<const float4*>(x + r * 64);
+    float s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float4 v = __ldg(x4 + i);
+      s2 = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, s2))));
+    }
+    m = fmaxf(m, sqrtf(s2));
   }
-  for (long long i = 4 * n4 + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
-    m = fmaxf(m, fabsf(x[i]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   __shared__ float wm[32];
@@ -346,12 +347,12 @@ __global__ void absmax_kernel(const float* __restrict__ x, long long n, uint32_t
   }
 }
 
-lsrm_status launch_absmax(const float* x, long long n, uint32_t* out, cudaStream_t s) {
+lsrm_status launch_rownorm_max(const float* x, long long rows, uint32_t* out, cudaStream_t s) {
   if (cudaMemsetAsync(out, 0, sizeof(uint32_t), s) != cudaSuccess) return LSRM_ERR_CUDA;
-  if (n <= 0) return LSRM_OK;
-  const long long want = (n / 4 + 255) / 256;
-  const unsigned blocks = (unsigned)(want < 148 * 8 ? (want > 0 ? want : 1) : 148 * 8);
-  absmax_kernel<<<blocks, 256, 0, s>>>(x, n, out);
+  if (rows <= 0) return LSRM_OK;
+  const long long want = (rows + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
+  rownorm_max_kernel<<<blocks, 256, 0, s>>>(x, rows, out);
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 

@@ -183,7 +183,7 @@ LSRM_API lsrm_status lsrm_route_geometric_noalloc(const lsrm_nsa_desc* desc, con
  * tensors [B][H][d] the tensor cores score with.  With qc32_or_null and
  * kc32_or_null (both or neither; fp32 [B][H][64], 16-byte aligned) the ranking is
  * that of the fp32 pooled means themselves: candidates are gathered from the bf16
- * logits with a gate widened by a bound on their error (2^-7 |qc32|_1 max|kc32|)
+ * logits with a gate widened by a bound on their error (2^-7 |qc32|_2 max_j |kc32_j|_2)
  * and ranked by fp32 dot products of the means; without them it is the ranking of
  * the bf16 operands, products accumulated in fp32.  idx is int32 [B][Hq][top_k]
  * (top_k at most 64, else LSRM_ERR_UNSUPPORTED; a row with fewer eligible blocks
