@@ -325,6 +325,42 @@ __device__ __noinline__ float topk_insert_full(float* val, int* id, int n, float
   return lo;
 }
 
+// The appends of one quarter (16 keys, logits -inf where not eligible) for k above kCand - 16:
+// append while the buffer has room, then each new candidate replaces the worst entry (with the
+// exact ranking, the buffer is re-scored in fp32 once and each newcomer on arrival); returns the
+// buffer count, the gate and whether the buffer holds fp32 logits.
+struct Quarter16 {
+  float v[16];
+};
+struct CandState {
+  int n;
+  float thr;
+  bool rescored;
+};
+__device__ __noinline__ CandState topk_quarter_full(Quarter16 q, int key0, CandState st, float* val, int* id,
+                                                    int cap, bool exact, const float* qrow, const float* kbase,
+                                                    size_t kstride, float err) {
+  for (int i = 0; i < 16; ++i) {
+    float sv = q.v[i];
+    if (!(sv > st.thr)) continue;
+    const int j = key0 + i;
+    if (st.n < cap) {
+      val[st.n * 128] = sv;
+      id[st.n * 128] = j;
+      ++st.n;
+      continue;
+    }
+    if (exact) {
+      if (!st.rescored) topk_rescore(val, id, st.n, qrow, kbase, kstride);
+      st.rescored = true;
+      sv = rescore_dot64(qrow, kbase + (size_t)j * kstride);
+    }
+    const float lo = topk_insert_full(val, id, st.n, sv, j);
+    st.thr = exact ? lo - err : lo;
+  }
+  return st;
+}
+
 // Emit the row's k best in order (logit desc, row asc); a row with fewer than k candidates pads
 // with -1.
 __device__ __noinline__ void topk_emit(const float* val, const int* id, int n, int k, int32_t* dst,
@@ -714,19 +750,9 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     bool rescored = false;  // a full buffer holds the fp32 logits of the means (exact ranking)
     auto topk_append = [&](float sv, int j) {
       if (sv > thr) {
-        if (ncand < C::kCand) {
-          cval[ncand * 128] = sv;
-          cid[ncand * 128] = key_base + j;
-          ++ncand;
-        } else {
-          if (exact && valid) {
-            if (!rescored) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
-            rescored = true;
-            sv = rescore_dot64(qrow, kbase + (size_t)(key_base + j) * kstride);
-          }
-          const float lo = topk_insert_full(cval, cid, ncand, sv, key_base + j);
-          thr = exact ? lo - err : lo;
-        }
+        cval[ncand * 128] = sv;
+        cid[ncand * 128] = key_base + j;
+        ++ncand;
       }
     };
     if (topk_on && p.topk_thr != nullptr && valid) {
@@ -826,10 +852,22 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           }
           // only quarters where some row of the warp has a key above its gate visit the keys
           if (__any_sync(0xffffffffu, qmx > thr)) {
+            if (!big_k) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) topk_append(sv[i], 16 * qd + i);
-            // a quarter appends at most 16 candidates per row
-            if (!big_k && __any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_compact();
+              for (int i = 0; i < 16; ++i) topk_append(sv[i], 16 * qd + i);
+              // a quarter appends at most 16 candidates per row
+              if (__any_sync(0xffffffffu, ncand > C::kCand - 16)) topk_compact();
+            } else {
+              // (one call site: the full-buffer insertion kept out of the unrolled appends)
+              Quarter16 qv;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) qv.v[i] = sv[i];
+              const CandState cs2 = topk_quarter_full(qv, key_base + 16 * qd, CandState{ncand, thr, rescored}, cval,
+                                                      cid, C::kCand, exact && valid, qrow, kbase, kstride, err);
+              ncand = cs2.n;
+              thr = cs2.thr;
+              rescored = cs2.rescored;
+            }
           }
         }
       };
