@@ -713,6 +713,7 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     int key_base = 0;    // block id of key 0 of the current chunk
     uint64_t fmask = 0;  // forced blocks among the chunk's 64 keys (never candidates)
     int ncand = 0;       // this row's buffered candidates
+    int n_exact = 0;     // leading entries that already hold fp32 logits (exact ranking)
     float* cval = acc;
     int* cid = &S.cand_id[t][0][row];
     // exact ranking (see TcParams::rescore_q): every bf16-operand logit lies within err of the
@@ -738,11 +739,15 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     }
     auto topk_compact = [&]() {
       if (ncand > p.topk_k) {
-        // with the exact ranking the buffer is re-scored in fp32 first (keeping the entries within
-        // the error slack of the k-th bf16 value instead was measured slower: too many of them stay)
-        if (exact && valid) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
+        // with the exact ranking the entries appended since the last compaction are re-scored in
+        // fp32 first (the kept ones, first in the buffer, already hold fp32 logits; keeping the
+        // entries within the error slack of the k-th bf16 value instead was measured slower: too
+        // many of them stay)
+        if (exact && valid)
+          topk_rescore(cval + n_exact * 128, cid + n_exact * 128, ncand - n_exact, qrow, kbase, kstride);
         const KeepBest kb = topk_keep_best(cval, cid, ncand, p.topk_k);
         ncand = kb.n;
+        n_exact = kb.n;
         thr = exact ? kb.thr - err : kb.thr;
       }
     };
@@ -1084,7 +1089,8 @@ nsa_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     // the mixture's cross slot over an empty stream: no keys, a zero output and LSE -inf
     if (kMode == kModeMix && cs.n_slc == 0 && valid && p.lse != nullptr) p.lse[orow * p.lse_stride + p.lse_first + 1] = -INFINITY;
     if (ok && topk_on && valid) {
-      if (exact) topk_rescore(cval, cid, ncand, qrow, kbase, kstride);
+      if (exact && rescored) n_exact = ncand;  // a full buffer is fp32 throughout
+      if (exact) topk_rescore(cval + n_exact * 128, cid + n_exact * 128, ncand - n_exact, qrow, kbase, kstride);
       topk_emit(cval, cid, ncand, p.topk_k, p.topk_idx + ((size_t)(t0 + R) * p.Hkv + g) * p.topk_k, p.topk_ids);
     }
     if (ok && cs.total > 0 && wait_all(&S.pv_done[t], (cs.total - 1) & 1)) {
