@@ -18,8 +18,7 @@ lsrm_status launch_route_camera(const lsrm_nsa_desc& d, const int32_t* off, cons
                                 int32_t tile_px, const int32_t* tile_block, int32_t radius, int32_t k_vol,
                                 int32_t* cen, int32_t* idx, uint32_t* status, cudaStream_t stream);
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
-                               int32_t* idx, float* score, uint32_t* status, cudaStream_t s, float* scratch,
-                               size_t scratch_bytes);
+                               int32_t* idx, float* score, uint32_t* status, cudaStream_t s);
 lsrm_status launch_gate_combine(const lsrm_nsa_desc& d, const float* oc, const float* os, const float* ow,
                                 const void* gates, void* out, cudaStream_t s);
 lsrm_status launch_attn(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const void* k, const void* v,
@@ -78,10 +77,6 @@ T* wsp(void* ws, size_t off) {
 
 uint32_t* status_of(void* ws) { return wsp<uint32_t>(ws, 0); }
 
-// bytes of the workspace's backward scratch region (as workspace_layout sizes it)
-size_t bwd_region_bytes(const lsrm_nsa_desc& d) {
-  return d.pooled_q ? pooled_bwd_layout(d).total : bwd_layout(d, d.n_kv_heads > 0 ? d.n_kv_heads : 1).total;
-}
 
 float tau_of(const lsrm_nsa_desc& d) { return d.scale > 0 ? d.scale : 1.0f / sqrtf((float)d.head_dim); }
 
@@ -152,10 +147,7 @@ lsrm_status lsrm_route_score_topk(const lsrm_nsa_desc* desc, const int32_t* off,
   LSRM_TRY(check_desc(desc));
   LSRM_TRY(check_ws(desc, ws));
   if (off == nullptr || q == nullptr || kc32 == nullptr || idx == nullptr) return LSRM_ERR_INVALID_ARG;
-  const Workspace w = workspace_layout(*desc);
-  // the backward scratch is idle during routing: it holds the per-split partial scores
-  return launch_route_score(*desc, off, q, kc32, idx, score_or_null, status_of(ws), (cudaStream_t)stream,
-                            wsp<float>(ws, w.bwd), bwd_region_bytes(*desc));
+  return launch_route_score(*desc, off, q, kc32, idx, score_or_null, status_of(ws), (cudaStream_t)stream);
 }
 
 lsrm_status lsrm_route_geometric(const lsrm_nsa_desc* desc, const int32_t* off, const int32_t* coords, int32_t* idx,
@@ -348,8 +340,7 @@ lsrm_status lsrm_nsa_forward(const lsrm_nsa_desc* desc, const int32_t* off, cons
       break;
     case LSRM_ROUTE_SCORE:
       idx_heads = d.n_kv_heads;
-      LSRM_TRY(launch_route_score(d, off, q, kc32, idx, nullptr, status_of(ws), s, wsp<float>(ws, w.bwd),
-                                  bwd_region_bytes(d)));
+      LSRM_TRY(launch_route_score(d, off, q, kc32, idx, nullptr, status_of(ws), s));
       break;
     case LSRM_ROUTE_GEOMETRIC:
       if (coords_or_null == nullptr) return LSRM_ERR_INVALID_ARG;

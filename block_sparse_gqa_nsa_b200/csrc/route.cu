@@ -14,6 +14,8 @@
 // shared memory across warps): round r returns the best candidate strictly after
 // the one returned by round r-1 in the total order (key, index), so no per-candidate
 // state is kept and ties always go to the lower block index.
+#include <cooperative_groups.h>
+
 #include "lsrm_common.cuh"
 
 namespace lsrm {
@@ -431,15 +433,16 @@ __device__ __forceinline__ void warp_key_sums(float (&acc)[kScoreChunk], int lan
   out[lane] = acc[0];
 }
 
-// One CTA per (query block a, KV group g, split of the block's rows).  With one split the CTA also
-// ranks the scores; with several it writes its partial sums part[((a Hkv + g) splits + split)][B]
-// and score_topk_kernel adds the splits in order and ranks.  Per key, the threads' partial sums are
-// added by a fixed shuffle tree within each warp (lane l ends with key l) and then warp by warp.
+// One CTA per (query block a, KV group g, split of the block's rows).  The splits of one (a, g) form
+// a thread-block cluster (grid z): each CTA leaves its per-key sums in its shared memory, and the
+// cluster's first CTA adds them in split order through distributed shared memory and ranks.  Per
+// key, the threads' partial sums are added by a fixed shuffle tree within each warp (lane l ends
+// with key l) and then warp by warp, so the scores are reproducible bit for bit.
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads)
 score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__ q, const float* __restrict__ kc32,
                    int32_t B, int32_t Hq, int32_t Hkv, int32_t k, float scale, int32_t* __restrict__ idx,
-                   float* __restrict__ score_out, float* __restrict__ part, uint32_t* status) {
+                   float* __restrict__ score_out, uint32_t* status) {
   extern __shared__ float smem[];
   float* s_k = smem;                                            // [kScoreChunk][D] compressed keys of the chunk
   float* s_wsum = s_k + kScoreChunk * D;                        // [warps][kScoreChunk] per-warp sums
@@ -463,6 +466,26 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
   const float sl2 = scale * 1.4426950408889634f;  // logits in log2 units
   const int nchunks = (B + kScoreChunk - 1) / kScoreChunk;
   constexpr int kRowsPerThread = kMaxScoreRows / kRouteThreads;
+  // the CTA's per-key sums are in s_score: add the cluster's splits in order (first CTA), then rank
+  auto finish = [&](float* sc) {
+    if (n_split > 1) {
+      cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+      cluster.sync();  // every split's sums are in its shared memory
+      if (split == 0) {
+        for (int j = tid; j < B; j += kRouteThreads) {
+          float sum = sc[j];
+          for (int r = 1; r < n_split; ++r) sum += cluster.map_shared_rank(sc, r)[j];
+          sc[j] = sum;
+        }
+      }
+      cluster.sync();  // the other splits keep their shared memory until it has been read
+      if (split != 0) return;
+    }
+    __syncthreads();
+    if (score_out)
+      for (int j = tid; j < B; j += kRouteThreads) score_out[((size_t)a * Hkv + g) * B + j] = sc[j];
+    score_topk_rounds(sc, B, k, idx + ((size_t)a * Hkv + g) * k, s_bv, s_bj, &s_lv, &s_lj);
+  };
 
   auto load_chunk = [&](int c) {
     __syncthreads();
@@ -531,16 +554,9 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
     if (tid < kScoreChunk && tid < B) {
       float sum = 0.0f;
       for (int w = 0; w < kRouteThreads / 32; ++w) sum += s_wsum[w * kScoreChunk + tid];
-      if (n_split > 1) {
-        part[(((size_t)a * Hkv + g) * n_split + split) * B + tid] = sum;
-      } else {
-        s_score[tid] = sum;
-        if (score_out) score_out[((size_t)a * Hkv + g) * B + tid] = sum;
-      }
+      s_score[tid] = sum;
     }
-    if (n_split > 1) return;
-    __syncthreads();
-    score_topk_rounds(s_score, B, k, idx + ((size_t)a * Hkv + g) * k, s_bv, s_bj, &s_lv, &s_lj);
+    finish(s_score);
     return;
   }
   // pass 1: every row's max and normaliser (each thread its rows r = r_lo + tid, + 256, ...)
@@ -591,99 +607,60 @@ score_route_kernel(const int32_t* __restrict__ off, const uint16_t* __restrict__
       const int j = c * kScoreChunk + tid;
       float sum = 0.0f;
       for (int w = 0; w < kRouteThreads / 32; ++w) sum += s_wsum[w * kScoreChunk + tid];
-      if (j < B) {
-        if (n_split > 1) {
-          part[(((size_t)a * Hkv + g) * n_split + split) * B + j] = sum;
-        } else {
-          s_score[j] = sum;
-          if (score_out) score_out[((size_t)a * Hkv + g) * B + j] = sum;
-        }
-      }
+      if (j < B) s_score[j] = sum;
     }
   }
-  if (n_split > 1) return;
-  __syncthreads();
-  score_topk_rounds(s_score, B, k, idx + ((size_t)a * Hkv + g) * k, s_bv, s_bj, &s_lv, &s_lj);
-}
-
-// One CTA per (query block, group): the splits' partial scores added in split order, then the top-k.
-__global__ void __launch_bounds__(kRouteThreads)
-score_topk_kernel(const float* __restrict__ part, int n_split, int32_t B, int32_t Hkv, int32_t k,
-                  int32_t* __restrict__ idx, float* __restrict__ score_out) {
-  extern __shared__ float s_score[];
-  __shared__ float s_bv[kRouteThreads / 32];
-  __shared__ int s_bj[kRouteThreads / 32];
-  __shared__ float s_lv;
-  __shared__ int s_lj;
-  const size_t ag = (size_t)blockIdx.x * Hkv + blockIdx.y;
-  // launched as a programmatic dependent of the partial-score kernel: wait for its results here
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  for (int j = threadIdx.x; j < B; j += kRouteThreads) {
-    float sum = 0.0f;
-    for (int sp = 0; sp < n_split; ++sp) sum += part[(ag * n_split + sp) * B + j];
-    s_score[j] = sum;
-    if (score_out) score_out[ag * B + j] = sum;
-  }
-  __syncthreads();
-  score_topk_rounds(s_score, B, k, idx + ag * k, s_bv, s_bj, &s_lv, &s_lj);
+  finish(s_score);
 }
 
 size_t score_route_smem(int B, int D) {
   return (size_t)kScoreChunk * D * 4 + (size_t)(kRouteThreads / 32) * kScoreChunk * 4 + (size_t)B * 4;
 }
 
-// scratch / scratch_bytes: room for the per-split partial scores; small problems (few query blocks)
-// split each block's rows over several CTAs so that the GPU is filled
+// Small problems (few query blocks) split each block's rows over a cluster of up to 8 CTAs so that
+// the GPU is filled.
+template <int D>
+lsrm_status launch_route_score_d(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
+                                 int32_t* idx, float* score, uint32_t* status, cudaStream_t stream, size_t smem,
+                                 int n_split) {
+  if (cudaFuncSetAttribute(score_route_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LSRM_ERR_CUDA;
+  const float scale = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)D);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)d.n_blocks, (unsigned)d.n_kv_heads, (unsigned)n_split);
+  cfg.blockDim = dim3(kRouteThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = (unsigned)n_split;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, score_route_kernel<D>, off, (const uint16_t*)q, kc32, (int32_t)d.n_blocks,
+                         (int32_t)d.n_q_heads, (int32_t)d.n_kv_heads, (int32_t)d.top_k, scale, idx, score,
+                         status) != cudaSuccess)
+    return LSRM_ERR_CUDA;
+  return LSRM_OK;
+}
+
 lsrm_status launch_route_score(const lsrm_nsa_desc& d, const int32_t* off, const void* q, const float* kc32,
-                               int32_t* idx, float* score, uint32_t* status, cudaStream_t stream, float* scratch,
-                               size_t scratch_bytes) {
+                               int32_t* idx, float* score, uint32_t* status, cudaStream_t stream) {
   const int B = d.n_blocks, D = d.head_dim;
   if ((size_t)d.max_block_len * (d.n_q_heads / d.n_kv_heads) > (size_t)kMaxScoreRows) return LSRM_ERR_UNSUPPORTED;
   const size_t smem = score_route_smem(B, D);
   if (smem > 200 * 1024) return LSRM_ERR_UNSUPPORTED;
-  const float scale = d.scale > 0 ? d.scale : 1.0f / sqrtf((float)D);
   const long long ctas = (long long)B * d.n_kv_heads;
   const int max_rows = d.max_block_len * (d.n_q_heads / d.n_kv_heads);
   int n_split = (int)((148LL * 4 + ctas - 1) / ctas);
   n_split = min(n_split, min(kMaxScoreSplits, (max_rows + kRouteThreads - 1) / kRouteThreads));
   if (n_split < 1) n_split = 1;
-  if (n_split > 1 && (scratch == nullptr || (size_t)ctas * n_split * B * 4 > scratch_bytes)) n_split = 1;
-  dim3 grid((unsigned)B, (unsigned)d.n_kv_heads, (unsigned)n_split);
-  float* part = n_split > 1 ? scratch : nullptr;
-  cudaError_t e;
-  if (D == 32) {
-    e = cudaFuncSetAttribute(score_route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return LSRM_ERR_CUDA;
-    score_route_kernel<32><<<grid, kRouteThreads, smem, stream>>>(off, (const uint16_t*)q, kc32, B, d.n_q_heads,
-                                                                  d.n_kv_heads, d.top_k, scale, idx, score, part,
-                                                                  status);
-  } else {
-    e = cudaFuncSetAttribute(score_route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return LSRM_ERR_CUDA;
-    score_route_kernel<64><<<grid, kRouteThreads, smem, stream>>>(off, (const uint16_t*)q, kc32, B, d.n_q_heads,
-                                                                  d.n_kv_heads, d.top_k, scale, idx, score, part,
-                                                                  status);
-  }
-  if (n_split > 1) {
-    const size_t tsmem = (size_t)B * 4;
-    if (cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
-        cudaSuccess)
-      return LSRM_ERR_CUDA;
-    // a programmatic dependent launch: its launch overlaps the tail of the partial-score kernel
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)B, (unsigned)d.n_kv_heads);
-    cfg.blockDim = dim3(kRouteThreads);
-    cfg.dynamicSmemBytes = tsmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, score_topk_kernel, (const float*)part, n_split, (int32_t)B, (int32_t)d.n_kv_heads,
-                           (int32_t)d.top_k, idx, score) != cudaSuccess)
-      return LSRM_ERR_CUDA;
-  }
+  if (d.n_kv_heads > 65535 || n_split > 8) return LSRM_ERR_UNSUPPORTED;
+  const lsrm_status st = D == 32 ? launch_route_score_d<32>(d, off, q, kc32, idx, score, status, stream, smem, n_split)
+                                 : launch_route_score_d<64>(d, off, q, kc32, idx, score, status, stream, smem, n_split);
+  if (st != LSRM_OK) return st;
   return cudaGetLastError() == cudaSuccess ? LSRM_OK : LSRM_ERR_CUDA;
 }
 
