@@ -8,11 +8,14 @@
  *   - compression: per-block mean of K and V (equations k^cmp, v^cmp; the
  *     ResBlock before the pool is a trained module and is not part of this ABI);
  *   - routing picks top-k KV blocks per query block, from compressed attention
- *     scores (standard NSA) or from 3D distances between block centres (the
- *     3D-aware routing paragraph);
+ *     scores (standard NSA), from 3D distances between block centres, or for
+ *     image blocks by projecting the query point into every view (the 3D-aware
+ *     routing paragraph);
  *   - a compressed branch, a selected-block branch and an in-block window branch
  *     run softmax attention and a sigmoid-gated sum combines them (gate
- *     equations w = Sigmoid(Linear(x)); the gate VALUES are inputs here).
+ *     equations w = Sigmoid(Linear(x)); the gate VALUES are inputs here);
+ *   - the dense blocks' decoupled self/cross gated mixture of the volume and
+ *     image streams (the gated cross-attention equations).
  * Speed3R page (gist.science "Speed3R", section 2.1 Global Sparse Attention):
  *   Q/K/V are average-pooled per block, the pooled scores pick the top-k blocks,
  *   the reference frame and camera tokens are always selected (section 2.2), and
@@ -40,7 +43,8 @@
  * Ownership and errors.  Every array pointer is DEVICE memory owned by the
  * caller; the library allocates nothing and keeps no global state (all scratch
  * lives in the caller's workspace, sized by lsrm_nsa_workspace_size and zeroed
- * once by lsrm_nsa_workspace_init).  The descriptor itself is host memory.
+ * once by lsrm_nsa_workspace_init), apart from the fixed centroid array of
+ * lsrm_route_geometric_noalloc (see there).  The descriptor itself is host memory.
  * Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
  * legacy default stream).  The return value reports argument validation and
  * launch errors only.  Faults found while running (a routed index outside
