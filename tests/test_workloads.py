@@ -121,3 +121,26 @@ def test_workloads_are_seeded():
     assert not np.array_equal(a.q, c.q)
     s = bf16_bits_to_f32(a.q).astype(np.float64)
     assert abs(s.std() * math.sqrt(32) - 1.0) < 0.02
+
+
+def test_mixture_workloads_split_the_streams_at_the_volume_blocks():
+    for name, n, nx_blocks in (("mixture", 20480, 64), ("mixture_small", 1024, 8), ("mixture_ragged", 1472, 56)):
+        w = make_workload(name)
+        assert w.n_tokens == n and w.n_blocks_x == nx_blocks and w.n_gates == 2
+        assert w.gates.shape == (n, w.n_q_heads, 2)
+        # volume blocks come first: every volume token lies on the voxel lattice (16 i + 8)
+        vol = w.coords[: w.off[w.n_blocks_x]]
+        assert np.all(vol % 16 == 8)
+
+
+def test_camera_inputs_tables_and_projection_shapes():
+    lay = lsrm_layout(16, 4, 32, 8, (0.3, 0.45), True)
+    from workloads import camera_inputs
+    proj, tiles, tile_px = camera_inputs(lay)
+    tpr = 32 // 8
+    assert proj.shape == (4, 3, 4) and proj.dtype == np.int32 and tiles.shape == (4, tpr, tpr)
+    assert tile_px == 8 and np.abs(proj).max() <= (1 << 23) + 1
+    kept = tiles[tiles >= 0]
+    # every image block appears exactly once, views in order
+    assert sorted(kept.tolist()) == list(range(lay.n_vol_blocks, lay.n_blocks))
+    assert (tiles >= 0).sum(axis=(1, 2)).tolist() == [8] * 4
